@@ -1,0 +1,179 @@
+"""fp64 CPU oracle of the SCOPE per-layer hot path -- TEST INFRASTRUCTURE ONLY.
+
+Only the tests, ``__graft_entry__.smoke()`` and the benchmark's CPU-baseline leg may
+import this package.  It shares no code with the CUDA library; both sides only share
+the seeded input generator.  Each function works on one (batch, head) slice and
+follows the SCOPE equations as cited in ``scope_oracle.c``.
+
+Parity status of each function (what pins it, in tests/test_oracle_pins.py):
+  kmeans     -- pinned: scipy.cluster.vq.kmeans2 (same Lloyd reading), brute-force
+                nearest-centroid, member means, non-increasing objective.
+  select     -- pinned: Eq. 27 closed form (numpy dot with the product-code key),
+                rho=1 keeps everything, uniform logits give ceil(rho*N), rho->0 gives
+                k_fix, k_head against exact rational arithmetic, Eq. 10 invariants,
+                lossless codebook.
+  attention  -- pinned: torch scaled_dot_product_attention (float64, CPU) with the
+                selection as a boolean mask; rho=1 equals dense attention.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+from .build import build as _build
+
+_lib = None
+
+_f32p = np.ctypeslib.ndpointer(np.float32, flags="C_CONTIGUOUS")
+_f64p = np.ctypeslib.ndpointer(np.float64, flags="C_CONTIGUOUS")
+_i32p = np.ctypeslib.ndpointer(np.int32, flags="C_CONTIGUOUS")
+_i64p = np.ctypeslib.ndpointer(np.int64, flags="C_CONTIGUOUS")
+_u16p = np.ctypeslib.ndpointer(np.uint16, flags="C_CONTIGUOUS")
+_u32p = np.ctypeslib.ndpointer(np.uint32, flags="C_CONTIGUOUS")
+_vp = ctypes.c_void_p
+_i64 = ctypes.c_int64
+_int = ctypes.c_int
+_dbl = ctypes.c_double
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        path = _build()
+        L = ctypes.CDLL(path)
+        L.oracle_num_threads.restype = _int
+        L.oracle_kfix.restype = _i64
+        L.oracle_kfix.argtypes = [_dbl, _i64]
+        L.oracle_kmeans.restype = _int
+        L.oracle_kmeans.argtypes = [_f32p, _i64, _i64, _int, _int, _int, _vp, _vp, _int,
+                                    _f64p, _u16p, _i32p, _vp, _vp, _vp]
+        L.oracle_select.restype = _int
+        L.oracle_select.argtypes = [_f64p, _i32p, _f64p, _u16p, _i64, _int, _int, _int, _int,
+                                    _int, _int, _dbl, _dbl, _vp, _i32p, _i32p, _i32p, _i32p,
+                                    _u32p, _vp]
+        L.oracle_attention.restype = _int
+        L.oracle_attention.argtypes = [_f32p, _f32p, _f32p, _i64, _int, _u16p, _u32p, _int,
+                                       _vp, _i64, _f64p]
+        _lib = L
+    return _lib
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def num_threads() -> int:
+    return lib().oracle_num_threads()
+
+
+def kfix(alpha: float, N: int) -> int:
+    return int(lib().oracle_kfix(float(alpha), int(N)))
+
+
+def kmeans(X, ch0, dm, C, iters, init_idx=None, init_cent=None, logs=False):
+    """Lloyd k-means on channels [ch0, ch0+dm) of the rows of X (float32 [N, ld])."""
+    X = np.ascontiguousarray(X, np.float32)
+    N, ld = X.shape
+    if init_idx is not None:
+        init_idx = np.ascontiguousarray(init_idx, np.int32)
+    if init_cent is not None:
+        init_cent = np.ascontiguousarray(init_cent, np.float64)
+    cent = np.empty((C, dm), np.float64)
+    assign = np.empty(N, np.uint16)
+    sizes = np.empty(C, np.int32)
+    margin = np.empty(N, np.float64) if logs else None
+    oa = np.empty(iters, np.float64) if logs else None
+    ou = np.empty(iters, np.float64) if logs else None
+    rc = lib().oracle_kmeans(X, N, ld, ch0, dm, C, _ptr(init_idx), _ptr(init_cent), iters,
+                             cent, assign, sizes, _ptr(margin), _ptr(oa), _ptr(ou))
+    if rc:
+        raise ValueError(f"oracle_kmeans failed ({rc})")
+    out = {"centroids": cent, "assign": assign, "sizes": sizes}
+    if logs:
+        out.update(margin=margin, obj_assign=oa, obj_update=ou)
+    return out
+
+
+def select(qcent, qsizes, kcent, codes, d_split, rho, alpha, want_scores=False):
+    """Eqs. 6-10 for one head.  qcent [Cq, d], kcent [Cm, d], codes [3, N] uint16."""
+    qcent = np.ascontiguousarray(qcent, np.float64)
+    kcent = np.ascontiguousarray(kcent, np.float64)
+    qsizes = np.ascontiguousarray(qsizes, np.int32)
+    codes = np.ascontiguousarray(codes, np.uint16)
+    Cq, d = qcent.shape
+    Cm = kcent.shape[0]
+    N = codes.shape[1]
+    dt, dh, dw = d_split
+    nw = (N + 31) // 32
+    scores = np.empty((Cq, N), np.float64) if want_scores else None
+    p = np.empty(Cq, np.int32)
+    b = np.empty(Cq, np.int32)
+    r = np.empty(Cq, np.int32)
+    kh = np.empty(1, np.int32)
+    mask = np.empty((Cq, nw), np.uint32)
+    margin = np.empty(Cq, np.float64)
+    rc = lib().oracle_select(qcent, qsizes, kcent, codes, N, d, dt, dh, dw, Cq, Cm, float(rho),
+                             float(alpha), _ptr(scores), p, b, kh, r, mask, _ptr(margin))
+    if rc:
+        raise ValueError(f"oracle_select failed ({rc})")
+    out = {"p": p, "b": b, "k_head": int(kh[0]), "r": r, "mask": mask, "topp_margin": margin}
+    if want_scores:
+        out["scores"] = scores
+    return out
+
+
+def attention(Q, K, V, qassign, mask, rows=None):
+    """Sparse attention of the listed query rows (all when None); float64 [nrows, d]."""
+    Q = np.ascontiguousarray(Q, np.float32)
+    K = np.ascontiguousarray(K, np.float32)
+    V = np.ascontiguousarray(V, np.float32)
+    qassign = np.ascontiguousarray(qassign, np.uint16)
+    mask = np.ascontiguousarray(mask, np.uint32)
+    N, d = Q.shape
+    Cq = mask.shape[0]
+    if rows is not None:
+        rows = np.ascontiguousarray(rows, np.int64)
+    nrows = N if rows is None else rows.shape[0]
+    O = np.empty((nrows, d), np.float64)
+    rc = lib().oracle_attention(Q, K, V, N, d, qassign, mask, Cq, _ptr(rows), nrows, O)
+    if rc:
+        raise ValueError(f"oracle_attention failed ({rc})")
+    return O
+
+
+def cluster_keys(K, d_split, Cm, iters, init_idx3=None, init_cent=None, logs=False):
+    """The three subspace k-means of one head's keys.
+
+    Returns centroids [Cm, d] (subspace m's centroid in m's channel range), codes
+    [3, N] uint16 and per-subspace logs.  init_idx3 is [3, Cm]; init_cent is [Cm, d].
+    """
+    N, d = K.shape
+    bounds = [0, d_split[0], d_split[0] + d_split[1], d]
+    cent = np.zeros((Cm, d), np.float64)
+    codes = np.empty((3, N), np.uint16)
+    sizes = np.empty((3, Cm), np.int32)
+    extra = []
+    for m in range(3):
+        ch0, dm = bounds[m], bounds[m + 1] - bounds[m]
+        res = kmeans(K, ch0, dm, Cm, iters,
+                     init_idx=None if init_idx3 is None else init_idx3[m],
+                     init_cent=None if init_cent is None else init_cent[:, ch0:ch0 + dm],
+                     logs=logs)
+        cent[:, ch0:ch0 + dm] = res["centroids"]
+        codes[m] = res["assign"]
+        sizes[m] = res["sizes"]
+        extra.append(res)
+    return {"centroids": cent, "codes": codes, "sizes": sizes, "per_subspace": extra}
+
+
+def forward_head(q, k, v, wl, q_init, k_init, rows=None, logs=False, rho=None):
+    """The whole hot path for one head: clustering, selection, sparse attention."""
+    rho = wl.rho if rho is None else rho
+    qc = kmeans(q, 0, wl.d, wl.Cq, wl.iters, init_idx=q_init, logs=logs)
+    kc = cluster_keys(k, (wl.d_t, wl.d_h, wl.d_w), wl.Cm, wl.iters, init_idx3=k_init, logs=logs)
+    sel = select(qc["centroids"], qc["sizes"], kc["centroids"], kc["codes"],
+                 (wl.d_t, wl.d_h, wl.d_w), rho, wl.alpha)
+    O = attention(q, k, v, qc["assign"], sel["mask"], rows=rows)
+    return {"q": qc, "k": kc, "sel": sel, "O": O}

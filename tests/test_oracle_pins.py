@@ -1,0 +1,273 @@
+"""Pins of the CPU oracle against facts that do not come from the oracle itself.
+
+Each test ties one oracle function to an independent source: a library routine that
+implements the same textbook step (scipy's Lloyd k-means, torch's attention), exact
+rational arithmetic, a closed form that the SCOPE equations imply for a special
+input, or brute force over all subsets of a tiny input.  A dropped term, a wrong sign
+or index, or a transposed operand in the oracle fails at least one of them.
+"""
+import itertools
+import math
+import warnings
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import scipy.cluster.vq as vq
+import torch
+
+import oracle
+from free_sparse_attention_b200 import synth
+from free_sparse_attention_b200.workloads import TINY
+
+
+def _blobs(rng, N, dm, C, spread=0.05):
+    centers = rng.standard_normal((C, dm)) * 3.0
+    lab = rng.integers(0, C, size=N)
+    X = centers[lab] + spread * rng.standard_normal((N, dm))
+    return X.astype(np.float32)
+
+
+# ----------------------------------------------------------------------------- k-means
+@pytest.mark.parametrize("iters", [1, 2, 5])
+@pytest.mark.parametrize("dm,C", [(4, 3), (16, 8), (24, 13)])
+def test_kmeans_matches_scipy_lloyd(iters, dm, C):
+    """Eq. 3 by Lloyd's iteration == scipy.cluster.vq.kmeans2 with the same init."""
+    rng = np.random.default_rng(1000 + 17 * dm + C + iters)
+    X = rng.standard_normal((300, dm)).astype(np.float32)
+    init = rng.choice(300, size=C, replace=False).astype(np.int32)
+    res = oracle.kmeans(X, 0, dm, C, iters, init_idx=init)
+    with warnings.catch_warnings():
+        warnings.simplefilter("ignore")
+        cb, lab = vq.kmeans2(X.astype(np.float64), X[init].astype(np.float64), iter=iters,
+                             minit="matrix", missing="warn")
+    np.testing.assert_array_equal(res["assign"].astype(np.int64), lab)
+    np.testing.assert_allclose(res["centroids"], cb, rtol=1e-12, atol=1e-12)
+    np.testing.assert_array_equal(res["sizes"], np.bincount(lab, minlength=C))
+
+
+def test_kmeans_subspace_channels_match_scipy():
+    """A channel range of a wider row is clustered on exactly those channels."""
+    rng = np.random.default_rng(7)
+    X = rng.standard_normal((257, 64)).astype(np.float32)
+    for ch0, dm in [(0, 16), (16, 24), (40, 24)]:
+        init = rng.choice(257, size=8, replace=False).astype(np.int32)
+        res = oracle.kmeans(X, ch0, dm, 8, 5, init_idx=init)
+        sub = X[:, ch0:ch0 + dm].astype(np.float64)
+        with warnings.catch_warnings():
+            warnings.simplefilter("ignore")
+            cb, lab = vq.kmeans2(sub, sub[init], iter=5, minit="matrix", missing="warn")
+        np.testing.assert_array_equal(res["assign"].astype(np.int64), lab)
+        np.testing.assert_allclose(res["centroids"], cb, rtol=1e-12, atol=1e-12)
+
+
+def test_kmeans_one_iteration_brute_force():
+    """One iteration: every row goes to its nearest init centroid (lowest index on a
+    tie) and every centroid becomes its members' mean (numpy mean)."""
+    rng = np.random.default_rng(3)
+    X = _blobs(rng, 200, 10, 6)
+    init = rng.choice(200, size=6, replace=False).astype(np.int32)
+    res = oracle.kmeans(X, 0, 10, 6, 1, init_idx=init)
+    X64 = X.astype(np.float64)
+    d2 = ((X64[:, None, :] - X64[init][None, :, :]) ** 2).sum(-1)
+    np.testing.assert_array_equal(res["assign"], np.argmin(d2, axis=1))
+    for c in range(6):
+        members = X64[res["assign"] == c]
+        expect = members.mean(0) if len(members) else X64[init[c]]
+        np.testing.assert_allclose(res["centroids"][c], expect, rtol=1e-13, atol=1e-13)
+
+
+def test_kmeans_tie_goes_to_lowest_index_and_empty_keeps_centroid():
+    X = np.array([[0.0], [2.0], [10.0]], np.float32)
+    # centroids -1 and 1 are equidistant from row 0; centroid 100 gets no member
+    res = oracle.kmeans(X, 0, 1, 3, 1, init_cent=np.array([[1.0], [-1.0], [100.0]]))
+    assert list(res["assign"]) == [0, 0, 0]
+    np.testing.assert_allclose(res["centroids"][:, 0], [4.0, -1.0, 100.0])
+    assert list(res["sizes"]) == [3, 0, 0]
+
+
+def test_kmeans_objective_non_increasing():
+    """Lloyd never increases the squared error: assign and update each lower it."""
+    rng = np.random.default_rng(11)
+    X = rng.standard_normal((500, 24)).astype(np.float32)
+    init = rng.choice(500, size=12, replace=False).astype(np.int32)
+    res = oracle.kmeans(X, 0, 24, 12, 8, init_idx=init, logs=True)
+    seq = np.stack([res["obj_assign"], res["obj_update"]], 1).reshape(-1)
+    assert np.all(np.diff(seq) <= 1e-9 * seq[0])
+    # the logged margin is the relative gap to the second-nearest centroid
+    assert np.all(res["margin"] >= 0)
+
+
+# ----------------------------------------------------------------------------- selection
+def _random_select_inputs(rng, N=97, d=16, split=(4, 6, 6), Cq=5, Cm=7):
+    qcent = rng.standard_normal((Cq, d))
+    kcent = rng.standard_normal((Cm, d))
+    codes = rng.integers(0, Cm, size=(3, N)).astype(np.uint16)
+    qsizes = rng.integers(0, 40, size=Cq).astype(np.int32)
+    qsizes[0] = max(qsizes[0], 1)
+    return qcent, qsizes, kcent, codes, split
+
+
+def test_proxy_logit_equals_product_code_inner_product():
+    """Eq. 27: the LUT sum equals <q_c, k_hat_j>/sqrt(d), k_hat_j the concatenation of
+    key j's three subspace centroids."""
+    rng = np.random.default_rng(5)
+    qcent, qsizes, kcent, codes, split = _random_select_inputs(rng)
+    sel = oracle.select(qcent, qsizes, kcent, codes, split, 0.9, 0.1, want_scores=True)
+    d = qcent.shape[1]
+    b = [0, split[0], split[0] + split[1], d]
+    khat = np.empty((codes.shape[1], d))
+    for m in range(3):
+        khat[:, b[m]:b[m + 1]] = kcent[codes[m], b[m]:b[m + 1]]
+    expect = qcent @ khat.T / math.sqrt(d)
+    np.testing.assert_allclose(sel["scores"], expect, rtol=1e-12, atol=1e-13)
+
+
+def _ranking(scores_row):
+    N = scores_row.shape[0]
+    return np.lexsort((np.arange(N), -scores_row))
+
+
+def test_topp_is_minimal_subset_by_brute_force():
+    """Eq. 7: p_c is the least number of keys whose softmax mass reaches rho; over ALL
+    subsets of a tiny key set, no smaller subset reaches it, and the selected keys are
+    the highest-scoring ones (index order on equal scores)."""
+    rng = np.random.default_rng(9)
+    for trial in range(6):
+        N = 11
+        qcent, qsizes, kcent, codes, split = _random_select_inputs(rng, N=N, Cq=3, Cm=3)
+        rho = [0.3, 0.5, 0.7, 0.8, 0.9, 0.95][trial]
+        sel = oracle.select(qcent, qsizes, kcent, codes, split, rho, 0.0, want_scores=True)
+        for c in range(3):
+            s = sel["scores"][c]
+            w = np.exp(s - s.max())
+            Z = w.sum()
+            best = min(len(S) for k in range(1, N + 1) for S in itertools.combinations(range(N), k)
+                       if w[list(S)].sum() >= rho * Z * (1 + 1e-12))
+            assert sel["p"][c] == best, (trial, c)
+
+
+def test_uniform_logits_give_ceil_rho_n():
+    """All keys equal => every key carries mass 1/N => p_c = ceil(rho*N) (closed form)."""
+    N, Cq, Cm, d = 1000, 4, 3, 16
+    rng = np.random.default_rng(2)
+    codes = np.zeros((3, N), np.uint16)
+    for rho in (0.3337, 0.5001, 0.9003, 0.0149):
+        sel = oracle.select(rng.standard_normal((Cq, d)), np.full(Cq, 10, np.int32),
+                            rng.standard_normal((Cm, d)), codes, (4, 6, 6), rho, 0.0)
+        assert np.all(sel["p"] == math.ceil(rho * N))
+
+
+def test_rho_one_keeps_every_key():
+    rng = np.random.default_rng(4)
+    qcent, qsizes, kcent, codes, split = _random_select_inputs(rng, N=70)
+    sel = oracle.select(qcent, qsizes, kcent, codes, split, 1.0, 0.1)
+    assert np.all(sel["p"] == 70) and np.all(sel["r"] == 70) and sel["k_head"] == 70
+    bits = np.unpackbits(sel["mask"].view(np.uint8), bitorder="little").reshape(len(qsizes), -1)
+    assert np.all(bits[:, :70] == 1) and np.all(bits[:, 70:] == 0)
+
+
+def test_tiny_rho_gives_fixed_topk_floor():
+    """rho -> 0 keeps one key by Top-p, so b_c = k_fix = ceil(alpha*N) everywhere and
+    k_head = k_fix; with one query cluster, k_head = b_1."""
+    rng = np.random.default_rng(6)
+    qcent, qsizes, kcent, codes, split = _random_select_inputs(rng, N=200)
+    sel = oracle.select(qcent, qsizes, kcent, codes, split, 1e-12, 0.1)
+    assert np.all(sel["p"] == 1)
+    assert np.all(sel["b"] == 20) and sel["k_head"] == 20 and np.all(sel["r"] == 20)
+    sel1 = oracle.select(qcent[:1], qsizes[:1], kcent, codes, split, 0.6, 0.0)
+    assert sel1["k_head"] == sel1["b"][0]
+
+
+def test_khead_is_exact_weighted_mean_ceiling_and_topup_invariants():
+    """Eq. 9 against exact rationals, Eq. 10 invariants, and the selected sets are
+    prefixes of each cluster's ranking of the sizes r_c."""
+    rng = np.random.default_rng(8)
+    for trial in range(5):
+        qcent, qsizes, kcent, codes, split = _random_select_inputs(rng, N=150, Cq=9, Cm=5)
+        sel = oracle.select(qcent, qsizes, kcent, codes, split, [0.5, 0.7, 0.9, 0.95, 0.99][trial],
+                            0.1, want_scores=True)
+        b, r, kh = sel["b"].astype(int), sel["r"].astype(int), sel["k_head"]
+        expect = math.ceil(Fraction(int(np.dot(qsizes.astype(int), b)), int(qsizes.sum())))
+        assert kh == expect
+        kfix = math.ceil(Fraction(1, 10) * 150)
+        assert np.all(b >= kfix) and np.all(b >= sel["p"]) and kh >= kfix
+        nz = qsizes > 0
+        assert b[nz].min() <= kh <= b[nz].max()
+        assert np.all(r >= kh) and np.all(r[b >= kh] == b[b >= kh]) and np.all(r == np.maximum(b, kh))
+        bits = np.unpackbits(sel["mask"].view(np.uint8), bitorder="little").reshape(9, -1)[:, :150]
+        for c in range(9):
+            top = _ranking(sel["scores"][c])[:r[c]]
+            expect_bits = np.zeros(150, np.uint8)
+            expect_bits[top] = 1
+            np.testing.assert_array_equal(bits[c], expect_bits)
+
+
+def test_lossless_codebook_gives_exact_logits():
+    """Keys whose subspace parts take at most Cm distinct values, clustered from those
+    values, are reproduced exactly (k_hat = k), so the proxy is the true logit."""
+    rng = np.random.default_rng(12)
+    N, d, split, Cm = 120, 16, (4, 6, 6), 5
+    b = [0, 4, 10, 16]
+    K = np.empty((N, d), np.float32)
+    vals = []
+    for m in range(3):
+        v = rng.standard_normal((Cm, b[m + 1] - b[m])).astype(np.float32)
+        pick = rng.integers(0, Cm, size=N)
+        pick[:Cm] = np.arange(Cm)          # every value occurs
+        K[:, b[m]:b[m + 1]] = v[pick]
+        vals.append(pick)
+    init = np.stack([np.arange(Cm, dtype=np.int32)] * 3)
+    kc = oracle.cluster_keys(K, split, Cm, 3, init_idx3=init)
+    for m in range(3):
+        np.testing.assert_array_equal(kc["codes"][m], vals[m])
+    q = rng.standard_normal((2, d))
+    sel = oracle.select(q, np.array([3, 4], np.int32), kc["centroids"], kc["codes"], split,
+                        0.9, 0.1, want_scores=True)
+    np.testing.assert_allclose(sel["scores"], q @ K.astype(np.float64).T / 4.0, rtol=1e-14, atol=1e-14)
+
+
+# ----------------------------------------------------------------------------- attention
+def _sdpa64(Q, K, V, allowed):
+    q = torch.from_numpy(Q.astype(np.float64))[None, None]
+    k = torch.from_numpy(K.astype(np.float64))[None, None]
+    v = torch.from_numpy(V.astype(np.float64))[None, None]
+    m = torch.from_numpy(allowed)[None, None]
+    return torch.nn.functional.scaled_dot_product_attention(q, k, v, attn_mask=m)[0, 0].numpy()
+
+
+def test_attention_equals_masked_sdpa():
+    """Sparse attention over S_c == torch SDPA (float64) with -inf on unselected keys."""
+    rng = np.random.default_rng(13)
+    N, d, Cq = 90, 32, 4
+    Q, K, V = (rng.standard_normal((N, d)).astype(np.float32) for _ in range(3))
+    qassign = rng.integers(0, Cq, size=N).astype(np.uint16)
+    bits = rng.random((Cq, 96)) < 0.4
+    bits[:, 90:] = False
+    bits[:, 0] = True
+    mask = np.packbits(bits.astype(np.uint8), axis=1, bitorder="little").view(np.uint32)
+    O = oracle.attention(Q, K, V, qassign, mask)
+    np.testing.assert_allclose(O, _sdpa64(Q, K, V, bits[qassign][:, :N]), rtol=1e-12, atol=1e-12)
+    rows = np.array([5, 0, 77], np.int64)
+    np.testing.assert_allclose(oracle.attention(Q, K, V, qassign, mask, rows=rows), O[rows],
+                               rtol=0, atol=0)
+
+
+def test_rho_one_forward_is_dense_attention():
+    """With rho = 1 every cluster keeps every key, so the whole hot path reduces to
+    dense softmax attention over the original Q, K, V."""
+    x = synth.layer_inputs(TINY)
+    q, k, v = x["q"][0], x["k"][0], x["v"][0]
+    res = oracle.forward_head(q, k, v, TINY, x["q_init"][0], x["k_init"][0], rho=1.0)
+    dense = _sdpa64(q, k, v, np.ones((TINY.N, TINY.N), bool))
+    np.testing.assert_allclose(res["O"], dense, rtol=1e-12, atol=1e-12)
+
+
+def test_tiny_forward_invariants():
+    x = synth.layer_inputs(TINY)
+    res = oracle.forward_head(x["q"][0], x["k"][0], x["v"][0], TINY, x["q_init"][0],
+                              x["k_init"][0], logs=True)
+    sel = res["sel"]
+    assert res["q"]["sizes"].sum() == TINY.N
+    assert np.all(sel["r"] >= sel["k_head"]) and sel["k_head"] >= oracle.kfix(TINY.alpha, TINY.N)
+    assert np.all(np.isfinite(res["O"]))
