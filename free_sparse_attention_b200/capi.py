@@ -1,0 +1,210 @@
+"""Thin Python binding of libscope.so (the C ABI in include/scope.h).
+
+Argument marshalling only: every step of the SCOPE path runs in the library's CUDA
+kernels.  PyTorch provides device memory and the current stream.  If the library is
+missing or cannot be loaded, every call raises: there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+from .workloads import Workload
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libscope.so")
+
+SCOPE_F32, SCOPE_BF16 = 0, 1
+STATUS = {0: "SCOPE_OK", 1: "SCOPE_ERR_INVALID_ARGUMENT", 2: "SCOPE_ERR_UNSUPPORTED",
+          3: "SCOPE_ERR_WORKSPACE_TOO_SMALL", 4: "SCOPE_ERR_CUDA", 5: "SCOPE_ERR_DEVICE_CHECK"}
+DEV_BAD_INIT_INDEX, DEV_SELECT_TIE, DEV_BAD_ASSIGN = 0x1, 0x2, 0x4
+
+EXPORTS = ("scope_workspace_bytes", "scope_cluster_queries", "scope_cluster_keys",
+           "scope_build_lut_and_select", "scope_sparse_attention", "scope_forward",
+           "scope_status_string", "scope_get_device_status")
+
+
+class ScopeError(RuntimeError):
+    def __init__(self, fn, code):
+        super().__init__(f"{fn} returned {STATUS.get(code, code)}")
+        self.code = code
+
+
+class Params(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("T", ctypes.c_int),
+                ("Hg", ctypes.c_int), ("Wg", ctypes.c_int), ("d", ctypes.c_int),
+                ("d_t", ctypes.c_int), ("d_h", ctypes.c_int), ("d_w", ctypes.c_int),
+                ("Cq", ctypes.c_int), ("Cm", ctypes.c_int), ("iters", ctypes.c_int),
+                ("rho", ctypes.c_double), ("alpha", ctypes.c_double), ("dtype", ctypes.c_int)]
+
+    @classmethod
+    def from_workload(cls, w: Workload, **over) -> "Params":
+        kw = dict(B=w.B, H=w.H, T=w.T, Hg=w.Hg, Wg=w.Wg, d=w.d, d_t=w.d_t, d_h=w.d_h,
+                  d_w=w.d_w, Cq=w.Cq, Cm=w.Cm, iters=w.iters, rho=w.rho, alpha=w.alpha,
+                  dtype=SCOPE_BF16 if w.dtype == "bf16" else SCOPE_F32)
+        kw.update(over)
+        return cls(**kw)
+
+    @property
+    def N(self) -> int:
+        return self.T * self.Hg * self.Wg
+
+    @property
+    def nw(self) -> int:
+        return (self.N + 31) // 32
+
+
+class Intermediates(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in
+                ("q_centroids", "q_assign", "q_sizes", "k_centroids", "k_codes", "topp_counts",
+                 "base_counts", "k_head", "final_counts", "sel_mask")]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Loads libscope.so (raises if it is missing: there is no CPU fallback)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing; build it with free_sparse_attention_b200.build")
+        L = ctypes.CDLL(LIB_PATH)
+        P, vp, sz, i = ctypes.POINTER(Params), ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int
+        L.scope_workspace_bytes.restype = sz
+        L.scope_workspace_bytes.argtypes = [P]
+        L.scope_cluster_queries.restype = i
+        L.scope_cluster_queries.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.scope_cluster_keys.restype = i
+        L.scope_cluster_keys.argtypes = [P, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.scope_build_lut_and_select.restype = i
+        L.scope_build_lut_and_select.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.scope_sparse_attention.restype = i
+        L.scope_sparse_attention.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.scope_forward.restype = i
+        L.scope_forward.argtypes = [P, vp, vp, vp, vp, vp, vp, ctypes.POINTER(Intermediates),
+                                    vp, sz, vp]
+        L.scope_status_string.restype = ctypes.c_char_p
+        L.scope_status_string.argtypes = [i]
+        L.scope_get_device_status.restype = i
+        L.scope_get_device_status.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_int32)]
+        _lib = L
+    return _lib
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(fn, code):
+    if code != 0:
+        raise ScopeError(fn, code)
+
+
+def torch_dtype(p: Params):
+    return torch.bfloat16 if p.dtype == SCOPE_BF16 else torch.float32
+
+
+def workspace_bytes(p: Params) -> int:
+    return int(lib().scope_workspace_bytes(ctypes.byref(p)))
+
+
+def alloc_workspace(p: Params, device="cuda") -> torch.Tensor:
+    n = workspace_bytes(p)
+    if n == 0:
+        raise ScopeError("scope_workspace_bytes", 1)
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def cluster_queries(p, Q, init_idx=None, init_cent=None, ws=None, stream=None):
+    dev = Q.device
+    ws = alloc_workspace(p, dev) if ws is None else ws
+    qc = torch.empty((p.B, p.H, p.Cq, p.d), dtype=torch.float64, device=dev)
+    qa = torch.empty((p.B, p.H, p.N), dtype=torch.uint16, device=dev)
+    qs = torch.empty((p.B, p.H, p.Cq), dtype=torch.int32, device=dev)
+    _check("scope_cluster_queries", lib().scope_cluster_queries(
+        ctypes.byref(p), _ptr(Q), _ptr(init_idx), _ptr(init_cent), _ptr(qc), _ptr(qa), _ptr(qs),
+        _ptr(ws), ws.numel(), _stream(stream)))
+    return qc, qa, qs
+
+
+def cluster_keys(p, K, init_idx=None, init_cent=None, ws=None, stream=None):
+    dev = K.device
+    ws = alloc_workspace(p, dev) if ws is None else ws
+    kc = torch.empty((p.B, p.H, p.Cm, p.d), dtype=torch.float64, device=dev)
+    kk = torch.empty((p.B, p.H, 3, p.N), dtype=torch.uint16, device=dev)
+    _check("scope_cluster_keys", lib().scope_cluster_keys(
+        ctypes.byref(p), _ptr(K), _ptr(init_idx), _ptr(init_cent), _ptr(kc), _ptr(kk), _ptr(ws),
+        ws.numel(), _stream(stream)))
+    return kc, kk
+
+
+def build_lut_and_select(p, q_centroids, q_sizes, k_centroids, k_codes, ws=None, stream=None):
+    dev = q_centroids.device
+    ws = alloc_workspace(p, dev) if ws is None else ws
+    shp = (p.B, p.H, p.Cq)
+    tp = torch.empty(shp, dtype=torch.int32, device=dev)
+    bc = torch.empty(shp, dtype=torch.int32, device=dev)
+    fc = torch.empty(shp, dtype=torch.int32, device=dev)
+    kh = torch.empty((p.B, p.H), dtype=torch.int32, device=dev)
+    mk = torch.empty((p.B, p.H, p.Cq, p.nw), dtype=torch.int32, device=dev)
+    _check("scope_build_lut_and_select", lib().scope_build_lut_and_select(
+        ctypes.byref(p), _ptr(q_centroids), _ptr(q_sizes), _ptr(k_centroids), _ptr(k_codes),
+        _ptr(tp), _ptr(bc), _ptr(kh), _ptr(fc), _ptr(mk), _ptr(ws), ws.numel(), _stream(stream)))
+    return {"topp_counts": tp, "base_counts": bc, "k_head": kh, "final_counts": fc, "sel_mask": mk}
+
+
+def sparse_attention(p, Q, K, V, q_assign, sel_mask, final_counts, ws=None, out=None, stream=None):
+    dev = Q.device
+    ws = alloc_workspace(p, dev) if ws is None else ws
+    O = torch.empty_like(Q) if out is None else out
+    _check("scope_sparse_attention", lib().scope_sparse_attention(
+        ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(V), _ptr(q_assign), _ptr(sel_mask),
+        _ptr(final_counts), _ptr(O), _ptr(ws), ws.numel(), _stream(stream)))
+    return O
+
+
+def forward(p, Q, K, V, q_init_idx, k_init_idx, ws=None, out=None, intermediates=False,
+            stream=None):
+    """The whole layer.  With intermediates=True also returns every stage's outputs."""
+    dev = Q.device
+    ws = alloc_workspace(p, dev) if ws is None else ws
+    O = torch.empty_like(Q) if out is None else out
+    inter = None
+    tensors = {}
+    if intermediates:
+        shp = (p.B, p.H)
+        tensors = {
+            "q_centroids": torch.empty(shp + (p.Cq, p.d), dtype=torch.float64, device=dev),
+            "q_assign": torch.empty(shp + (p.N,), dtype=torch.uint16, device=dev),
+            "q_sizes": torch.empty(shp + (p.Cq,), dtype=torch.int32, device=dev),
+            "k_centroids": torch.empty(shp + (p.Cm, p.d), dtype=torch.float64, device=dev),
+            "k_codes": torch.empty(shp + (3, p.N), dtype=torch.uint16, device=dev),
+            "topp_counts": torch.empty(shp + (p.Cq,), dtype=torch.int32, device=dev),
+            "base_counts": torch.empty(shp + (p.Cq,), dtype=torch.int32, device=dev),
+            "k_head": torch.empty(shp, dtype=torch.int32, device=dev),
+            "final_counts": torch.empty(shp + (p.Cq,), dtype=torch.int32, device=dev),
+            "sel_mask": torch.empty(shp + (p.Cq, p.nw), dtype=torch.int32, device=dev),
+        }
+        inter = Intermediates(**{k: v.data_ptr() for k, v in tensors.items()})
+    _check("scope_forward", lib().scope_forward(
+        ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(V), _ptr(q_init_idx), _ptr(k_init_idx), _ptr(O),
+        ctypes.byref(inter) if inter is not None else None, _ptr(ws), ws.numel(), _stream(stream)))
+    if intermediates:
+        return O, tensors
+    return O
+
+
+def get_device_status(ws, stream=None) -> int:
+    out = ctypes.c_int32(0)
+    code = lib().scope_get_device_status(_ptr(ws), _stream(stream), ctypes.byref(out))
+    if code not in (0, 5):
+        raise ScopeError("scope_get_device_status", code)
+    return int(out.value)

@@ -1,0 +1,115 @@
+// Internal declarations shared by the SCOPE CUDA sources (not part of the C ABI).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/scope.h"
+
+namespace scope {
+
+constexpr int kMaxC = 2048;         // max centroids per problem (LUT and histogram sizes)
+constexpr int kSortChunk = 512;     // tokens per warp in the stable counting sort
+constexpr int kAttnTile = 128;      // queries per attention tile
+
+// ---------------------------------------------------------------------------------
+// Clustering problems.  Role 0 = queries (all d channels, C = Cq); roles 1..3 = the
+// key subspaces T, H, W (their channel range, C = Cm).  A launch covers a contiguous
+// range of roles for every (b, h): problem index p = bh * nroles + (role - role0).
+struct RoleDesc {
+    const void *X;        // [BH, N, d] input (Q or K)
+    int ch0, dm, C;       // channel range and centroid count
+    double *cent;         // fp64 centroids, element (bh, c, i) at cent[bh*C*d + c*d + i]
+    uint16_t *assign;     // assignments, element (bh, j) at assign[bh*assign_bh + j]
+    long long assign_bh;  // bh stride of assign
+    int32_t *sizes;       // member counts, (bh, c) at sizes[bh*sizes_bh + c]
+    long long sizes_bh;
+    const int32_t *init_idx;   // initial centroid rows, (bh, c) at init_idx[bh*init_bh + c]
+    long long init_bh;
+    const double *init_cent;   // or initial centroids, same layout as cent
+};
+
+struct KmArgs {
+    RoleDesc role[4];
+    int role0, nroles;
+    int BH, N, d;
+    int is_bf16;
+    // per-problem scratch (problem p = bh*nroles + r)
+    float *cent32;        // [P, ds, Cs] fp32 centroids, transposed
+    float *cnorm;         // [P, Cs]  ||mu32_c|| rounded up
+    float *cnrm2;         // [P, Cs]  ||mu_c||^2 rounded to fp32
+    float *cslack;        // [P, Cs]  2^-22 ||mu_c||^2 rounded up (error-bound term)
+    int Cs, ds;           // strides: max C and max dm over the launched roles
+    int32_t *perm;        // [P, N] members sorted by cluster, token order inside
+    int32_t *off;         // [P, Cs+1] segment offsets into perm
+    int32_t *chunk_hist;  // [P, nchunk, Cs] per-chunk counts -> prefix
+    int nchunk;
+    int32_t *status;      // device status word
+};
+
+// Workspace layout (byte offsets); computed identically by every entry point.
+struct WsLayout {
+    size_t status, counters;
+    size_t cent32, cnorm, cnrm2, cslack, perm, off, chunk_hist;
+    size_t q_cent, q_assign, q_sizes, k_cent, k_codes, k_sizes;
+    size_t topp, base, khead, final_cnt, mask, sel_state;
+    size_t q_perm, q_off, q_hist, work_items, attn_counter;
+    size_t total;
+};
+
+WsLayout ws_layout(const scope_params &p);
+
+// Launchers (enqueue only; return cudaGetLastError()).
+cudaError_t km_run(KmArgs a, int iters, cudaStream_t s);
+cudaError_t sort_by_cluster(KmArgs a, cudaStream_t s);  // stable counting sort, all problems
+
+struct SelArgs {
+    const double *qcent;      // [BH, Cq, d]
+    const int32_t *qsizes;    // [BH, Cq]
+    const double *kcent;      // [BH, Cm, d]
+    const uint16_t *codes;    // [BH, 3, N]
+    int32_t *topp, *base, *khead, *final_cnt;
+    uint32_t *mask;           // [BH, Cq, nw]
+    double *state;            // [BH*Cq, 8] per-unit selection state
+    int BH, N, d, dt, dh, dw, Cq, Cm, nw;
+    double rho, inv_sqrt_d;
+    int kfix;
+    int32_t *status;
+};
+cudaError_t select_run(const SelArgs &a, cudaStream_t s);
+
+struct AttnArgs {
+    const void *Q, *K, *V;
+    void *O;
+    const int32_t *perm;      // queries sorted by cluster, (bh, m) at perm[bh*perm_bh + m]
+    const int32_t *off;       // cluster offsets into perm, (bh, c) at off[bh*off_bh + c]
+    long long perm_bh, off_bh;
+    const uint32_t *mask;     // [BH, Cq, nw]
+    const int32_t *final_cnt; // [BH, Cq]
+    int4 *items;              // work list (bh, c, q0, nq)
+    int32_t *counter;         // [2]: item count, dynamic scheduler
+    int BH, N, d, Cq, nw, is_bf16;
+    int use_tc;               // bf16 on the tensor cores (else CUDA cores)
+    float scale_log2;         // log2(e)/sqrt(d)
+    int32_t *status;
+    int num_sms;
+};
+cudaError_t attention_run(const AttnArgs &a, cudaStream_t s);
+cudaError_t attention_simt_run(const AttnArgs &a, cudaStream_t s);
+size_t select_smem_bytes(int Cm, int d);
+
+// ---------------------------------------------------------------------------------
+__device__ __forceinline__ float load_x(const void *X, long long idx, int is_bf16)
+{
+    if (is_bf16)
+        return __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(X)[idx]);
+    return reinterpret_cast<const float *>(X)[idx];
+}
+
+__device__ __forceinline__ void set_status(int32_t *status, int bits)
+{
+    if (status) atomicOr(status, bits);
+}
+
+}  // namespace scope

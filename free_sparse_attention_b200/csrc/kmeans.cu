@@ -1,0 +1,492 @@
+// Lloyd k-means for SCOPE's query clustering and key-subspace clustering.
+//
+// SCOPE (arXiv 2608.12780) clusters post-RoPE queries (Cq centroids) and, per 3D-RoPE
+// subspace, post-RoPE keys (Cm centroids each) with k-means minimising the Euclidean
+// reconstruction error (review page, load_bearing_attack: Eq. 3).  One iteration:
+// every token goes to its nearest centroid (lowest index on a tie), then every
+// non-empty centroid moves to the mean of its members.
+//
+// Design (B200): the assignment is a [tokens x dm] x [dm x C] contraction followed by
+// an argmin.  It runs on the fp32 FMA pipes with centroids staged in shared memory;
+// each distance carries a rigorous error bound, and a token whose best and runner-up
+// cannot be told apart under that bound is re-decided in binary64 with the channels
+// summed in order (one rounding per operation).  Hence the assignment equals a
+// binary64 evaluation of the definition exactly.  The update sums each centroid's
+// members in increasing token order in binary64: a stable counting sort by cluster
+// gives every (centroid, channel) pair its member list, so the sum is sequential and
+// the means are bit-identical to an in-order binary64 evaluation.
+#include "common.cuh"
+
+#include <cfloat>
+
+namespace scope {
+
+namespace {
+
+constexpr int kTok = 128;     // tokens per CTA in the fast assignment
+constexpr int kCC = 64;       // centroids per shared-memory chunk
+constexpr int kAssignThreads = 256;
+constexpr uint16_t kUnsure = 0xFFFF;
+
+__device__ __forceinline__ const RoleDesc &role_of(const KmArgs &a, int p, int &bh, int &r)
+{
+    r = p % a.nroles;
+    bh = p / a.nroles;
+    return a.role[a.role0 + r];
+}
+
+// Squared distance in binary64, channels in order, separate multiply and add.
+__device__ __forceinline__ double sqdist64(const void *X, long long xrow, int is_bf16,
+                                           const double *mu, int dm)
+{
+    double acc = 0.0;
+    for (int i = 0; i < dm; ++i) {
+        double diff = __dsub_rn((double)load_x(X, xrow + i, is_bf16), mu[i]);
+        acc = __dadd_rn(acc, __dmul_rn(diff, diff));
+    }
+    return acc;
+}
+
+// fp32 copy, norms and the error-bound term of one centroid row (cent64 has dm
+// values, all written before the caller's barrier).  Thread i handles channel i.
+__device__ void finalize_row(const KmArgs &a, int p, int c, const double *cent64, int dm, int i)
+{
+    float *cent32T = a.cent32 + (size_t)p * a.Cs * a.ds;
+    cent32T[(size_t)i * a.Cs + c] = __double2float_rn(cent64[i]);
+    if (i == 0) {
+        double n2 = 0.0, n32 = 0.0;
+        for (int k = 0; k < dm; ++k) {
+            double m = cent64[k];
+            double m32 = (double)__double2float_rn(m);
+            n2 += m * m;
+            n32 += m32 * m32;
+        }
+        a.cnrm2[(size_t)p * a.Cs + c] = __double2float_rn(n2);
+        a.cnorm[(size_t)p * a.Cs + c] = __double2float_ru(sqrt(n32));
+        a.cslack[(size_t)p * a.Cs + c] = __double2float_ru(ldexp(n2, -22));
+    }
+}
+
+// ------------------------------------------------------------------------- init
+// grid (ceil(Cs/G), P), block 128: a group of dm threads per centroid.
+__global__ void __launch_bounds__(128) km_init_kernel(KmArgs a)
+{
+    int bh, r;
+    const int p = blockIdx.y;
+    const RoleDesc &R = role_of(a, p, bh, r);
+    const int dm = R.dm, G = max(1, 128 / dm);
+    const int g = threadIdx.x / dm, i = threadIdx.x % dm;
+    const int c = blockIdx.x * G + g;
+    const bool active = g < G && c < R.C;
+    double *cent = R.cent + ((size_t)bh * R.C + c) * a.d + R.ch0;
+    if (active) {
+        if (R.init_idx) {
+            int row = R.init_idx[(size_t)bh * R.init_bh + c];
+            if (row < 0 || row >= a.N) {
+                if (i == 0) set_status(a.status, SCOPE_DEV_BAD_INIT_INDEX);
+                row = 0;
+            }
+            cent[i] = (double)load_x(R.X, ((long long)bh * a.N + row) * a.d + R.ch0 + i, a.is_bf16);
+        } else {
+            cent[i] = R.init_cent[((size_t)bh * R.C + c) * a.d + R.ch0 + i];
+        }
+    }
+    __syncthreads();
+    if (active) finalize_row(a, p, c, cent, dm, i);
+}
+
+// ------------------------------------------------------------------------- fast assignment
+// grid (ceil(N/kTok), P), block 256.  Thread (ty, tx): tokens ty*8..+8, chunk
+// centroids tx*4..+4.  For every pair the fp32 score A = |mu|^2 - 2 x.mu approximates
+// S = |mu|^2 - 2 x.mu (exact, binary64 mu) within
+//     E = 2^-22 ((dm+3) |x| |mu| + |mu|^2) + 2^-40 |x|^2,
+// twice the first-order bound of the three roundings (mu to fp32, the fp32 dot
+// product, the final subtraction) plus the binary64 rounding of the reference sum.
+// With L = A - E and U = A + E, the token's winner is certain when the second-smallest
+// L exceeds the smallest U; otherwise the token is marked for the exact path.
+__global__ void __launch_bounds__(kAssignThreads) km_assign_fast_kernel(KmArgs a)
+{
+    int bh, r;
+    const int p = blockIdx.y;
+    const RoleDesc &R = role_of(a, p, bh, r);
+    const int dm = R.dm, C = R.C;
+    const int j0 = blockIdx.x * kTok;
+    if (j0 >= a.N) return;
+    extern __shared__ __align__(16) float sm[];
+    float *Xs = sm;                     // [dm][kTok]
+    float *Ms = Xs + dm * kTok;         // [dm][kCC]
+    float *Mn2 = Ms + dm * kCC;         // [kCC]
+    float *Mnorm = Mn2 + kCC;           // [kCC]
+    float *Mslack = Mnorm + kCC;        // [kCC]
+    float *Xn = Mslack + kCC;           // [kTok]
+
+    const int tid = threadIdx.x;
+    for (int idx = tid; idx < kTok * dm; idx += kAssignThreads) {
+        int t = idx / dm, i = idx - t * dm;
+        int j = j0 + t;
+        float v = 0.f;
+        if (j < a.N) v = load_x(R.X, ((long long)bh * a.N + j) * a.d + R.ch0 + i, a.is_bf16);
+        Xs[i * kTok + t] = v;
+    }
+    __syncthreads();
+    if (tid < kTok) {
+        float s = 0.f;
+        for (int i = 0; i < dm; ++i) s = fmaf(Xs[i * kTok + tid], Xs[i * kTok + tid], s);
+        Xn[tid] = sqrtf(s) * (1.0f + 0x1p-12f);
+    }
+    const int ty = tid >> 4, tx = tid & 15;
+    float xk[8], e0[8], minL[8], min2L[8], minU[8];
+    int idxL[8];
+    __syncthreads();
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+        float xn = Xn[ty * 8 + t];
+        xk[t] = 0x1p-22f * (float)(dm + 3) * xn;
+        e0[t] = 0x1p-40f * xn * xn;
+        minL[t] = FLT_MAX;
+        min2L[t] = FLT_MAX;
+        minU[t] = FLT_MAX;
+        idxL[t] = 0;
+    }
+    const float *cent32T = a.cent32 + (size_t)p * a.Cs * a.ds;
+    const float *cn2 = a.cnrm2 + (size_t)p * a.Cs;
+    const float *cnm = a.cnorm + (size_t)p * a.Cs;
+    const float *csl = a.cslack + (size_t)p * a.Cs;
+
+    for (int c0 = 0; c0 < C; c0 += kCC) {
+        __syncthreads();
+        for (int idx = tid; idx < dm * kCC; idx += kAssignThreads) {
+            int i = idx / kCC, cc = idx - i * kCC;
+            Ms[idx] = (c0 + cc < C) ? cent32T[(size_t)i * a.Cs + c0 + cc] : 0.f;
+        }
+        if (tid < kCC) {
+            bool ok = c0 + tid < C;
+            Mn2[tid] = ok ? cn2[c0 + tid] : INFINITY;
+            Mnorm[tid] = ok ? cnm[c0 + tid] : 0.f;
+            Mslack[tid] = ok ? csl[c0 + tid] : 0.f;
+        }
+        __syncthreads();
+        float acc[8][4];
+#pragma unroll
+        for (int t = 0; t < 8; ++t)
+#pragma unroll
+            for (int b = 0; b < 4; ++b) acc[t][b] = 0.f;
+#pragma unroll 4
+        for (int i = 0; i < dm; ++i) {
+            const float4 xa = *reinterpret_cast<const float4 *>(Xs + i * kTok + ty * 8);
+            const float4 xb = *reinterpret_cast<const float4 *>(Xs + i * kTok + ty * 8 + 4);
+            const float4 m = *reinterpret_cast<const float4 *>(Ms + i * kCC + tx * 4);
+            const float xv[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+            const float mv[4] = {m.x, m.y, m.z, m.w};
+#pragma unroll
+            for (int t = 0; t < 8; ++t)
+#pragma unroll
+                for (int b = 0; b < 4; ++b) acc[t][b] = fmaf(xv[t], mv[b], acc[t][b]);
+        }
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+            const int cc = tx * 4 + b;
+            const float n2 = Mn2[cc], nm = Mnorm[cc], sl = Mslack[cc];
+#pragma unroll
+            for (int t = 0; t < 8; ++t) {
+                float A = fmaf(-2.f, acc[t][b], n2);
+                float E = fmaf(xk[t], nm, sl + e0[t]);
+                float L = A - E, U = A + E;
+                if (L < minL[t]) {
+                    min2L[t] = minL[t];
+                    minL[t] = L;
+                    idxL[t] = c0 + cc;
+                } else if (L < min2L[t]) {
+                    min2L[t] = L;
+                }
+                minU[t] = fminf(minU[t], U);
+            }
+        }
+    }
+    // merge the 16 partial states of each token (lanes sharing ty)
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+#pragma unroll
+        for (int off = 1; off < 16; off <<= 1) {
+            float oL = __shfl_xor_sync(0xffffffffu, minL[t], off);
+            float o2 = __shfl_xor_sync(0xffffffffu, min2L[t], off);
+            float oU = __shfl_xor_sync(0xffffffffu, minU[t], off);
+            int oi = __shfl_xor_sync(0xffffffffu, idxL[t], off);
+            if (oL < minL[t] || (oL == minL[t] && oi < idxL[t])) {
+                min2L[t] = fminf(o2, minL[t]);
+                minL[t] = oL;
+                idxL[t] = oi;
+            } else {
+                min2L[t] = fminf(min2L[t], oL);
+            }
+            minU[t] = fminf(minU[t], oU);
+        }
+    }
+    // lane tx writes token ty*8 + tx for tx < 8
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+        if (tx == t) {
+            int j = j0 + ty * 8 + t;
+            if (j < a.N) {
+                bool sure = min2L[t] > minU[t];
+                R.assign[(size_t)bh * R.assign_bh + j] = sure ? (uint16_t)idxL[t] : kUnsure;
+            }
+        }
+    }
+}
+
+// ------------------------------------------------------------------------- exact assignment
+// One warp per group of 32 tokens (grid-stride); every unsure token is re-decided in
+// binary64 against all centroids, lanes striding over the centroids.
+__global__ void __launch_bounds__(256) km_assign_exact_kernel(KmArgs a)
+{
+    const int lane = threadIdx.x & 31;
+    const int ngroups = (a.N + 31) / 32;
+    const long long total = (long long)a.BH * a.nroles * ngroups;
+    const long long nwarps = (long long)gridDim.x * (blockDim.x / 32);
+    for (long long g = (long long)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32; g < total;
+         g += nwarps) {
+        const int p = (int)(g / ngroups);
+        int bh, r;
+        const RoleDesc &R = role_of(a, p, bh, r);
+        const int j = (int)(g % ngroups) * 32 + lane;
+        uint16_t *asg = R.assign + (size_t)bh * R.assign_bh;
+        bool unsure = j < a.N && asg[j] == kUnsure;
+        unsigned todo = __ballot_sync(0xffffffffu, unsure);
+        while (todo) {
+            const int src = __ffs(todo) - 1;
+            todo &= todo - 1;
+            const int jj = (int)(g % ngroups) * 32 + src;
+            const long long xrow = ((long long)bh * a.N + jj) * a.d + R.ch0;
+            double best = INFINITY;
+            int bi = 0x7fffffff;
+            for (int c = lane; c < R.C; c += 32) {
+                const double *mu = R.cent + ((size_t)bh * R.C + c) * a.d + R.ch0;
+                double dd = sqdist64(R.X, xrow, a.is_bf16, mu, R.dm);
+                if (dd < best) {
+                    best = dd;
+                    bi = c;
+                }
+            }
+            for (int off = 16; off; off >>= 1) {
+                double ob = __shfl_xor_sync(0xffffffffu, best, off);
+                int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+                if (ob < best || (ob == best && oi < bi)) {
+                    best = ob;
+                    bi = oi;
+                }
+            }
+            if (lane == 0) asg[jj] = (uint16_t)bi;
+        }
+    }
+}
+
+// ------------------------------------------------------------------------- counting sort
+// Chunk histogram: one warp per chunk of kSortChunk tokens, block of 4 warps.
+__global__ void __launch_bounds__(128) sort_hist_kernel(KmArgs a)
+{
+    extern __shared__ int hs[];
+    const int w = threadIdx.x / 32, lane = threadIdx.x & 31;
+    const int k = blockIdx.x * 4 + w;
+    const int p = blockIdx.y;
+    int bh, r;
+    const RoleDesc &R = role_of(a, p, bh, r);
+    if (k >= a.nchunk) return;
+    int *h = hs + w * a.Cs;
+    for (int c = lane; c < R.C; c += 32) h[c] = 0;
+    __syncwarp();
+    const uint16_t *asg = R.assign + (size_t)bh * R.assign_bh;
+    const int jend = min(a.N, (k + 1) * kSortChunk);
+    for (int j = k * kSortChunk + lane; j < jend; j += 32) {
+        int z = asg[j];
+        if (z >= R.C) {   // only a caller-supplied assignment can be out of range
+            set_status(a.status, SCOPE_DEV_BAD_ASSIGN);
+            z = R.C - 1;
+        }
+        atomicAdd(&h[z], 1);
+    }
+    __syncwarp();
+    int32_t *out = a.chunk_hist + ((size_t)p * a.nchunk + k) * a.Cs;
+    for (int c = lane; c < R.C; c += 32) out[c] = h[c];
+}
+
+// Per problem: prefix over chunks for every cluster, sizes, and cluster offsets.
+__global__ void __launch_bounds__(1024) sort_scan_kernel(KmArgs a)
+{
+    __shared__ int wsum[32];
+    const int p = blockIdx.x;
+    int bh, r;
+    const RoleDesc &R = role_of(a, p, bh, r);
+    const int C = R.C;
+    const int per = (C + 1023) / 1024;
+    int loc[4];  // C <= 4096
+    int tot = 0;
+    for (int q = 0; q < per; ++q) {
+        int c = threadIdx.x * per + q;
+        int run = 0;
+        if (c < C) {
+            int32_t *col = a.chunk_hist + (size_t)p * a.nchunk * a.Cs + c;
+            for (int k = 0; k < a.nchunk; ++k) {
+                int h = col[(size_t)k * a.Cs];
+                col[(size_t)k * a.Cs] = run;
+                run += h;
+            }
+            R.sizes[(size_t)bh * R.sizes_bh + c] = run;
+        }
+        loc[q] = run;
+        tot += run;
+    }
+    // exclusive block scan of tot
+    const int lane = threadIdx.x & 31, wid = threadIdx.x / 32;
+    int v = tot;
+    for (int o = 1; o < 32; o <<= 1) {
+        int n = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += n;
+    }
+    if (lane == 31) wsum[wid] = v;
+    __syncthreads();
+    if (wid == 0) {
+        int s = wsum[lane];
+        for (int o = 1; o < 32; o <<= 1) {
+            int n = __shfl_up_sync(0xffffffffu, s, o);
+            if (lane >= o) s += n;
+        }
+        wsum[lane] = s;
+    }
+    __syncthreads();
+    int excl = v - tot + (wid ? wsum[wid - 1] : 0);
+    int32_t *off = a.off + (size_t)p * (a.Cs + 1);
+    for (int q = 0; q < per; ++q) {
+        int c = threadIdx.x * per + q;
+        if (c < C) off[c] = excl;
+        excl += loc[q];
+    }
+    if (threadIdx.x == 0) off[C] = a.N;
+}
+
+// Stable scatter: warp k walks its chunk in token order, 32 tokens at a time.
+__global__ void __launch_bounds__(128) sort_scatter_kernel(KmArgs a)
+{
+    extern __shared__ int cs[];
+    const int w = threadIdx.x / 32, lane = threadIdx.x & 31;
+    const int k = blockIdx.x * 4 + w;
+    const int p = blockIdx.y;
+    int bh, r;
+    const RoleDesc &R = role_of(a, p, bh, r);
+    if (k >= a.nchunk) return;
+    int *cnt = cs + w * a.Cs;
+    const int32_t *off = a.off + (size_t)p * (a.Cs + 1);
+    const int32_t *pre = a.chunk_hist + ((size_t)p * a.nchunk + k) * a.Cs;
+    for (int c = lane; c < R.C; c += 32) cnt[c] = off[c] + pre[c];
+    __syncwarp();
+    const uint16_t *asg = R.assign + (size_t)bh * R.assign_bh;
+    int32_t *perm = a.perm + (size_t)p * a.N;
+    const int jend = min(a.N, (k + 1) * kSortChunk);
+    for (int jb = k * kSortChunk; jb < jend; jb += 32) {
+        const int j = jb + lane;
+        const int z = j < jend ? min((int)asg[j], R.C - 1) : -1;
+        const unsigned peers = __match_any_sync(0xffffffffu, z);
+        const int leader = __ffs(peers) - 1;
+        const int rank = __popc(peers & ((1u << lane) - 1u));
+        int base = (lane == leader && z >= 0) ? cnt[z] : 0;
+        base = __shfl_sync(0xffffffffu, base, leader);
+        if (z >= 0) perm[base + rank] = j;
+        __syncwarp();
+        if (lane == leader && z >= 0) cnt[z] = base + __popc(peers);
+        __syncwarp();
+    }
+}
+
+// ------------------------------------------------------------------------- update
+// grid (ceil(Cs/G), P), block 128: a group of dm threads per centroid sums its
+// members in token order (binary64) and divides by the count.
+__global__ void __launch_bounds__(128) km_update_kernel(KmArgs a)
+{
+    int bh, r;
+    const int p = blockIdx.y;
+    const RoleDesc &R = role_of(a, p, bh, r);
+    const int dm = R.dm, G = max(1, 128 / dm);
+    const int g = threadIdx.x / dm, i = threadIdx.x % dm;
+    const int c = blockIdx.x * G + g;
+    const bool active = g < G && c < R.C;
+    const int32_t *off = a.off + (size_t)p * (a.Cs + 1);
+    const int32_t *perm = a.perm + (size_t)p * a.N;
+    const int beg = active ? off[c] : 0, end = active ? off[c + 1] : 0;
+    double *cent = R.cent + ((size_t)bh * R.C + c) * a.d + R.ch0;
+    if (active && end > beg) {
+        const long long base = (long long)bh * a.N * a.d + R.ch0 + i;
+        double acc = 0.0;
+        int m = beg;
+        for (; m + 4 <= end; m += 4) {
+            const int ja = perm[m], jb = perm[m + 1], jc = perm[m + 2], jd = perm[m + 3];
+            const double xa = (double)load_x(R.X, base + (long long)ja * a.d, a.is_bf16);
+            const double xb = (double)load_x(R.X, base + (long long)jb * a.d, a.is_bf16);
+            const double xc = (double)load_x(R.X, base + (long long)jc * a.d, a.is_bf16);
+            const double xd = (double)load_x(R.X, base + (long long)jd * a.d, a.is_bf16);
+            acc = __dadd_rn(acc, xa);
+            acc = __dadd_rn(acc, xb);
+            acc = __dadd_rn(acc, xc);
+            acc = __dadd_rn(acc, xd);
+        }
+        for (; m < end; ++m)
+            acc = __dadd_rn(acc, (double)load_x(R.X, base + (long long)perm[m] * a.d, a.is_bf16));
+        cent[i] = __ddiv_rn(acc, (double)(end - beg));
+    }
+    __syncthreads();
+    if (active) finalize_row(a, p, c, cent, dm, i);
+}
+
+int max_blocks_for_groups(const KmArgs &a)
+{
+    int mx = 1;
+    for (int r = 0; r < a.nroles; ++r) {
+        const RoleDesc &R = a.role[a.role0 + r];
+        int G = R.dm >= 128 ? 1 : 128 / R.dm;
+        mx = max(mx, (R.C + G - 1) / G);
+    }
+    return mx;
+}
+
+}  // namespace
+
+cudaError_t sort_by_cluster(KmArgs a, cudaStream_t s)
+{
+    const int P = a.BH * a.nroles;
+    const size_t hsm = (size_t)4 * a.Cs * sizeof(int);
+    dim3 gh((a.nchunk + 3) / 4, P);
+    sort_hist_kernel<<<gh, 128, hsm, s>>>(a);
+    sort_scan_kernel<<<P, 1024, 0, s>>>(a);
+    sort_scatter_kernel<<<gh, 128, hsm, s>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t km_run(KmArgs a, int iters, cudaStream_t s)
+{
+    static bool attr_done = false;
+    const int P = a.BH * a.nroles;
+    const size_t fsm = ((size_t)a.ds * (kTok + kCC) + 3 * kCC + kTok) * sizeof(float);
+    if (!attr_done) {
+        cudaFuncSetAttribute(km_assign_fast_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)(((size_t)128 * (kTok + kCC) + 3 * kCC + kTok) * sizeof(float)));
+        cudaFuncSetAttribute(sort_hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             4 * kMaxC * (int)sizeof(int));
+        cudaFuncSetAttribute(sort_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             4 * kMaxC * (int)sizeof(int));
+        attr_done = true;
+    }
+    const int gb = max_blocks_for_groups(a);
+    km_init_kernel<<<dim3(gb, P), 128, 0, s>>>(a);
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    for (int it = 0; it < iters; ++it) {
+        km_assign_fast_kernel<<<dim3((a.N + kTok - 1) / kTok, P), kAssignThreads, fsm, s>>>(a);
+        km_assign_exact_kernel<<<sms * 4, 256, 0, s>>>(a);
+        cudaError_t e = sort_by_cluster(a, s);
+        if (e != cudaSuccess) return e;
+        km_update_kernel<<<dim3(gb, P), 128, 0, s>>>(a);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace scope

@@ -1,0 +1,610 @@
+// Lookup tables, proxy logits and the hybrid Top-p / fixed Top-k / online k_head
+// selection of SCOPE (arXiv 2608.12780; review page, key_machinery: Eq. 6 and Eq. 9;
+// major_comments[1]: Eqs. 7, 8 and 10).
+//
+// Per unit (b, h, query cluster c), with q_c the cluster centroid:
+//   P^m[c, z] = sum_{i in m} q_c[i] mu^m_z[i]                       (LUT, shared memory)
+//   s_j       = (1/sqrt d) ((P^T[z^T_j] + P^H[z^H_j]) + P^W[z^W_j])   (Eq. 6)
+// Keys are ranked by s_j descending, index ascending.  Both are evaluated in binary64
+// with one rounding per operation, in the order written, so logits and ranks are exact.
+//
+// Selection without a sort: a block-wide select finds the ranking position where the
+// cumulative weight (softmax mass for Top-p, one per key for a count) first reaches
+// a target.  Keys are histogrammed into 2048 bins by value; the crossing bin is
+// resolved exactly (its keys gathered and ranked in shared memory) when it holds at
+// most 2048 keys, otherwise it is binned again over its own value range; keys with
+// identical logits are binned by index instead.
+//
+// The softmax mass of key j is exp(s_j - max s) up to the factorisation
+//   exp(s_j) = exp(P^T/sqrt d) exp(P^H/sqrt d) exp(P^W/sqrt d),
+// i.e. three table lookups and two products instead of an exponential per key
+// (relative error ~1e-15).  Masses are accumulated as fixed-point integers
+// (2^-63 units, split 32/32 bits), so every sum is exact and independent of order:
+// results are deterministic run to run.
+#include "common.cuh"
+
+#include <cfloat>
+
+namespace scope {
+
+namespace {
+
+constexpr int kSelThreads = 512;
+constexpr int kBins = 2048;
+constexpr int kCap = 2048;
+constexpr int kMaxLevels = 6;
+constexpr int kBinsPerThread = kBins / kSelThreads;
+
+struct SelSmem {
+    double *lut, *E, *qc;
+    int *cnt;
+    unsigned long long *mhi, *mlo;
+    double *cs;
+    int *cj;
+    unsigned long long *cw;
+    int *order;
+    double *red;                 // reduction scratch, 32 doubles
+    unsigned long long *ured;    // 3 x 32 words
+    int *misc;                   // 8 ints
+};
+
+__host__ __device__ size_t sel_smem_bytes(int Cm, int d)
+{
+    return sizeof(double) * (6 * (size_t)Cm + d) + sizeof(int) * kBins +
+           2 * sizeof(unsigned long long) * kBins + sizeof(double) * kCap + sizeof(int) * kCap +
+           sizeof(unsigned long long) * kCap + sizeof(int) * kCap + sizeof(double) * 32 +
+           sizeof(unsigned long long) * 96 + sizeof(int) * 8;
+}
+
+__device__ SelSmem carve(char *base, int Cm, int d)
+{
+    SelSmem s;
+    double *dp = reinterpret_cast<double *>(base);
+    s.lut = dp;
+    s.E = dp + 3 * Cm;
+    s.qc = dp + 6 * Cm;
+    s.cs = s.qc + d;
+    s.red = s.cs + kCap;
+    unsigned long long *up = reinterpret_cast<unsigned long long *>(s.red + 32);
+    s.mhi = up;
+    s.mlo = up + kBins;
+    s.cw = up + 2 * kBins;
+    s.ured = s.cw + kCap;
+    int *ip = reinterpret_cast<int *>(s.ured + 96);
+    s.cnt = ip;
+    s.cj = ip + kBins;
+    s.order = s.cj + kCap;
+    s.misc = s.order + kCap;
+    return s;
+}
+
+struct Unit {
+    const uint16_t *zt, *zh, *zw;
+    int Cm, N;
+    double inv;          // 1/sqrt(d)
+    double inv_umax;     // mass normalisation
+};
+
+// Codes are clamped to [0, Cm) so that a malformed caller-supplied code cannot read
+// outside the tables (sel_check_kernel reports such codes in the status word).
+__device__ __forceinline__ double key_score(const SelSmem &S, const Unit &u, int j)
+{
+    const int zt = min((int)u.zt[j], u.Cm - 1), zh = min((int)u.zh[j], u.Cm - 1),
+              zw = min((int)u.zw[j], u.Cm - 1);
+    const double a = S.lut[zt], b = S.lut[u.Cm + zh], c = S.lut[2 * u.Cm + zw];
+    return __dmul_rn(u.inv, __dadd_rn(__dadd_rn(a, b), c));
+}
+
+__device__ __forceinline__ double key_u(const SelSmem &S, const Unit &u, int j)
+{
+    const int zt = min((int)u.zt[j], u.Cm - 1), zh = min((int)u.zh[j], u.Cm - 1),
+              zw = min((int)u.zw[j], u.Cm - 1);
+    return __dmul_rn(__dmul_rn(S.E[zt], S.E[u.Cm + zh]), S.E[2 * u.Cm + zw]);
+}
+
+// fixed-point mass in units of 2^-63, clamped to [0, 2^63]
+__device__ __forceinline__ unsigned long long key_mass(const SelSmem &S, const Unit &u, int j)
+{
+    double w = fmin(__dmul_rn(key_u(S, u, j), u.inv_umax), 1.0);
+    return __double2ull_rn(w * 9223372036854775808.0);
+}
+
+__device__ __forceinline__ double mass_to_double(unsigned long long hi, unsigned long long lo)
+{
+    return ldexp((double)hi, -31) + ldexp((double)lo, -63);
+}
+
+__device__ __forceinline__ int vbin(double s, double hi, double scale)
+{
+    const double t = __dmul_rn(__dsub_rn(hi, s), scale);
+    if (!(t > 0.0)) return 0;
+    if (t >= (double)kBins) return kBins - 1;
+    return (int)t;
+}
+
+__device__ __forceinline__ int jbin(int j, int N)
+{
+    return (int)(((long long)j * kBins) / N);
+}
+
+struct Levels {
+    int n;
+    double hi[kMaxLevels], scale[kMaxLevels];
+    int bstar[kMaxLevels];
+    bool jmode, jexact;
+    double tie_s;
+};
+
+__device__ __forceinline__ bool in_candidates(const Levels &L, double s)
+{
+    for (int k = 0; k < L.n; ++k)
+        if (vbin(s, L.hi[k], L.scale[k]) != L.bstar[k]) return false;
+    if (L.jmode && L.jexact && s != L.tie_s) return false;
+    return true;
+}
+
+// ---- block reductions (all threads call; result broadcast)
+__device__ double block_max(double v, double *red)
+{
+    for (int o = 16; o; o >>= 1) v = fmax(v, __shfl_xor_sync(0xffffffffu, v, o));
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    __syncthreads();
+    if (lane == 0) red[w] = v;
+    __syncthreads();
+    if (w == 0) {
+        v = lane < (int)(blockDim.x >> 5) ? red[lane] : -DBL_MAX;
+        for (int o = 16; o; o >>= 1) v = fmax(v, __shfl_xor_sync(0xffffffffu, v, o));
+        if (lane == 0) red[0] = v;
+    }
+    __syncthreads();
+    return red[0];
+}
+
+__device__ double block_min(double v, double *red)
+{
+    return -block_max(-v, red);
+}
+
+// inclusive warp scan of three 64-bit components
+__device__ __forceinline__ void warp_scan3(unsigned long long &a, unsigned long long &b,
+                                           unsigned long long &c)
+{
+    const int lane = threadIdx.x & 31;
+    for (int o = 1; o < 32; o <<= 1) {
+        unsigned long long x = __shfl_up_sync(0xffffffffu, a, o);
+        unsigned long long y = __shfl_up_sync(0xffffffffu, b, o);
+        unsigned long long z = __shfl_up_sync(0xffffffffu, c, o);
+        if (lane >= o) {
+            a += x;
+            b += y;
+            c += z;
+        }
+    }
+}
+
+// Exclusive block scan of (a, b, c); returns the block totals through tot[3].
+__device__ void block_excl_scan3(unsigned long long &a, unsigned long long &b, unsigned long long &c,
+                                 unsigned long long *ured, unsigned long long tot[3])
+{
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    unsigned long long ia = a, ib = b, ic = c;
+    warp_scan3(ia, ib, ic);
+    __syncthreads();
+    if (lane == 31) {
+        ured[w] = ia;
+        ured[32 + w] = ib;
+        ured[64 + w] = ic;
+    }
+    __syncthreads();
+    if (w == 0) {
+        unsigned long long xa = lane < nw ? ured[lane] : 0ull;
+        unsigned long long xb = lane < nw ? ured[32 + lane] : 0ull;
+        unsigned long long xc = lane < nw ? ured[64 + lane] : 0ull;
+        warp_scan3(xa, xb, xc);
+        ured[lane] = xa;
+        ured[32 + lane] = xb;
+        ured[64 + lane] = xc;
+    }
+    __syncthreads();
+    const unsigned long long pa = w ? ured[w - 1] : 0ull, pb = w ? ured[32 + w - 1] : 0ull,
+                             pc = w ? ured[64 + w - 1] : 0ull;
+    tot[0] = ured[nw - 1];
+    tot[1] = ured[32 + nw - 1];
+    tot[2] = ured[64 + nw - 1];
+    a = pa + ia - a;
+    b = pb + ib - b;
+    c = pc + ic - c;
+}
+
+struct SelectOut {
+    double s;
+    int j;
+    long long rank;   // keys before it in the ranking
+};
+
+// Finds the first key of the ranking at which the cumulative weight reaches the target.
+// mass_mode: weight = softmax mass, target = rho * (total mass); else weight = 1 and
+// target = count (1 <= count <= N).  Called by all threads of the block.
+__device__ SelectOut block_select(const SelSmem &S, const Unit &u, bool mass_mode, double rho,
+                                  long long count, double smax, double smin, int32_t *status)
+{
+    Levels L;
+    L.n = 0;
+    L.jmode = false;
+    L.jexact = false;
+    L.tie_s = 0.0;
+    double hi = smax, lo = smin;
+    unsigned long long bhi = 0, blo = 0;   // mass before the candidate set (fixed point)
+    long long bcnt = 0;                    // keys before the candidate set
+    double target = 0.0;
+    bool have_target = !mass_mode;
+    const int tid = threadIdx.x;
+    SelectOut out{smax, 0, 0};
+
+    for (int iter = 0; iter < kMaxLevels + 3; ++iter) {
+        const double scale = (hi > lo) ? (double)kBins / (hi - lo) : 0.0;
+        for (int b = tid; b < kBins; b += kSelThreads) {
+            S.cnt[b] = 0;
+            S.mhi[b] = 0;
+            S.mlo[b] = 0;
+        }
+        __syncthreads();
+        double cmin = DBL_MAX, cmax = -DBL_MAX;
+        for (int j = tid; j < u.N; j += kSelThreads) {
+            const double s = key_score(S, u, j);
+            if (!in_candidates(L, s)) continue;
+            const int b = L.jmode ? jbin(j, u.N) : vbin(s, hi, scale);
+            atomicAdd(&S.cnt[b], 1);
+            if (mass_mode) {
+                const unsigned long long W = key_mass(S, u, j);
+                atomicAdd(&S.mhi[b], W >> 32);
+                atomicAdd(&S.mlo[b], W & 0xffffffffull);
+            }
+            cmin = fmin(cmin, s);
+            cmax = fmax(cmax, s);
+        }
+        cmin = block_min(cmin, S.red);
+        cmax = block_max(cmax, S.red);
+        if (!L.jmode && cmin == cmax) {
+            // every candidate has the same logit: the ranking among them is by index
+            L.jmode = true;
+            L.jexact = true;
+            L.tie_s = cmin;
+            continue;
+        }
+        // per-thread sums of its bins, then block scan
+        unsigned long long th = 0, tl = 0, tc = 0;
+        const int b0 = tid * kBinsPerThread;
+        for (int q = 0; q < kBinsPerThread; ++q) {
+            th += S.mhi[b0 + q];
+            tl += S.mlo[b0 + q];
+            tc += (unsigned long long)S.cnt[b0 + q];
+        }
+        unsigned long long tot[3];
+        block_excl_scan3(th, tl, tc, S.ured, tot);
+        if (!have_target) {
+            // first scan covers every key: its total is the softmax normaliser Z
+            target = rho * mass_to_double(tot[0], tot[1]);
+            have_target = true;
+        }
+        if (tid == 0) S.misc[0] = -1;
+        __syncthreads();
+        {
+            unsigned long long eh = bhi + th, el = blo + tl;
+            long long ec = bcnt + (long long)tc;
+            for (int q = 0; q < kBinsPerThread; ++q) {
+                const int b = b0 + q;
+                const unsigned long long ih = eh + S.mhi[b], il = el + S.mlo[b];
+                const long long ic = ec + S.cnt[b];
+                bool before_ok, incl_ok;
+                if (mass_mode) {
+                    before_ok = mass_to_double(eh, el) >= target;
+                    incl_ok = mass_to_double(ih, il) >= target;
+                } else {
+                    before_ok = ec >= count;
+                    incl_ok = ic >= count;
+                }
+                if (!before_ok && incl_ok) {
+                    S.misc[0] = b;
+                    S.ured[0] = eh;   // safe: scan results already consumed above
+                    S.ured[1] = el;
+                    reinterpret_cast<long long *>(S.ured)[2] = ec;
+                }
+                eh = ih;
+                el = il;
+                ec = ic;
+            }
+        }
+        __syncthreads();
+        int bstar = S.misc[0];
+        if (bstar < 0) {
+            // cannot happen for consistent inputs; fall back to the last non-empty bin
+            if (tid == 0) set_status(status, SCOPE_DEV_SELECT_TIE);
+            return out;
+        }
+        bhi = S.ured[0];
+        blo = S.ured[1];
+        bcnt = reinterpret_cast<long long *>(S.ured)[2];
+        const int nb = S.cnt[bstar];
+        __syncthreads();
+
+        if (nb <= kCap || L.jmode) {
+            if (nb > kCap) {
+                if (tid == 0) set_status(status, SCOPE_DEV_SELECT_TIE);
+            }
+            // gather the crossing bin's keys
+            if (tid == 0) S.misc[1] = 0;
+            __syncthreads();
+            for (int j = tid; j < u.N; j += kSelThreads) {
+                const double s = key_score(S, u, j);
+                if (!in_candidates(L, s)) continue;
+                const int b = L.jmode ? jbin(j, u.N) : vbin(s, hi, scale);
+                if (b != bstar) continue;
+                const int slot = atomicAdd(&S.misc[1], 1);
+                if (slot < kCap) {
+                    S.cs[slot] = s;
+                    S.cj[slot] = j;
+                    if (mass_mode) S.cw[slot] = key_mass(S, u, j);
+                }
+            }
+            __syncthreads();
+            const int n = min(S.misc[1], kCap);
+            if (n == 0) {   // the gather pass always finds the crossing bin's keys
+                if (tid == 0) set_status(status, SCOPE_DEV_SELECT_TIE);
+                __syncthreads();
+                return out;
+            }
+            // rank among the gathered keys: logit descending, index ascending
+            for (int i = tid; i < n; i += kSelThreads) {
+                const double si = S.cs[i];
+                const int ji = S.cj[i];
+                int r = 0;
+                for (int k = 0; k < n; ++k) {
+                    const double sk = S.cs[k];
+                    r += (sk > si) || (sk == si && S.cj[k] < ji);
+                }
+                S.order[r] = i;
+            }
+            __syncthreads();
+            int pos = -1;
+            if (mass_mode) {
+                if (tid < 32) {
+                    unsigned long long rh = bhi, rl = blo;
+                    for (int base = 0; base < n && pos < 0; base += 32) {
+                        const int idx = base + tid;
+                        unsigned long long W = idx < n ? S.cw[S.order[idx]] : 0ull;
+                        unsigned long long h = W >> 32, l = W & 0xffffffffull, z = 0;
+                        warp_scan3(h, l, z);
+                        const bool ok = idx < n && mass_to_double(rh + h, rl + l) >= target;
+                        const unsigned bal = __ballot_sync(0xffffffffu, ok);
+                        if (bal) pos = base + __ffs(bal) - 1;
+                        rh += __shfl_sync(0xffffffffu, h, 31);
+                        rl += __shfl_sync(0xffffffffu, l, 31);
+                    }
+                    if (tid == 0) S.misc[2] = pos < 0 ? n - 1 : pos;
+                }
+            } else if (tid == 0) {
+                long long q = count - 1 - bcnt;
+                S.misc[2] = (int)(q < 0 ? 0 : (q >= n ? n - 1 : q));
+            }
+            __syncthreads();
+            pos = S.misc[2];
+            const int i = S.order[pos];
+            out.s = S.cs[i];
+            out.j = S.cj[i];
+            out.rank = bcnt + pos;
+            __syncthreads();
+            return out;
+        }
+        // refine inside the crossing bin
+        if (L.n >= kMaxLevels) {
+            if (tid == 0) set_status(status, SCOPE_DEV_SELECT_TIE);
+            L.jmode = true;   // order the remaining candidates by index
+            continue;
+        }
+        L.hi[L.n] = hi;
+        L.scale[L.n] = scale;
+        L.bstar[L.n] = bstar;
+        L.n += 1;
+        const double nhi = hi - (double)bstar / scale, nlo = hi - (double)(bstar + 1) / scale;
+        hi = nhi;
+        lo = nlo;
+        __syncthreads();
+    }
+    if (tid == 0) set_status(status, SCOPE_DEV_SELECT_TIE);
+    return out;
+}
+
+// Builds the LUT (and, with want_E, the per-subspace exponential tables) for unit c.
+__device__ void build_tables(const SelArgs &a, const SelSmem &S, int bh, int c, bool want_E)
+{
+    const int tid = threadIdx.x, Cm = a.Cm, d = a.d;
+    const double *qc = a.qcent + ((size_t)bh * a.Cq + c) * d;
+    for (int i = tid; i < d; i += kSelThreads) S.qc[i] = qc[i];
+    __syncthreads();
+    const int bnd[4] = {0, a.dt, a.dt + a.dh, d};
+    const double *kc = a.kcent + (size_t)bh * Cm * d;
+    for (int idx = tid; idx < 3 * Cm; idx += kSelThreads) {
+        const int m = idx / Cm, z = idx - m * Cm;
+        double acc = 0.0;
+        for (int i = bnd[m]; i < bnd[m + 1]; ++i)
+            acc = __dadd_rn(acc, __dmul_rn(S.qc[i], kc[(size_t)z * d + i]));
+        S.lut[idx] = acc;
+    }
+    __syncthreads();
+    if (!want_E) return;
+    for (int m = 0; m < 3; ++m) {
+        double mx = -DBL_MAX;
+        for (int z = tid; z < Cm; z += kSelThreads) mx = fmax(mx, S.lut[m * Cm + z]);
+        mx = block_max(mx, S.red);
+        for (int z = tid; z < Cm; z += kSelThreads)
+            S.E[m * Cm + z] = exp(__dmul_rn(__dsub_rn(S.lut[m * Cm + z], mx), a.inv_sqrt_d));
+        __syncthreads();
+    }
+}
+
+// ------------------------------------------------------------------------- kernels
+// Reports caller-supplied codes outside [0, Cm) (the tables clamp them).
+__global__ void sel_check_kernel(SelArgs a)
+{
+    const long long total = (long long)a.BH * 3 * a.N;
+    bool bad = false;
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+         i += (long long)gridDim.x * blockDim.x)
+        bad |= a.codes[i] >= a.Cm;
+    if (__syncthreads_or(bad) && threadIdx.x == 0) set_status(a.status, SCOPE_DEV_BAD_ASSIGN);
+}
+
+// Top-p count p_c and base count b_c (Eqs. 7-8).  grid (Cq, BH).
+__global__ void __launch_bounds__(kSelThreads) sel_topp_kernel(SelArgs a)
+{
+    extern __shared__ __align__(16) char smem_raw[];
+    const SelSmem S = carve(smem_raw, a.Cm, a.d);
+    const int c = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
+    build_tables(a, S, bh, c, true);
+    Unit u;
+    u.zt = a.codes + (size_t)bh * 3 * a.N;
+    u.zh = u.zt + a.N;
+    u.zw = u.zh + a.N;
+    u.Cm = a.Cm;
+    u.N = a.N;
+    u.inv = a.inv_sqrt_d;
+    double smax = -DBL_MAX, smin = DBL_MAX, umax = 0.0;
+    for (int j = tid; j < a.N; j += kSelThreads) {
+        const double s = key_score(S, u, j);
+        smax = fmax(smax, s);
+        smin = fmin(smin, s);
+        umax = fmax(umax, key_u(S, u, j));
+    }
+    smax = block_max(smax, S.red);
+    smin = block_min(smin, S.red);
+    umax = block_max(umax, S.red);
+    u.inv_umax = 1.0 / umax;
+    long long p = a.N;
+    SelectOut so{smax, 0, 0};
+    if (a.rho < 1.0) {
+        so = block_select(S, u, true, a.rho, 0, smax, smin, a.status);
+        p = so.rank + 1;
+    }
+    if (tid == 0) {
+        const size_t unit = (size_t)bh * a.Cq + c;
+        const long long b = p > a.kfix ? p : a.kfix;
+        if (a.topp) a.topp[unit] = (int32_t)p;
+        a.base[unit] = (int32_t)b;
+        double *st = a.state + unit * 8;
+        st[0] = smax;
+        st[1] = smin;
+        st[2] = so.s;
+        st[3] = (double)so.j;
+        st[4] = (double)p;
+    }
+}
+
+// k_head (Eq. 9) and final counts r_c (Eq. 10).  grid BH.
+__global__ void __launch_bounds__(256) sel_khead_kernel(SelArgs a)
+{
+    __shared__ long long rn[8], rd[8];
+    const int bh = blockIdx.x, tid = threadIdx.x;
+    long long num = 0, den = 0;
+    for (int c = tid; c < a.Cq; c += 256) {
+        const long long n = a.qsizes[(size_t)bh * a.Cq + c];
+        num += n * (long long)a.base[(size_t)bh * a.Cq + c];
+        den += n;
+    }
+    for (int o = 16; o; o >>= 1) {
+        num += __shfl_xor_sync(0xffffffffu, num, o);
+        den += __shfl_xor_sync(0xffffffffu, den, o);
+    }
+    if ((tid & 31) == 0) {
+        rn[tid >> 5] = num;
+        rd[tid >> 5] = den;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        num = 0;
+        den = 0;
+        for (int w = 0; w < 8; ++w) {
+            num += rn[w];
+            den += rd[w];
+        }
+        rn[0] = den > 0 ? (num + den - 1) / den : a.N;
+        a.khead[bh] = (int32_t)rn[0];
+    }
+    __syncthreads();
+    const long long kh = rn[0];
+    for (int c = tid; c < a.Cq; c += 256) {
+        const long long b = a.base[(size_t)bh * a.Cq + c];
+        a.final_cnt[(size_t)bh * a.Cq + c] = (int32_t)(b < kh ? kh : b);
+    }
+}
+
+// Selected set S_c = the first r_c keys of the ranking, as a bitmask.  grid (Cq, BH).
+__global__ void __launch_bounds__(kSelThreads) sel_mask_kernel(SelArgs a)
+{
+    extern __shared__ __align__(16) char smem_raw[];
+    const SelSmem S = carve(smem_raw, a.Cm, a.d);
+    const int c = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
+    const size_t unit = (size_t)bh * a.Cq + c;
+    uint32_t *row = a.mask + unit * a.nw;
+    const long long r = a.final_cnt[unit];
+    const int lane = tid & 31, warp = tid >> 5;
+    if (r >= a.N) {
+        for (int w = tid; w < a.nw; w += kSelThreads) {
+            const int rem = a.N - w * 32;
+            row[w] = rem >= 32 ? 0xffffffffu : ((1u << rem) - 1u);
+        }
+        return;
+    }
+    build_tables(a, S, bh, c, false);
+    Unit u;
+    u.zt = a.codes + (size_t)bh * 3 * a.N;
+    u.zh = u.zt + a.N;
+    u.zw = u.zh + a.N;
+    u.Cm = a.Cm;
+    u.N = a.N;
+    u.inv = a.inv_sqrt_d;
+    u.inv_umax = 1.0;
+    const double *st = a.state + unit * 8;
+    double s_star;
+    int j_star;
+    if ((long long)st[4] == r) {
+        s_star = st[2];
+        j_star = (int)st[3];
+    } else {
+        const SelectOut so = block_select(S, u, false, 0.0, r, st[0], st[1], a.status);
+        s_star = so.s;
+        j_star = so.j;
+    }
+    for (int w = warp; w < a.nw; w += kSelThreads / 32) {
+        const int j = w * 32 + lane;
+        bool sel = false;
+        if (j < a.N) {
+            const double s = key_score(S, u, j);
+            sel = (s > s_star) || (s == s_star && j <= j_star);
+        }
+        const unsigned bits = __ballot_sync(0xffffffffu, sel);
+        if (lane == 0) row[w] = bits;
+    }
+}
+
+}  // namespace
+
+size_t select_smem_bytes(int Cm, int d)
+{
+    return sel_smem_bytes(Cm, d);
+}
+
+cudaError_t select_run(const SelArgs &a, cudaStream_t s)
+{
+    const size_t smem = sel_smem_bytes(a.Cm, a.d);
+    cudaFuncSetAttribute(sel_topp_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaFuncSetAttribute(sel_mask_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    dim3 grid(a.Cq, a.BH);
+    sel_check_kernel<<<256, 256, 0, s>>>(a);
+    sel_topp_kernel<<<grid, kSelThreads, smem, s>>>(a);
+    sel_khead_kernel<<<a.BH, 256, 0, s>>>(a);
+    sel_mask_kernel<<<grid, kSelThreads, smem, s>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace scope

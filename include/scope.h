@@ -1,0 +1,197 @@
+/*
+ * scope.h -- C ABI of the SCOPE per-layer sparse-attention hot path on B200 (sm_100a).
+ *
+ * SCOPE ("Subspace Clustering with Online Per-Head Top-K Estimation for Sparse Video
+ * Attention", arXiv 2608.12780) runs, per attention layer of a video diffusion
+ * transformer and per (batch, head):
+ *   1. clustering: post-RoPE queries into Cq clusters; post-RoPE keys split into the
+ *      temporal / height / width channel ranges of 3D RoPE and each range clustered
+ *      independently into Cm centroids (abstract; review page "major_comments": Eq. 3);
+ *   2. selection: per query cluster c, lookup tables of centroid dot products summed
+ *      into a proxy logit per key (Eq. 6), hybrid Top-p / fixed Top-k base counts
+ *      (Eqs. 7-8), the online per-head Top-k k_head (Eq. 9) and the top-up of clusters
+ *      below it (Eq. 10) (review page "key_machinery");
+ *   3. exact softmax attention of each query over its cluster's selected ORIGINAL
+ *      keys and values (abstract; review page "forward_implications").
+ *
+ * Conventions for every entry point
+ *  - Tensors are dense, row-major, on the device of the current CUDA context:
+ *    Q, K, V, O are [B, H, N, d] with N = T*Hg*Wg and token n = t*Hg*Wg + h*Wg + w;
+ *    channels [0, d_t) / [d_t, d_t+d_h) / [d_t+d_h, d) are the temporal / height /
+ *    width subspaces.  Element type of Q, K, V, O is params->dtype.
+ *  - The caller owns every buffer, including the workspace `ws` of at least
+ *    scope_workspace_bytes(params) bytes (256-byte aligned).  The library allocates
+ *    no device memory, keeps no state between calls and never synchronises the
+ *    stream, except scope_get_device_status.  Calls on one workspace must not overlap.
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream).  Work is enqueued;
+ *    results are valid once the stream has completed and the status is SCOPE_OK.
+ *  - Arguments are validated on the host before anything is enqueued; a failure
+ *    returns SCOPE_ERR_INVALID_ARGUMENT / SCOPE_ERR_UNSUPPORTED /
+ *    SCOPE_ERR_WORKSPACE_TOO_SMALL and enqueues nothing.  A failed launch returns
+ *    SCOPE_ERR_CUDA.  Conditions only the device can see (an init index out of range,
+ *    an unresolvable selection tie) set bits in a status word inside the workspace,
+ *    read by scope_get_device_status; each entry point clears that word first.
+ *  - Limits: d in {64, 128}; d_t, d_h, d_w >= 1 with d_t + d_h + d_w = d;
+ *    1 <= Cq, Cm <= min(N, 4096); 1 <= iters <= 64; 0 < rho <= 1; 0 <= alpha <= 1;
+ *    N <= 2^24; B*H*N < 2^31.  Device pointers must be 16-byte aligned.
+ */
+#ifndef SCOPE_H
+#define SCOPE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SCOPE_OK = 0,
+    SCOPE_ERR_INVALID_ARGUMENT = 1,
+    SCOPE_ERR_UNSUPPORTED = 2,
+    SCOPE_ERR_WORKSPACE_TOO_SMALL = 3,
+    SCOPE_ERR_CUDA = 4,
+    SCOPE_ERR_DEVICE_CHECK = 5
+} scope_status;
+
+typedef enum { SCOPE_F32 = 0, SCOPE_BF16 = 1 } scope_dtype;
+
+/* Device status bits (scope_get_device_status). */
+#define SCOPE_DEV_BAD_INIT_INDEX 0x1   /* an init index was outside [0, N); row 0 was used */
+#define SCOPE_DEV_SELECT_TIE     0x2   /* a selection boundary could not be resolved exactly */
+#define SCOPE_DEV_BAD_ASSIGN     0x4   /* a cluster index >= C reached the attention stage */
+
+/* Shape and hyperparameters of one layer.  rho: Top-p threshold of Eq. 7 (the paper
+ * does not report it; 0.9 is the usual choice).  alpha: fixed Top-k minimum as a
+ * fraction of N, k_fix = ceil(alpha * N) (the paper gives alpha = 0.1).  iters: Lloyd
+ * iterations of every k-means. */
+typedef struct {
+    int B, H;
+    int T, Hg, Wg;
+    int d, d_t, d_h, d_w;
+    int Cq, Cm;
+    int iters;
+    double rho, alpha;
+    scope_dtype dtype;
+} scope_params;
+
+/* Optional intermediate outputs of scope_forward (device pointers; NULL = keep the
+ * value in the workspace only).  Layouts as in the stage functions below. */
+typedef struct {
+    double *q_centroids;   /* [B, H, Cq, d] */
+    uint16_t *q_assign;    /* [B, H, N] */
+    int32_t *q_sizes;      /* [B, H, Cq] */
+    double *k_centroids;   /* [B, H, Cm, d] */
+    uint16_t *k_codes;     /* [B, H, 3, N] */
+    int32_t *topp_counts;  /* [B, H, Cq]  p_c */
+    int32_t *base_counts;  /* [B, H, Cq]  b_c */
+    int32_t *k_head;       /* [B, H] */
+    int32_t *final_counts; /* [B, H, Cq]  r_c */
+    uint32_t *sel_mask;    /* [B, H, Cq, ceil(N/32)] */
+} scope_intermediates;
+
+/* Bytes of workspace every entry point below needs for `p` (0 if p is invalid). */
+size_t scope_workspace_bytes(const scope_params *p);
+
+/*
+ * Query clustering (abstract: "query clusters"; review page, major_comments[0]: the
+ * cluster centroid q_c; major_comments[1]: Cq = 300).  Lloyd k-means on all d
+ * channels, params->iters iterations.  One iteration assigns every token to its
+ * nearest centroid in squared Euclidean distance (lowest index on a tie), then moves
+ * every non-empty centroid to the mean of its members; empty centroids stay.
+ *   Q            [B,H,N,d] dtype
+ *   init_idx     [B,H,Cq] int32 token indices of the initial centroids, or NULL
+ *   init_cent    [B,H,Cq,d] double initial centroids (used when init_idx is NULL)
+ *   q_centroids  out [B,H,Cq,d] double: means of the final members
+ *   q_assign     out [B,H,N] uint16: final assignments
+ *   q_sizes      out [B,H,Cq] int32: final member counts n_c
+ * Assignments are exact: distances are certified against binary64 sums over the
+ * channels in order, so they equal a binary64 evaluation of the definition.
+ */
+scope_status scope_cluster_queries(const scope_params *p, const void *Q, const int32_t *init_idx,
+                                   const double *init_cent, double *q_centroids,
+                                   uint16_t *q_assign, int32_t *q_sizes, void *ws,
+                                   size_t ws_bytes, void *stream);
+
+/*
+ * Key subspace clustering (abstract: keys partitioned into temporal, height and width
+ * subspaces and clustered independently; review page, load_bearing_attack: Eq. 3,
+ * k-means minimising Euclidean reconstruction error per subspace; Cm = 333).  Three
+ * independent Lloyd k-means, one per channel range, same rules as the queries.
+ *   K            [B,H,N,d] dtype
+ *   init_idx     [B,H,3,Cm] int32 (subspace-major), or NULL
+ *   init_cent    [B,H,Cm,d] double (used when init_idx is NULL)
+ *   k_centroids  out [B,H,Cm,d] double: centroid z of subspace m in m's channel range
+ *   k_codes      out [B,H,3,N] uint16: z^T_j, z^H_j, z^W_j
+ */
+scope_status scope_cluster_keys(const scope_params *p, const void *K, const int32_t *init_idx,
+                                const double *init_cent, double *k_centroids, uint16_t *k_codes,
+                                void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Lookup tables, proxy logits and selection (review page, key_machinery: Eq. 6
+ * s_cj = (1/sqrt d) sum_m P^m[c, z^m_j] and Eq. 9 k_head = ceil(sum n_c b_c / sum n_c);
+ * major_comments[1]: hybrid Top-p / fixed Top-k (Eq. 7), base counts b_c (Eq. 8),
+ * top-up (Eq. 10)).  Per (b, h, c):
+ *   P^m[c,z] = sum_{i in m} q_c[i] * mu^m_z[i];  s_cj = (1/sqrt d)((P^T + P^H) + P^W);
+ *   keys ranked by s_cj descending, key index ascending on equal logits;
+ *   p_c = least r whose first r keys hold softmax mass >= rho (rho = 1: p_c = N);
+ *   b_c = max(p_c, ceil(alpha N)); k_head = ceil(sum_c n_c b_c / N);
+ *   r_c = max(b_c, k_head); S_c = first r_c keys of the ranking.
+ *   q_centroids [B,H,Cq,d] double, q_sizes [B,H,Cq] int32,
+ *   k_centroids [B,H,Cm,d] double, k_codes [B,H,3,N] uint16  (as produced above)
+ *   topp_counts  out [B,H,Cq] int32 p_c (may be NULL)
+ *   base_counts  out [B,H,Cq] int32 b_c
+ *   k_head       out [B,H] int32
+ *   final_counts out [B,H,Cq] int32 r_c
+ *   sel_mask     out [B,H,Cq,ceil(N/32)] uint32: bit (j%32) of word j/32 set iff j in S_c
+ * Logits and ranks are binary64 and exact; the softmax mass is summed in binary64, so
+ * p_c can differ from another binary64 evaluation only where the mass of a prefix is
+ * within ~1e-12 (relative) of rho.
+ */
+scope_status scope_build_lut_and_select(const scope_params *p, const double *q_centroids,
+                                        const int32_t *q_sizes, const double *k_centroids,
+                                        const uint16_t *k_codes, int32_t *topp_counts,
+                                        int32_t *base_counts, int32_t *k_head,
+                                        int32_t *final_counts, uint32_t *sel_mask, void *ws,
+                                        size_t ws_bytes, void *stream);
+
+/*
+ * Sparse attention over the selected original keys and values (abstract: "sparse
+ * attention is then computed over the selected original keys and values"):
+ *   O_i = sum_{j in S_c} softmax_j(q_i . k_j / sqrt d) v_j  for every token i, c = q_assign[i].
+ * Queries are grouped by cluster on the device; bf16 runs on the tensor cores
+ * (tcgen05, fp32 accumulation and softmax), fp32 on the CUDA cores.
+ *   Q, K, V      [B,H,N,d] dtype;  O out [B,H,N,d] dtype
+ *   q_assign     [B,H,N] uint16;  sel_mask [B,H,Cq,ceil(N/32)] uint32
+ *   final_counts [B,H,Cq] int32 r_c (popcount of each mask row; used for scheduling)
+ * A query whose cluster selects no key gets O_i = 0.
+ */
+scope_status scope_sparse_attention(const scope_params *p, const void *Q, const void *K,
+                                    const void *V, const uint16_t *q_assign,
+                                    const uint32_t *sel_mask, const int32_t *final_counts,
+                                    void *O, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * The whole layer: query and key clustering (initial centroids from q_init_idx
+ * [B,H,Cq] and k_init_idx [B,H,3,Cm]), selection and sparse attention, enqueued with
+ * no host synchronisation.  `inter` may be NULL or name buffers that receive the
+ * intermediates.
+ */
+scope_status scope_forward(const scope_params *p, const void *Q, const void *K, const void *V,
+                           const int32_t *q_init_idx, const int32_t *k_init_idx, void *O,
+                           const scope_intermediates *inter, void *ws, size_t ws_bytes,
+                           void *stream);
+
+/* Human-readable name of a status code (static storage). */
+const char *scope_status_string(scope_status s);
+
+/* Synchronises `stream` and returns the device status word of the last call that used
+ * `ws` in *out (0 = clean; SCOPE_DEV_* bits otherwise). */
+scope_status scope_get_device_status(const void *ws, void *stream, int32_t *out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SCOPE_H */
