@@ -1,12 +1,605 @@
-// Tensor-core (tcgen05) sparse attention for bf16 -- routed to the CUDA-core kernel
-// until the tcgen05 kernel passes its parity tests.
+// Gathered sparse attention on the Blackwell tensor cores (tcgen05, sm_100a), bf16.
+//
+// SCOPE computes exact softmax attention of every query over the ORIGINAL keys and
+// values its query cluster selected (arXiv 2608.12780, abstract;
+// review page, forward_implications[1]).  Queries are grouped by cluster, so one work
+// item = up to 128 queries of one (b, h, c) against the r_c keys of S_c.
+//
+// Per CTA (persistent, one per SM, static round-robin over the head-major work list):
+//   warps 0-3  softmax + epilogue: thread r owns query row r = TMEM lane r
+//   warp 4     gathers the Q tile once per item and the selected K rows per key tile
+//   warp 5     gathers the selected V rows per key tile
+//   warp 6     allocates TMEM and issues the MMAs (one elected thread)
+// The selected key indices come straight from the selection bitmask (each gather warp
+// expands it with popc + warp prefix sums).  Rows are copied with 16-byte cp.async into
+// the 128B-swizzled K-major layout the tensor core reads, two stages deep.
+//   S_b = Q K^T   tcgen05.mma kind::f16, M=128, N=128, K=d, fp32 in TMEM (2 buffers)
+//   O  += P V     M=128, N=d, K=128, P bf16 in shared memory, O fp32 in TMEM
+// The softmax keeps a running row maximum and rescales O (TMEM load/store) only when
+// the maximum grows by more than 2^8, so P stays <= 256 and the final O / l is exact
+// softmax arithmetic.  Every mbarrier wait gives up after ~4 s, sets a status bit and
+// lets the CTA drain and free its TMEM.
 #include "common.cuh"
 
 namespace scope {
 
+namespace {
+
+constexpr int kBM = 128;           // queries per tile
+constexpr int kBN = 128;           // keys per tile
+constexpr int kStages = 2;
+constexpr int kThreads = 224;      // 7 warps
+constexpr uint32_t kTmemCols = 512;
+constexpr unsigned long long kWaitNs = 4000000000ull;
+
+struct __align__(8) Bars {
+    uint64_t q_full, q_empty;
+    uint64_t k_full[kStages], v_full[kStages], kv_empty[kStages];
+    uint64_t s_full[2], s_empty[2];
+    uint64_t p_full, o_done, o_free;
+};
+
+template <int D>
+struct Smem {
+    static constexpr int kTile = kBM * D * 2;          // bytes of a 128 x D bf16 tile
+    static constexpr int kQ = 0;
+    static constexpr int kK = kQ + kTile;
+    static constexpr int kV = kK + kStages * kTile;
+    static constexpr int kP = kV + kStages * kTile;
+    static constexpr int kIdx = kP + kBM * kBN * 2;    // 2 warps x 128 int indices
+    static constexpr int kBars = kIdx + 2 * kBN * 4;
+    static constexpr int kMisc = kBars + (int)sizeof(Bars);
+    static constexpr int kBytes = kMisc + 64;
+    // room to align the base to 1 KB; at least 120 KB so that one CTA holds an SM (and
+    // its 512 TMEM columns) alone
+    static constexpr int kAlloc = (kBytes + 1024) > 122880 ? (kBytes + 1024) : 122880;
+};
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p)
+{
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ unsigned long long global_ns()
+{
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ void bar_init(uint64_t *b, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(b)), "r"(count));
+}
+
+__device__ __forceinline__ void bar_arrive(uint64_t *b)
+{
+    asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(smem_u32(b))
+                 : "memory");
+}
+
+__device__ __forceinline__ bool bar_test(uint64_t *b, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(b)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait by one thread; on timeout sets the CTA abort flag and the device status.
+__device__ __forceinline__ bool bar_wait(uint64_t *b, uint32_t parity, volatile int *abort_flag,
+                                         int32_t *status)
+{
+    if (bar_test(b, parity)) return true;
+    const unsigned long long t0 = global_ns();
+    while (!bar_test(b, parity)) {
+        if (*abort_flag) return false;
+        if (global_ns() - t0 > kWaitNs) {
+            *abort_flag = 1;
+            set_status(status, SCOPE_DEV_TIMEOUT);
+            return false;
+        }
+    }
+    return true;
+}
+
+// Warp-uniform wait: lane 0 polls, every lane gets the same answer.
+__device__ __forceinline__ bool warp_wait(uint64_t *b, uint32_t parity, volatile int *abort_flag,
+                                          int32_t *status)
+{
+    int ok = 0;
+    if ((threadIdx.x & 31) == 0) ok = bar_wait(b, parity, abort_flag, status) ? 1 : 0;
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    __syncwarp();
+    return ok != 0;
+}
+
+__device__ __forceinline__ bool warp_aborted(volatile int *abort_flag)
+{
+    return __any_sync(0xffffffffu, *abort_flag != 0);
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void cp_async_arrive(uint64_t *b)
+{
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(b)) : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async()
+{
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before()
+{
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void tc_fence_after()
+{
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor, 128-byte swizzle (sm_100 layout: version 1 at bit 46,
+// swizzle mode 2 at bits 61-63); addresses and offsets in 16-byte units.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t addr, uint32_t lbo, uint32_t sbo)
+{
+    return (uint64_t)((addr & 0x3FFFFu) >> 4) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// Instruction descriptor, kind::f16: fp32 accumulator, bf16 A and B, A K-major.
+__host__ __device__ constexpr uint32_t f16_idesc(int M, int N, bool b_mn_major)
+{
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) |
+           ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                         uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void mma_commit(uint64_t *b)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     smem_u32(b))
+                 : "memory");
+}
+
+// 32 consecutive fp32 columns of this thread's TMEM lane; valid after tmem_wait_ld().
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float *v)
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+        "%12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, "
+        "%30, %31}, [%32];"
+        : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]), "=f"(v[6]),
+          "=f"(v[7]), "=f"(v[8]), "=f"(v[9]), "=f"(v[10]), "=f"(v[11]), "=f"(v[12]), "=f"(v[13]),
+          "=f"(v[14]), "=f"(v[15]), "=f"(v[16]), "=f"(v[17]), "=f"(v[18]), "=f"(v[19]),
+          "=f"(v[20]), "=f"(v[21]), "=f"(v[22]), "=f"(v[23]), "=f"(v[24]), "=f"(v[25]),
+          "=f"(v[26]), "=f"(v[27]), "=f"(v[28]), "=f"(v[29]), "=f"(v[30]), "=f"(v[31])
+        : "r"(taddr)
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32])
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+        "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, "
+        "%29, %30, %31, %32};" ::"r"(taddr),
+        "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+        "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+        "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+        "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+        "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+        "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])),
+        "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])), "r"(__float_as_uint(v[20])),
+        "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
+        "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
+        "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
+        "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_ld()
+{
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_st()
+{
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ float fast_exp2(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// Byte offset of (row r, 16-byte chunk ch) in a 128B-swizzled K-major tile of kBM rows.
+__device__ __forceinline__ uint32_t sw_off(int r, int ch)
+{
+    return (uint32_t)((ch >> 3) * (kBM * 128) + (r >> 3) * 1024 + (r & 7) * 128 +
+                      (((ch & 7) ^ (r & 7)) << 4));
+}
+
+// Expands the next n (<= 128) selected key indices of a mask row into idx[0..n).
+// Warp-cooperative; (wpos, rem) is the cursor: word index and its unconsumed bits.
+__device__ __forceinline__ void next_indices(const uint32_t *row, int nw, int N, int n, int &wpos,
+                                             uint32_t &rem, int *idx)
+{
+    const int lane = threadIdx.x & 31;
+    int count = 0;
+    while (count < n && wpos < nw) {
+        const int w = wpos + lane;
+        uint32_t bits = 0;
+        if (w < nw) {
+            bits = lane == 0 ? rem : row[w];
+            if (w == nw - 1 && (N & 31)) bits &= (1u << (N & 31)) - 1u;
+        }
+        const int pc = __popc(bits);
+        int incl = pc;
+        for (int o = 1; o < 32; o <<= 1) {
+            const int t = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += t;
+        }
+        const int excl = incl - pc;
+        const int total = __shfl_sync(0xffffffffu, incl, 31);
+        const int need = n - count;
+        // lane writes the first min(pc, need - excl) of its bits
+        int take = min(pc, max(0, need - excl));
+        uint32_t b = bits;
+        for (int k = 0; k < take; ++k) {
+            const int bit = __ffs(b) - 1;
+            b &= b - 1;
+            idx[count + excl + k] = w * 32 + bit;
+        }
+        if (total <= need) {
+            count += total;
+            wpos += 32;
+            rem = (wpos < nw) ? row[wpos] : 0u;
+        } else {
+            // the crossing lane keeps its unconsumed bits
+            const unsigned cross = __ballot_sync(0xffffffffu, excl < need && incl > need);
+            const unsigned full = __ballot_sync(0xffffffffu, incl == need && pc > 0);
+            int src;
+            uint32_t left;
+            if (cross) {
+                src = __ffs(cross) - 1;
+                left = __shfl_sync(0xffffffffu, b, src);
+            } else {
+                src = __ffs(full) - 1 + 1;   // next word starts fresh
+                left = 0xffffffffu;          // placeholder, replaced below
+            }
+            const int neww = wpos + src;
+            if (!cross) left = (neww < nw) ? row[neww] : 0u;
+            wpos = neww;
+            rem = left;
+            count = n;
+        }
+        __syncwarp();
+    }
+    // a mask row with fewer bits than requested (inconsistent input): pad with key 0
+    for (int k = count + lane; k < n; k += 32) idx[k] = 0;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a)
+{
+    using L = Smem<D>;
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    unsigned char *sm = reinterpret_cast<unsigned char *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    Bars *bars = reinterpret_cast<Bars *>(sm + L::kBars);
+    int *misc = reinterpret_cast<int *>(sm + L::kMisc);
+    volatile int *abort_flag = misc;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(misc + 1);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t sbase = smem_u32(sm);
+
+    if (threadIdx.x == 0) {
+        misc[0] = 0;
+        bar_init(&bars->q_full, 32);
+        bar_init(&bars->q_empty, 1);
+        for (int s = 0; s < kStages; ++s) {
+            bar_init(&bars->k_full[s], 32);
+            bar_init(&bars->v_full[s], 32);
+            bar_init(&bars->kv_empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            bar_init(&bars->s_full[b], 1);
+            bar_init(&bars->s_empty[b], 4);
+        }
+        bar_init(&bars->p_full, 4);
+        bar_init(&bars->o_done, 1);
+        bar_init(&bars->o_free, 4);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 6) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(tmem_slot)),
+                     "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const int n_items = a.counter[0];
+
+    if (warp == 4 || warp == 5) {
+        // ------------------------------------------------------------ gather warps
+        const bool is_k = warp == 4;
+        const __nv_bfloat16 *src = reinterpret_cast<const __nv_bfloat16 *>(is_k ? a.K : a.V);
+        const __nv_bfloat16 *Qp = reinterpret_cast<const __nv_bfloat16 *>(a.Q);
+        int *idx = reinterpret_cast<int *>(sm + L::kIdx) + (is_k ? 0 : kBN);
+        uint32_t stage_it = 0, q_it = 0;
+        constexpr int CH = D / 8;   // 16-byte chunks per row
+        for (int it = blockIdx.x; it < n_items && !warp_aborted(abort_flag); it += gridDim.x) {
+            const int4 item = a.items[it];
+            const int bh = item.x, c = item.y, q0 = item.z, nq = item.w;
+            const long long r = a.final_cnt[(size_t)bh * a.Cq + c];
+            const int T = (int)((r + kBN - 1) / kBN);
+            const __nv_bfloat16 *base = src + (size_t)bh * a.N * D;
+            if (is_k) {
+                // Q tile: rows perm[q0 .. q0+nq), zero rows beyond nq
+                if (!warp_wait(&bars->q_empty, (q_it & 1) ^ 1, abort_flag, a.status)) break;
+                const int32_t *perm = a.perm + (size_t)bh * a.perm_bh;
+                const __nv_bfloat16 *qb = Qp + (size_t)bh * a.N * D;
+                for (int id = lane; id < kBM * CH; id += 32) {
+                    const int row = id / CH, ch = id - row * CH;
+                    const bool ok = row < nq;
+                    const int tok = ok ? perm[q0 + row] : 0;
+                    cp_async16(sbase + L::kQ + sw_off(row, ch), qb + (size_t)tok * D + ch * 8, ok ? 16 : 0);
+                }
+                cp_async_arrive(&bars->q_full);
+                ++q_it;
+            }
+            const uint32_t *mrow = a.mask + ((size_t)bh * a.Cq + c) * a.nw;
+            int wpos = 0;
+            uint32_t rem = mrow[0];
+            for (int t = 0; t < T; ++t) {
+                const int s = stage_it % kStages;
+                if (!warp_wait(&bars->kv_empty[s], ((stage_it / kStages) & 1) ^ 1, abort_flag, a.status))
+                    break;
+                const int nvalid = (int)min((long long)kBN, r - (long long)t * kBN);
+                next_indices(mrow, a.nw, a.N, nvalid, wpos, rem, idx);
+                __syncwarp();
+                const uint32_t dst0 = sbase + (is_k ? L::kK : L::kV) + s * L::kTile;
+                for (int id = lane; id < kBN * CH; id += 32) {
+                    const int row = id / CH, ch = id - row * CH;
+                    const bool ok = row < nvalid;
+                    const int key = ok ? idx[row] : 0;
+                    cp_async16(dst0 + sw_off(row, ch), base + (size_t)key * D + ch * 8, ok ? 16 : 0);
+                }
+                cp_async_arrive(is_k ? &bars->k_full[s] : &bars->v_full[s]);
+                __syncwarp();
+                ++stage_it;
+            }
+        }
+        asm volatile("cp.async.wait_all;" ::: "memory");
+    } else if (warp == 6) {
+        // ------------------------------------------------------------ MMA issuer
+        constexpr uint32_t idesc_qk = f16_idesc(kBM, kBN, false);
+        constexpr uint32_t idesc_pv = f16_idesc(kBM, D, true);
+        uint32_t stage_it = 0, q_it = 0, s_it = 0, p_it = 0, item_it = 0;
+        const bool leader = lane == 0;
+        for (int it = blockIdx.x; it < n_items && !warp_aborted(abort_flag); it += gridDim.x, ++item_it) {
+            const int4 item = a.items[it];
+            const long long r = a.final_cnt[(size_t)item.x * a.Cq + item.y];
+            const int T = (int)((r + kBN - 1) / kBN);
+            if (!warp_wait(&bars->q_full, q_it & 1, abort_flag, a.status)) break;
+            ++q_it;
+            bool ok = true;
+            for (int t = 0; t <= T && ok; ++t) {
+                if (t < T) {
+                    const int s = (stage_it + t) % kStages;
+                    const int b = (s_it) & 1;
+                    ok = warp_wait(&bars->k_full[s], ((stage_it + t) / kStages) & 1, abort_flag, a.status) &&
+                         warp_wait(&bars->s_empty[b], ((s_it >> 1) & 1) ^ 1, abort_flag, a.status);
+                    if (!ok) break;
+                    fence_proxy_async();
+                    tc_fence_after();
+                    if (leader) {
+                        const uint32_t qa = sbase + L::kQ, ka = sbase + L::kK + s * L::kTile;
+#pragma unroll
+                        for (int kk = 0; kk < D / 16; ++kk) {
+                            const uint32_t off = (kk >> 2) * (kBM * 128) + (kk & 3) * 32;
+                            mma_bf16(tmem + b * kBN, sw128_desc(qa + off, 16, 1024),
+                                     sw128_desc(ka + off, 16, 1024), idesc_qk, kk > 0);
+                        }
+                        mma_commit(&bars->s_full[b]);
+                        if (t == T - 1) mma_commit(&bars->q_empty);
+                    }
+                    __syncwarp();
+                    ++s_it;
+                }
+                if (t >= 1) {
+                    // O += P_{t-1} V_{t-1}
+                    const int tp = t - 1;
+                    const int s = (stage_it + tp) % kStages;
+                    ok = warp_wait(&bars->p_full, p_it & 1, abort_flag, a.status) &&
+                         warp_wait(&bars->v_full[s], ((stage_it + tp) / kStages) & 1, abort_flag, a.status);
+                    if (ok && tp == 0)
+                        ok = warp_wait(&bars->o_free, (item_it & 1) ^ 1, abort_flag, a.status);
+                    if (!ok) break;
+                    ++p_it;
+                    fence_proxy_async();
+                    tc_fence_after();
+                    if (leader) {
+                        const uint32_t pa = sbase + L::kP, va = sbase + L::kV + s * L::kTile;
+#pragma unroll
+                        for (int kk = 0; kk < kBN / 16; ++kk) {
+                            const uint32_t poff = (kk >> 2) * (kBM * 128) + (kk & 3) * 32;
+                            mma_bf16(tmem + 2 * kBN, sw128_desc(pa + poff, 16, 1024),
+                                     sw128_desc(va + kk * 2048, kBM * 128, 1024), idesc_pv,
+                                     (tp > 0 || kk > 0) ? 1u : 0u);
+                        }
+                        mma_commit(&bars->o_done);
+                        mma_commit(&bars->kv_empty[s]);
+                    }
+                    __syncwarp();
+                }
+            }
+            stage_it += T;
+        }
+    } else if (warp < 4) {
+        // ------------------------------------------------------------ softmax + epilogue
+        const int row = threadIdx.x;   // 0..127 = TMEM lane
+        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        uint32_t s_it = 0, o_it = 0;
+        const float c = a.scale_log2;
+        unsigned char *P = sm + L::kP;
+        for (int it = blockIdx.x; it < n_items && !warp_aborted(abort_flag); it += gridDim.x) {
+            const int4 item = a.items[it];
+            const int bh = item.x, cl = item.y, q0 = item.z, nq = item.w;
+            const long long r = a.final_cnt[(size_t)bh * a.Cq + cl];
+            const int T = (int)((r + kBN - 1) / kBN);
+            float m_run = -INFINITY, l = 0.f;
+            bool ok = true;
+            for (int t = 0; t < T; ++t) {
+                const int b = s_it & 1;
+                ok = warp_wait(&bars->s_full[b], (s_it >> 1) & 1, abort_flag, a.status);
+                if (!ok) break;
+                tc_fence_after();
+                float s[kBN];
+#pragma unroll
+                for (int q = 0; q < kBN / 32; ++q)
+                    tmem_ld32(tmem + lane_base + b * kBN + q * 32, s + q * 32);
+                tmem_wait_ld();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) bar_arrive(&bars->s_empty[b]);
+                ++s_it;
+                const int nvalid = (int)min((long long)kBN, r - (long long)t * kBN);
+                float mt = -INFINITY;
+#pragma unroll
+                for (int j = 0; j < kBN; ++j) {
+                    s[j] = (j < nvalid) ? s[j] * c : -INFINITY;
+                    mt = fmaxf(mt, s[j]);
+                }
+                // PV of the previous tile must be done: P buffer free, O stable
+                if (t > 0) {
+                    ok = warp_wait(&bars->o_done, o_it & 1, abort_flag, a.status);
+                    if (!ok) break;
+                    ++o_it;
+                    tc_fence_after();
+                }
+                const bool need = mt > m_run + 8.f;
+                if (t > 0 && __any_sync(0xffffffffu, need)) {
+                    const float alpha = need ? fast_exp2(m_run - mt) : 1.f;
+#pragma unroll 1
+                    for (int q = 0; q < D / 32; ++q) {
+                        float o[32];
+                        tmem_ld32(tmem + lane_base + 2 * kBN + q * 32, o);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) o[e] *= alpha;
+                        tmem_st32(tmem + lane_base + 2 * kBN + q * 32, o);
+                    }
+                    tmem_wait_st();
+                    if (need) l *= alpha;
+                }
+                if (need) m_run = mt;
+                float ls = 0.f;
+#pragma unroll
+                for (int j = 0; j < kBN; j += 8) {
+                    uint32_t pk[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float p0 = fast_exp2(s[j + 2 * e] - m_run);
+                        const float p1 = fast_exp2(s[j + 2 * e + 1] - m_run);
+                        ls += p0 + p1;
+                        __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
+                        pk[e] = *reinterpret_cast<uint32_t *>(&h);
+                    }
+                    *reinterpret_cast<uint4 *>(P + sw_off(row, j >> 3)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                }
+                l += ls;
+                fence_proxy_async();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) bar_arrive(&bars->p_full);
+            }
+            if (!ok) break;
+            // epilogue: O / l for the valid rows
+            if (!warp_wait(&bars->o_done, o_it & 1, abort_flag, a.status)) break;
+            ++o_it;
+            tc_fence_after();
+            const float inv = l > 0.f ? 1.f / l : 0.f;
+            const bool valid = row < nq;
+            __nv_bfloat16 *dst = nullptr;
+            if (valid) {
+                const int tok = a.perm[(size_t)bh * a.perm_bh + q0 + row];
+                dst = reinterpret_cast<__nv_bfloat16 *>(a.O) + ((size_t)bh * a.N + tok) * D;
+            }
+#pragma unroll 1
+            for (int q = 0; q < D / 32; ++q) {
+                float o[32];
+                tmem_ld32(tmem + lane_base + 2 * kBN + q * 32, o);
+                tmem_wait_ld();
+                if (valid) {
+#pragma unroll
+                    for (int e = 0; e < 32; e += 8) {
+                        uint32_t pk[4];
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            __nv_bfloat162 h = __floats2bfloat162_rn(o[e + 2 * k] * inv, o[e + 2 * k + 1] * inv);
+                            pk[k] = *reinterpret_cast<uint32_t *>(&h);
+                        }
+                        *reinterpret_cast<uint4 *>(dst + q * 32 + e) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) bar_arrive(&bars->o_free);
+        }
+    }
+    // drain and free TMEM
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 6)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
+                     : "memory");
+}
+
+}  // namespace
+
 cudaError_t attention_tc_run(const AttnArgs &a, cudaStream_t s)
 {
-    return attention_simt_run(a, s);
+    if (a.d == 128) {
+        const int smem = Smem<128>::kAlloc;
+        cudaFuncSetAttribute(attn_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        attn_tc_kernel<128><<<a.num_sms, kThreads, smem, s>>>(a);
+    } else {
+        const int smem = Smem<64>::kAlloc;
+        cudaFuncSetAttribute(attn_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        attn_tc_kernel<64><<<a.num_sms, kThreads, smem, s>>>(a);
+    }
+    return cudaGetLastError();
 }
 
 }  // namespace scope

@@ -32,8 +32,8 @@
  *    an unresolvable selection tie) set bits in a status word inside the workspace,
  *    read by scope_get_device_status; each entry point clears that word first.
  *  - Limits: d in {64, 128}; d_t, d_h, d_w >= 1 with d_t + d_h + d_w = d;
- *    1 <= Cq, Cm <= min(N, 4096); 1 <= iters <= 64; 0 < rho <= 1; 0 <= alpha <= 1;
- *    N <= 2^24; B*H*N < 2^31.  Device pointers must be 16-byte aligned.
+ *    1 <= Cq, Cm <= min(N, 2048); 1 <= iters <= 64; 0 < rho <= 1; 0 <= alpha <= 1;
+ *    N <= 2^22; B*H <= 16383; B*H*N < 2^31.  Device pointers must be 16-byte aligned.
  */
 #ifndef SCOPE_H
 #define SCOPE_H
@@ -59,7 +59,8 @@ typedef enum { SCOPE_F32 = 0, SCOPE_BF16 = 1 } scope_dtype;
 /* Device status bits (scope_get_device_status). */
 #define SCOPE_DEV_BAD_INIT_INDEX 0x1   /* an init index was outside [0, N); row 0 was used */
 #define SCOPE_DEV_SELECT_TIE     0x2   /* a selection boundary could not be resolved exactly */
-#define SCOPE_DEV_BAD_ASSIGN     0x4   /* a cluster index >= C reached the attention stage */
+#define SCOPE_DEV_BAD_ASSIGN     0x4   /* a cluster index >= C or a code >= Cm was supplied (clamped) */
+#define SCOPE_DEV_TIMEOUT        0x8   /* an on-chip pipeline wait gave up (~4 s); outputs invalid */
 
 /* Shape and hyperparameters of one layer.  rho: Top-p threshold of Eq. 7 (the paper
  * does not report it; 0.9 is the usual choice).  alpha: fixed Top-k minimum as a
