@@ -1,0 +1,406 @@
+#!/usr/bin/env python
+"""Benchmark of the SCOPE per-layer sparse-attention hot path on B200.
+
+One step = one SCOPE layer through the C ABI (scope_forward): query clustering, key
+subspace clustering, LUT / Top-p / k_head / top-up selection and the gathered sparse
+attention, on the HunyuanVideo-shaped 720p layer (B=1, 24 heads, 33x45x80 = 118800
+tokens, d=128 split 16/56/56, bf16, Cq=300, Cm=333, rho=0.9, alpha=0.1, 5 Lloyd
+iterations), synthetic inputs from the seeded generator.
+
+Metric: effective TFLOP/s of the layer = 4 * sum_c n_c * r_c * d / layer time (the
+attention FLOPs over the selected pairs only), plus the layer time in ms.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl scope|reference]
+
+Multi-GPU (torchrun, one rank per GPU): every rank runs its own layer (weak scaling,
+no collective on the data path); the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from free_sparse_attention_b200 import synth  # noqa: E402
+from free_sparse_attention_b200.workloads import ALL, HUNYUAN720  # noqa: E402
+
+FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12   # FMA pipes at the max SM clock
+METRIC = "SCOPE layer effective TFLOP/s (4*sum n_c*r_c*d / layer time) at 118800 tokens"
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16": p["bf16_tflops"],
+                "bf16_sustained": p.get("bf16_tflops_sustained", p["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "source": "fallback"}
+
+
+def kernels_per_forward(iters: int) -> int:
+    # clustering: init + iters x (fast assign, exact assign, hist, scan, scatter, update)
+    # selection: check, top-p, k_head, mask; attention: items, zero-fill, attention
+    return 1 + 6 * iters + 4 + 3
+
+
+def workload_desc(w):
+    return (f"{w.name}: B={w.B} H={w.H} grid {w.T}x{w.Hg}x{w.Wg} (N={w.N}) d={w.d} "
+            f"({w.d_t}/{w.d_h}/{w.d_w}) {w.dtype} Cq={w.Cq} Cm={w.Cm} rho={w.rho} "
+            f"alpha={w.alpha} iters={w.iters}")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = f"/tmp/scope_clocks_{os.getpid()}.csv"
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        load = [s for s in sm if mx is None or s > 0.3 * mx] or sm
+        return {"sm_mhz": statistics.median(load), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+def oracle_sample(w, T_sample=6):
+    """The oracle on a bounded sub-layer: head (0, 0) of the same workload with the
+    grid cut to the first T_sample frames (N_s = T_sample*Hg*Wg tokens); every stage
+    runs in full on it.  Each stage's cost is extrapolated to the whole layer by its
+    complexity (clustering and selection linear in N per head, attention by its
+    effective FLOPs).  Returns (layer seconds, description, threads)."""
+    import oracle
+    ws = w.with_(T=T_sample, H=1, B=1)
+    x = synth.layer_inputs(ws)
+    q, k, v = x["q"][0], x["k"][0], x["v"][0]
+    t0 = time.perf_counter()
+    rq = oracle.kmeans(q, 0, ws.d, ws.Cq, ws.iters, init_idx=x["q_init"][0])
+    rk = oracle.cluster_keys(k, (ws.d_t, ws.d_h, ws.d_w), ws.Cm, ws.iters, init_idx3=x["k_init"][0])
+    t1 = time.perf_counter()
+    sel = oracle.select(rq["centroids"], rq["sizes"], rk["centroids"], rk["codes"],
+                        (ws.d_t, ws.d_h, ws.d_w), ws.rho, ws.alpha)
+    t2 = time.perf_counter()
+    oracle.attention(q, k, v, rq["assign"], sel["mask"])
+    t3 = time.perf_counter()
+    eff = 4.0 * float(np.dot(rq["sizes"].astype(np.float64), sel["r"].astype(np.float64))) * ws.d
+    scale = (w.N / ws.N) * w.H * w.B
+    desc = (f"oracle on head (0,0) cut to the first {T_sample} frames (N_s={ws.N}): clustering "
+            f"{t1 - t0:.2f}s, selection {t2 - t1:.2f}s, attention {t3 - t2:.2f}s "
+            f"({eff / (t3 - t2) / 1e9:.2f} GFLOP/s); clustering and selection scaled by "
+            f"N/N_s x heads, attention by the layer's effective FLOPs")
+    return {"clust_s": (t1 - t0) * scale, "sel_s": (t2 - t1) * scale, "attn_rate": eff / (t3 - t2),
+            "desc": desc, "threads": oracle.num_threads()}
+
+
+def layer_seconds_from_sample(s, flops):
+    return s["clust_s"] + s["sel_s"] + flops / s["attn_rate"]
+
+
+def expected_layer_flops(w):
+    """Effective FLOPs of the layer when r_c is unknown (reference arm): dense x 0.89,
+    the realised density the oracle measures on this generator at rho = 0.9."""
+    return 4.0 * w.B * w.H * w.N * w.N * w.d * 0.89
+
+
+def run_reference(args, w):
+    world, rank, _ = dist_setup()
+    if rank != 0:
+        return 0
+    for _ in range(args.warmup):
+        oracle_sample(w, T_sample=4)
+    times, desc, threads = [], "", 1
+    flops = expected_layer_flops(w)
+    for _ in range(args.steps):
+        s = oracle_sample(w, T_sample=4)
+        times.append(layer_seconds_from_sample(s, flops))
+        desc, threads = s["desc"], s["threads"]
+    sec = statistics.mean(times)
+    value = flops / sec / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": sec * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded generator G)",
+            "config": {"workload": workload_desc(w), "parallelism": "oracle, OpenMP threads"},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                             "sample": desc + "; effective FLOPs taken at density 0.89"},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- GPU arm
+def traffic_from_profile(kernel_file):
+    """DRAM bytes per attention launch from the committed ncu summary, if the kernel
+    source is unchanged since it was captured (else None)."""
+    prof = os.path.join(ROOT, "profiles", "attn_tc_hunyuan720p.json")
+    if not os.path.exists(prof):
+        return None
+    with open(prof) as f:
+        p = json.load(f)
+    with open(kernel_file, "rb") as f:
+        h = hashlib.sha256(f.read()).hexdigest()
+    if p.get("kernel_sha256") != h:
+        return None
+    return p.get("dram_bytes_per_launch")
+
+
+def run_scope(args, w):
+    import torch
+    import torch.distributed as dist
+    from free_sparse_attention_b200 import capi
+
+    world, rank, local = dist_setup()
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    capi.lib()
+    p = capi.Params.from_workload(w)
+    x = synth.layer_inputs(w)
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    host = {n: torch.from_numpy(x[n]).reshape(w.B, w.H, w.N, w.d).to(dt).pin_memory() for n in "qkv"}
+    host["qi"] = torch.from_numpy(x["q_init"]).reshape(w.B, w.H, w.Cq).pin_memory()
+    host["ki"] = torch.from_numpy(x["k_init"]).reshape(w.B, w.H, 3, w.Cm).pin_memory()
+    del x
+    dev = {n: t.cuda() for n, t in host.items()}
+    ws = capi.alloc_workspace(p)
+    O = torch.empty_like(dev["q"])
+    _, it = capi.forward(p, dev["q"], dev["k"], dev["v"], dev["qi"], dev["ki"], ws=ws, out=O,
+                         intermediates=True)
+    torch.cuda.synchronize()
+    status = capi.get_device_status(ws)
+    n_c = it["q_sizes"].double()
+    r_c = it["final_counts"].double()
+    flops = float(4.0 * (n_c * r_c).sum().item() * w.d)
+    density = float((n_c * r_c).sum().item() / (w.B * w.H * w.N * w.N))
+    del it
+
+    def mk_events():
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+        for e in evs:
+            e.record()
+        return evs
+
+    for _ in range(args.warmup):
+        capi.forward(p, dev["q"], dev["k"], dev["v"], dev["qi"], dev["ki"], ws=ws, out=O)
+    stage_evs = [mk_events() for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for s in range(args.steps):
+        capi.forward(p, dev["q"], dev["k"], dev["v"], dev["qi"], dev["ki"], ws=ws, out=O,
+                     stage_events=stage_evs[s])
+    e1.record()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1) / args.steps
+    st = np.array([[ev[i].elapsed_time(ev[i + 1]) for i in range(4)] for ev in stage_evs])
+    stage_ms = st.mean(axis=0)
+    if world > 1:
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    status |= capi.get_device_status(ws)
+
+    # end to end through the C ABI with host buffers: H2D inputs, layer, D2H output
+    Oh = torch.empty(O.shape, dtype=O.dtype, pin_memory=True)
+    h2d = sum(host[n].numel() * host[n].element_size() for n in host)
+    d2h = Oh.numel() * Oh.element_size()
+
+    def e2e_step():
+        for n in host:
+            dev[n].copy_(host[n], non_blocking=True)
+        capi.forward(p, dev["q"], dev["k"], dev["v"], dev["qi"], dev["ki"], ws=ws, out=O)
+        Oh.copy_(O, non_blocking=True)
+
+    for _ in range(max(1, min(args.warmup, 2))):
+        e2e_step()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / args.steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    # dense attention on the same shape (library comparator, not part of the path)
+    dense_ms = None
+    if not args.no_dense:
+        import torch.nn.functional as F
+        for _ in range(2):
+            F.scaled_dot_product_attention(dev["q"], dev["k"], dev["v"])
+        torch.cuda.synchronize()
+        e0.record()
+        for _ in range(3):
+            F.scaled_dot_product_attention(dev["q"], dev["k"], dev["v"])
+        e1.record()
+        torch.cuda.synchronize()
+        dense_ms = e0.elapsed_time(e1) / 3
+
+    pk = peaks()
+    attn_ms = float(stage_ms[3])
+    achieved = flops / (attn_ms * 1e-3) / 1e12
+    traffic = traffic_from_profile(os.path.join(ROOT, "free_sparse_attention_b200", "csrc",
+                                                "attention_tc.cu"))
+    clust_bytes = w.iters * 2 * w.B * w.H * w.N * w.d * 2
+    clust_flops = 2.0 * w.iters * w.B * w.H * w.N * (w.Cq * w.d + w.Cm * w.d)
+    nw = (w.N + 31) // 32
+    sel_bytes = w.B * w.H * (6 * w.N + w.Cq * nw * 4)
+    value = world * flops / (ms * 1e-3) / 1e12
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded generator G: smooth field + noise, 3D RoPE)",
+        "config": {"workload": workload_desc(w), "global_batch": world * w.B, "seq_len": w.N,
+                   "parallelism": f"{world} independent layers, one per GPU (no collective)",
+                   "l2": "inputs larger than L2 (Q, K, V = 2.19 GB resident in HBM)"},
+        "roofline": {"bound": "tensor", "kernel": "attn_tc_kernel (tcgen05 sparse attention)",
+                     "achieved": achieved, "peak": pk["bf16_sustained"], "unit": "TFLOP/s",
+                     "frac": achieved / pk["bf16_sustained"], "traffic": traffic,
+                     "peak_source": f"{pk['source']} bf16 sustained (kernel timed inside the step)"},
+        "stages_ms": {"clustering": float(stage_ms[0]), "selection": float(stage_ms[1]),
+                      "worklist": float(stage_ms[2]), "attention": attn_ms},
+        "stage_fractions": {
+            "clustering_hbm": clust_bytes / (stage_ms[0] * 1e-3) / 1e9 / pk["hbm_gbs"],
+            "clustering_fp32_alu": clust_flops / (stage_ms[0] * 1e-3) / 1e12 / FP32_ALU_TFLOPS,
+            "selection_hbm": sel_bytes / (stage_ms[1] * 1e-3) / 1e9 / pk["hbm_gbs"]},
+        "density": density, "effective_tflop_per_layer": flops / 1e12,
+        "dense_sdpa_ms": dense_ms,
+        "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
+        "gpu_launches": kernels_per_forward(w.iters) * args.steps,
+        "device_status": status,
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        s = oracle_sample(w)
+        sec = layer_seconds_from_sample(s, flops)
+        line["cpu_baseline"] = {"value": flops / sec / 1e12, "unit": "TFLOP/s", "cores": s["threads"],
+                                "kind": "oracle", "sample": s["desc"]}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def profile_once(w):
+    """One warm-up layer and one layer, nothing else (the command ncu captures)."""
+    import torch
+    from free_sparse_attention_b200 import capi
+    p = capi.Params.from_workload(w)
+    x = synth.layer_inputs(w)
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    Q, K, V = (torch.from_numpy(x[n]).reshape(w.B, w.H, w.N, w.d).to("cuda", dt) for n in "qkv")
+    qi = torch.from_numpy(x["q_init"]).reshape(w.B, w.H, w.Cq).cuda()
+    ki = torch.from_numpy(x["k_init"]).reshape(w.B, w.H, 3, w.Cm).cuda()
+    ws = capi.alloc_workspace(p)
+    for _ in range(2):
+        O = capi.forward(p, Q, K, V, qi, ki, ws=ws)
+    torch.cuda.synchronize()
+    st = capi.get_device_status(ws)
+    print(json.dumps({"workload": workload_desc(w), "device_status": st,
+                      "out_finite": bool(torch.isfinite(O.float()).all().item())}))
+    return 0 if st == 0 else 1
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["scope", "reference"], default="scope")
+    ap.add_argument("--workload", default=HUNYUAN720.name, choices=sorted(ALL))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--heads", type=int, default=0,
+                    help="override the head count (small cases for profiling)")
+    ap.add_argument("--profile-once", action="store_true",
+                    help="run the layer once (after one warm-up) and exit; for ncu captures")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    w = ALL[args.workload]
+    if args.heads:
+        w = w.with_(H=args.heads)
+    if args.profile_once:
+        return profile_once(w)
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_scope(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

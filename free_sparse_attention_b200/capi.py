@@ -59,7 +59,8 @@ class Params(ctypes.Structure):
 class Intermediates(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
                 ("q_centroids", "q_assign", "q_sizes", "k_centroids", "k_codes", "topp_counts",
-                 "base_counts", "k_head", "final_counts", "sel_mask")]
+                 "base_counts", "k_head", "final_counts", "sel_mask")] + \
+               [("stage_events", ctypes.c_void_p * 5)]
 
 
 _lib = None
@@ -172,13 +173,20 @@ def sparse_attention(p, Q, K, V, q_assign, sel_mask, final_counts, ws=None, out=
 
 
 def forward(p, Q, K, V, q_init_idx, k_init_idx, ws=None, out=None, intermediates=False,
-            stream=None):
-    """The whole layer.  With intermediates=True also returns every stage's outputs."""
+            stage_events=None, stream=None):
+    """The whole layer.  With intermediates=True also returns every stage's outputs.
+
+    stage_events: optional list of 5 recorded torch.cuda.Event (timing enabled) that
+    the library records at the stage boundaries (see scope_intermediates)."""
     dev = Q.device
     ws = alloc_workspace(p, dev) if ws is None else ws
     O = torch.empty_like(Q) if out is None else out
     inter = None
     tensors = {}
+    if stage_events is not None:
+        inter = Intermediates()
+        for k, ev in enumerate(stage_events):
+            inter.stage_events[k] = ev.cuda_event
     if intermediates:
         shp = (p.B, p.H)
         tensors = {
@@ -193,7 +201,9 @@ def forward(p, Q, K, V, q_init_idx, k_init_idx, ws=None, out=None, intermediates
             "final_counts": torch.empty(shp + (p.Cq,), dtype=torch.int32, device=dev),
             "sel_mask": torch.empty(shp + (p.Cq, p.nw), dtype=torch.int32, device=dev),
         }
-        inter = Intermediates(**{k: v.data_ptr() for k, v in tensors.items()})
+        inter = Intermediates() if inter is None else inter
+        for k, v in tensors.items():
+            setattr(inter, k, v.data_ptr())
     _check("scope_forward", lib().scope_forward(
         ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(V), _ptr(q_init_idx), _ptr(k_init_idx), _ptr(O),
         ctypes.byref(inter) if inter is not None else None, _ptr(ws), ws.numel(), _stream(stream)))

@@ -170,12 +170,17 @@ cudaError_t attention_simt_run(const AttnArgs &a, cudaStream_t s)
     return cudaGetLastError();
 }
 
+cudaError_t attention_kernel(const AttnArgs &a, cudaStream_t s)
+{
+    if (a.is_bf16 && a.use_tc) return attention_tc_run(a, s);
+    return attention_simt_run(a, s);
+}
+
 cudaError_t attention_run(const AttnArgs &a, cudaStream_t s)
 {
     cudaError_t e = attention_items(a, s);
     if (e != cudaSuccess) return e;
-    if (a.is_bf16 && a.use_tc) return attention_tc_run(a, s);
-    return attention_simt_run(a, s);
+    return attention_kernel(a, s);
 }
 
 }  // namespace scope

@@ -95,7 +95,9 @@ struct AttnArgs {
     int32_t *status;
     int num_sms;
 };
-cudaError_t attention_run(const AttnArgs &a, cudaStream_t s);
+cudaError_t attention_run(const AttnArgs &a, cudaStream_t s);     // items + kernel
+cudaError_t attention_items(const AttnArgs &a, cudaStream_t s);   // work list only
+cudaError_t attention_kernel(const AttnArgs &a, cudaStream_t s);  // kernel only
 cudaError_t attention_simt_run(const AttnArgs &a, cudaStream_t s);
 size_t select_smem_bytes(int Cm, int d);
 

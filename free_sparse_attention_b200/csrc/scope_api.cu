@@ -423,6 +423,11 @@ scope_status scope_forward(const scope_params *p, const void *Q, const void *K, 
     int32_t *fc = I.final_counts ? I.final_counts : at<int32_t>(ws, L.final_cnt);
     uint32_t *mk = I.sel_mask ? I.sel_mask : at<uint32_t>(ws, L.mask);
     if ((st = clear_status(ws, L, s)) != SCOPE_OK) return st;
+    auto mark = [&](int k) {
+        return I.stage_events[k] ? cudaEventRecord(static_cast<cudaEvent_t>(I.stage_events[k]), s)
+                                 : cudaSuccess;
+    };
+    if (mark(0) != cudaSuccess) return SCOPE_ERR_CUDA;
 
     // stage 1: query clustering and the three key-subspace clusterings, one launch set
     KmArgs a = km_base(*p, L, ws);
@@ -434,17 +439,21 @@ scope_status scope_forward(const scope_params *p, const void *Q, const void *K, 
     a.Cs = std::max(p->Cq, p->Cm);
     a.ds = p->d;
     cudaError_t e = km_run(a, p->iters, s);
-    if (e != cudaSuccess) return SCOPE_ERR_CUDA;
+    if (e != cudaSuccess || mark(1) != cudaSuccess) return SCOPE_ERR_CUDA;
 
     // stage 2: LUT, proxy logits, Top-p, k_head, top-up, masks
     SelArgs sa = sel_args(*p, L, ws, qc, qs, kc, kk, tp, bc, kh, fc, mk);
     e = select_run(sa, s);
-    if (e != cudaSuccess) return SCOPE_ERR_CUDA;
+    if (e != cudaSuccess || mark(2) != cudaSuccess) return SCOPE_ERR_CUDA;
 
     // stage 3: attention; the last clustering iteration already grouped the queries
     const Dims D = dims_of(*p);
     AttnArgs t = attn_args(*p, L, ws, Q, K, V, O, a.perm, 4 * D.N, a.off, 4 * (a.Cs + 1), mk, fc);
-    return cuda_status(attention_run(t, s));
+    e = attention_items(t, s);
+    if (e != cudaSuccess || mark(3) != cudaSuccess) return SCOPE_ERR_CUDA;
+    e = attention_kernel(t, s);
+    if (e != cudaSuccess || mark(4) != cudaSuccess) return SCOPE_ERR_CUDA;
+    return SCOPE_OK;
 }
 
 }  // extern "C"

@@ -89,6 +89,10 @@ typedef struct {
     int32_t *k_head;       /* [B, H] */
     int32_t *final_counts; /* [B, H, Cq]  r_c */
     uint32_t *sel_mask;    /* [B, H, Cq, ceil(N/32)] */
+    /* Optional cudaEvent_t handles (NULL = skip) recorded on the stream at the stage
+     * boundaries: [0] start, [1] after clustering, [2] after selection, [3] after the
+     * attention work list is built, [4] after the attention kernel. */
+    void *stage_events[5];
 } scope_intermediates;
 
 /* Bytes of workspace every entry point below needs for `p` (0 if p is invalid). */
