@@ -27,25 +27,29 @@ namespace {
 
 constexpr int kBM = 128;           // queries per tile
 constexpr int kBN = 128;           // keys per tile
-constexpr int kStages = 2;
+constexpr int kMaxStages = 4;
 constexpr int kThreads = 224;      // 7 warps
 constexpr uint32_t kTmemCols = 512;
 constexpr unsigned long long kWaitNs = 4000000000ull;
 
 struct __align__(8) Bars {
     uint64_t q_full, q_empty;
-    uint64_t k_full[kStages], v_full[kStages], kv_empty[kStages];
+    uint64_t k_full[kMaxStages], k_empty[kMaxStages];
+    uint64_t v_full[kMaxStages], v_empty[kMaxStages];
     uint64_t s_full[2], s_empty[2];
     uint64_t p_full, o_done, o_free;
 };
 
+// K tiles are released right after Q K^T, V tiles after P V; K runs one stage deeper.
 template <int D>
 struct Smem {
+    static constexpr int kKS = D == 128 ? 3 : 4;       // K ring depth
+    static constexpr int kVS = D == 128 ? 2 : 4;       // V ring depth
     static constexpr int kTile = kBM * D * 2;          // bytes of a 128 x D bf16 tile
     static constexpr int kQ = 0;
     static constexpr int kK = kQ + kTile;
-    static constexpr int kV = kK + kStages * kTile;
-    static constexpr int kP = kV + kStages * kTile;
+    static constexpr int kV = kK + kKS * kTile;
+    static constexpr int kP = kV + kVS * kTile;
     static constexpr int kIdx = kP + kBM * kBN * 2;    // 2 warps x 128 int indices
     static constexpr int kBars = kIdx + 2 * kBN * 4;
     static constexpr int kMisc = kBars + (int)sizeof(Bars);
@@ -53,6 +57,7 @@ struct Smem {
     // room to align the base to 1 KB; at least 120 KB so that one CTA holds an SM (and
     // its 512 TMEM columns) alone
     static constexpr int kAlloc = (kBytes + 1024) > 122880 ? (kBytes + 1024) : 122880;
+    static_assert(kAlloc <= 232448, "shared memory budget");
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p)
@@ -78,15 +83,17 @@ __device__ __forceinline__ void bar_arrive(uint64_t *b)
                  : "memory");
 }
 
+// try_wait with a suspend-time hint: the thread sleeps until the phase completes (or
+// the hint, 1 ms, elapses) instead of spinning on the issue slots.
 __device__ __forceinline__ bool bar_test(uint64_t *b, uint32_t parity)
 {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(smem_u32(b)), "r"(parity)
+        : "r"(smem_u32(b)), "r"(parity), "r"(1000000u)
         : "memory");
     return ok != 0;
 }
@@ -321,10 +328,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a)
         misc[0] = 0;
         bar_init(&bars->q_full, 32);
         bar_init(&bars->q_empty, 1);
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < kMaxStages; ++s) {
             bar_init(&bars->k_full[s], 32);
             bar_init(&bars->v_full[s], 32);
-            bar_init(&bars->kv_empty[s], 1);
+            bar_init(&bars->k_empty[s], 1);
+            bar_init(&bars->v_empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
             bar_init(&bars->s_full[b], 1);
@@ -379,9 +387,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a)
             const uint32_t *mrow = a.mask + ((size_t)bh * a.Cq + c) * a.nw;
             int wpos = 0;
             uint32_t rem = mrow[0];
+            const int NS = is_k ? L::kKS : L::kVS;
             for (int t = 0; t < T; ++t) {
-                const int s = stage_it % kStages;
-                if (!warp_wait(&bars->kv_empty[s], ((stage_it / kStages) & 1) ^ 1, abort_flag, a.status))
+                const int s = stage_it % NS;
+                if (!warp_wait(is_k ? &bars->k_empty[s] : &bars->v_empty[s], ((stage_it / NS) & 1) ^ 1,
+                               abort_flag, a.status))
                     break;
                 const int nvalid = (int)min((long long)kBN, r - (long long)t * kBN);
                 next_indices(mrow, a.nw, a.N, nvalid, wpos, rem, idx);
@@ -403,7 +413,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a)
         // ------------------------------------------------------------ MMA issuer
         constexpr uint32_t idesc_qk = f16_idesc(kBM, kBN, false);
         constexpr uint32_t idesc_pv = f16_idesc(kBM, D, true);
-        uint32_t stage_it = 0, q_it = 0, s_it = 0, p_it = 0, item_it = 0;
+        uint32_t k_it = 0, v_it = 0, q_it = 0, s_it = 0, p_it = 0, item_it = 0;
         const bool leader = lane == 0;
         for (int it = blockIdx.x; it < n_items && !warp_aborted(abort_flag); it += gridDim.x, ++item_it) {
             const int4 item = a.items[it];
@@ -414,9 +424,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a)
             bool ok = true;
             for (int t = 0; t <= T && ok; ++t) {
                 if (t < T) {
-                    const int s = (stage_it + t) % kStages;
+                    const int s = k_it % L::kKS;
                     const int b = (s_it) & 1;
-                    ok = warp_wait(&bars->k_full[s], ((stage_it + t) / kStages) & 1, abort_flag, a.status) &&
+                    ok = warp_wait(&bars->k_full[s], (k_it / L::kKS) & 1, abort_flag, a.status) &&
                          warp_wait(&bars->s_empty[b], ((s_it >> 1) & 1) ^ 1, abort_flag, a.status);
                     if (!ok) break;
                     fence_proxy_async();
@@ -430,17 +440,19 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a)
                                      sw128_desc(ka + off, 16, 1024), idesc_qk, kk > 0);
                         }
                         mma_commit(&bars->s_full[b]);
+                        mma_commit(&bars->k_empty[s]);
                         if (t == T - 1) mma_commit(&bars->q_empty);
                     }
                     __syncwarp();
                     ++s_it;
+                    ++k_it;
                 }
                 if (t >= 1) {
                     // O += P_{t-1} V_{t-1}
                     const int tp = t - 1;
-                    const int s = (stage_it + tp) % kStages;
+                    const int s = v_it % L::kVS;
                     ok = warp_wait(&bars->p_full, p_it & 1, abort_flag, a.status) &&
-                         warp_wait(&bars->v_full[s], ((stage_it + tp) / kStages) & 1, abort_flag, a.status);
+                         warp_wait(&bars->v_full[s], (v_it / L::kVS) & 1, abort_flag, a.status);
                     if (ok && tp == 0)
                         ok = warp_wait(&bars->o_free, (item_it & 1) ^ 1, abort_flag, a.status);
                     if (!ok) break;
@@ -457,12 +469,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a)
                                      (tp > 0 || kk > 0) ? 1u : 0u);
                         }
                         mma_commit(&bars->o_done);
-                        mma_commit(&bars->kv_empty[s]);
+                        mma_commit(&bars->v_empty[s]);
                     }
                     __syncwarp();
+                    ++v_it;
                 }
             }
-            stage_it += T;
         }
     } else if (warp < 4) {
         // ------------------------------------------------------------ softmax + epilogue
@@ -493,12 +505,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a)
                 if (lane == 0) bar_arrive(&bars->s_empty[b]);
                 ++s_it;
                 const int nvalid = (int)min((long long)kBN, r - (long long)t * kBN);
-                float mt = -INFINITY;
+                if (nvalid < kBN) {
 #pragma unroll
-                for (int j = 0; j < kBN; ++j) {
-                    s[j] = (j < nvalid) ? s[j] * c : -INFINITY;
-                    mt = fmaxf(mt, s[j]);
+                    for (int j = 0; j < kBN; ++j)
+                        if (j >= nvalid) s[j] = -INFINITY;
                 }
+                float mraw = -INFINITY;
+#pragma unroll
+                for (int j = 0; j < kBN; ++j) mraw = fmaxf(mraw, s[j]);
+                const float mt = mraw * c;   // c > 0: the maximum of the scaled logits
                 // PV of the previous tile must be done: P buffer free, O stable
                 if (t > 0) {
                     ok = warp_wait(&bars->o_done, o_it & 1, abort_flag, a.status);
@@ -528,8 +543,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a)
                     uint32_t pk[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const float p0 = fast_exp2(s[j + 2 * e] - m_run);
-                        const float p1 = fast_exp2(s[j + 2 * e + 1] - m_run);
+                        const float p0 = fast_exp2(fmaf(s[j + 2 * e], c, -m_run));
+                        const float p1 = fast_exp2(fmaf(s[j + 2 * e + 1], c, -m_run));
                         ls += p0 + p1;
                         __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
                         pk[e] = *reinterpret_cast<uint32_t *>(&h);
