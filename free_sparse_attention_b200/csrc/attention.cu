@@ -68,6 +68,50 @@ __global__ void __launch_bounds__(1024) attn_items_kernel(AttnArgs a)
     }
 }
 
+// Expands the selection bitmask of every (bh, cluster) that has queries into its
+// ascending list of selected key indices (the gather order of the attention kernel).
+// grid = BH*Cq units, 256 threads: one mask word per thread per chunk, block prefix sum
+// of the popcounts, then each thread writes its word's set bits.
+__global__ void __launch_bounds__(256) attn_lists_kernel(AttnArgs a)
+{
+    __shared__ int wsum[8];
+    const int u = blockIdx.x, tid = threadIdx.x, lane = tid & 31, w8 = tid >> 5;
+    const int bh = u / a.Cq, c = u - bh * a.Cq;
+    const int32_t *off = a.off + (size_t)bh * a.off_bh;
+    if (off[c + 1] == off[c] || a.final_cnt[u] <= 0) return;
+    const uint32_t *row = a.mask + (size_t)u * a.nw;
+    int32_t *out = a.lists + (size_t)u * a.list_stride;
+    int base = 0;
+    for (int w0 = 0; w0 < a.nw; w0 += 256) {
+        const int w = w0 + tid;
+        uint32_t bits = 0;
+        if (w < a.nw) {
+            bits = row[w];
+            if (w == a.nw - 1 && (a.N & 31)) bits &= (1u << (a.N & 31)) - 1u;
+        }
+        const int pc = __popc(bits);
+        int incl = pc;
+        for (int o = 1; o < 32; o <<= 1) {
+            const int t = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += t;
+        }
+        if (lane == 31) wsum[w8] = incl;
+        __syncthreads();
+        int before = 0, total = 0;
+        for (int k = 0; k < 8; ++k) {
+            before += k < w8 ? wsum[k] : 0;
+            total += wsum[k];
+        }
+        int pos = base + before + incl - pc;
+        while (bits) {
+            out[pos++] = w * 32 + __ffs(bits) - 1;
+            bits &= bits - 1;
+        }
+        base += total;
+        __syncthreads();
+    }
+}
+
 // Queries of clusters that select no key get zeros.
 __global__ void attn_zero_empty_kernel(AttnArgs a)
 {
@@ -156,6 +200,7 @@ cudaError_t attention_items(const AttnArgs &a, cudaStream_t s)
 {
     attn_items_kernel<<<1, 1024, 0, s>>>(a);
     attn_zero_empty_kernel<<<a.BH * a.Cq, 128, 0, s>>>(a);
+    if (a.is_bf16 && a.use_tc) attn_lists_kernel<<<a.BH * a.Cq, 256, 0, s>>>(a);
     return cudaGetLastError();
 }
 

@@ -10,9 +10,11 @@
 //   warp 4     gathers the Q tile once per item and the selected K rows per key tile
 //   warp 5     gathers the selected V rows per key tile
 //   warp 6     allocates TMEM and issues the MMAs (one elected thread)
-// The selected key indices come straight from the selection bitmask (each gather warp
-// expands it with popc + warp prefix sums).  Rows are copied with 16-byte cp.async into
-// the 128B-swizzled K-major layout the tensor core reads, two stages deep.
+// Each cluster's selected key indices are expanded once from the bitmask into an
+// ascending list (attn_lists_kernel).  Rows are gathered with TMA tile::gather4 (four
+// arbitrary rows of one 64-column, 128-byte box per instruction, each lane issuing its
+// own four rows) straight into the 128B-swizzled K-major layout the tensor core reads;
+// K tiles run three stages deep, V tiles two.
 //   S_b = Q K^T   tcgen05.mma kind::f16, M=128, N=128, K=d, fp32 in TMEM (2 buffers)
 //   O  += P V     M=128, N=d, K=128, P bf16 in shared memory, O fp32 in TMEM
 // The softmax keeps a running row maximum and rescales O (TMEM load/store) only when
@@ -20,6 +22,9 @@
 // softmax arithmetic.  Every mbarrier wait gives up after ~4 s, sets a status bit and
 // lets the CTA drain and free its TMEM.
 #include "common.cuh"
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
 
 namespace scope {
 
@@ -50,8 +55,7 @@ struct Smem {
     static constexpr int kK = kQ + kTile;
     static constexpr int kV = kK + kKS * kTile;
     static constexpr int kP = kV + kVS * kTile;
-    static constexpr int kIdx = kP + kBM * kBN * 2;    // 2 warps x 128 int indices
-    static constexpr int kBars = kIdx + 2 * kBN * 4;
+    static constexpr int kBars = kP + kBM * kBN * 2;
     static constexpr int kMisc = kBars + (int)sizeof(Bars);
     static constexpr int kBytes = kMisc + 64;
     // room to align the base to 1 KB; at least 120 KB so that one CTA holds an SM (and
@@ -131,15 +135,23 @@ __device__ __forceinline__ bool warp_aborted(volatile int *abort_flag)
     return __any_sync(0xffffffffu, *abort_flag != 0);
 }
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes)
+__device__ __forceinline__ void bar_expect_tx(uint64_t *b, uint32_t bytes)
 {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%1], %0;" ::"r"(bytes), "r"(smem_u32(b))
                  : "memory");
 }
 
-__device__ __forceinline__ void cp_async_arrive(uint64_t *b)
+// Four rows (r0..r3) x 64 columns starting at column `col` of a 2-D bf16 tensor map
+// into 4 x 128 bytes of shared memory at dst, completing on mbarrier `bar`.
+__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap *tm, int col, int r0,
+                                            int r1, int r2, int r3, uint64_t *bar)
 {
-    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(b)) : "memory");
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(tm)), "r"(col), "r"(r0), "r"(r1), "r"(r2), "r"(r3),
+        "r"(smem_u32(bar))
+        : "memory");
 }
 
 __device__ __forceinline__ void fence_proxy_async()
@@ -250,68 +262,10 @@ __device__ __forceinline__ uint32_t sw_off(int r, int ch)
                       (((ch & 7) ^ (r & 7)) << 4));
 }
 
-// Expands the next n (<= 128) selected key indices of a mask row into idx[0..n).
-// Warp-cooperative; (wpos, rem) is the cursor: word index and its unconsumed bits.
-__device__ __forceinline__ void next_indices(const uint32_t *row, int nw, int N, int n, int &wpos,
-                                             uint32_t &rem, int *idx)
-{
-    const int lane = threadIdx.x & 31;
-    int count = 0;
-    while (count < n && wpos < nw) {
-        const int w = wpos + lane;
-        uint32_t bits = 0;
-        if (w < nw) {
-            bits = lane == 0 ? rem : row[w];
-            if (w == nw - 1 && (N & 31)) bits &= (1u << (N & 31)) - 1u;
-        }
-        const int pc = __popc(bits);
-        int incl = pc;
-        for (int o = 1; o < 32; o <<= 1) {
-            const int t = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += t;
-        }
-        const int excl = incl - pc;
-        const int total = __shfl_sync(0xffffffffu, incl, 31);
-        const int need = n - count;
-        // lane writes the first min(pc, need - excl) of its bits
-        int take = min(pc, max(0, need - excl));
-        uint32_t b = bits;
-        for (int k = 0; k < take; ++k) {
-            const int bit = __ffs(b) - 1;
-            b &= b - 1;
-            idx[count + excl + k] = w * 32 + bit;
-        }
-        if (total <= need) {
-            count += total;
-            wpos += 32;
-            rem = (wpos < nw) ? row[wpos] : 0u;
-        } else {
-            // the crossing lane keeps its unconsumed bits
-            const unsigned cross = __ballot_sync(0xffffffffu, excl < need && incl > need);
-            const unsigned full = __ballot_sync(0xffffffffu, incl == need && pc > 0);
-            int src;
-            uint32_t left;
-            if (cross) {
-                src = __ffs(cross) - 1;
-                left = __shfl_sync(0xffffffffu, b, src);
-            } else {
-                src = __ffs(full) - 1 + 1;   // next word starts fresh
-                left = 0xffffffffu;          // placeholder, replaced below
-            }
-            const int neww = wpos + src;
-            if (!cross) left = (neww < nw) ? row[neww] : 0u;
-            wpos = neww;
-            rem = left;
-            count = n;
-        }
-        __syncwarp();
-    }
-    // a mask row with fewer bits than requested (inconsistent input): pad with key 0
-    for (int k = count + lane; k < n; k += 32) idx[k] = 0;
-}
-
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a)
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, AttnArgs a)
 {
     using L = Smem<D>;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -326,11 +280,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a)
 
     if (threadIdx.x == 0) {
         misc[0] = 0;
-        bar_init(&bars->q_full, 32);
+        bar_init(&bars->q_full, 1);
         bar_init(&bars->q_empty, 1);
         for (int s = 0; s < kMaxStages; ++s) {
-            bar_init(&bars->k_full[s], 32);
-            bar_init(&bars->v_full[s], 32);
+            bar_init(&bars->k_full[s], 1);
+            bar_init(&bars->v_full[s], 1);
             bar_init(&bars->k_empty[s], 1);
             bar_init(&bars->v_empty[s], 1);
         }
@@ -359,56 +313,62 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a)
     if (warp == 4 || warp == 5) {
         // ------------------------------------------------------------ gather warps
         const bool is_k = warp == 4;
-        const __nv_bfloat16 *src = reinterpret_cast<const __nv_bfloat16 *>(is_k ? a.K : a.V);
-        const __nv_bfloat16 *Qp = reinterpret_cast<const __nv_bfloat16 *>(a.Q);
-        int *idx = reinterpret_cast<int *>(sm + L::kIdx) + (is_k ? 0 : kBN);
+        const CUtensorMap *tm = is_k ? &tmK : &tmV;
+        constexpr int NB = D / 64;                    // 64-column boxes per row
+        constexpr uint32_t kTileBytes = kBM * D * 2;
+        const int NS = is_k ? L::kKS : L::kVS;
         uint32_t stage_it = 0, q_it = 0;
-        constexpr int CH = D / 8;   // 16-byte chunks per row
         for (int it = blockIdx.x; it < n_items && !warp_aborted(abort_flag); it += gridDim.x) {
             const int4 item = a.items[it];
             const int bh = item.x, c = item.y, q0 = item.z, nq = item.w;
             const long long r = a.final_cnt[(size_t)bh * a.Cq + c];
             const int T = (int)((r + kBN - 1) / kBN);
-            const __nv_bfloat16 *base = src + (size_t)bh * a.N * D;
+            const int rowbase = bh * a.N;
             if (is_k) {
-                // Q tile: rows perm[q0 .. q0+nq), zero rows beyond nq
+                // Q tile: rows perm[q0 .. q0+nq); rows beyond nq repeat the first query
                 if (!warp_wait(&bars->q_empty, (q_it & 1) ^ 1, abort_flag, a.status)) break;
-                const int32_t *perm = a.perm + (size_t)bh * a.perm_bh;
-                const __nv_bfloat16 *qb = Qp + (size_t)bh * a.N * D;
-                for (int id = lane; id < kBM * CH; id += 32) {
-                    const int row = id / CH, ch = id - row * CH;
-                    const bool ok = row < nq;
-                    const int tok = ok ? perm[q0 + row] : 0;
-                    cp_async16(sbase + L::kQ + sw_off(row, ch), qb + (size_t)tok * D + ch * 8, ok ? 16 : 0);
-                }
-                cp_async_arrive(&bars->q_full);
+                if (lane == 0) bar_expect_tx(&bars->q_full, kTileBytes);
+                __syncwarp();
+                const int32_t *perm = a.perm + (size_t)bh * a.perm_bh + q0;
+                int g[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) g[k] = rowbase + perm[min(4 * lane + k, nq - 1)];
+#pragma unroll
+                for (int blk = 0; blk < NB; ++blk)
+                    tma_gather4(sbase + L::kQ + blk * (kBM * 128) + lane * 512, &tmQ, blk * 64, g[0], g[1],
+                                g[2], g[3], &bars->q_full);
                 ++q_it;
             }
-            const uint32_t *mrow = a.mask + ((size_t)bh * a.Cq + c) * a.nw;
-            int wpos = 0;
-            uint32_t rem = mrow[0];
-            const int NS = is_k ? L::kKS : L::kVS;
+            const int32_t *list = a.lists + ((size_t)bh * a.Cq + c) * a.list_stride;
             for (int t = 0; t < T; ++t) {
                 const int s = stage_it % NS;
                 if (!warp_wait(is_k ? &bars->k_empty[s] : &bars->v_empty[s], ((stage_it / NS) & 1) ^ 1,
                                abort_flag, a.status))
                     break;
-                const int nvalid = (int)min((long long)kBN, r - (long long)t * kBN);
-                next_indices(mrow, a.nw, a.N, nvalid, wpos, rem, idx);
+                uint64_t *full = is_k ? &bars->k_full[s] : &bars->v_full[s];
+                if (lane == 0) bar_expect_tx(full, kTileBytes);
                 __syncwarp();
-                const uint32_t dst0 = sbase + (is_k ? L::kK : L::kV) + s * L::kTile;
-                for (int id = lane; id < kBN * CH; id += 32) {
-                    const int row = id / CH, ch = id - row * CH;
-                    const bool ok = row < nvalid;
-                    const int key = ok ? idx[row] : 0;
-                    cp_async16(dst0 + sw_off(row, ch), base + (size_t)key * D + ch * 8, ok ? 16 : 0);
+                // this lane's four keys; keys past r_c (last tile) load key 0 and are masked
+                const long long j0 = (long long)t * kBN + 4 * lane;
+                int g[4];
+                if (j0 + 3 < r) {
+                    const int4 v = *reinterpret_cast<const int4 *>(list + j0);
+                    g[0] = v.x;
+                    g[1] = v.y;
+                    g[2] = v.z;
+                    g[3] = v.w;
+                } else {
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) g[k] = (j0 + k < r) ? list[j0 + k] : 0;
                 }
-                cp_async_arrive(is_k ? &bars->k_full[s] : &bars->v_full[s]);
-                __syncwarp();
+                const uint32_t dst0 = sbase + (is_k ? L::kK : L::kV) + s * L::kTile + lane * 512;
+#pragma unroll
+                for (int blk = 0; blk < NB; ++blk)
+                    tma_gather4(dst0 + blk * (kBM * 128), tm, blk * 64, rowbase + g[0], rowbase + g[1],
+                                rowbase + g[2], rowbase + g[3], full);
                 ++stage_it;
             }
         }
-        asm volatile("cp.async.wait_all;" ::: "memory");
     } else if (warp == 6) {
         // ------------------------------------------------------------ MMA issuer
         constexpr uint32_t idesc_qk = f16_idesc(kBM, kBN, false);
@@ -603,18 +563,54 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a)
 
 }  // namespace
 
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+// [rows, D] bf16 row-major; box = 64 columns x 1 row (tile::gather4), 128-byte swizzle.
+bool row_gather_map(CUtensorMap *m, const void *base, long long rows, int D)
+{
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+    cuuint32_t box[2] = {64, 1};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D>
+cudaError_t launch_tc(const AttnArgs &a, cudaStream_t s)
+{
+    CUtensorMap tq, tk, tv;
+    const long long rows = (long long)a.BH * a.N;
+    if (!row_gather_map(&tq, a.Q, rows, D) || !row_gather_map(&tk, a.K, rows, D) ||
+        !row_gather_map(&tv, a.V, rows, D))
+        return cudaErrorInvalidValue;
+    const int smem = Smem<D>::kAlloc;
+    cudaFuncSetAttribute(attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    attn_tc_kernel<D><<<a.num_sms, kThreads, smem, s>>>(tq, tk, tv, a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
 cudaError_t attention_tc_run(const AttnArgs &a, cudaStream_t s)
 {
-    if (a.d == 128) {
-        const int smem = Smem<128>::kAlloc;
-        cudaFuncSetAttribute(attn_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        attn_tc_kernel<128><<<a.num_sms, kThreads, smem, s>>>(a);
-    } else {
-        const int smem = Smem<64>::kAlloc;
-        cudaFuncSetAttribute(attn_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        attn_tc_kernel<64><<<a.num_sms, kThreads, smem, s>>>(a);
-    }
-    return cudaGetLastError();
+    return a.d == 128 ? launch_tc<128>(a, s) : launch_tc<64>(a, s);
 }
 
 }  // namespace scope

@@ -54,7 +54,7 @@ struct WsLayout {
     size_t cent32, cnorm, cnrm2, cslack, perm, off, chunk_hist;
     size_t q_cent, q_assign, q_sizes, k_cent, k_codes, k_sizes;
     size_t topp, base, khead, final_cnt, mask, sel_state;
-    size_t q_perm, q_off, q_hist, work_items, attn_counter;
+    size_t q_perm, q_off, q_hist, work_items, attn_counter, key_lists;
     size_t total;
 };
 
@@ -88,6 +88,8 @@ struct AttnArgs {
     const uint32_t *mask;     // [BH, Cq, nw]
     const int32_t *final_cnt; // [BH, Cq]
     int4 *items;              // work list (bh, c, q0, nq)
+    int32_t *lists;           // selected key indices of unit u at lists[u*list_stride ...], ascending
+    long long list_stride;    // N rounded up to a multiple of 4
     int32_t *counter;         // [2]: item count, dynamic scheduler
     int BH, N, d, Cq, nw, is_bf16;
     int use_tc;               // bf16 on the tensor cores (else CUDA cores)
