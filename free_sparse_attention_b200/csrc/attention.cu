@@ -15,7 +15,7 @@ cudaError_t attention_tc_run(const AttnArgs &a, cudaStream_t s);
 
 namespace {
 
-// Work list: one item per tile of kAttnTile queries of one (bh, cluster), head-major.
+// Work list: one item per kAttnTile queries of one (bh, cluster), head-major.
 // Single block; counter[0] = number of items, counter[1] = 0 (scheduler).
 __global__ void __launch_bounds__(1024) attn_items_kernel(AttnArgs a)
 {

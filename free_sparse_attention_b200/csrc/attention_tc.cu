@@ -30,10 +30,11 @@ namespace scope {
 
 namespace {
 
-constexpr int kBM = 128;           // queries per tile
-constexpr int kBN = 128;           // keys per tile
-constexpr int kMaxStages = 4;
-constexpr int kThreads = 224;      // 7 warps
+constexpr int kBM = 128;           // queries per Q tile (TMEM lanes)
+constexpr int kQT = 2;             // Q tiles per CTA, both against every gathered K/V tile
+constexpr int kBN = 64;            // keys per K/V tile
+constexpr int kThreads = 352;      // 11 warps
+constexpr int kMaxStages = 8;
 constexpr uint32_t kTmemCols = 512;
 constexpr unsigned long long kWaitNs = 4000000000ull;
 
@@ -41,27 +42,29 @@ struct __align__(8) Bars {
     uint64_t q_full, q_empty;
     uint64_t k_full[kMaxStages], k_empty[kMaxStages];
     uint64_t v_full[kMaxStages], v_empty[kMaxStages];
-    uint64_t s_full[2], s_empty[2];
-    uint64_t p_full, o_done, o_free;
+    uint64_t s_full[kQT][2], s_empty[kQT][2];
+    uint64_t p_full[kQT], o_done[kQT], o_free[kQT];
 };
 
-// K tiles are released right after Q K^T, V tiles after P V; K runs one stage deeper.
+// Shared memory: two Q tiles, K and V rings, one P tile per Q tile (all bf16, 128-byte
+// swizzled, K-major).  TMEM: S[q][b] (fp32, 64 columns each, double-buffered) at
+// columns q*128 + b*64, O[q] (fp32, D columns) at 256 + q*D.
 template <int D>
 struct Smem {
-    static constexpr int kKS = D == 128 ? 3 : 4;       // K ring depth
-    static constexpr int kVS = D == 128 ? 2 : 4;       // V ring depth
-    static constexpr int kTile = kBM * D * 2;          // bytes of a 128 x D bf16 tile
+    static constexpr int kStages = D == 128 ? 4 : 8;   // K ring and V ring depth
+    static constexpr int kQTile = kBM * D * 2;
+    static constexpr int kKVTile = kBN * D * 2;
+    static constexpr int kPTile = kBM * kBN * 2;
     static constexpr int kQ = 0;
-    static constexpr int kK = kQ + kTile;
-    static constexpr int kV = kK + kKS * kTile;
-    static constexpr int kP = kV + kVS * kTile;
-    static constexpr int kBars = kP + kBM * kBN * 2;
+    static constexpr int kK = kQ + kQT * kQTile;
+    static constexpr int kV = kK + kStages * kKVTile;
+    static constexpr int kP = kV + kStages * kKVTile;
+    static constexpr int kBars = kP + kQT * kPTile;
     static constexpr int kMisc = kBars + (int)sizeof(Bars);
     static constexpr int kBytes = kMisc + 64;
-    // room to align the base to 1 KB; at least 120 KB so that one CTA holds an SM (and
-    // its 512 TMEM columns) alone
-    static constexpr int kAlloc = (kBytes + 1024) > 122880 ? (kBytes + 1024) : 122880;
+    static constexpr int kAlloc = kBytes + 1024;       // room to align the base to 1 KB
     static_assert(kAlloc <= 232448, "shared memory budget");
+    static_assert(kAlloc > 232448 / 2, "one CTA (and its 512 TMEM columns) per SM");
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p)
@@ -255,10 +258,12 @@ __device__ __forceinline__ float fast_exp2(float x)
     return y;
 }
 
-// Byte offset of (row r, 16-byte chunk ch) in a 128B-swizzled K-major tile of kBM rows.
-__device__ __forceinline__ uint32_t sw_off(int r, int ch)
+
+// Byte offset of (row r, 16-byte chunk ch) in a 128B-swizzled K-major tile of `rows`
+// rows: 64-column blocks of rows x 128 bytes, 8-row atoms of 1024 bytes.
+__device__ __forceinline__ uint32_t sw_off(int rows, int r, int ch)
 {
-    return (uint32_t)((ch >> 3) * (kBM * 128) + (r >> 3) * 1024 + (r & 7) * 128 +
+    return (uint32_t)((ch >> 3) * (rows * 128) + (r >> 3) * 1024 + (r & 7) * 128 +
                       (((ch & 7) ^ (r & 7)) << 4));
 }
 
@@ -268,6 +273,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                    const __grid_constant__ CUtensorMap tmV, AttnArgs a)
 {
     using L = Smem<D>;
+    constexpr int NB = D / 64;     // 64-column boxes per row
+    constexpr int KS = L::kStages;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char *sm = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -288,16 +295,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             bar_init(&bars->k_empty[s], 1);
             bar_init(&bars->v_empty[s], 1);
         }
-        for (int b = 0; b < 2; ++b) {
-            bar_init(&bars->s_full[b], 1);
-            bar_init(&bars->s_empty[b], 4);
+        for (int q = 0; q < kQT; ++q) {
+            for (int b = 0; b < 2; ++b) {
+                bar_init(&bars->s_full[q][b], 1);
+                bar_init(&bars->s_empty[q][b], 4);
+            }
+            bar_init(&bars->p_full[q], 4);
+            bar_init(&bars->o_done[q], 1);
+            bar_init(&bars->o_free[q], 4);
         }
-        bar_init(&bars->p_full, 4);
-        bar_init(&bars->o_done, 1);
-        bar_init(&bars->o_free, 4);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    if (warp == 6) {
+    if (warp == 10) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                          smem_u32(tmem_slot)),
                      "r"(kTmemCols)
@@ -310,13 +319,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem = *tmem_slot;
     const int n_items = a.counter[0];
 
-    if (warp == 4 || warp == 5) {
+    if (warp == 8 || warp == 9) {
         // ------------------------------------------------------------ gather warps
-        const bool is_k = warp == 4;
+        const bool is_k = warp == 8;
         const CUtensorMap *tm = is_k ? &tmK : &tmV;
-        constexpr int NB = D / 64;                    // 64-column boxes per row
-        constexpr uint32_t kTileBytes = kBM * D * 2;
-        const int NS = is_k ? L::kKS : L::kVS;
+        constexpr uint32_t kTileBytes = kBN * D * 2;
+        const int grp = lane & 15, blk = lane >> 4;     // rows 4*grp..+3 of 64-column box blk
         uint32_t stage_it = 0, q_it = 0;
         for (int it = blockIdx.x; it < n_items && !warp_aborted(abort_flag); it += gridDim.x) {
             const int4 item = a.items[it];
@@ -325,214 +333,238 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int T = (int)((r + kBN - 1) / kBN);
             const int rowbase = bh * a.N;
             if (is_k) {
-                // Q tile: rows perm[q0 .. q0+nq); rows beyond nq repeat the first query
+                // both Q tiles: rows perm[q0 .. q0+nq); rows beyond nq repeat the last query
                 if (!warp_wait(&bars->q_empty, (q_it & 1) ^ 1, abort_flag, a.status)) break;
-                if (lane == 0) bar_expect_tx(&bars->q_full, kTileBytes);
+                if (lane == 0) bar_expect_tx(&bars->q_full, kQT * kBM * D * 2);
                 __syncwarp();
                 const int32_t *perm = a.perm + (size_t)bh * a.perm_bh + q0;
-                int g[4];
 #pragma unroll
-                for (int k = 0; k < 4; ++k) g[k] = rowbase + perm[min(4 * lane + k, nq - 1)];
+                for (int h = 0; h < 2; ++h) {
+                    const int g = lane + 32 * h;             // row group 0..63 over both tiles
+                    const int q = g >> 5, r0 = (g & 31) * 4;
+                    int rr[4];
 #pragma unroll
-                for (int blk = 0; blk < NB; ++blk)
-                    tma_gather4(sbase + L::kQ + blk * (kBM * 128) + lane * 512, &tmQ, blk * 64, g[0], g[1],
-                                g[2], g[3], &bars->q_full);
+                    for (int k = 0; k < 4; ++k) rr[k] = rowbase + perm[min(q * kBM + r0 + k, nq - 1)];
+#pragma unroll
+                    for (int b = 0; b < NB; ++b)
+                        tma_gather4(sbase + L::kQ + q * L::kQTile + b * (kBM * 128) + r0 * 128, &tmQ, b * 64,
+                                    rr[0], rr[1], rr[2], rr[3], &bars->q_full);
+                }
                 ++q_it;
             }
             const int32_t *list = a.lists + ((size_t)bh * a.Cq + c) * a.list_stride;
+            // this lane's four keys of tile t; keys past r_c (last tile) load key 0 and are
+            // masked by the softmax.  Indices are loaded two tiles ahead of their gathers.
+            auto keys_of = [&](int t) {
+                const long long j0 = (long long)t * kBN + 4 * grp;
+                int4 v;
+                if (j0 + 3 < r) {
+                    v = *reinterpret_cast<const int4 *>(list + j0);
+                } else {
+                    v.x = j0 < r ? list[j0] : 0;
+                    v.y = j0 + 1 < r ? list[j0 + 1] : 0;
+                    v.z = j0 + 2 < r ? list[j0 + 2] : 0;
+                    v.w = 0;
+                }
+                return v;
+            };
+            int4 g0 = keys_of(0), g1 = T > 1 ? keys_of(1) : make_int4(0, 0, 0, 0);
             for (int t = 0; t < T; ++t) {
-                const int s = stage_it % NS;
-                if (!warp_wait(is_k ? &bars->k_empty[s] : &bars->v_empty[s], ((stage_it / NS) & 1) ^ 1,
+                const int s = stage_it % KS;
+                if (!warp_wait(is_k ? &bars->k_empty[s] : &bars->v_empty[s], ((stage_it / KS) & 1) ^ 1,
                                abort_flag, a.status))
                     break;
                 uint64_t *full = is_k ? &bars->k_full[s] : &bars->v_full[s];
                 if (lane == 0) bar_expect_tx(full, kTileBytes);
                 __syncwarp();
-                // this lane's four keys; keys past r_c (last tile) load key 0 and are masked
-                const long long j0 = (long long)t * kBN + 4 * lane;
-                int g[4];
-                if (j0 + 3 < r) {
-                    const int4 v = *reinterpret_cast<const int4 *>(list + j0);
-                    g[0] = v.x;
-                    g[1] = v.y;
-                    g[2] = v.z;
-                    g[3] = v.w;
-                } else {
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) g[k] = (j0 + k < r) ? list[j0 + k] : 0;
-                }
-                const uint32_t dst0 = sbase + (is_k ? L::kK : L::kV) + s * L::kTile + lane * 512;
-#pragma unroll
-                for (int blk = 0; blk < NB; ++blk)
-                    tma_gather4(dst0 + blk * (kBM * 128), tm, blk * 64, rowbase + g[0], rowbase + g[1],
-                                rowbase + g[2], rowbase + g[3], full);
+                if (blk < NB)
+                    tma_gather4(sbase + (is_k ? L::kK : L::kV) + s * L::kKVTile + blk * (kBN * 128) + grp * 512,
+                                tm, blk * 64, rowbase + g0.x, rowbase + g0.y, rowbase + g0.z,
+                                rowbase + g0.w, full);
+                g0 = g1;
+                if (t + 2 < T) g1 = keys_of(t + 2);
                 ++stage_it;
             }
         }
-    } else if (warp == 6) {
+    } else if (warp == 10) {
         // ------------------------------------------------------------ MMA issuer
         constexpr uint32_t idesc_qk = f16_idesc(kBM, kBN, false);
         constexpr uint32_t idesc_pv = f16_idesc(kBM, D, true);
-        uint32_t k_it = 0, v_it = 0, q_it = 0, s_it = 0, p_it = 0, item_it = 0;
+        uint32_t k_it = 0, v_it = 0, q_it = 0;
+        uint32_t s_cnt[kQT] = {0, 0}, p_cnt[kQT] = {0, 0}, o_items[kQT] = {0, 0};
         const bool leader = lane == 0;
-        for (int it = blockIdx.x; it < n_items && !warp_aborted(abort_flag); it += gridDim.x, ++item_it) {
+        for (int it = blockIdx.x; it < n_items && !warp_aborted(abort_flag); it += gridDim.x) {
             const int4 item = a.items[it];
             const long long r = a.final_cnt[(size_t)item.x * a.Cq + item.y];
             const int T = (int)((r + kBN - 1) / kBN);
+            const int nqt = item.w > kBM ? 2 : 1;     // active Q tiles
             if (!warp_wait(&bars->q_full, q_it & 1, abort_flag, a.status)) break;
             ++q_it;
             bool ok = true;
             for (int t = 0; t <= T && ok; ++t) {
                 if (t < T) {
-                    const int s = k_it % L::kKS;
-                    const int b = (s_it) & 1;
-                    ok = warp_wait(&bars->k_full[s], (k_it / L::kKS) & 1, abort_flag, a.status) &&
-                         warp_wait(&bars->s_empty[b], ((s_it >> 1) & 1) ^ 1, abort_flag, a.status);
-                    if (!ok) break;
-                    fence_proxy_async();
-                    tc_fence_after();
-                    if (leader) {
-                        const uint32_t qa = sbase + L::kQ, ka = sbase + L::kK + s * L::kTile;
+                    const int s = k_it % KS;
+                    ok = warp_wait(&bars->k_full[s], (k_it / KS) & 1, abort_flag, a.status);
+                    for (int q = 0; q < nqt && ok; ++q) {
+                        const int b = s_cnt[q] & 1;
+                        ok = warp_wait(&bars->s_empty[q][b], ((s_cnt[q] >> 1) & 1) ^ 1, abort_flag, a.status);
+                        if (!ok) break;
+                        tc_fence_after();
+                        if (leader) {
+                            const uint32_t qa = sbase + L::kQ + q * L::kQTile, ka = sbase + L::kK + s * L::kKVTile;
 #pragma unroll
-                        for (int kk = 0; kk < D / 16; ++kk) {
-                            const uint32_t off = (kk >> 2) * (kBM * 128) + (kk & 3) * 32;
-                            mma_bf16(tmem + b * kBN, sw128_desc(qa + off, 16, 1024),
-                                     sw128_desc(ka + off, 16, 1024), idesc_qk, kk > 0);
+                            for (int kk = 0; kk < D / 16; ++kk)
+                                mma_bf16(tmem + q * 128 + b * kBN,
+                                         sw128_desc(qa + (kk >> 2) * (kBM * 128) + (kk & 3) * 32, 16, 1024),
+                                         sw128_desc(ka + (kk >> 2) * (kBN * 128) + (kk & 3) * 32, 16, 1024),
+                                         idesc_qk, kk > 0);
+                            mma_commit(&bars->s_full[q][b]);
                         }
-                        mma_commit(&bars->s_full[b]);
+                        __syncwarp();
+                        ++s_cnt[q];
+                    }
+                    if (!ok) break;
+                    if (leader) {
                         mma_commit(&bars->k_empty[s]);
                         if (t == T - 1) mma_commit(&bars->q_empty);
                     }
                     __syncwarp();
-                    ++s_it;
                     ++k_it;
                 }
                 if (t >= 1) {
-                    // O += P_{t-1} V_{t-1}
-                    const int tp = t - 1;
-                    const int s = v_it % L::kVS;
-                    ok = warp_wait(&bars->p_full, p_it & 1, abort_flag, a.status) &&
-                         warp_wait(&bars->v_full[s], (v_it / L::kVS) & 1, abort_flag, a.status);
-                    if (ok && tp == 0)
-                        ok = warp_wait(&bars->o_free, (item_it & 1) ^ 1, abort_flag, a.status);
-                    if (!ok) break;
-                    ++p_it;
-                    fence_proxy_async();
-                    tc_fence_after();
-                    if (leader) {
-                        const uint32_t pa = sbase + L::kP, va = sbase + L::kV + s * L::kTile;
+                    const int s = v_it % KS;
+                    ok = warp_wait(&bars->v_full[s], (v_it / KS) & 1, abort_flag, a.status);
+                    for (int q = 0; q < nqt && ok; ++q) {
+                        ok = warp_wait(&bars->p_full[q], p_cnt[q] & 1, abort_flag, a.status);
+                        if (ok && t == 1)
+                            ok = warp_wait(&bars->o_free[q], (o_items[q] & 1) ^ 1, abort_flag, a.status);
+                        if (!ok) break;
+                        ++p_cnt[q];
+                        fence_proxy_async();
+                        tc_fence_after();
+                        if (leader) {
+                            const uint32_t pa = sbase + L::kP + q * L::kPTile, va = sbase + L::kV + s * L::kKVTile;
 #pragma unroll
-                        for (int kk = 0; kk < kBN / 16; ++kk) {
-                            const uint32_t poff = (kk >> 2) * (kBM * 128) + (kk & 3) * 32;
-                            mma_bf16(tmem + 2 * kBN, sw128_desc(pa + poff, 16, 1024),
-                                     sw128_desc(va + kk * 2048, kBM * 128, 1024), idesc_pv,
-                                     (tp > 0 || kk > 0) ? 1u : 0u);
+                            for (int kk = 0; kk < kBN / 16; ++kk)
+                                mma_bf16(tmem + 256 + q * D, sw128_desc(pa + kk * 32, 16, 1024),
+                                         sw128_desc(va + kk * 2048, kBN * 128, 1024), idesc_pv,
+                                         (t > 1 || kk > 0) ? 1u : 0u);
+                            mma_commit(&bars->o_done[q]);
                         }
-                        mma_commit(&bars->o_done);
-                        mma_commit(&bars->v_empty[s]);
+                        __syncwarp();
                     }
+                    if (!ok) break;
+                    if (leader) mma_commit(&bars->v_empty[s]);
                     __syncwarp();
                     ++v_it;
                 }
             }
+            if (!ok) break;
+            for (int q = 0; q < nqt; ++q) ++o_items[q];
         }
-    } else if (warp < 4) {
+    } else if (warp < 8) {
         // ------------------------------------------------------------ softmax + epilogue
-        const int row = threadIdx.x;   // 0..127 = TMEM lane
-        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-        uint32_t s_it = 0, o_it = 0;
+        const int q = warp >> 2;                       // Q tile of this warpgroup
+        const int row = threadIdx.x - q * kBM;         // 0..127 = TMEM lane
+        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+        const uint32_t s_col = q * 128, o_col = 256 + q * D;
+        uint32_t s_cnt = 0, o_cnt = 0;
         const float c = a.scale_log2;
-        unsigned char *P = sm + L::kP;
+        unsigned char *P = sm + L::kP + q * L::kPTile;
         for (int it = blockIdx.x; it < n_items && !warp_aborted(abort_flag); it += gridDim.x) {
             const int4 item = a.items[it];
             const int bh = item.x, cl = item.y, q0 = item.z, nq = item.w;
+            if (q == 1 && nq <= kBM) continue;        // this Q tile is idle for the item
             const long long r = a.final_cnt[(size_t)bh * a.Cq + cl];
             const int T = (int)((r + kBN - 1) / kBN);
             float m_run = -INFINITY, l = 0.f;
             bool ok = true;
             for (int t = 0; t < T; ++t) {
-                const int b = s_it & 1;
-                ok = warp_wait(&bars->s_full[b], (s_it >> 1) & 1, abort_flag, a.status);
+                const int b = s_cnt & 1;
+                ok = warp_wait(&bars->s_full[q][b], (s_cnt >> 1) & 1, abort_flag, a.status);
                 if (!ok) break;
                 tc_fence_after();
                 float s[kBN];
 #pragma unroll
-                for (int q = 0; q < kBN / 32; ++q)
-                    tmem_ld32(tmem + lane_base + b * kBN + q * 32, s + q * 32);
+                for (int h = 0; h < kBN / 32; ++h) tmem_ld32(tmem + lane_base + s_col + b * kBN + h * 32, s + h * 32);
                 tmem_wait_ld();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) bar_arrive(&bars->s_empty[b]);
-                ++s_it;
+                if (lane == 0) bar_arrive(&bars->s_empty[q][b]);
+                ++s_cnt;
                 const int nvalid = (int)min((long long)kBN, r - (long long)t * kBN);
                 if (nvalid < kBN) {
 #pragma unroll
                     for (int j = 0; j < kBN; ++j)
                         if (j >= nvalid) s[j] = -INFINITY;
                 }
-                float mraw = -INFINITY;
+                float m8[8];
 #pragma unroll
-                for (int j = 0; j < kBN; ++j) mraw = fmaxf(mraw, s[j]);
-                const float mt = mraw * c;   // c > 0: the maximum of the scaled logits
-                // PV of the previous tile must be done: P buffer free, O stable
+                for (int k = 0; k < 8; ++k) m8[k] = s[k];
+#pragma unroll
+                for (int j = 8; j < kBN; ++j) m8[j & 7] = fmaxf(m8[j & 7], s[j]);
+                const float mt = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                                       fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) * c;
+                // the previous P V of this Q tile must be done: P buffer free, O stable
                 if (t > 0) {
-                    ok = warp_wait(&bars->o_done, o_it & 1, abort_flag, a.status);
+                    ok = warp_wait(&bars->o_done[q], o_cnt & 1, abort_flag, a.status);
                     if (!ok) break;
-                    ++o_it;
+                    ++o_cnt;
                     tc_fence_after();
                 }
                 const bool need = mt > m_run + 8.f;
                 if (t > 0 && __any_sync(0xffffffffu, need)) {
                     const float alpha = need ? fast_exp2(m_run - mt) : 1.f;
 #pragma unroll 1
-                    for (int q = 0; q < D / 32; ++q) {
+                    for (int h = 0; h < D / 32; ++h) {
                         float o[32];
-                        tmem_ld32(tmem + lane_base + 2 * kBN + q * 32, o);
+                        tmem_ld32(tmem + lane_base + o_col + h * 32, o);
                         tmem_wait_ld();
 #pragma unroll
                         for (int e = 0; e < 32; ++e) o[e] *= alpha;
-                        tmem_st32(tmem + lane_base + 2 * kBN + q * 32, o);
+                        tmem_st32(tmem + lane_base + o_col + h * 32, o);
                     }
                     tmem_wait_st();
                     if (need) l *= alpha;
                 }
                 if (need) m_run = mt;
-                float ls = 0.f;
+                float ls[4] = {0.f, 0.f, 0.f, 0.f};
+                const float nm = -m_run;
 #pragma unroll
                 for (int j = 0; j < kBN; j += 8) {
                     uint32_t pk[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const float p0 = fast_exp2(fmaf(s[j + 2 * e], c, -m_run));
-                        const float p1 = fast_exp2(fmaf(s[j + 2 * e + 1], c, -m_run));
-                        ls += p0 + p1;
-                        __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
-                        pk[e] = *reinterpret_cast<uint32_t *>(&h);
+                        const float p0 = fast_exp2(fmaf(s[j + 2 * e], c, nm));
+                        const float p1 = fast_exp2(fmaf(s[j + 2 * e + 1], c, nm));
+                        ls[e] += p0 + p1;
+                        __nv_bfloat162 hh = __floats2bfloat162_rn(p0, p1);
+                        pk[e] = *reinterpret_cast<uint32_t *>(&hh);
                     }
-                    *reinterpret_cast<uint4 *>(P + sw_off(row, j >> 3)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                    *reinterpret_cast<uint4 *>(P + sw_off(kBM, row, j >> 3)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
                 }
-                l += ls;
+                l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
                 fence_proxy_async();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) bar_arrive(&bars->p_full);
+                if (lane == 0) bar_arrive(&bars->p_full[q]);
             }
             if (!ok) break;
-            // epilogue: O / l for the valid rows
-            if (!warp_wait(&bars->o_done, o_it & 1, abort_flag, a.status)) break;
-            ++o_it;
+            // epilogue: O / l for the valid rows of this Q tile
+            if (!warp_wait(&bars->o_done[q], o_cnt & 1, abort_flag, a.status)) break;
+            ++o_cnt;
             tc_fence_after();
             const float inv = l > 0.f ? 1.f / l : 0.f;
-            const bool valid = row < nq;
+            const bool valid = q * kBM + row < nq;
             __nv_bfloat16 *dst = nullptr;
             if (valid) {
-                const int tok = a.perm[(size_t)bh * a.perm_bh + q0 + row];
+                const int tok = a.perm[(size_t)bh * a.perm_bh + q0 + q * kBM + row];
                 dst = reinterpret_cast<__nv_bfloat16 *>(a.O) + ((size_t)bh * a.N + tok) * D;
             }
 #pragma unroll 1
-            for (int q = 0; q < D / 32; ++q) {
+            for (int h = 0; h < D / 32; ++h) {
                 float o[32];
-                tmem_ld32(tmem + lane_base + 2 * kBN + q * 32, o);
+                tmem_ld32(tmem + lane_base + o_col + h * 32, o);
                 tmem_wait_ld();
                 if (valid) {
 #pragma unroll
@@ -540,23 +572,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                         uint32_t pk[4];
 #pragma unroll
                         for (int k = 0; k < 4; ++k) {
-                            __nv_bfloat162 h = __floats2bfloat162_rn(o[e + 2 * k] * inv, o[e + 2 * k + 1] * inv);
-                            pk[k] = *reinterpret_cast<uint32_t *>(&h);
+                            __nv_bfloat162 hh = __floats2bfloat162_rn(o[e + 2 * k] * inv, o[e + 2 * k + 1] * inv);
+                            pk[k] = *reinterpret_cast<uint32_t *>(&hh);
                         }
-                        *reinterpret_cast<uint4 *>(dst + q * 32 + e) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                        *reinterpret_cast<uint4 *>(dst + h * 32 + e) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
                     }
                 }
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) bar_arrive(&bars->o_free);
+            if (lane == 0) bar_arrive(&bars->o_free[q]);
         }
     }
     // drain and free TMEM
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 6)
+    if (warp == 10)
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
                      : "memory");
 }

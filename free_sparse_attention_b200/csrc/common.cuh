@@ -11,7 +11,7 @@ namespace scope {
 
 constexpr int kMaxC = 2048;         // max centroids per problem (LUT and histogram sizes)
 constexpr int kSortChunk = 512;     // tokens per warp in the stable counting sort
-constexpr int kAttnTile = 128;      // queries per attention tile
+constexpr int kAttnTile = 256;      // queries per attention work item (two 128-row tiles)
 
 // ---------------------------------------------------------------------------------
 // Clustering problems.  Role 0 = queries (all d channels, C = Cq); roles 1..3 = the
