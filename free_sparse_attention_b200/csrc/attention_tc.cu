@@ -3,24 +3,28 @@
 // SCOPE computes exact softmax attention of every query over the ORIGINAL keys and
 // values its query cluster selected (arXiv 2608.12780, abstract;
 // review page, forward_implications[1]).  Queries are grouped by cluster, so one work
-// item = up to 128 queries of one (b, h, c) against the r_c keys of S_c.
+// item = up to 256 queries of one (b, h, c) against the r_c keys of S_c.
 //
 // Per CTA (persistent, one per SM, static round-robin over the head-major work list):
-//   warps 0-3  softmax + epilogue: thread r owns query row r = TMEM lane r
-//   warp 4     gathers the Q tile once per item and the selected K rows per key tile
-//   warp 5     gathers the selected V rows per key tile
-//   warp 6     allocates TMEM and issues the MMAs (one elected thread)
+//   warps 0-3 / 4-7  softmax + epilogue of Q tile 0 / 1 (thread r owns row r = TMEM lane r)
+//   warp 8           gathers both Q tiles once per item and the selected K rows per key tile
+//   warp 9           gathers the selected V rows per key tile
+//   warp 10          allocates TMEM and issues the MMAs (one elected thread)
 // Each cluster's selected key indices are expanded once from the bitmask into an
 // ascending list (attn_lists_kernel).  Rows are gathered with TMA tile::gather4 (four
 // arbitrary rows of one 64-column, 128-byte box per instruction, each lane issuing its
-// own four rows) straight into the 128B-swizzled K-major layout the tensor core reads;
-// K tiles run three stages deep, V tiles two.
-//   S_b = Q K^T   tcgen05.mma kind::f16, M=128, N=128, K=d, fp32 in TMEM (2 buffers)
-//   O  += P V     M=128, N=d, K=128, P bf16 in shared memory, O fp32 in TMEM
-// The softmax keeps a running row maximum and rescales O (TMEM load/store) only when
-// the maximum grows by more than 2^8, so P stays <= 256 and the final O / l is exact
-// softmax arithmetic.  Every mbarrier wait gives up after ~4 s, sets a status bit and
-// lets the CTA drain and free its TMEM.
+// own four rows) straight into the 128B-swizzled K-major layout the tensor core reads.
+//   S_q  = Q_q K^T     tcgen05.mma kind::f16, M=128, N=128, K=d, fp32 in TMEM
+//   O_q += P_q V       M=128, N=d, K=128, P_q bf16 written by the softmax over its own
+//                      S_q columns in TMEM (A operand from TMEM), V from shared memory
+// Both Q tiles reuse every gathered K/V tile.  The MMA warp issues in ping-pong order
+// PV_0(t), QK_0(t+1), PV_1(t), QK_1(t+1), so the tensor core works on one Q tile while
+// the other tile's softmax runs; in-order execution of the tensor pipe keeps QK_q(t+1)
+// from overwriting P_q(t) before PV_q(t) has read it.  The softmax keeps a running row
+// maximum and rescales O (TMEM load/store) only when the maximum grows by more than
+// 2^8, so P stays <= 256 and the final O / l is exact softmax arithmetic.  Every
+// mbarrier wait gives up after ~4 s, sets a status bit and lets the CTA drain and free
+// its TMEM.
 #include "common.cuh"
 
 #include <cuda.h>
@@ -32,9 +36,9 @@ namespace {
 
 constexpr int kBM = 128;           // queries per Q tile (TMEM lanes)
 constexpr int kQT = 2;             // Q tiles per CTA, both against every gathered K/V tile
-constexpr int kBN = 64;            // keys per K/V tile
+constexpr int kBN = 128;           // keys per K/V tile
 constexpr int kThreads = 352;      // 11 warps
-constexpr int kMaxStages = 8;
+constexpr int kMaxStages = 6;
 constexpr uint32_t kTmemCols = 512;
 constexpr unsigned long long kWaitNs = 4000000000ull;
 
@@ -42,24 +46,22 @@ struct __align__(8) Bars {
     uint64_t q_full, q_empty;
     uint64_t k_full[kMaxStages], k_empty[kMaxStages];
     uint64_t v_full[kMaxStages], v_empty[kMaxStages];
-    uint64_t s_full[kQT][2], s_empty[kQT][2];
-    uint64_t p_full[kQT], o_done[kQT], o_free[kQT];
+    uint64_t s_full[kQT], p_full[kQT], o_done[kQT], o_free[kQT];
 };
 
-// Shared memory: two Q tiles, K and V rings, one P tile per Q tile (all bf16, 128-byte
-// swizzled, K-major).  TMEM: S[q][b] (fp32, 64 columns each, double-buffered) at
-// columns q*128 + b*64, O[q] (fp32, D columns) at 256 + q*D.
+// Shared memory: two Q tiles, a K ring and a V ring (bf16, 128-byte swizzled, K-major).
+// TMEM: S_q (fp32, 128 columns; P_q bf16 pairs over its first 64) at q*128, O_q (fp32,
+// D columns) at 256 + q*D.
 template <int D>
 struct Smem {
-    static constexpr int kStages = D == 128 ? 4 : 8;   // K ring and V ring depth
+    static constexpr int kKS = D == 128 ? 3 : 6;       // K ring depth
+    static constexpr int kVS = D == 128 ? 2 : 6;       // V ring depth
     static constexpr int kQTile = kBM * D * 2;
     static constexpr int kKVTile = kBN * D * 2;
-    static constexpr int kPTile = kBM * kBN * 2;
     static constexpr int kQ = 0;
     static constexpr int kK = kQ + kQT * kQTile;
-    static constexpr int kV = kK + kStages * kKVTile;
-    static constexpr int kP = kV + kStages * kKVTile;
-    static constexpr int kBars = kP + kQT * kPTile;
+    static constexpr int kV = kK + kKS * kKVTile;
+    static constexpr int kBars = kV + kVS * kKVTile;
     static constexpr int kMisc = kBars + (int)sizeof(Bars);
     static constexpr int kBytes = kMisc + 64;
     static constexpr int kAlloc = kBytes + 1024;       // room to align the base to 1 KB
@@ -259,12 +261,28 @@ __device__ __forceinline__ float fast_exp2(float x)
 }
 
 
-// Byte offset of (row r, 16-byte chunk ch) in a 128B-swizzled K-major tile of `rows`
-// rows: 64-column blocks of rows x 128 bytes, 8-row atoms of 1024 bytes.
-__device__ __forceinline__ uint32_t sw_off(int rows, int r, int ch)
+
+// A operand from TMEM (P), B from shared memory (V).
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc,
+                                            uint32_t accumulate)
 {
-    return (uint32_t)((ch >> 3) * (rows * 128) + (r >> 3) * 1024 + (r & 7) * 128 +
-                      (((ch & 7) ^ (r & 7)) << 4));
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%5, %5, %5, %5}, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b), "r"(idesc), "r"(accumulate), "r"(0u)
+        : "memory");
+}
+
+// 16 consecutive 32-bit columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16])
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+        "%11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+        "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+        : "memory");
 }
 
 template <int D>
@@ -274,7 +292,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 {
     using L = Smem<D>;
     constexpr int NB = D / 64;     // 64-column boxes per row
-    constexpr int KS = L::kStages;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char *sm = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -296,10 +313,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             bar_init(&bars->v_empty[s], 1);
         }
         for (int q = 0; q < kQT; ++q) {
-            for (int b = 0; b < 2; ++b) {
-                bar_init(&bars->s_full[q][b], 1);
-                bar_init(&bars->s_empty[q][b], 4);
-            }
+            bar_init(&bars->s_full[q], 1);
             bar_init(&bars->p_full[q], 4);
             bar_init(&bars->o_done[q], 1);
             bar_init(&bars->o_free[q], 4);
@@ -324,7 +338,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool is_k = warp == 8;
         const CUtensorMap *tm = is_k ? &tmK : &tmV;
         constexpr uint32_t kTileBytes = kBN * D * 2;
-        const int grp = lane & 15, blk = lane >> 4;     // rows 4*grp..+3 of 64-column box blk
+        const int NS = is_k ? L::kKS : L::kVS;
         uint32_t stage_it = 0, q_it = 0;
         for (int it = blockIdx.x; it < n_items && !warp_aborted(abort_flag); it += gridDim.x) {
             const int4 item = a.items[it];
@@ -339,16 +353,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __syncwarp();
                 const int32_t *perm = a.perm + (size_t)bh * a.perm_bh + q0;
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int g = lane + 32 * h;             // row group 0..63 over both tiles
-                    const int q = g >> 5, r0 = (g & 31) * 4;
+                for (int q = 0; q < kQT; ++q) {
                     int rr[4];
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) rr[k] = rowbase + perm[min(q * kBM + r0 + k, nq - 1)];
+                    for (int k = 0; k < 4; ++k) rr[k] = rowbase + perm[min(q * kBM + 4 * lane + k, nq - 1)];
 #pragma unroll
                     for (int b = 0; b < NB; ++b)
-                        tma_gather4(sbase + L::kQ + q * L::kQTile + b * (kBM * 128) + r0 * 128, &tmQ, b * 64,
-                                    rr[0], rr[1], rr[2], rr[3], &bars->q_full);
+                        tma_gather4(sbase + L::kQ + q * L::kQTile + b * (kBM * 128) + lane * 512, &tmQ,
+                                    b * 64, rr[0], rr[1], rr[2], rr[3], &bars->q_full);
                 }
                 ++q_it;
             }
@@ -356,7 +368,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // this lane's four keys of tile t; keys past r_c (last tile) load key 0 and are
             // masked by the softmax.  Indices are loaded two tiles ahead of their gathers.
             auto keys_of = [&](int t) {
-                const long long j0 = (long long)t * kBN + 4 * grp;
+                const long long j0 = (long long)t * kBN + 4 * lane;
                 int4 v;
                 if (j0 + 3 < r) {
                     v = *reinterpret_cast<const int4 *>(list + j0);
@@ -370,17 +382,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             };
             int4 g0 = keys_of(0), g1 = T > 1 ? keys_of(1) : make_int4(0, 0, 0, 0);
             for (int t = 0; t < T; ++t) {
-                const int s = stage_it % KS;
-                if (!warp_wait(is_k ? &bars->k_empty[s] : &bars->v_empty[s], ((stage_it / KS) & 1) ^ 1,
+                const int s = stage_it % NS;
+                if (!warp_wait(is_k ? &bars->k_empty[s] : &bars->v_empty[s], ((stage_it / NS) & 1) ^ 1,
                                abort_flag, a.status))
                     break;
                 uint64_t *full = is_k ? &bars->k_full[s] : &bars->v_full[s];
                 if (lane == 0) bar_expect_tx(full, kTileBytes);
                 __syncwarp();
-                if (blk < NB)
-                    tma_gather4(sbase + (is_k ? L::kK : L::kV) + s * L::kKVTile + blk * (kBN * 128) + grp * 512,
-                                tm, blk * 64, rowbase + g0.x, rowbase + g0.y, rowbase + g0.z,
-                                rowbase + g0.w, full);
+                const uint32_t dst0 = sbase + (is_k ? L::kK : L::kV) + s * L::kKVTile + lane * 512;
+#pragma unroll
+                for (int b = 0; b < NB; ++b)
+                    tma_gather4(dst0 + b * (kBN * 128), tm, b * 64, rowbase + g0.x, rowbase + g0.y,
+                                rowbase + g0.z, rowbase + g0.w, full);
                 g0 = g1;
                 if (t + 2 < T) g1 = keys_of(t + 2);
                 ++stage_it;
@@ -391,8 +404,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         constexpr uint32_t idesc_qk = f16_idesc(kBM, kBN, false);
         constexpr uint32_t idesc_pv = f16_idesc(kBM, D, true);
         uint32_t k_it = 0, v_it = 0, q_it = 0;
-        uint32_t s_cnt[kQT] = {0, 0}, p_cnt[kQT] = {0, 0}, o_items[kQT] = {0, 0};
+        uint32_t p_cnt[kQT] = {0, 0}, o_items[kQT] = {0, 0};
         const bool leader = lane == 0;
+        auto issue_qk = [&](int q, int ks) {
+            if (leader) {
+                const uint32_t qa = sbase + L::kQ + q * L::kQTile, ka = sbase + L::kK + ks * L::kKVTile;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * (kBM * 128) + (kk & 3) * 32;
+                    mma_bf16(tmem + q * 128, sw128_desc(qa + off, 16, 1024), sw128_desc(ka + off, 16, 1024),
+                             idesc_qk, kk > 0);
+                }
+                mma_commit(&bars->s_full[q]);
+            }
+            __syncwarp();
+        };
         for (int it = blockIdx.x; it < n_items && !warp_aborted(abort_flag); it += gridDim.x) {
             const int4 item = a.items[it];
             const long long r = a.final_cnt[(size_t)item.x * a.Cq + item.y];
@@ -400,67 +426,71 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int nqt = item.w > kBM ? 2 : 1;     // active Q tiles
             if (!warp_wait(&bars->q_full, q_it & 1, abort_flag, a.status)) break;
             ++q_it;
+            // prologue: S_q(0) = Q_q K(0)^T
+            int ks = k_it % L::kKS;
+            if (!warp_wait(&bars->k_full[ks], (k_it / L::kKS) & 1, abort_flag, a.status)) break;
+            tc_fence_after();
+#pragma unroll
+            for (int q = 0; q < kQT; ++q)
+                if (q < nqt) issue_qk(q, ks);
+            if (leader) {
+                mma_commit(&bars->k_empty[ks]);
+                if (T == 1) mma_commit(&bars->q_empty);
+            }
+            __syncwarp();
+            ++k_it;
             bool ok = true;
-            for (int t = 0; t <= T && ok; ++t) {
-                if (t < T) {
-                    const int s = k_it % KS;
-                    ok = warp_wait(&bars->k_full[s], (k_it / KS) & 1, abort_flag, a.status);
-                    for (int q = 0; q < nqt && ok; ++q) {
-                        const int b = s_cnt[q] & 1;
-                        ok = warp_wait(&bars->s_empty[q][b], ((s_cnt[q] >> 1) & 1) ^ 1, abort_flag, a.status);
-                        if (!ok) break;
-                        tc_fence_after();
-                        if (leader) {
-                            const uint32_t qa = sbase + L::kQ + q * L::kQTile, ka = sbase + L::kK + s * L::kKVTile;
+            for (int t = 0; t < T && ok; ++t) {
+                const int vs = v_it % L::kVS;
+                ok = warp_wait(&bars->v_full[vs], (v_it / L::kVS) & 1, abort_flag, a.status);
+                const bool more = t + 1 < T;
+                ks = k_it % L::kKS;
 #pragma unroll
-                            for (int kk = 0; kk < D / 16; ++kk)
-                                mma_bf16(tmem + q * 128 + b * kBN,
-                                         sw128_desc(qa + (kk >> 2) * (kBM * 128) + (kk & 3) * 32, 16, 1024),
-                                         sw128_desc(ka + (kk >> 2) * (kBN * 128) + (kk & 3) * 32, 16, 1024),
-                                         idesc_qk, kk > 0);
-                            mma_commit(&bars->s_full[q][b]);
-                        }
-                        __syncwarp();
-                        ++s_cnt[q];
-                    }
+                for (int q = 0; q < kQT; ++q) {
+                    if (q >= nqt || !ok) break;
+                    ok = warp_wait(&bars->p_full[q], p_cnt[q] & 1, abort_flag, a.status);
+                    if (ok && t == 0)
+                        ok = warp_wait(&bars->o_free[q], (o_items[q] & 1) ^ 1, abort_flag, a.status);
                     if (!ok) break;
+                    ++p_cnt[q];
+                    tc_fence_after();
+                    // O_q += P_q(t) V(t), P_q from TMEM (columns q*128 + [0, 64))
                     if (leader) {
-                        mma_commit(&bars->k_empty[s]);
-                        if (t == T - 1) mma_commit(&bars->q_empty);
-                    }
-                    __syncwarp();
-                    ++k_it;
-                }
-                if (t >= 1) {
-                    const int s = v_it % KS;
-                    ok = warp_wait(&bars->v_full[s], (v_it / KS) & 1, abort_flag, a.status);
-                    for (int q = 0; q < nqt && ok; ++q) {
-                        ok = warp_wait(&bars->p_full[q], p_cnt[q] & 1, abort_flag, a.status);
-                        if (ok && t == 1)
-                            ok = warp_wait(&bars->o_free[q], (o_items[q] & 1) ^ 1, abort_flag, a.status);
-                        if (!ok) break;
-                        ++p_cnt[q];
-                        fence_proxy_async();
-                        tc_fence_after();
-                        if (leader) {
-                            const uint32_t pa = sbase + L::kP + q * L::kPTile, va = sbase + L::kV + s * L::kKVTile;
+                        const uint32_t va = sbase + L::kV + vs * L::kKVTile;
 #pragma unroll
-                            for (int kk = 0; kk < kBN / 16; ++kk)
-                                mma_bf16(tmem + 256 + q * D, sw128_desc(pa + kk * 32, 16, 1024),
-                                         sw128_desc(va + kk * 2048, kBN * 128, 1024), idesc_pv,
-                                         (t > 1 || kk > 0) ? 1u : 0u);
-                            mma_commit(&bars->o_done[q]);
-                        }
-                        __syncwarp();
+                        for (int kk = 0; kk < kBN / 16; ++kk)
+                            mma_bf16_ts(tmem + 256 + q * D, tmem + q * 128 + kk * 8,
+                                        sw128_desc(va + kk * 2048, kBN * 128, 1024), idesc_pv,
+                                        (t > 0 || kk > 0) ? 1u : 0u);
+                        mma_commit(&bars->o_done[q]);
                     }
-                    if (!ok) break;
-                    if (leader) mma_commit(&bars->v_empty[s]);
                     __syncwarp();
-                    ++v_it;
+                    // S_q(t+1) = Q_q K(t+1)^T, issued after PV_q(t) has read P_q(t)
+                    if (more) {
+                        if (q == 0) {
+                            ok = warp_wait(&bars->k_full[ks], (k_it / L::kKS) & 1, abort_flag, a.status);
+                            if (!ok) break;
+                            tc_fence_after();
+                        }
+                        issue_qk(q, ks);
+                    }
                 }
+                if (!ok) break;
+                if (leader) {
+                    mma_commit(&bars->v_empty[vs]);
+                    if (more) {
+                        mma_commit(&bars->k_empty[ks]);
+                        if (t + 2 == T) mma_commit(&bars->q_empty);
+                    }
+                }
+                __syncwarp();
+                ++v_it;
+                if (more) ++k_it;
             }
             if (!ok) break;
-            for (int q = 0; q < nqt; ++q) ++o_items[q];
+#pragma unroll
+            for (int q = 0; q < kQT; ++q)
+                if (q < nqt) ++o_items[q];
         }
     } else if (warp < 8) {
         // ------------------------------------------------------------ softmax + epilogue
@@ -470,7 +500,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t s_col = q * 128, o_col = 256 + q * D;
         uint32_t s_cnt = 0, o_cnt = 0;
         const float c = a.scale_log2;
-        unsigned char *P = sm + L::kP + q * L::kPTile;
         for (int it = blockIdx.x; it < n_items && !warp_aborted(abort_flag); it += gridDim.x) {
             const int4 item = a.items[it];
             const int bh = item.x, cl = item.y, q0 = item.z, nq = item.w;
@@ -480,18 +509,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             float m_run = -INFINITY, l = 0.f;
             bool ok = true;
             for (int t = 0; t < T; ++t) {
-                const int b = s_cnt & 1;
-                ok = warp_wait(&bars->s_full[q][b], (s_cnt >> 1) & 1, abort_flag, a.status);
+                ok = warp_wait(&bars->s_full[q], s_cnt & 1, abort_flag, a.status);
                 if (!ok) break;
+                ++s_cnt;
                 tc_fence_after();
                 float s[kBN];
 #pragma unroll
-                for (int h = 0; h < kBN / 32; ++h) tmem_ld32(tmem + lane_base + s_col + b * kBN + h * 32, s + h * 32);
+                for (int h = 0; h < kBN / 32; ++h) tmem_ld32(tmem + lane_base + s_col + h * 32, s + h * 32);
                 tmem_wait_ld();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) bar_arrive(&bars->s_empty[q][b]);
-                ++s_cnt;
                 const int nvalid = (int)min((long long)kBN, r - (long long)t * kBN);
                 if (nvalid < kBN) {
 #pragma unroll
@@ -505,7 +530,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int j = 8; j < kBN; ++j) m8[j & 7] = fmaxf(m8[j & 7], s[j]);
                 const float mt = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
                                        fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) * c;
-                // the previous P V of this Q tile must be done: P buffer free, O stable
+                // P V of the previous tile is complete (it preceded Q K^T of this one)
                 if (t > 0) {
                     ok = warp_wait(&bars->o_done[q], o_cnt & 1, abort_flag, a.status);
                     if (!ok) break;
@@ -524,27 +549,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                         for (int e = 0; e < 32; ++e) o[e] *= alpha;
                         tmem_st32(tmem + lane_base + o_col + h * 32, o);
                     }
-                    tmem_wait_st();
                     if (need) l *= alpha;
                 }
                 if (need) m_run = mt;
+                // P = 2^(s*c - m) as bf16 pairs over the first 64 columns of S_q
                 float ls[4] = {0.f, 0.f, 0.f, 0.f};
                 const float nm = -m_run;
 #pragma unroll
-                for (int j = 0; j < kBN; j += 8) {
-                    uint32_t pk[4];
+                for (int h = 0; h < kBN / 32; ++h) {
+                    uint32_t pk[16];
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float p0 = fast_exp2(fmaf(s[j + 2 * e], c, nm));
-                        const float p1 = fast_exp2(fmaf(s[j + 2 * e + 1], c, nm));
-                        ls[e] += p0 + p1;
+                    for (int e = 0; e < 16; ++e) {
+                        const float p0 = fast_exp2(fmaf(s[h * 32 + 2 * e], c, nm));
+                        const float p1 = fast_exp2(fmaf(s[h * 32 + 2 * e + 1], c, nm));
+                        ls[e & 3] += p0 + p1;
                         __nv_bfloat162 hh = __floats2bfloat162_rn(p0, p1);
                         pk[e] = *reinterpret_cast<uint32_t *>(&hh);
                     }
-                    *reinterpret_cast<uint4 *>(P + sw_off(kBM, row, j >> 3)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                    tmem_st16(tmem + lane_base + s_col + h * 16, pk);
                 }
                 l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
-                fence_proxy_async();
+                tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) bar_arrive(&bars->p_full[q]);
