@@ -7,9 +7,13 @@
 //
 // Per CTA (persistent, one per SM, static round-robin over the head-major work list):
 //   warps 0-3 / 4-7  softmax + epilogue of Q tile 0 / 1 (thread r owns row r = TMEM lane r)
-//   warp 8           gathers both Q tiles once per item and the selected K rows per key tile
-//   warp 9           gathers the selected V rows per key tile
-//   warp 10          allocates TMEM and issues the MMAs (one elected thread)
+//   warps 8-11       gather both Q tiles once per item and the selected K rows per key tile
+//   warps 12-14      gather the selected V rows per key tile
+//   warp 15          allocates TMEM and issues the MMAs (one elected thread)
+// A TMA gather4 stream sustains ~15 GB/s per issuing warp, so each tile is split over
+// four (K) or three (V) warps; every warp signals its own share with arrive.expect_tx.
+// Registers are rebalanced per warpgroup with setmaxnreg: the softmax warpgroups hold a
+// whole 128-column row of logits (192 registers), the gather / MMA warpgroups need 64.
 // Each cluster's selected key indices are expanded once from the bitmask into an
 // ascending list (attn_lists_kernel).  Rows are gathered with TMA tile::gather4 (four
 // arbitrary rows of one 64-column, 128-byte box per instruction, each lane issuing its
@@ -37,7 +41,12 @@ namespace {
 constexpr int kBM = 128;           // queries per Q tile (TMEM lanes)
 constexpr int kQT = 2;             // Q tiles per CTA, both against every gathered K/V tile
 constexpr int kBN = 128;           // keys per K/V tile
-constexpr int kThreads = 352;      // 11 warps
+constexpr int kThreads = 512;      // 16 warps = 4 warpgroups
+constexpr int kKWarps = 4;         // K (and Q) gather warps
+constexpr int kVWarps = 3;         // V gather warps
+constexpr int kLaunchRegs = 128;   // 65536 / 512; the setmaxnreg split below sums to it
+constexpr int kSoftmaxRegs = 192;  // 2 warpgroups x 128 threads x 192
+constexpr int kOtherRegs = 64;     //  + 2 warpgroups x 128 threads x 64 = 65536
 constexpr int kMaxStages = 6;
 constexpr uint32_t kTmemCols = 512;
 constexpr unsigned long long kWaitNs = 4000000000ull;
@@ -304,11 +313,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (threadIdx.x == 0) {
         misc[0] = 0;
-        bar_init(&bars->q_full, 1);
+        bar_init(&bars->q_full, kKWarps);
         bar_init(&bars->q_empty, 1);
         for (int s = 0; s < kMaxStages; ++s) {
-            bar_init(&bars->k_full[s], 1);
-            bar_init(&bars->v_full[s], 1);
+            bar_init(&bars->k_full[s], kKWarps);
+            bar_init(&bars->v_full[s], kVWarps);
             bar_init(&bars->k_empty[s], 1);
             bar_init(&bars->v_empty[s], 1);
         }
@@ -320,7 +329,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    if (warp == 10) {
+    if (warp == 15) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                          smem_u32(tmem_slot)),
                      "r"(kTmemCols)
@@ -333,12 +342,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem = *tmem_slot;
     const int n_items = a.counter[0];
 
-    if (warp == 8 || warp == 9) {
+    if (warp >= 8) {
+    // warpgroups 2 and 3 give registers back (one setmaxnreg site for all their warps)
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kOtherRegs));
+    if (warp < 15) {
         // ------------------------------------------------------------ gather warps
-        const bool is_k = warp == 8;
+        const bool is_k = warp < 12;
+        const int gw = is_k ? warp - 8 : warp - 12;   // this warp's share of each tile
         const CUtensorMap *tm = is_k ? &tmK : &tmV;
-        constexpr uint32_t kTileBytes = kBN * D * 2;
         const int NS = is_k ? L::kKS : L::kVS;
+        // K/V tile: 32 groups of 4 rows x NB boxes; K warps take 8 groups each, V warps
+        // 11, 11 and 10
+        const int per = is_k ? 8 : 11, g_lo = gw * per, cnt = min(per, 32 - g_lo);
+        const int grp = g_lo + lane / NB, blk = lane % NB;
+        const bool active = lane < cnt * NB;
+        const uint32_t kShareBytes = (uint32_t)cnt * 4 * D * 2;
         uint32_t stage_it = 0, q_it = 0;
         for (int it = blockIdx.x; it < n_items && !warp_aborted(abort_flag); it += gridDim.x) {
             const int4 item = a.items[it];
@@ -347,20 +365,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int T = (int)((r + kBN - 1) / kBN);
             const int rowbase = bh * a.N;
             if (is_k) {
-                // both Q tiles: rows perm[q0 .. q0+nq); rows beyond nq repeat the last query
+                // both Q tiles: rows perm[q0 .. q0+nq); rows beyond nq repeat the last query.
+                // 64 groups of 4 rows over the two tiles; warp gw takes groups 16*gw .. +15.
                 if (!warp_wait(&bars->q_empty, (q_it & 1) ^ 1, abort_flag, a.status)) break;
-                if (lane == 0) bar_expect_tx(&bars->q_full, kQT * kBM * D * 2);
+                if (lane == 0) bar_expect_tx(&bars->q_full, 16 * 4 * D * 2);
                 __syncwarp();
-                const int32_t *perm = a.perm + (size_t)bh * a.perm_bh + q0;
-#pragma unroll
-                for (int q = 0; q < kQT; ++q) {
+                if (lane < 16) {
+                    const int32_t *perm = a.perm + (size_t)bh * a.perm_bh + q0;
+                    const int g = gw * 16 + lane, q = g >> 5, r0 = (g & 31) * 4;
                     int rr[4];
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) rr[k] = rowbase + perm[min(q * kBM + 4 * lane + k, nq - 1)];
+                    for (int k = 0; k < 4; ++k) rr[k] = rowbase + perm[min(q * kBM + r0 + k, nq - 1)];
 #pragma unroll
                     for (int b = 0; b < NB; ++b)
-                        tma_gather4(sbase + L::kQ + q * L::kQTile + b * (kBM * 128) + lane * 512, &tmQ,
-                                    b * 64, rr[0], rr[1], rr[2], rr[3], &bars->q_full);
+                        tma_gather4(sbase + L::kQ + q * L::kQTile + b * (kBM * 128) + r0 * 128, &tmQ, b * 64,
+                                    rr[0], rr[1], rr[2], rr[3], &bars->q_full);
                 }
                 ++q_it;
             }
@@ -368,7 +387,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // this lane's four keys of tile t; keys past r_c (last tile) load key 0 and are
             // masked by the softmax.  Indices are loaded two tiles ahead of their gathers.
             auto keys_of = [&](int t) {
-                const long long j0 = (long long)t * kBN + 4 * lane;
+                const long long j0 = (long long)t * kBN + 4 * grp;
                 int4 v;
                 if (j0 + 3 < r) {
                     v = *reinterpret_cast<const int4 *>(list + j0);
@@ -387,20 +406,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                                abort_flag, a.status))
                     break;
                 uint64_t *full = is_k ? &bars->k_full[s] : &bars->v_full[s];
-                if (lane == 0) bar_expect_tx(full, kTileBytes);
+                if (lane == 0) bar_expect_tx(full, kShareBytes);
                 __syncwarp();
-                const uint32_t dst0 = sbase + (is_k ? L::kK : L::kV) + s * L::kKVTile + lane * 512;
-#pragma unroll
-                for (int b = 0; b < NB; ++b)
-                    tma_gather4(dst0 + b * (kBN * 128), tm, b * 64, rowbase + g0.x, rowbase + g0.y,
-                                rowbase + g0.z, rowbase + g0.w, full);
+                if (active)
+                    tma_gather4(sbase + (is_k ? L::kK : L::kV) + s * L::kKVTile + blk * (kBN * 128) + grp * 512,
+                                tm, blk * 64, rowbase + g0.x, rowbase + g0.y, rowbase + g0.z,
+                                rowbase + g0.w, full);
                 g0 = g1;
                 if (t + 2 < T) g1 = keys_of(t + 2);
                 ++stage_it;
             }
         }
-    } else if (warp == 10) {
-        // ------------------------------------------------------------ MMA issuer
+    } else {
+        // ------------------------------------------------------------ MMA issuer (warp 15)
         constexpr uint32_t idesc_qk = f16_idesc(kBM, kBN, false);
         constexpr uint32_t idesc_pv = f16_idesc(kBM, D, true);
         uint32_t k_it = 0, v_it = 0, q_it = 0;
@@ -492,8 +510,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int q = 0; q < kQT; ++q)
                 if (q < nqt) ++o_items[q];
         }
-    } else if (warp < 8) {
+    }
+    } else {
         // ------------------------------------------------------------ softmax + epilogue
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
         const int q = warp >> 2;                       // Q tile of this warpgroup
         const int row = threadIdx.x - q * kBM;         // 0..127 = TMEM lane
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
@@ -613,7 +633,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 10)
+    if (warp == 15)
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
                      : "memory");
 }
@@ -657,6 +677,11 @@ cudaError_t launch_tc(const AttnArgs &a, cudaStream_t s)
     if (!row_gather_map(&tq, a.Q, rows, D) || !row_gather_map(&tk, a.K, rows, D) ||
         !row_gather_map(&tv, a.V, rows, D))
         return cudaErrorInvalidValue;
+    // setmaxnreg moves registers between warpgroups inside the block's launch allocation;
+    // the split only adds up if the kernel was compiled to exactly kLaunchRegs
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, attn_tc_kernel<D>) != cudaSuccess || fa.numRegs != kLaunchRegs)
+        return cudaErrorInvalidDeviceFunction;
     const int smem = Smem<D>::kAlloc;
     cudaFuncSetAttribute(attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     attn_tc_kernel<D><<<a.num_sms, kThreads, smem, s>>>(tq, tk, tv, a);
