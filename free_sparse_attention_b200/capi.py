@@ -23,7 +23,7 @@ DEV_BAD_INIT_INDEX, DEV_SELECT_TIE, DEV_BAD_ASSIGN = 0x1, 0x2, 0x4
 
 EXPORTS = ("scope_workspace_bytes", "scope_cluster_queries", "scope_cluster_keys",
            "scope_build_lut_and_select", "scope_sparse_attention", "scope_forward",
-           "scope_status_string", "scope_get_device_status")
+           "scope_status_string", "scope_get_device_status", "scope_build_lut_and_select_noalloc")
 
 
 class ScopeError(RuntimeError):
@@ -87,6 +87,8 @@ def lib() -> ctypes.CDLL:
         L.scope_forward.restype = i
         L.scope_forward.argtypes = [P, vp, vp, vp, vp, vp, vp, ctypes.POINTER(Intermediates),
                                     vp, sz, vp]
+        L.scope_build_lut_and_select_noalloc.restype = i
+        L.scope_build_lut_and_select_noalloc.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
         L.scope_status_string.restype = ctypes.c_char_p
         L.scope_status_string.argtypes = [i]
         L.scope_get_device_status.restype = i
@@ -159,6 +161,25 @@ def build_lut_and_select(p, q_centroids, q_sizes, k_centroids, k_codes, ws=None,
     _check("scope_build_lut_and_select", lib().scope_build_lut_and_select(
         ctypes.byref(p), _ptr(q_centroids), _ptr(q_sizes), _ptr(k_centroids), _ptr(k_codes),
         _ptr(tp), _ptr(bc), _ptr(kh), _ptr(fc), _ptr(mk), _ptr(ws), ws.numel(), _stream(stream)))
+    return {"topp_counts": tp, "base_counts": bc, "k_head": kh, "final_counts": fc, "sel_mask": mk}
+
+
+def build_lut_and_select_noalloc(p, q_centroids, q_sizes, k_centroids, k_codes, stream=None):
+    """scope_build_lut_and_select without a workspace: for callers that cannot allocate
+    device memory at run time.  The library keeps the scratch in a fixed device array
+    shared by all calls, so calls must not overlap on the GPU (the output tensors below
+    are the caller's; a caller that cannot allocate passes its own preallocated ones
+    through the C ABI directly)."""
+    dev = q_centroids.device
+    shp = (p.B, p.H, p.Cq)
+    tp = torch.empty(shp, dtype=torch.int32, device=dev)
+    bc = torch.empty(shp, dtype=torch.int32, device=dev)
+    fc = torch.empty(shp, dtype=torch.int32, device=dev)
+    kh = torch.empty((p.B, p.H), dtype=torch.int32, device=dev)
+    mk = torch.empty((p.B, p.H, p.Cq, p.nw), dtype=torch.int32, device=dev)
+    _check("scope_build_lut_and_select_noalloc", lib().scope_build_lut_and_select_noalloc(
+        ctypes.byref(p), _ptr(q_centroids), _ptr(q_sizes), _ptr(k_centroids), _ptr(k_codes),
+        _ptr(tp), _ptr(bc), _ptr(kh), _ptr(fc), _ptr(mk), _stream(stream)))
     return {"topp_counts": tp, "base_counts": bc, "k_head": kh, "final_counts": fc, "sel_mask": mk}
 
 

@@ -190,6 +190,34 @@ scope_status scope_forward(const scope_params *p, const void *Q, const void *K, 
                            const scope_intermediates *inter, void *ws, size_t ws_bytes,
                            void *stream);
 
+/*
+ * Selection without a workspace.  The SCOPE paper has no counterpart: this is an
+ * integration variant of scope_build_lut_and_select (same arguments minus the workspace,
+ * same kernels, same outputs) for callers that cannot call cudaMalloc, such as a host
+ * application that owns every device allocation through its own pool and does not let
+ * libraries allocate, or a latency-critical loop in which cudaMalloc / cudaFree (which
+ * may synchronise the device) are not allowed.  Its scratch -- a status word and 64
+ * bytes per (b, h, query cluster) unit -- lives in a fixed device array of the library
+ * (256 B + 1 MiB, held by every GPU that loads the library until the process exits).
+ *  - B*H*Cq must not exceed SCOPE_NOALLOC_MAX_UNITS; larger layers are rejected with
+ *    SCOPE_ERR_UNSUPPORTED before anything is enqueued.
+ *  - The first call on a device looks up the array's device address on that device
+ *    (cudaGetSymbolAddress); make that first call before any stream capture.
+ *  - Every call shares the array and it keeps the last call's contents; each call clears
+ *    the status word it needs.  Calls whose work overlaps on the GPU (other streams, or
+ *    other host threads on the same device) race on the array: serialise them.
+ *  - The device status word of this variant is not readable through
+ *    scope_get_device_status (use the workspace entry point when the status is needed).
+ * Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ */
+#define SCOPE_NOALLOC_MAX_UNITS 16384
+scope_status scope_build_lut_and_select_noalloc(const scope_params *p, const double *q_centroids,
+                                                const int32_t *q_sizes, const double *k_centroids,
+                                                const uint16_t *k_codes, int32_t *topp_counts,
+                                                int32_t *base_counts, int32_t *k_head,
+                                                int32_t *final_counts, uint32_t *sel_mask,
+                                                void *stream);
+
 /* Human-readable name of a status code (static storage). */
 const char *scope_status_string(scope_status s);
 
