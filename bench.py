@@ -113,6 +113,18 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+def max_over_ranks(value: float, device="cpu") -> float:
+    """Maximum of a per-rank time over all ranks (no-op in a single process).  Every rank
+    must call it at the same point."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def dist_setup():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -261,10 +273,7 @@ def run_scope(args, w):
     ms = e0.elapsed_time(e1) / args.steps
     st = np.array([[ev[i].elapsed_time(ev[i + 1]) for i in range(4)] for ev in stage_evs])
     stage_ms = st.mean(axis=0)
-    if world > 1:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, device="cuda")
     status |= capi.get_device_status(ws)
 
     # end to end through the C ABI with host buffers: H2D inputs, layer, D2H output
@@ -288,11 +297,7 @@ def run_scope(args, w):
         e2e_step()
     e1.record()
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / args.steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, device="cuda")
 
     # dense attention on the same shape (library comparator, not part of the path)
     dense_ms = None

@@ -1,0 +1,145 @@
+"""Edge cases of the SCOPE path on the GPU, each against the binary64 oracle or a closed
+form: empty clusters, a single centroid, rho = 1 (dense attention), explicit initial
+centroids (warm start), and the device status word for an out-of-range init index."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from free_sparse_attention_b200 import capi, synth
+from free_sparse_attention_b200.workloads import Workload
+
+from gpu_common import compare_attention, to_np
+
+pytestmark = pytest.mark.gpu
+
+W = Workload("edge", 1, 2, 3, 12, 10, 44, 42, 42, "bf16", 16, 12, seed=21)
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    from free_sparse_attention_b200.build import build
+    build()
+    capi.lib()
+
+
+def _dev(w, x, q_init=None, k_init=None):
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    t = {n: torch.from_numpy(x[n]).reshape(w.B, w.H, w.N, w.d).to("cuda", dt) for n in "qkv"}
+    qi = x["q_init"] if q_init is None else q_init
+    ki = x["k_init"] if k_init is None else k_init
+    t["qi"] = torch.from_numpy(np.ascontiguousarray(qi)).reshape(w.B, w.H, w.Cq).cuda()
+    t["ki"] = torch.from_numpy(np.ascontiguousarray(ki)).reshape(w.B, w.H, 3, w.Cm).cuda()
+    return t
+
+
+def _forward_and_compare(w, x, t, q_init, k_init, rho=None):
+    p = capi.Params.from_workload(w, **({} if rho is None else {"rho": rho}))
+    ws = capi.alloc_workspace(p)
+    O, it = capi.forward(p, t["q"], t["k"], t["v"], t["qi"], t["ki"], ws=ws, intermediates=True)
+    torch.cuda.synchronize()
+    assert capi.get_device_status(ws) == 0
+    g = {k: to_np(v) for k, v in it.items()}
+    O = O.float().cpu().numpy().reshape(w.B * w.H, w.N, w.d)
+    for i in range(w.B * w.H):
+        ref = oracle.forward_head(x["q"][i], x["k"][i], x["v"][i], w, q_init[i], k_init[i], rho=rho)
+        np.testing.assert_array_equal(g["q_assign"][0, i], ref["q"]["assign"])
+        np.testing.assert_array_equal(g["q_centroids"][0, i], ref["q"]["centroids"])
+        np.testing.assert_array_equal(g["k_codes"][0, i], ref["k"]["codes"])
+        np.testing.assert_array_equal(g["k_centroids"][0, i], ref["k"]["centroids"])
+        np.testing.assert_array_equal(g["final_counts"][0, i], ref["sel"]["r"])
+        np.testing.assert_array_equal(g["sel_mask"][0, i].view(np.uint32), ref["sel"]["mask"])
+        compare_attention(w, O[i], ref["O"])
+    return g, O
+
+
+def test_duplicate_init_rows_give_empty_clusters():
+    """Two initial centroids on the same token tie everywhere: after the first iteration
+    the higher index has no member and keeps its centroid; the whole layer (where the
+    stale duplicate may win members again later) still matches the oracle."""
+    x = synth.layer_inputs(W)
+    qi = x["q_init"].copy()
+    ki = x["k_init"].copy()
+    qi[:, 5] = qi[:, 2]
+    ki[:, 1, 7] = ki[:, 1, 3]
+    t = _dev(W, x, qi, ki)
+    _forward_and_compare(W, x, t, qi, ki)
+    p1 = capi.Params.from_workload(W, iters=1)
+    qc, qa, qs = capi.cluster_queries(p1, t["q"], init_idx=t["qi"])
+    torch.cuda.synchronize()
+    assert np.all(to_np(qs)[0, :, 5] == 0)
+    first = np.stack([x["q"][h][qi[h, 2]] for h in range(W.H)]).astype(np.float64)
+    np.testing.assert_array_equal(to_np(qc)[0, :, 5], first)
+
+
+def test_single_centroid_everywhere():
+    w = W.with_(Cq=1, Cm=1)
+    x = synth.layer_inputs(w)
+    t = _dev(w, x)
+    g, _ = _forward_and_compare(w, x, t, x["q_init"], x["k_init"])
+    assert np.all(g["k_head"] == g["base_counts"][..., 0])
+
+
+def test_rho_one_is_dense_attention():
+    x = synth.layer_inputs(W)
+    t = _dev(W, x)
+    p = capi.Params.from_workload(W, rho=1.0)
+    O, it = capi.forward(p, t["q"], t["k"], t["v"], t["qi"], t["ki"], intermediates=True)
+    dense = torch.nn.functional.scaled_dot_product_attention(t["q"].float(), t["k"].float(), t["v"].float())
+    torch.cuda.synchronize()
+    assert torch.all(it["final_counts"] == W.N)
+    err = (O.float() - dense).abs()
+    assert err.max().item() <= 2e-2
+    assert (err.pow(2).mean().sqrt() / dense.pow(2).mean().sqrt()).item() <= 5e-3
+
+
+def test_explicit_initial_centroids_warm_start():
+    """Clustering started from caller centroids (e.g. the previous step's) equals the
+    oracle started from the same centroids."""
+    x = synth.layer_inputs(W)
+    t = _dev(W, x)
+    p = capi.Params.from_workload(W)
+    rng = np.random.default_rng(3)
+    qc0 = rng.standard_normal((W.B, W.H, W.Cq, W.d))
+    kc0 = rng.standard_normal((W.B, W.H, W.Cm, W.d))
+    qc, qa, qs = capi.cluster_queries(p, t["q"], init_cent=torch.from_numpy(qc0).cuda())
+    kc, kk = capi.cluster_keys(p, t["k"], init_cent=torch.from_numpy(kc0).cuda())
+    torch.cuda.synchronize()
+    for h in range(W.H):
+        rq = oracle.kmeans(x["q"][h], 0, W.d, W.Cq, W.iters, init_cent=qc0[0, h])
+        rk = oracle.cluster_keys(x["k"][h], (W.d_t, W.d_h, W.d_w), W.Cm, W.iters, init_cent=kc0[0, h])
+        np.testing.assert_array_equal(to_np(qa)[0, h], rq["assign"])
+        np.testing.assert_array_equal(to_np(qc)[0, h], rq["centroids"])
+        np.testing.assert_array_equal(to_np(kk)[0, h], rk["codes"])
+        np.testing.assert_array_equal(to_np(kc)[0, h], rk["centroids"])
+
+
+def test_bad_init_index_sets_status():
+    x = synth.layer_inputs(W)
+    qi = x["q_init"].copy()
+    qi[0, 0] = W.N + 5
+    t = _dev(W, x, qi, x["k_init"])
+    p = capi.Params.from_workload(W)
+    ws = capi.alloc_workspace(p)
+    capi.cluster_queries(p, t["q"], init_idx=t["qi"], ws=ws)
+    assert capi.get_device_status(ws) & capi.DEV_BAD_INIT_INDEX
+    # the next call on the same workspace starts clean
+    capi.cluster_queries(p, t["q"], init_idx=_dev(W, x)["qi"], ws=ws)
+    assert capi.get_device_status(ws) == 0
+
+
+def test_fp32_and_bf16_paths_agree_on_selection():
+    """The same values as fp32 and as bf16 give identical clustering and selection
+    (the inputs are bf16-exact), and attention within tolerance of each other."""
+    x = synth.layer_inputs(W)
+    w32 = W.with_(dtype="f32")
+    t16, t32 = _dev(W, x), _dev(w32, x)
+    O16, i16 = capi.forward(capi.Params.from_workload(W), t16["q"], t16["k"], t16["v"], t16["qi"],
+                            t16["ki"], intermediates=True)
+    O32, i32 = capi.forward(capi.Params.from_workload(w32), t32["q"], t32["k"], t32["v"], t32["qi"],
+                            t32["ki"], intermediates=True)
+    torch.cuda.synchronize()
+    for k in ("q_assign", "k_codes", "final_counts", "sel_mask", "k_head"):
+        assert torch.equal(i16[k], i32[k]), k
+    assert (O16.float() - O32).abs().max().item() <= 2e-2
