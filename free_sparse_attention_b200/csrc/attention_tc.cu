@@ -269,6 +269,36 @@ __device__ __forceinline__ float fast_exp2(float x)
     return y;
 }
 
+// Packed fp32 pairs (sm_100 f32x2 arithmetic): two lanes of work per FMA-pipe instruction.
+__device__ __forceinline__ unsigned long long f2pack(float a, float b)
+{
+    unsigned long long r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+
+__device__ __forceinline__ float2 f2unpack(unsigned long long r)
+{
+    float a, b;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
+    return make_float2(a, b);
+}
+
+__device__ __forceinline__ unsigned long long f2fma(unsigned long long a, unsigned long long b,
+                                                    unsigned long long c)
+{
+    unsigned long long d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
+__device__ __forceinline__ unsigned long long f2add(unsigned long long a, unsigned long long b)
+{
+    unsigned long long d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
 
 
 // A operand from TMEM (P), B from shared memory (V).
@@ -424,14 +454,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t k_it = 0, v_it = 0, q_it = 0;
         uint32_t p_cnt[kQT] = {0, 0}, o_items[kQT] = {0, 0};
         const bool leader = lane == 0;
+        // descriptors: a base per tile, K steps add their byte offset / 16 to the start
+        // address field (offsets stay inside the 14-bit field)
         auto issue_qk = [&](int q, int ks) {
             if (leader) {
-                const uint32_t qa = sbase + L::kQ + q * L::kQTile, ka = sbase + L::kK + ks * L::kKVTile;
+                const uint64_t qd = sw128_desc(sbase + L::kQ + q * L::kQTile, 16, 1024);
+                const uint64_t kd = sw128_desc(sbase + L::kK + ks * L::kKVTile, 16, 1024);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * (kBM * 128) + (kk & 3) * 32;
-                    mma_bf16(tmem + q * 128, sw128_desc(qa + off, 16, 1024), sw128_desc(ka + off, 16, 1024),
-                             idesc_qk, kk > 0);
+                    const uint64_t off = (uint64_t)(((kk >> 2) * (kBM * 128) + (kk & 3) * 32) >> 4);
+                    mma_bf16(tmem + q * 128, qd + off, kd + off, idesc_qk, kk > 0);
                 }
                 mma_commit(&bars->s_full[q]);
             }
@@ -474,12 +506,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc_fence_after();
                     // O_q += P_q(t) V(t), P_q from TMEM (columns q*128 + [0, 64))
                     if (leader) {
-                        const uint32_t va = sbase + L::kV + vs * L::kKVTile;
+                        const uint64_t vd = sw128_desc(sbase + L::kV + vs * L::kKVTile, kBN * 128, 1024);
 #pragma unroll
                         for (int kk = 0; kk < kBN / 16; ++kk)
-                            mma_bf16_ts(tmem + 256 + q * D, tmem + q * 128 + kk * 8,
-                                        sw128_desc(va + kk * 2048, kBN * 128, 1024), idesc_pv,
-                                        (t > 0 || kk > 0) ? 1u : 0u);
+                            mma_bf16_ts(tmem + 256 + q * D, tmem + q * 128 + kk * 8, vd + (uint64_t)(kk * 2048 >> 4),
+                                        idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
                         mma_commit(&bars->o_done[q]);
                     }
                     __syncwarp();
@@ -572,22 +603,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (need) l *= alpha;
                 }
                 if (need) m_run = mt;
-                // P = 2^(s*c - m) as bf16 pairs over the first 64 columns of S_q
-                float ls[4] = {0.f, 0.f, 0.f, 0.f};
-                const float nm = -m_run;
+                // P = 2^(s*c - m) as bf16 pairs over the first 64 columns of S_q; exponent
+                // arguments and row sums on packed fp32 pairs
+                const unsigned long long c2 = f2pack(c, c), nm2 = f2pack(-m_run, -m_run);
+                unsigned long long ls2[2] = {0ull, 0ull};
 #pragma unroll
                 for (int h = 0; h < kBN / 32; ++h) {
                     uint32_t pk[16];
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
-                        const float p0 = fast_exp2(fmaf(s[h * 32 + 2 * e], c, nm));
-                        const float p1 = fast_exp2(fmaf(s[h * 32 + 2 * e + 1], c, nm));
-                        ls[e & 3] += p0 + p1;
+                        const float2 av = f2unpack(f2fma(f2pack(s[h * 32 + 2 * e], s[h * 32 + 2 * e + 1]), c2, nm2));
+                        const float p0 = fast_exp2(av.x), p1 = fast_exp2(av.y);
+                        ls2[e & 1] = f2add(ls2[e & 1], f2pack(p0, p1));
                         __nv_bfloat162 hh = __floats2bfloat162_rn(p0, p1);
                         pk[e] = *reinterpret_cast<uint32_t *>(&hh);
                     }
                     tmem_st16(tmem + lane_base + s_col + h * 16, pk);
                 }
+                const float2 la = f2unpack(ls2[0]), lb = f2unpack(ls2[1]);
+                float ls[4] = {la.x, la.y, lb.x, lb.y};
                 l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
                 tmem_wait_st();
                 tc_fence_before();
