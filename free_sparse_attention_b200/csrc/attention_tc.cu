@@ -8,10 +8,13 @@
 // Per CTA (persistent, one per SM, static round-robin over the head-major work list):
 //   warps 0-3 / 4-7  softmax + epilogue of Q tile 0 / 1 (thread r owns row r = TMEM lane r)
 //   warps 8-11       gather both Q tiles once per item and the selected K rows per key tile
-//   warps 12-14      gather the selected V rows per key tile
-//   warp 15          allocates TMEM and issues the MMAs (one elected thread)
+//   warps 12-13      gather the selected V rows per key tile
+//   warps 14 / 15    issue the MMAs of Q tile 0 / 1 (one elected thread each; warp 14 also
+//                    allocates TMEM)
 // A TMA gather4 stream sustains ~15 GB/s per issuing warp, so each tile is split over
-// four (K) or three (V) warps; every warp signals its own share with arrive.expect_tx.
+// four (K) or two (V) warps; every warp signals its own share with arrive.expect_tx.
+// One issuing thread sustains an M=128, N=128 tcgen05.mma only every ~170 cycles, about
+// 0.6x of the tensor core's rate; two issuers (one per Q tile) feed it at ~0.8-0.9x.
 // Registers are rebalanced per warpgroup with setmaxnreg: the softmax warpgroups hold a
 // whole 128-column row of logits (192 registers), the gather / MMA warpgroups need 64.
 // Each cluster's selected key indices are expanded once from the bitmask into an
@@ -43,7 +46,8 @@ constexpr int kQT = 2;             // Q tiles per CTA, both against every gather
 constexpr int kBN = 128;           // keys per K/V tile
 constexpr int kThreads = 512;      // 16 warps = 4 warpgroups
 constexpr int kKWarps = 4;         // K (and Q) gather warps
-constexpr int kVWarps = 3;         // V gather warps
+constexpr int kVWarps = 2;         // V gather warps
+constexpr int kMmaWarps = 2;       // one MMA-issuing warp per Q tile
 constexpr int kLaunchRegs = 128;   // 65536 / 512; the setmaxnreg split below sums to it
 constexpr int kSoftmaxRegs = 192;  // 2 warpgroups x 128 threads x 192
 constexpr int kOtherRegs = 64;     //  + 2 warpgroups x 128 threads x 64 = 65536
@@ -344,12 +348,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
         misc[0] = 0;
         bar_init(&bars->q_full, kKWarps);
-        bar_init(&bars->q_empty, 1);
+        bar_init(&bars->q_empty, kMmaWarps);
         for (int s = 0; s < kMaxStages; ++s) {
             bar_init(&bars->k_full[s], kKWarps);
             bar_init(&bars->v_full[s], kVWarps);
-            bar_init(&bars->k_empty[s], 1);
-            bar_init(&bars->v_empty[s], 1);
+            bar_init(&bars->k_empty[s], kMmaWarps);
+            bar_init(&bars->v_empty[s], kMmaWarps);
         }
         for (int q = 0; q < kQT; ++q) {
             bar_init(&bars->s_full[q], 1);
@@ -359,7 +363,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    if (warp == 15) {
+    if (warp == 14) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                          smem_u32(tmem_slot)),
                      "r"(kTmemCols)
@@ -375,15 +379,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp >= 8) {
     // warpgroups 2 and 3 give registers back (one setmaxnreg site for all their warps)
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kOtherRegs));
-    if (warp < 15) {
+    if (warp < 14) {
         // ------------------------------------------------------------ gather warps
         const bool is_k = warp < 12;
         const int gw = is_k ? warp - 8 : warp - 12;   // this warp's share of each tile
         const CUtensorMap *tm = is_k ? &tmK : &tmV;
         const int NS = is_k ? L::kKS : L::kVS;
-        // K/V tile: 32 groups of 4 rows x NB boxes; K warps take 8 groups each, V warps
-        // 11, 11 and 10
-        const int per = is_k ? 8 : 11, g_lo = gw * per, cnt = min(per, 32 - g_lo);
+        // K/V tile: 32 groups of 4 rows x NB boxes; K warps take 8 groups each, V warps 16
+        const int per = is_k ? 8 : 16, g_lo = gw * per, cnt = min(per, 32 - g_lo);
         const int grp = g_lo + lane / NB, blk = lane % NB;
         const bool active = lane < cnt * NB;
         const uint32_t kShareBytes = (uint32_t)cnt * 4 * D * 2;
@@ -448,17 +451,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
     } else {
-        // ------------------------------------------------------------ MMA issuer (warp 15)
+        // ------------------------------------------------------------ MMA issuers (warps 14, 15)
+        // Warp 14 + q issues Q tile q's products: S_q(t+1) = Q_q K(t+1)^T after
+        // O_q += P_q(t) V(t), so the in-order pipe of this thread keeps S_q(t+1) from
+        // overwriting P_q(t) before it is read.  Both warps consume every K and V stage (an
+        // idle Q tile only waits for the data and releases the stage), so the ring phases
+        // advance in step.
+        const int q = warp - 14;
         constexpr uint32_t idesc_qk = f16_idesc(kBM, kBN, false);
         constexpr uint32_t idesc_pv = f16_idesc(kBM, D, true);
-        uint32_t k_it = 0, v_it = 0, q_it = 0;
-        uint32_t p_cnt[kQT] = {0, 0}, o_items[kQT] = {0, 0};
+        uint32_t k_it = 0, v_it = 0, q_it = 0, p_cnt = 0, o_items = 0;
         const bool leader = lane == 0;
-        // descriptors: a base per tile, K steps add their byte offset / 16 to the start
-        // address field (offsets stay inside the 14-bit field)
-        auto issue_qk = [&](int q, int ks) {
+        const uint64_t qd = sw128_desc(sbase + L::kQ + q * L::kQTile, 16, 1024);
+        auto issue_qk = [&](int ks) {
             if (leader) {
-                const uint64_t qd = sw128_desc(sbase + L::kQ + q * L::kQTile, 16, 1024);
                 const uint64_t kd = sw128_desc(sbase + L::kK + ks * L::kKVTile, 16, 1024);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
@@ -469,77 +475,63 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             __syncwarp();
         };
+        auto release = [&](uint64_t *b) {
+            if (leader) mma_commit(b);
+            __syncwarp();
+        };
         for (int it = blockIdx.x; it < n_items && !warp_aborted(abort_flag); it += gridDim.x) {
             const int4 item = a.items[it];
             const long long r = a.final_cnt[(size_t)item.x * a.Cq + item.y];
             const int T = (int)((r + kBN - 1) / kBN);
-            const int nqt = item.w > kBM ? 2 : 1;     // active Q tiles
+            const bool active = q == 0 || item.w > kBM;   // Q tile 1 idles on items of <= 128 queries
             if (!warp_wait(&bars->q_full, q_it & 1, abort_flag, a.status)) break;
             ++q_it;
             // prologue: S_q(0) = Q_q K(0)^T
             int ks = k_it % L::kKS;
             if (!warp_wait(&bars->k_full[ks], (k_it / L::kKS) & 1, abort_flag, a.status)) break;
             tc_fence_after();
-#pragma unroll
-            for (int q = 0; q < kQT; ++q)
-                if (q < nqt) issue_qk(q, ks);
-            if (leader) {
-                mma_commit(&bars->k_empty[ks]);
-                if (T == 1) mma_commit(&bars->q_empty);
-            }
-            __syncwarp();
+            if (active) issue_qk(ks);
+            release(&bars->k_empty[ks]);
+            if (T == 1) release(&bars->q_empty);
             ++k_it;
             bool ok = true;
             for (int t = 0; t < T && ok; ++t) {
                 const int vs = v_it % L::kVS;
                 ok = warp_wait(&bars->v_full[vs], (v_it / L::kVS) & 1, abort_flag, a.status);
-                const bool more = t + 1 < T;
-                ks = k_it % L::kKS;
+                if (ok && active) {
+                    ok = warp_wait(&bars->p_full[q], p_cnt & 1, abort_flag, a.status);
+                    if (ok && t == 0) ok = warp_wait(&bars->o_free[q], (o_items & 1) ^ 1, abort_flag, a.status);
+                    if (ok) {
+                        ++p_cnt;
+                        tc_fence_after();
+                        // O_q += P_q(t) V(t), P_q from TMEM (columns q*128 + [0, 64))
+                        if (leader) {
+                            const uint64_t vd = sw128_desc(sbase + L::kV + vs * L::kKVTile, kBN * 128, 1024);
 #pragma unroll
-                for (int q = 0; q < kQT; ++q) {
-                    if (q >= nqt || !ok) break;
-                    ok = warp_wait(&bars->p_full[q], p_cnt[q] & 1, abort_flag, a.status);
-                    if (ok && t == 0)
-                        ok = warp_wait(&bars->o_free[q], (o_items[q] & 1) ^ 1, abort_flag, a.status);
-                    if (!ok) break;
-                    ++p_cnt[q];
-                    tc_fence_after();
-                    // O_q += P_q(t) V(t), P_q from TMEM (columns q*128 + [0, 64))
-                    if (leader) {
-                        const uint64_t vd = sw128_desc(sbase + L::kV + vs * L::kKVTile, kBN * 128, 1024);
-#pragma unroll
-                        for (int kk = 0; kk < kBN / 16; ++kk)
-                            mma_bf16_ts(tmem + 256 + q * D, tmem + q * 128 + kk * 8, vd + (uint64_t)(kk * 2048 >> 4),
-                                        idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
-                        mma_commit(&bars->o_done[q]);
-                    }
-                    __syncwarp();
-                    // S_q(t+1) = Q_q K(t+1)^T, issued after PV_q(t) has read P_q(t)
-                    if (more) {
-                        if (q == 0) {
-                            ok = warp_wait(&bars->k_full[ks], (k_it / L::kKS) & 1, abort_flag, a.status);
-                            if (!ok) break;
-                            tc_fence_after();
+                            for (int kk = 0; kk < kBN / 16; ++kk)
+                                mma_bf16_ts(tmem + 256 + q * D, tmem + q * 128 + kk * 8, vd + (uint64_t)(kk * 2048 >> 4),
+                                            idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
+                            mma_commit(&bars->o_done[q]);
                         }
-                        issue_qk(q, ks);
+                        __syncwarp();
                     }
                 }
                 if (!ok) break;
-                if (leader) {
-                    mma_commit(&bars->v_empty[vs]);
-                    if (more) {
-                        mma_commit(&bars->k_empty[ks]);
-                        if (t + 2 == T) mma_commit(&bars->q_empty);
-                    }
-                }
-                __syncwarp();
+                release(&bars->v_empty[vs]);
                 ++v_it;
-                if (more) ++k_it;
+                if (t + 1 < T) {
+                    ks = k_it % L::kKS;
+                    ok = warp_wait(&bars->k_full[ks], (k_it / L::kKS) & 1, abort_flag, a.status);
+                    if (!ok) break;
+                    tc_fence_after();
+                    if (active) issue_qk(ks);
+                    release(&bars->k_empty[ks]);
+                    if (t + 2 == T) release(&bars->q_empty);
+                    ++k_it;
+                }
             }
             if (!ok) break;
-#pragma unroll
-            for (int q = 0; q < kQT; ++q)
-                if (q < nqt) ++o_items[q];
+            if (active) ++o_items;
         }
     }
     } else {
@@ -667,7 +659,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 15)
+    if (warp == 14)
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
                      : "memory");
 }
