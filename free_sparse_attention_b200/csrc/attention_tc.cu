@@ -9,25 +9,25 @@
 //   warps 0-3 / 4-7  softmax + epilogue of Q tile 0 / 1 (thread r owns row r = TMEM lane r)
 //   warps 8-11       gather both Q tiles once per item and the selected K rows per key tile
 //   warps 12-13      gather the selected V rows per key tile
-//   warps 14 / 15    issue the MMAs of Q tile 0 / 1 (one elected thread each; warp 14 also
+//   warps 14 / 15    issue the MMAs of Q tile 0 / 1 (one thread each; warp 14 also
 //                    allocates TMEM)
 // A TMA gather4 stream sustains ~15 GB/s per issuing warp, so each tile is split over
 // four (K) or two (V) warps; every warp signals its own share with arrive.expect_tx.
-// One issuing thread sustains an M=128, N=128 tcgen05.mma only every ~170 cycles, about
-// 0.6x of the tensor core's rate; two issuers (one per Q tile) feed it at ~0.8-0.9x.
 // Registers are rebalanced per warpgroup with setmaxnreg: the softmax warpgroups hold a
-// whole 128-column row of logits (192 registers), the gather / MMA warpgroups need 64.
+// row of logits (192 registers), the gather / MMA warpgroups need 64.
 // Each cluster's selected key indices are expanded once from the bitmask into an
 // ascending list (attn_lists_kernel).  Rows are gathered with TMA tile::gather4 (four
 // arbitrary rows of one 64-column, 128-byte box per instruction, each lane issuing its
 // own four rows) straight into the 128B-swizzled K-major layout the tensor core reads.
-//   S_q  = Q_q K^T     tcgen05.mma kind::f16, M=128, N=128, K=d, fp32 in TMEM
-//   O_q += P_q V       M=128, N=d, K=128, P_q bf16 written by the softmax over its own
-//                      S_q columns in TMEM (A operand from TMEM), V from shared memory
-// Both Q tiles reuse every gathered K/V tile.  The MMA warp issues in ping-pong order
-// PV_0(t), QK_0(t+1), PV_1(t), QK_1(t+1), so the tensor core works on one Q tile while
-// the other tile's softmax runs; in-order execution of the tensor pipe keeps QK_q(t+1)
-// from overwriting P_q(t) before PV_q(t) has read it.  The softmax keeps a running row
+//   S_q  = Q_q K^T     tcgen05.mma kind::f16, M=128, N=64 keys, K=d, fp32 in TMEM
+//   O_q += P_q V       M=128, N=d, K=64, P_q bf16 written by the softmax over the first
+//                      columns of its own S buffer (A operand from TMEM), V from smem
+// Both Q tiles reuse every gathered K/V tile.  S is double-buffered per Q tile (two
+// 64-column buffers; 2 x (2 x 64 + 128) = 512 TMEM columns at d = 128): the MMA thread
+// of tile q issues S(0), S(1), then P(t) V(t) followed by S(t+2) into the buffer P(t)
+// occupied, so the softmax of step t+1 runs while the tensor core works on step t.  A
+// thread's tcgen05.commit costs it roughly one pipe latency before its next MMA starts,
+// which is why each Q tile has its own issuing thread.  The softmax keeps a running row
 // maximum and rescales O (TMEM load/store) only when the maximum grows by more than
 // 2^8, so P stays <= 256 and the final O / l is exact softmax arithmetic.  Every
 // mbarrier wait gives up after ~4 s, sets a status bit and lets the CTA drain and free
@@ -43,7 +43,7 @@ namespace {
 
 constexpr int kBM = 128;           // queries per Q tile (TMEM lanes)
 constexpr int kQT = 2;             // Q tiles per CTA, both against every gathered K/V tile
-constexpr int kBN = 128;           // keys per K/V tile
+constexpr int kBN = 64;            // keys per K/V tile (one S buffer)
 constexpr int kThreads = 512;      // 16 warps = 4 warpgroups
 constexpr int kKWarps = 4;         // K (and Q) gather warps
 constexpr int kVWarps = 2;         // V gather warps
@@ -51,7 +51,7 @@ constexpr int kMmaWarps = 2;       // one MMA-issuing warp per Q tile
 constexpr int kLaunchRegs = 128;   // 65536 / 512; the setmaxnreg split below sums to it
 constexpr int kSoftmaxRegs = 192;  // 2 warpgroups x 128 threads x 192
 constexpr int kOtherRegs = 64;     //  + 2 warpgroups x 128 threads x 64 = 65536
-constexpr int kMaxStages = 6;
+constexpr int kMaxStages = 8;
 constexpr uint32_t kTmemCols = 512;
 constexpr unsigned long long kWaitNs = 4000000000ull;
 
@@ -59,16 +59,19 @@ struct __align__(8) Bars {
     uint64_t q_full, q_empty;
     uint64_t k_full[kMaxStages], k_empty[kMaxStages];
     uint64_t v_full[kMaxStages], v_empty[kMaxStages];
-    uint64_t s_full[kQT], p_full[kQT], o_done[kQT], o_free[kQT];
+    // per Q tile and S buffer: S ready (MMA commit), P written (softmax), P V done (commit)
+    uint64_t s_full[kQT][2], p_full[kQT][2], o_done[kQT][2];
+    uint64_t o_free[kQT];  // epilogue has read O_q
+    uint64_t turn[kQT];    // softmax warpgroups take turns: turn[q] = "Q tile q's softmax may run"
 };
 
 // Shared memory: two Q tiles, a K ring and a V ring (bf16, 128-byte swizzled, K-major).
-// TMEM: S_q (fp32, 128 columns; P_q bf16 pairs over its first 64) at q*128, O_q (fp32,
-// D columns) at 256 + q*D.
+// TMEM: two S buffers per Q tile (fp32, 64 columns each; P bf16 pairs over the first 32
+// columns of its own buffer) at q*128 + b*64, O_q (fp32, D columns) at 256 + q*D.
 template <int D>
 struct Smem {
-    static constexpr int kKS = D == 128 ? 3 : 6;       // K ring depth
-    static constexpr int kVS = D == 128 ? 2 : 6;       // V ring depth
+    static constexpr int kKS = D == 128 ? 5 : 8;       // K ring depth
+    static constexpr int kVS = D == 128 ? 5 : 8;       // V ring depth
     static constexpr int kQTile = kBM * D * 2;
     static constexpr int kKVTile = kBN * D * 2;
     static constexpr int kQ = 0;
@@ -79,6 +82,7 @@ struct Smem {
     static constexpr int kBytes = kMisc + 64;
     static constexpr int kAlloc = kBytes + 1024;       // room to align the base to 1 KB
     static_assert(kAlloc <= 232448, "shared memory budget");
+    static_assert(kKS <= kMaxStages && kVS <= kMaxStages, "ring depth");
     static_assert(kAlloc > 232448 / 2, "one CTA (and its 512 TMEM columns) per SM");
 };
 
@@ -105,28 +109,32 @@ __device__ __forceinline__ void bar_arrive(uint64_t *b)
                  : "memory");
 }
 
-// try_wait with a suspend-time hint: the thread sleeps until the phase completes (or
-// the hint, 1 ms, elapses) instead of spinning on the issue slots.
+// Non-blocking test of an mbarrier phase.
 __device__ __forceinline__ bool bar_test(uint64_t *b, uint32_t parity)
 {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(smem_u32(b)), "r"(parity), "r"(1000000u)
+        : "r"(smem_u32(b)), "r"(parity)
         : "memory");
     return ok != 0;
 }
 
-// Bounded wait by one thread; on timeout sets the CTA abort flag and the device status.
+// Bounded wait by one thread: polls with a short nanosleep backoff (a few tens of ns, so
+// a completed phase is seen quickly without taking issue slots from the busy warps); on
+// timeout sets the CTA abort flag and the device status.
 __device__ __forceinline__ bool bar_wait(uint64_t *b, uint32_t parity, volatile int *abort_flag,
                                          int32_t *status)
 {
     if (bar_test(b, parity)) return true;
     const unsigned long long t0 = global_ns();
+    unsigned ns = 8;
     while (!bar_test(b, parity)) {
+        __nanosleep(ns);
+        ns = ns < 64 ? ns * 2 : 64;
         if (*abort_flag) return false;
         if (global_ns() - t0 > kWaitNs) {
             *abort_flag = 1;
@@ -356,10 +364,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             bar_init(&bars->v_empty[s], kMmaWarps);
         }
         for (int q = 0; q < kQT; ++q) {
-            bar_init(&bars->s_full[q], 1);
-            bar_init(&bars->p_full[q], 4);
-            bar_init(&bars->o_done[q], 1);
+            for (int b = 0; b < 2; ++b) {
+                bar_init(&bars->s_full[q][b], 1);
+                bar_init(&bars->p_full[q][b], 4);
+                bar_init(&bars->o_done[q][b], 1);
+            }
             bar_init(&bars->o_free[q], 4);
+            bar_init(&bars->turn[q], 4);
         }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -385,8 +396,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int gw = is_k ? warp - 8 : warp - 12;   // this warp's share of each tile
         const CUtensorMap *tm = is_k ? &tmK : &tmV;
         const int NS = is_k ? L::kKS : L::kVS;
-        // K/V tile: 32 groups of 4 rows x NB boxes; K warps take 8 groups each, V warps 16
-        const int per = is_k ? 8 : 16, g_lo = gw * per, cnt = min(per, 32 - g_lo);
+        // K/V tile: kBN/4 groups of 4 rows x NB boxes, split evenly over the K (or V) warps
+        constexpr int kGroups = kBN / 4;
+        const int per = is_k ? kGroups / kKWarps : kGroups / kVWarps, g_lo = gw * per,
+                  cnt = min(per, kGroups - g_lo);
         const int grp = g_lo + lane / NB, blk = lane % NB;
         const bool active = lane < cnt * NB;
         const uint32_t kShareBytes = (uint32_t)cnt * 4 * D * 2;
@@ -452,29 +465,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // ------------------------------------------------------------ MMA issuers (warps 14, 15)
-        // Warp 14 + q issues Q tile q's products: S_q(t+1) = Q_q K(t+1)^T after
-        // O_q += P_q(t) V(t), so the in-order pipe of this thread keeps S_q(t+1) from
-        // overwriting P_q(t) before it is read.  Both warps consume every K and V stage (an
-        // idle Q tile only waits for the data and releases the stage), so the ring phases
-        // advance in step.
+        // Warp 14 + q issues Q tile q's products.  S is double-buffered: S_q(j) goes to
+        // buffer j & 1, so S_q(t+1) is ready while the softmax still works on S_q(t).  The
+        // order per tile is S(0), S(1), then for every t: O += P(t) V(t), S(t+2).  S(t+2)
+        // reuses the buffer whose first columns hold P(t); issuing it after P(t) V(t) from
+        // the same thread keeps the in-order tensor pipe from overwriting P(t) early.  Both
+        // warps consume every K and V stage in the same order (an idle Q tile only waits
+        // for the data and releases the stage), so the ring phases advance in step.
         const int q = warp - 14;
         constexpr uint32_t idesc_qk = f16_idesc(kBM, kBN, false);
         constexpr uint32_t idesc_pv = f16_idesc(kBM, D, true);
-        uint32_t k_it = 0, v_it = 0, q_it = 0, p_cnt = 0, o_items = 0;
+        uint32_t k_it = 0, v_it = 0, q_it = 0, o_items = 0;
+        uint32_t p_par = 0;   // bit b: parity of the next p_full[q][b] phase
         const bool leader = lane == 0;
         const uint64_t qd = sw128_desc(sbase + L::kQ + q * L::kQTile, 16, 1024);
-        auto issue_qk = [&](int ks) {
-            if (leader) {
-                const uint64_t kd = sw128_desc(sbase + L::kK + ks * L::kKVTile, 16, 1024);
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint64_t off = (uint64_t)(((kk >> 2) * (kBM * 128) + (kk & 3) * 32) >> 4);
-                    mma_bf16(tmem + q * 128, qd + off, kd + off, idesc_qk, kk > 0);
-                }
-                mma_commit(&bars->s_full[q]);
-            }
-            __syncwarp();
-        };
         auto release = [&](uint64_t *b) {
             if (leader) mma_commit(b);
             __syncwarp();
@@ -486,32 +490,49 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool active = q == 0 || item.w > kBM;   // Q tile 1 idles on items of <= 128 queries
             if (!warp_wait(&bars->q_full, q_it & 1, abort_flag, a.status)) break;
             ++q_it;
-            // prologue: S_q(0) = Q_q K(0)^T
-            int ks = k_it % L::kKS;
-            if (!warp_wait(&bars->k_full[ks], (k_it / L::kKS) & 1, abort_flag, a.status)) break;
-            tc_fence_after();
-            if (active) issue_qk(ks);
-            release(&bars->k_empty[ks]);
-            if (T == 1) release(&bars->q_empty);
-            ++k_it;
-            bool ok = true;
+            // S_q(j) = Q_q K(j)^T into buffer j & 1
+            auto qk_step = [&](int j) -> bool {
+                const int ks = k_it % L::kKS;
+                if (!warp_wait(&bars->k_full[ks], (k_it / L::kKS) & 1, abort_flag, a.status)) return false;
+                tc_fence_after();
+                if (active && leader) {
+                    const uint64_t kd = sw128_desc(sbase + L::kK + ks * L::kKVTile, 16, 1024);
+                    const uint32_t dst = tmem + q * 128 + (j & 1) * kBN;
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint64_t offa = (uint64_t)(((kk >> 2) * (kBM * 128) + (kk & 3) * 32) >> 4);
+                        const uint64_t offb = (uint64_t)(((kk >> 2) * (kBN * 128) + (kk & 3) * 32) >> 4);
+                        mma_bf16(dst, qd + offa, kd + offb, idesc_qk, kk > 0);
+                    }
+                    mma_commit(&bars->s_full[q][j & 1]);
+                }
+                __syncwarp();
+                release(&bars->k_empty[ks]);
+                if (j == T - 1) release(&bars->q_empty);
+                ++k_it;
+                return true;
+            };
+            bool ok = qk_step(0);
+            if (ok && T > 1) ok = qk_step(1);
             for (int t = 0; t < T && ok; ++t) {
                 const int vs = v_it % L::kVS;
+                const int b = t & 1;
                 ok = warp_wait(&bars->v_full[vs], (v_it / L::kVS) & 1, abort_flag, a.status);
                 if (ok && active) {
-                    ok = warp_wait(&bars->p_full[q], p_cnt & 1, abort_flag, a.status);
+                    ok = warp_wait(&bars->p_full[q][b], (p_par >> b) & 1u, abort_flag, a.status);
                     if (ok && t == 0) ok = warp_wait(&bars->o_free[q], (o_items & 1) ^ 1, abort_flag, a.status);
                     if (ok) {
-                        ++p_cnt;
+                        p_par ^= 1u << b;
                         tc_fence_after();
-                        // O_q += P_q(t) V(t), P_q from TMEM (columns q*128 + [0, 64))
+                        // O_q += P_q(t) V(t), P_q(t) from TMEM (columns q*128 + b*64 + [0, 32))
                         if (leader) {
                             const uint64_t vd = sw128_desc(sbase + L::kV + vs * L::kKVTile, kBN * 128, 1024);
 #pragma unroll
                             for (int kk = 0; kk < kBN / 16; ++kk)
-                                mma_bf16_ts(tmem + 256 + q * D, tmem + q * 128 + kk * 8, vd + (uint64_t)(kk * 2048 >> 4),
-                                            idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
-                            mma_commit(&bars->o_done[q]);
+                                mma_bf16_ts(tmem + 256 + q * D, tmem + q * 128 + b * kBN + kk * 8,
+                                            vd + (uint64_t)(kk * 2048 >> 4), idesc_pv,
+                                            (t > 0 || kk > 0) ? 1u : 0u);
+                            mma_commit(&bars->o_done[q][b]);
                         }
                         __syncwarp();
                     }
@@ -519,16 +540,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!ok) break;
                 release(&bars->v_empty[vs]);
                 ++v_it;
-                if (t + 1 < T) {
-                    ks = k_it % L::kKS;
-                    ok = warp_wait(&bars->k_full[ks], (k_it / L::kKS) & 1, abort_flag, a.status);
-                    if (!ok) break;
-                    tc_fence_after();
-                    if (active) issue_qk(ks);
-                    release(&bars->k_empty[ks]);
-                    if (t + 2 == T) release(&bars->q_empty);
-                    ++k_it;
-                }
+                if (t + 2 < T) ok = qk_step(t + 2);
             }
             if (!ok) break;
             if (active) ++o_items;
@@ -541,24 +553,35 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int row = threadIdx.x - q * kBM;         // 0..127 = TMEM lane
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
         const uint32_t s_col = q * 128, o_col = 256 + q * D;
-        uint32_t s_cnt = 0, o_cnt = 0;
+        // bit b of s_par: parity of the next s_full[q][b] phase; bit b of o_par: parity of
+        // the P V commits on o_done[q][b] before the current item (the softmax waits on
+        // o_done only when it must, so it counts the phases per item instead)
+        uint32_t s_par = 0, o_par = 0, turn_cnt = 0;
         const float c = a.scale_log2;
+        // parity of the o_done[q][j & 1] phase that completes when P(j) V(j) is done
+        auto pv_parity = [&](int j) -> uint32_t { return ((o_par >> (j & 1)) + (uint32_t)(j >> 1)) & 1u; };
         for (int it = blockIdx.x; it < n_items && !warp_aborted(abort_flag); it += gridDim.x) {
             const int4 item = a.items[it];
             const int bh = item.x, cl = item.y, q0 = item.z, nq = item.w;
             if (q == 1 && nq <= kBM) continue;        // this Q tile is idle for the item
+            // With both Q tiles active the two warpgroups take turns on the exponentials
+            // (tile 0 first), so one tile's exponentials overlap the other tile's MMAs
+            // instead of both competing for the special-function units at once.
+            const bool take_turns = nq > kBM;
             const long long r = a.final_cnt[(size_t)bh * a.Cq + cl];
             const int T = (int)((r + kBN - 1) / kBN);
             float m_run = -INFINITY, l = 0.f;
             bool ok = true;
             for (int t = 0; t < T; ++t) {
-                ok = warp_wait(&bars->s_full[q], s_cnt & 1, abort_flag, a.status);
+                const int b = t & 1;
+                ok = warp_wait(&bars->s_full[q][b], (s_par >> b) & 1u, abort_flag, a.status);
                 if (!ok) break;
-                ++s_cnt;
+                s_par ^= 1u << b;
                 tc_fence_after();
+                const uint32_t sb_col = s_col + b * kBN;
                 float s[kBN];
 #pragma unroll
-                for (int h = 0; h < kBN / 32; ++h) tmem_ld32(tmem + lane_base + s_col + h * 32, s + h * 32);
+                for (int h = 0; h < kBN / 32; ++h) tmem_ld32(tmem + lane_base + sb_col + h * 32, s + h * 32);
                 tmem_wait_ld();
                 const int nvalid = (int)min((long long)kBN, r - (long long)t * kBN);
                 if (nvalid < kBN) {
@@ -573,15 +596,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int j = 8; j < kBN; ++j) m8[j & 7] = fmaxf(m8[j & 7], s[j]);
                 const float mt = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
                                        fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) * c;
-                // P V of the previous tile is complete (it preceded Q K^T of this one)
-                if (t > 0) {
-                    ok = warp_wait(&bars->o_done[q], o_cnt & 1, abort_flag, a.status);
-                    if (!ok) break;
-                    ++o_cnt;
-                    tc_fence_after();
-                }
                 const bool need = mt > m_run + 8.f;
                 if (t > 0 && __any_sync(0xffffffffu, need)) {
+                    // rescaling O needs every earlier P V done; the last one is P(t-1) V(t-1)
+                    ok = warp_wait(&bars->o_done[q][(t - 1) & 1], pv_parity(t - 1), abort_flag, a.status);
+                    if (!ok) break;
+                    tc_fence_after();
                     const float alpha = need ? fast_exp2(m_run - mt) : 1.f;
 #pragma unroll 1
                     for (int h = 0; h < D / 32; ++h) {
@@ -595,8 +615,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (need) l *= alpha;
                 }
                 if (need) m_run = mt;
-                // P = 2^(s*c - m) as bf16 pairs over the first 64 columns of S_q; exponent
-                // arguments and row sums on packed fp32 pairs
+                if (take_turns) {
+                    ok = warp_wait(&bars->turn[q], (turn_cnt & 1) ^ (q == 0 ? 1u : 0u), abort_flag, a.status);
+                    if (!ok) break;
+                    ++turn_cnt;
+                }
+                // P = 2^(s*c - m) as bf16 pairs over the first kBN/2 columns of this S
+                // buffer; exponent arguments and row sums on packed fp32 pairs
                 const unsigned long long c2 = f2pack(c, c), nm2 = f2pack(-m_run, -m_run);
                 unsigned long long ls2[2] = {0ull, 0ull};
 #pragma unroll
@@ -610,7 +635,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                         __nv_bfloat162 hh = __floats2bfloat162_rn(p0, p1);
                         pk[e] = *reinterpret_cast<uint32_t *>(&hh);
                     }
-                    tmem_st16(tmem + lane_base + s_col + h * 16, pk);
+                    tmem_st16(tmem + lane_base + sb_col + h * 16, pk);
+                }
+                if (take_turns) {
+                    __syncwarp();
+                    if (lane == 0) bar_arrive(&bars->turn[q ^ 1]);
                 }
                 const float2 la = f2unpack(ls2[0]), lb = f2unpack(ls2[1]);
                 float ls[4] = {la.x, la.y, lb.x, lb.y};
@@ -618,12 +647,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) bar_arrive(&bars->p_full[q]);
+                if (lane == 0) bar_arrive(&bars->p_full[q][b]);
             }
             if (!ok) break;
-            // epilogue: O / l for the valid rows of this Q tile
-            if (!warp_wait(&bars->o_done[q], o_cnt & 1, abort_flag, a.status)) break;
-            ++o_cnt;
+            // epilogue: O / l for the valid rows of this Q tile, once P(T-1) V(T-1) is done
+            if (!warp_wait(&bars->o_done[q][(T - 1) & 1], pv_parity(T - 1), abort_flag, a.status)) break;
+            o_par ^= (uint32_t)(((T + 1) >> 1) & 1) | ((uint32_t)((T >> 1) & 1) << 1);
             tc_fence_after();
             const float inv = l > 0.f ? 1.f / l : 0.f;
             const bool valid = q * kBM + row < nq;
