@@ -46,12 +46,15 @@ struct KmArgs {
     int32_t *chunk_hist;  // [P, nchunk, Cs] per-chunk counts -> prefix
     int nchunk;
     int32_t *status;      // device status word
+    // tensor-core assignment (bf16 inputs): packed centroid operands, Cpad = Cs rounded up to 16
+    __nv_bfloat16 *cent_bf;   // [P, 2 (hi, lo), Cpad, d] bf16 split of the centroids
+    float *cn2p;              // [P, Cpad + 4] |mu|^2 (+inf padding), max |mu|, max slack
 };
 
 // Workspace layout (byte offsets); computed identically by every entry point.
 struct WsLayout {
     size_t status, counters;
-    size_t cent32, cnorm, cnrm2, cslack, perm, off, chunk_hist;
+    size_t cent32, cnorm, cnrm2, cslack, perm, off, chunk_hist, cent_bf, cn2p;
     size_t q_cent, q_assign, q_sizes, k_cent, k_codes, k_sizes;
     size_t topp, base, khead, final_cnt, mask, sel_state;
     size_t q_perm, q_off, q_hist, work_items, attn_counter, key_lists;
@@ -63,6 +66,9 @@ WsLayout ws_layout(const scope_params &p);
 // Launchers (enqueue only; return cudaGetLastError()).
 cudaError_t km_run(KmArgs a, int iters, cudaStream_t s);
 cudaError_t sort_by_cluster(KmArgs a, cudaStream_t s);  // stable counting sort, all problems
+bool km_assign_tc_supported(const KmArgs &a);            // bf16 and the operands fit on chip
+cudaError_t km_pack(const KmArgs &a, cudaStream_t s);     // centroids -> cent_bf, cn2p
+cudaError_t km_assign_tc(const KmArgs &a, int num_sms, cudaStream_t s);
 
 struct SelArgs {
     const double *qcent;      // [BH, Cq, d]

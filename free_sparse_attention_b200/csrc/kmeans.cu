@@ -7,7 +7,9 @@
 // non-empty centroid moves to the mean of its members.
 //
 // Design (B200): the assignment is a [tokens x dm] x [dm x C] contraction followed by
-// an argmin.  It runs on the fp32 FMA pipes with centroids staged in shared memory;
+// an argmin.  For bf16 inputs it runs on the tensor cores (kmeans_tc.cu); otherwise
+// (fp32 inputs, or centroid sets too large for shared memory) on the fp32 FMA pipes
+// with centroids staged in shared memory (km_assign_fast_kernel below);
 // each distance carries a rigorous error bound, and a token whose best and runner-up
 // cannot be told apart under that bound is re-decided in binary64 with the channels
 // summed in order (one rounding per operation).  Hence the assignment equals a
@@ -479,8 +481,18 @@ cudaError_t km_run(KmArgs a, int iters, cudaStream_t s)
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    // bf16 inputs whose centroid operands fit in shared memory take the tensor-core
+    // assignment (kmeans_tc.cu); both paths certify their winners the same way and leave
+    // the undecided tokens to the binary64 kernel.
+    const bool tc = km_assign_tc_supported(a);
     for (int it = 0; it < iters; ++it) {
-        km_assign_fast_kernel<<<dim3((a.N + kTok - 1) / kTok, P), kAssignThreads, fsm, s>>>(a);
+        if (tc) {
+            cudaError_t e = km_pack(a, s);
+            if (e == cudaSuccess) e = km_assign_tc(a, sms, s);
+            if (e != cudaSuccess) return e;
+        } else {
+            km_assign_fast_kernel<<<dim3((a.N + kTok - 1) / kTok, P), kAssignThreads, fsm, s>>>(a);
+        }
         km_assign_exact_kernel<<<sms * 4, 256, 0, s>>>(a);
         cudaError_t e = sort_by_cluster(a, s);
         if (e != cudaSuccess) return e;

@@ -1,0 +1,488 @@
+// k-means assignment on the Blackwell tensor cores (tcgen05, sm_100a), bf16 inputs.
+//
+// The assignment step of Lloyd's k-means (SCOPE's query clustering and the per-subspace
+// key clustering, review page, load_bearing_attack: Eq. 3) picks, for every token x,
+// the centroid c minimising |x - mu_c|^2, i.e. minimising S_c = |mu_c|^2 - 2 x.mu_c.
+// x.mu_c for a tile of 128 tokens against every centroid is a dense [128 x K] x [K x C]
+// product, so it runs as tcgen05 MMAs with the fp32 accumulator in TMEM:
+//   * x is bf16 already (the layer's Q or K), loaded by TMA straight into the 128-byte
+//     swizzled K-major layout.  A subspace uses the 16-channel-aligned window around its
+//     channel range; the centroid matrix is zero outside the range, so channels of other
+//     subspaces contribute exactly nothing.
+//   * each binary64 centroid is split as mu = hi + lo + r with hi = bf16(mu),
+//     lo = bf16(mu - hi), |r| <= 2^-16 |mu|; both halves accumulate into one TMEM
+//     accumulator (x.hi + x.lo), products being exact in fp32.
+//   * the epilogue (one thread per token = TMEM lane) keeps the smallest and the
+//     second-smallest fp32 score and the winner.  The winner is certain when the gap
+//     exceeds twice a rigorous bound on |score - S_c| (the bf16 split remainder, the
+//     fp32 accumulation, the rounding of |mu|^2 and of the score, and the binary64
+//     rounding of the reference); otherwise the token is marked unsure and the binary64
+//     kernel of kmeans.cu re-decides it exactly.  So the assignment equals the binary64
+//     evaluation of the definition, as on the CUDA-core path.
+//
+// Per CTA (persistent, one per SM, a contiguous range of (problem, 128-token tile) units):
+//   warp 0     TMA producer: the problem's centroid matrix (hi, lo) and |mu|^2 row once
+//              per problem, the token tile into a 2-deep ring
+//   warp 1     TMEM allocation and MMA issue (one thread)
+//   warps 2-5  epilogue: token norms from the shared-memory tile, TMEM loads, argmin
+// The centroids are split in chunks of at most 256 columns, double-buffered in TMEM
+// (2 x 256 columns), so the epilogue of one chunk overlaps the MMAs of the next.
+// Every mbarrier wait gives up after ~4 s, sets a status bit and lets the CTA drain.
+#include "tc_common.cuh"
+
+#include <cfloat>
+
+namespace scope {
+
+namespace {
+
+constexpr int kTile = 128;             // tokens per unit (TMEM lanes)
+constexpr int kThreadsTc = 192;        // 6 warps
+constexpr int kChunkMax = 256;         // centroid columns per TMEM buffer
+constexpr uint32_t kTmemColsTc = 512;  // two accumulator buffers
+constexpr uint16_t kUnsureTc = 0xFFFF;
+constexpr int kBoxRows = 16;           // centroid rows per TMA box
+constexpr int kSmemLimit = 232448;
+
+struct __align__(8) TcBars {
+    uint64_t b_full, b_empty;
+    uint64_t x_full[2], x_empty[2];
+    uint64_t acc_full[2], acc_empty[2];
+    uint64_t drain;
+};
+
+// Channel window of a role: [ws, ws + 16*ks), ks 16-channel MMA steps in nbox 64-channel boxes.
+struct Window {
+    int ws, ks, nbox;
+};
+
+__host__ __device__ inline Window window_of(int ch0, int dm)
+{
+    Window w;
+    w.ws = ch0 & ~15;
+    const int we = (ch0 + dm + 15) & ~15;
+    w.ks = (we - w.ws) / 16;
+    w.nbox = (we - w.ws + 63) / 64;
+    return w;
+}
+
+// Per role: C padded to 16 (Cr), split into nch chunks of at most 256 columns.
+struct Chunks {
+    int Cr, nch, chunk0;   // chunk0 = size of every chunk but the last (a multiple of 16)
+};
+
+__host__ __device__ inline Chunks chunks_of(int C)
+{
+    Chunks k;
+    k.Cr = (C + 15) & ~15;
+    k.nch = (k.Cr + kChunkMax - 1) / kChunkMax;
+    k.chunk0 = ((k.Cr + k.nch - 1) / k.nch + 15) & ~15;
+    return k;
+}
+
+struct TcLayout {
+    int Cpad;               // row stride of the packed centroid arrays (all roles)
+    int nbox_max, cr_max;
+    size_t b_bytes, x_stage, n2_off, bars_off, total;
+};
+
+TcLayout tc_layout(const KmArgs &a)
+{
+    TcLayout L{};
+    L.Cpad = (a.Cs + 15) & ~15;
+    size_t bmax = 0;
+    int nbm = 1, crm = 16;
+    for (int r = 0; r < a.nroles; ++r) {
+        const RoleDesc &R = a.role[a.role0 + r];
+        const Window w = window_of(R.ch0, R.dm);
+        const Chunks k = chunks_of(R.C);
+        nbm = w.nbox > nbm ? w.nbox : nbm;
+        crm = k.Cr > crm ? k.Cr : crm;
+        const size_t b = (size_t)2 * w.nbox * k.Cr * 128;
+        bmax = b > bmax ? b : bmax;
+    }
+    L.nbox_max = nbm;
+    L.cr_max = crm;
+    L.b_bytes = bmax;
+    L.x_stage = (size_t)nbm * kTile * 128;
+    L.n2_off = L.b_bytes + 2 * L.x_stage;
+    L.bars_off = (L.n2_off + (size_t)(crm + 4) * 4 + 15) & ~size_t(15);
+    L.total = L.bars_off + sizeof(TcBars) + 16 + 1024;
+    return L;
+}
+
+struct TcParams {
+    int TT;                 // token tiles per problem
+    int Cpad;               // row stride of cent_bf / cn2p
+    long long n_units;      // problems x TT
+    unsigned x_off, x_stage, n2_off, bars_off;   // shared-memory offsets
+};
+
+// A bounded wait without the abort check, for draining copies and MMAs already issued.
+__device__ __forceinline__ void drain_wait(uint64_t *b, uint32_t parity)
+{
+    const unsigned long long t0 = global_ns();
+    while (!bar_test(b, parity) && global_ns() - t0 < kTcWaitNs) __nanosleep(64);
+}
+
+// Coefficient of |x| max|mu| in the bound on |score - S_c| for a window of ks MMA steps:
+// 2 x (bf16 split remainder 2^-16 + fp32 accumulation, taken as 2^-19 of sum |x_i mu_i|
+// per MMA step over the hi and the lo steps with a 1% allowance) + 4 x 2^-22 for the
+// rounding of the score itself.
+__device__ __forceinline__ float bound_coef(int ks)
+{
+    return 2.f * (0x1p-16f + 2.02f * (float)ks * 0x1p-19f) + 4.f * 0x1p-22f;
+}
+
+__device__ __forceinline__ void bulk_copy(uint32_t dst, const void *src, uint32_t bytes, uint64_t *bar)
+{
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// ------------------------------------------------------------------------- pack
+// One block per problem: the bf16 hi / lo split of every centroid row over all d channels
+// (zero outside the role's channel range and for padded rows), |mu|^2 in fp32 with +inf
+// for padded rows, then max |mu| (rounded up) and the largest slack term.
+__global__ void __launch_bounds__(256) km_pack_kernel(KmArgs a, int Cpad)
+{
+    const int p = blockIdx.x;
+    const int r = p % a.nroles, bh = p / a.nroles;
+    const RoleDesc &R = a.role[a.role0 + r];
+    __nv_bfloat16 *hi = a.cent_bf + (size_t)p * 2 * Cpad * a.d;
+    __nv_bfloat16 *lo = hi + (size_t)Cpad * a.d;
+    for (int idx = threadIdx.x; idx < Cpad * a.d; idx += blockDim.x) {
+        const int c = idx / a.d, i = idx - c * a.d;
+        float h = 0.f, l = 0.f;
+        if (c < R.C && i >= R.ch0 && i < R.ch0 + R.dm) {
+            const double m = R.cent[((size_t)bh * R.C + c) * a.d + i];
+            const __nv_bfloat16 hb = __double2bfloat16(m);
+            const double rem = m - (double)__bfloat162float(hb);   // exact in binary64
+            h = __bfloat162float(hb);
+            l = __bfloat162float(__double2bfloat16(rem));
+        }
+        hi[idx] = __float2bfloat16(h);
+        lo[idx] = __float2bfloat16(l);
+    }
+    float *n2 = a.cn2p + (size_t)p * (Cpad + 4);
+    double mx = 0.0;
+    float msl = 0.f;
+    for (int c = threadIdx.x; c < Cpad; c += blockDim.x) {
+        if (c < R.C) {
+            const double *mu = R.cent + ((size_t)bh * R.C + c) * a.d + R.ch0;
+            double s = 0.0;
+            for (int i = 0; i < R.dm; ++i) s += mu[i] * mu[i];
+            mx = fmax(mx, s);
+            n2[c] = a.cnrm2[(size_t)p * a.Cs + c];
+            msl = fmaxf(msl, a.cslack[(size_t)p * a.Cs + c]);
+        } else {
+            n2[c] = INFINITY;
+        }
+    }
+    __shared__ double smx[256];
+    __shared__ float ssl[256];
+    smx[threadIdx.x] = mx;
+    ssl[threadIdx.x] = msl;
+    __syncthreads();
+    for (int o = 128; o; o >>= 1) {
+        if (threadIdx.x < o) {
+            smx[threadIdx.x] = fmax(smx[threadIdx.x], smx[threadIdx.x + o]);
+            ssl[threadIdx.x] = fmaxf(ssl[threadIdx.x], ssl[threadIdx.x + o]);
+        }
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) {
+        // sqrt of the binary64 sum (itself within ~1e-14 of |mu|^2), rounded up, plus margin
+        n2[Cpad] = __double2float_ru(sqrt(smx[0]) * (1.0 + 0x1p-20));
+        n2[Cpad + 1] = ssl[0];
+        n2[Cpad + 2] = 0.f;
+        n2[Cpad + 3] = 0.f;
+    }
+}
+
+// ------------------------------------------------------------------------- assignment
+__global__ void __launch_bounds__(kThreadsTc, 1)
+    km_assign_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                        const __grid_constant__ CUtensorMap tmB, KmArgs a, TcParams t)
+{
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    unsigned char *sm = reinterpret_cast<unsigned char *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    TcBars *bars = reinterpret_cast<TcBars *>(sm + t.bars_off);
+    int *misc = reinterpret_cast<int *>(sm + t.bars_off + sizeof(TcBars));
+    volatile int *abort_flag = misc;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(misc + 1);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t sbase = smem_u32(sm);
+    const long long ub = t.n_units * blockIdx.x / gridDim.x;
+    const long long ue = t.n_units * (blockIdx.x + 1) / gridDim.x;
+
+    if (threadIdx.x == 0) {
+        misc[0] = 0;
+        bar_init(&bars->b_full, 1);
+        bar_init(&bars->b_empty, 1 + 4);
+        for (int s = 0; s < 2; ++s) {
+            bar_init(&bars->x_full[s], 1);
+            bar_init(&bars->x_empty[s], 1 + 4);
+            bar_init(&bars->acc_full[s], 1);
+            bar_init(&bars->acc_empty[s], 4);
+        }
+        bar_init(&bars->drain, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(tmem_slot)),
+                     "r"(kTmemColsTc)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int cur_p = -1;
+            uint32_t nb = 0, xi = 0;
+            for (long long u = ub; u < ue && !*abort_flag; ++u) {
+                const int p = (int)(u / t.TT), tile = (int)(u % t.TT);
+                const int ra = a.role0 + p % a.nroles, bh = p / a.nroles;
+                const RoleDesc &R = a.role[ra];
+                const Window w = window_of(R.ch0, R.dm);
+                if (p != cur_p) {
+                    const Chunks k = chunks_of(R.C);
+                    if (nb > 0 && !bar_wait(&bars->b_empty, (nb - 1) & 1, abort_flag, a.status)) break;
+                    bar_expect_tx(&bars->b_full, 2u * w.nbox * k.Cr * 128 + (uint32_t)(k.Cr + 4) * 4);
+                    for (int sp = 0; sp < 2; ++sp)
+                        for (int b = 0; b < w.nbox; ++b)
+                            for (int c0 = 0; c0 < k.Cr; c0 += kBoxRows)
+                                tma_tile2d(sbase + ((sp * w.nbox + b) * k.Cr + c0) * 128, &tmB, w.ws + 64 * b,
+                                           (p * 2 + sp) * t.Cpad + c0, &bars->b_full);
+                    const float *n2g = a.cn2p + (size_t)p * (t.Cpad + 4);
+                    bulk_copy(sbase + t.n2_off, n2g, (uint32_t)k.Cr * 4, &bars->b_full);
+                    bulk_copy(sbase + t.n2_off + k.Cr * 4, n2g + t.Cpad, 16, &bars->b_full);
+                    cur_p = p;
+                    ++nb;
+                }
+                const int s = xi & 1;
+                if (!bar_wait(&bars->x_empty[s], ((xi >> 1) & 1) ^ 1, abort_flag, a.status)) break;
+                bar_expect_tx(&bars->x_full[s], (uint32_t)w.nbox * kTile * 128);
+                const CUtensorMap *tm = ra == 0 ? &tmQ : &tmK;
+                for (int b = 0; b < w.nbox; ++b)
+                    tma_tile2d(sbase + t.x_off + s * t.x_stage + b * (kTile * 128), tm, w.ws + 64 * b,
+                               bh * a.N + tile * kTile, &bars->x_full[s]);
+                ++xi;
+            }
+            // copies still in flight complete before the CTA exits
+            if (nb > 0) drain_wait(&bars->b_full, (nb - 1) & 1);
+            for (uint32_t k = xi > 2 ? xi - 2 : 0; k < xi; ++k) drain_wait(&bars->x_full[k & 1], (k >> 1) & 1);
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issue
+        if (lane == 0) {
+            int cur_p = -1;
+            uint32_t nb = 0, xi = 0, g = 0;
+            for (long long u = ub; u < ue && !*abort_flag; ++u) {
+                const int p = (int)(u / t.TT);
+                const RoleDesc &R = a.role[a.role0 + p % a.nroles];
+                const Window w = window_of(R.ch0, R.dm);
+                const Chunks k = chunks_of(R.C);
+                if (p != cur_p) {
+                    if (!bar_wait(&bars->b_full, nb & 1, abort_flag, a.status)) break;
+                    ++nb;
+                    cur_p = p;
+                }
+                const int s = xi & 1;
+                if (!bar_wait(&bars->x_full[s], (xi >> 1) & 1, abort_flag, a.status)) break;
+                tc_fence_after();
+                const uint32_t xa = sbase + t.x_off + s * t.x_stage;
+                bool ok = true;
+                for (int ch = 0; ch < k.nch; ++ch) {
+                    const int n0 = ch * k.chunk0, nc = min(k.chunk0, k.Cr - n0);
+                    const int buf = g & 1;
+                    if (!bar_wait(&bars->acc_empty[buf], ((g >> 1) & 1) ^ 1, abort_flag, a.status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t idesc = f16_idesc(kTile, nc, false);
+                    const uint32_t dst = tmem + buf * kChunkMax;
+                    for (int sp = 0; sp < 2; ++sp)
+                        for (int kk = 0; kk < w.ks; ++kk) {
+                            const uint64_t ad = sw128_desc(xa + (kk >> 2) * (kTile * 128) + (kk & 3) * 32, 16, 1024);
+                            const uint64_t bd = sw128_desc(
+                                sbase + ((sp * w.nbox + (kk >> 2)) * k.Cr + n0) * 128 + (kk & 3) * 32, 16, 1024);
+                            mma_bf16(dst, ad, bd, idesc, (sp | kk) != 0 ? 1u : 0u);
+                        }
+                    mma_commit(&bars->acc_full[buf]);
+                    ++g;
+                }
+                if (!ok) break;
+                mma_commit(&bars->x_empty[s]);
+                ++xi;
+                // the CTA's last unit of this problem releases the centroids
+                if (u + 1 == ue || (int)((u + 1) / t.TT) != p) mma_commit(&bars->b_empty);
+            }
+            // every issued MMA completes before TMEM is freed
+            mma_commit(&bars->drain);
+            drain_wait(&bars->drain, 0);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ epilogue (warps 2-5)
+        const int q4 = warp & 3;                       // TMEM lane quarter of this warp
+        const int row = q4 * 32 + lane;                // token row of the tile = TMEM lane
+        const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
+        const float *n2s = reinterpret_cast<const float *>(sm + t.n2_off);
+        int cur_p = -1;
+        uint32_t nb = 0, xi = 0, g = 0;
+        float maxnm = 0.f, maxsl = 0.f;
+        for (long long u = ub; u < ue; ++u) {
+            if (warp_aborted(abort_flag)) break;
+            const int p = (int)(u / t.TT), tile = (int)(u % t.TT);
+            const int bh = p / a.nroles;
+            const RoleDesc &R = a.role[a.role0 + p % a.nroles];
+            const Window w = window_of(R.ch0, R.dm);
+            const Chunks k = chunks_of(R.C);
+            if (p != cur_p) {
+                if (!warp_wait(&bars->b_full, nb & 1, abort_flag, a.status)) break;
+                ++nb;
+                cur_p = p;
+                maxnm = n2s[k.Cr];
+                maxsl = n2s[k.Cr + 1];
+            }
+            const int s = xi & 1;
+            if (!warp_wait(&bars->x_full[s], (xi >> 1) & 1, abort_flag, a.status)) break;
+            // |x|^2 over the role's channels, read from the 128-byte swizzled tile
+            const unsigned char *xt = sm + t.x_off + s * t.x_stage;
+            const int lo_c = R.ch0 - w.ws, hi_c = lo_c + R.dm;   // window-relative range
+            float ss = 0.f;
+            for (int j = lo_c >> 3; j <= (hi_c - 1) >> 3; ++j) {
+                const uint4 v = *reinterpret_cast<const uint4 *>(
+                    xt + (j >> 3) * (kTile * 128) + row * 128 + (((j & 7) ^ (row & 7)) << 4));
+                const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int c = j * 8 + e;
+                    const float x = __uint_as_float((e & 1) ? (wv[e >> 1] & 0xFFFF0000u) : (wv[e >> 1] << 16));
+                    if (c >= lo_c && c < hi_c) ss = fmaf(x, x, ss);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) bar_arrive(&bars->x_empty[s]);
+            ++xi;
+            const float xn = sqrtf(ss) * (1.0f + 0x1p-12f);
+            const float E = fmaf(bound_coef(w.ks) * xn, maxnm, fmaf(0x1p-40f * xn, xn, maxsl));
+            float m1 = INFINITY, m2 = INFINITY;
+            int idx = 0;
+            bool ok = true;
+            for (int ch = 0; ch < k.nch; ++ch) {
+                const int n0 = ch * k.chunk0, nc = min(k.chunk0, k.Cr - n0);
+                const int buf = g & 1;
+                if (!warp_wait(&bars->acc_full[buf], (g >> 1) & 1, abort_flag, a.status)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                for (int c = 0; c < nc; c += 32) {
+                    float v[32];
+                    const uint32_t ta = tmem + lane_base + buf * kChunkMax + c;
+                    const bool two = c + 16 < nc;
+                    tmem_ld16(ta, v);
+                    if (two) tmem_ld16(ta + 16, v + 16);
+                    tmem_wait_ld();
+                    const float4 *n4 = reinterpret_cast<const float4 *>(n2s + n0 + c);
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        if (q < 4 || two) {
+                            const float4 nn = n4[q];
+                            const float nv[4] = {nn.x, nn.y, nn.z, nn.w};
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const float A = fmaf(-2.f, v[4 * q + e], nv[e]);
+                                m2 = fminf(m2, fmaxf(m1, A));
+                                if (A < m1) {
+                                    m1 = A;
+                                    idx = n0 + c + 4 * q + e;
+                                }
+                            }
+                        }
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) bar_arrive(&bars->acc_empty[buf]);
+                ++g;
+            }
+            if (!ok) break;
+            if (u + 1 == ue || (int)((u + 1) / t.TT) != p) {
+                __syncwarp();
+                if (lane == 0) bar_arrive(&bars->b_empty);
+            }
+            const int j = tile * kTile + row;
+            if (j < a.N) {
+                const bool sure = (m2 - m1) > (E + E) * (1.0f + 0x1p-20f);
+                R.assign[(size_t)bh * R.assign_bh + j] = sure ? (uint16_t)idx : kUnsureTc;
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemColsTc)
+                     : "memory");
+}
+
+}  // namespace
+
+bool km_assign_tc_supported(const KmArgs &a)
+{
+    if (!a.is_bf16 || (a.d != 64 && a.d != 128) || !a.cent_bf || !a.cn2p) return false;
+    return tc_layout(a).total <= (size_t)kSmemLimit;
+}
+
+cudaError_t km_pack(const KmArgs &a, cudaStream_t s)
+{
+    const TcLayout L = tc_layout(a);
+    km_pack_kernel<<<a.BH * a.nroles, 256, 0, s>>>(a, L.Cpad);
+    return cudaGetLastError();
+}
+
+cudaError_t km_assign_tc(const KmArgs &a, int num_sms, cudaStream_t s)
+{
+    const TcLayout L = tc_layout(a);
+    const int P = a.BH * a.nroles;
+    CUtensorMap tq, tk, tb;
+    const long long rows = (long long)a.BH * a.N;
+    const bool has_q = a.role0 == 0, has_k = a.role0 + a.nroles > 1;
+    const void *xq = has_q ? a.role[0].X : a.role[a.role0].X;
+    const void *xk = has_k ? a.role[a.role0 + a.nroles - 1].X : xq;
+    if (!bf16_tile_map(&tq, has_q ? xq : xk, rows, a.d, 64, kTile) ||
+        !bf16_tile_map(&tk, xk, rows, a.d, 64, kTile) ||
+        !bf16_tile_map(&tb, a.cent_bf, (long long)P * 2 * L.Cpad, a.d, 64, kBoxRows))
+        return cudaErrorInvalidValue;
+    TcParams t;
+    t.TT = (a.N + kTile - 1) / kTile;
+    t.Cpad = L.Cpad;
+    t.n_units = (long long)P * t.TT;
+    t.x_off = (unsigned)L.b_bytes;
+    t.x_stage = (unsigned)L.x_stage;
+    t.n2_off = (unsigned)L.n2_off;
+    t.bars_off = (unsigned)L.bars_off;
+    // more than half of the SM's shared memory: one CTA (and one 512-column TMEM
+    // allocation) per SM
+    const size_t smem = L.total > (size_t)kSmemLimit / 2 + 1024 ? L.total : (size_t)kSmemLimit / 2 + 1024;
+    cudaFuncSetAttribute(km_assign_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const int grid = (int)(t.n_units < num_sms ? t.n_units : num_sms);
+    km_assign_tc_kernel<<<grid, kThreadsTc, smem, s>>>(tq, tk, tb, a, t);
+    return cudaGetLastError();
+}
+
+}  // namespace scope

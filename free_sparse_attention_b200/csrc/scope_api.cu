@@ -90,6 +90,8 @@ KmArgs km_base(const scope_params &p, const WsLayout &L, void *ws)
     a.perm = at<int32_t>(ws, L.perm);
     a.off = at<int32_t>(ws, L.off);
     a.chunk_hist = at<int32_t>(ws, L.chunk_hist);
+    a.cent_bf = at<__nv_bfloat16>(ws, L.cent_bf);
+    a.cn2p = at<float>(ws, L.cn2p);
     a.nchunk = (int)D.nchunk;
     a.status = at<int32_t>(ws, L.status);
     return a;
@@ -249,6 +251,9 @@ WsLayout ws_layout(const scope_params &p)
     L.perm = take(sizeof(int32_t) * D.P * D.N);
     L.off = take(sizeof(int32_t) * D.P * (D.Cs + 1));
     L.chunk_hist = take(sizeof(int32_t) * D.P * D.nchunk * D.Cs);
+    const long long Cpad = (D.Cs + 15) / 16 * 16;
+    L.cent_bf = take(sizeof(__nv_bfloat16) * D.P * 2 * Cpad * D.d);
+    L.cn2p = take(sizeof(float) * D.P * (Cpad + 4));
     L.q_cent = take(sizeof(double) * D.BH * p.Cq * p.d);
     L.q_assign = take(sizeof(uint16_t) * D.BH * D.N);
     L.q_sizes = take(sizeof(int32_t) * D.BH * p.Cq);
