@@ -37,6 +37,7 @@ struct KmArgs {
     int is_bf16;
     // per-problem scratch (problem p = bh*nroles + r)
     float *cent32;        // [P, ds, Cs] fp32 centroids, transposed
+    double *cent64T;      // [P, ds, Cs] binary64 centroids, transposed (exact re-decisions)
     float *cnorm;         // [P, Cs]  ||mu32_c|| rounded up
     float *cnrm2;         // [P, Cs]  ||mu_c||^2 rounded to fp32
     float *cslack;        // [P, Cs]  2^-22 ||mu_c||^2 rounded up (error-bound term)
@@ -54,7 +55,7 @@ struct KmArgs {
 // Workspace layout (byte offsets); computed identically by every entry point.
 struct WsLayout {
     size_t status, counters;
-    size_t cent32, cnorm, cnrm2, cslack, perm, off, chunk_hist, cent_bf, cn2p;
+    size_t cent32, cent64T, cnorm, cnrm2, cslack, perm, off, chunk_hist, cent_bf, cn2p;
     size_t q_cent, q_assign, q_sizes, k_cent, k_codes, k_sizes;
     size_t topp, base, khead, final_cnt, mask, sel_state;
     size_t q_perm, q_off, q_hist, work_items, attn_counter, key_lists;

@@ -37,24 +37,14 @@ __device__ __forceinline__ const RoleDesc &role_of(const KmArgs &a, int p, int &
     return a.role[a.role0 + r];
 }
 
-// Squared distance in binary64, channels in order, separate multiply and add.
-__device__ __forceinline__ double sqdist64(const void *X, long long xrow, int is_bf16,
-                                           const double *mu, int dm)
-{
-    double acc = 0.0;
-    for (int i = 0; i < dm; ++i) {
-        double diff = __dsub_rn((double)load_x(X, xrow + i, is_bf16), mu[i]);
-        acc = __dadd_rn(acc, __dmul_rn(diff, diff));
-    }
-    return acc;
-}
-
-// fp32 copy, norms and the error-bound term of one centroid row (cent64 has dm
-// values, all written before the caller's barrier).  Thread i handles channel i.
+// fp32 and binary64 transposed copies, norms and the error-bound term of one centroid
+// row (cent64 has dm values, all written before the caller's barrier).  Thread i
+// handles channel i.
 __device__ void finalize_row(const KmArgs &a, int p, int c, const double *cent64, int dm, int i)
 {
     float *cent32T = a.cent32 + (size_t)p * a.Cs * a.ds;
     cent32T[(size_t)i * a.Cs + c] = __double2float_rn(cent64[i]);
+    a.cent64T[(size_t)p * a.Cs * a.ds + (size_t)i * a.Cs + c] = cent64[i];
     if (i == 0) {
         double n2 = 0.0, n32 = 0.0;
         for (int k = 0; k < dm; ++k) {
@@ -239,15 +229,20 @@ __global__ void __launch_bounds__(kAssignThreads) km_assign_fast_kernel(KmArgs a
 
 // ------------------------------------------------------------------------- exact assignment
 // One warp per group of 32 tokens (grid-stride); every unsure token is re-decided in
-// binary64 against all centroids, lanes striding over the centroids.
-__global__ void __launch_bounds__(256) km_assign_exact_kernel(KmArgs a)
+// binary64 against all centroids.  The token's channels go to shared memory; lane l
+// takes centroids l, l+32, ... two at a time, reading the channel-major binary64 copy
+// (consecutive lanes, consecutive centroids), and sums the squared differences in
+// channel order with one rounding per operation, as the definition is evaluated.
+constexpr int kExactWarps = 8;
+
+__global__ void __launch_bounds__(kExactWarps * 32) km_assign_exact_kernel(KmArgs a)
 {
-    const int lane = threadIdx.x & 31;
+    __shared__ double xs[kExactWarps][128];
+    const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
     const int ngroups = (a.N + 31) / 32;
     const long long total = (long long)a.BH * a.nroles * ngroups;
-    const long long nwarps = (long long)gridDim.x * (blockDim.x / 32);
-    for (long long g = (long long)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32; g < total;
-         g += nwarps) {
+    const long long nwarps = (long long)gridDim.x * kExactWarps;
+    for (long long g = (long long)blockIdx.x * kExactWarps + wib; g < total; g += nwarps) {
         const int p = (int)(g / ngroups);
         int bh, r;
         const RoleDesc &R = role_of(a, p, bh, r);
@@ -255,19 +250,34 @@ __global__ void __launch_bounds__(256) km_assign_exact_kernel(KmArgs a)
         uint16_t *asg = R.assign + (size_t)bh * R.assign_bh;
         bool unsure = j < a.N && asg[j] == kUnsure;
         unsigned todo = __ballot_sync(0xffffffffu, unsure);
+        const double *muT = a.cent64T + (size_t)p * a.Cs * a.ds;
         while (todo) {
             const int src = __ffs(todo) - 1;
             todo &= todo - 1;
             const int jj = (int)(g % ngroups) * 32 + src;
             const long long xrow = ((long long)bh * a.N + jj) * a.d + R.ch0;
+            for (int i = lane; i < R.dm; i += 32) xs[wib][i] = (double)load_x(R.X, xrow + i, a.is_bf16);
+            __syncwarp();
             double best = INFINITY;
             int bi = 0x7fffffff;
-            for (int c = lane; c < R.C; c += 32) {
-                const double *mu = R.cent + ((size_t)bh * R.C + c) * a.d + R.ch0;
-                double dd = sqdist64(R.X, xrow, a.is_bf16, mu, R.dm);
-                if (dd < best) {
-                    best = dd;
+            for (int c = lane; c < R.C; c += 64) {
+                const bool two = c + 32 < R.C;
+                const int c2 = two ? c + 32 : c;
+                double d0 = 0.0, d1 = 0.0;
+                for (int i = 0; i < R.dm; ++i) {
+                    const double x = xs[wib][i];
+                    const double e0 = __dsub_rn(x, muT[(size_t)i * a.Cs + c]);
+                    const double e1 = __dsub_rn(x, muT[(size_t)i * a.Cs + c2]);
+                    d0 = __dadd_rn(d0, __dmul_rn(e0, e0));
+                    d1 = __dadd_rn(d1, __dmul_rn(e1, e1));
+                }
+                if (d0 < best) {
+                    best = d0;
                     bi = c;
+                }
+                if (two && d1 < best) {
+                    best = d1;
+                    bi = c2;
                 }
             }
             for (int off = 16; off; off >>= 1) {
@@ -279,6 +289,7 @@ __global__ void __launch_bounds__(256) km_assign_exact_kernel(KmArgs a)
                 }
             }
             if (lane == 0) asg[jj] = (uint16_t)bi;
+            __syncwarp();
         }
     }
 }
@@ -493,7 +504,7 @@ cudaError_t km_run(KmArgs a, int iters, cudaStream_t s)
         } else {
             km_assign_fast_kernel<<<dim3((a.N + kTok - 1) / kTok, P), kAssignThreads, fsm, s>>>(a);
         }
-        km_assign_exact_kernel<<<sms * 4, 256, 0, s>>>(a);
+        km_assign_exact_kernel<<<sms * 4, kExactWarps * 32, 0, s>>>(a);
         cudaError_t e = sort_by_cluster(a, s);
         if (e != cudaSuccess) return e;
         km_update_kernel<<<dim3(gb, P), 128, 0, s>>>(a);

@@ -10,8 +10,9 @@
 //     channel range; the centroid matrix is zero outside the range, so channels of other
 //     subspaces contribute exactly nothing.
 //   * each binary64 centroid is split as mu = hi + lo + r with hi = bf16(mu),
-//     lo = bf16(mu - hi), |r| <= 2^-16 |mu|; both halves accumulate into one TMEM
-//     accumulator (x.hi + x.lo), products being exact in fp32.
+//     lo = bf16(mu - hi), |r| <= 2^-16 |mu| (the largest |r| of the centroid set enters
+//     the bound); both halves accumulate into one TMEM accumulator (x.hi + x.lo),
+//     products being exact in fp32.
 //   * the epilogue (one thread per token = TMEM lane) keeps the smallest and the
 //     second-smallest fp32 score and the winner.  The winner is certain when the gap
 //     exceeds twice a rigorous bound on |score - S_c| (the bf16 split remainder, the
@@ -24,7 +25,8 @@
 //   warp 0     TMA producer: the problem's centroid matrix (hi, lo) and |mu|^2 row once
 //              per problem, the token tile into a 2-deep ring
 //   warp 1     TMEM allocation and MMA issue (one thread)
-//   warps 2-5  epilogue: token norms from the shared-memory tile, TMEM loads, argmin
+//   warps 2-9  epilogue, two warpgroups splitting every chunk's columns: token norms
+//              from the shared-memory tile, TMEM loads, running minima, certification
 // The centroids are split in chunks of at most 256 columns, double-buffered in TMEM
 // (2 x 256 columns), so the epilogue of one chunk overlaps the MMAs of the next.
 // Every mbarrier wait gives up after ~4 s, sets a status bit and lets the CTA drain.
@@ -37,7 +39,7 @@ namespace scope {
 namespace {
 
 constexpr int kTile = 128;             // tokens per unit (TMEM lanes)
-constexpr int kThreadsTc = 192;        // 6 warps
+constexpr int kThreadsTc = 320;        // 10 warps
 constexpr int kChunkMax = 256;         // centroid columns per TMEM buffer
 constexpr uint32_t kTmemColsTc = 512;  // two accumulator buffers
 constexpr uint16_t kUnsureTc = 0xFFFF;
@@ -48,6 +50,7 @@ struct __align__(8) TcBars {
     uint64_t b_full, b_empty;
     uint64_t x_full[2], x_empty[2];
     uint64_t acc_full[2], acc_empty[2];
+    uint64_t mg_full[2], mg_empty[2];   // epilogue warpgroup 1 -> 0 hand-off slots
     uint64_t drain;
 };
 
@@ -83,7 +86,7 @@ __host__ __device__ inline Chunks chunks_of(int C)
 struct TcLayout {
     int Cpad;               // row stride of the packed centroid arrays (all roles)
     int nbox_max, cr_max;
-    size_t b_bytes, x_stage, n2_off, bars_off, total;
+    size_t b_bytes, x_stage, n2_off, merge_off, bars_off, total;
 };
 
 TcLayout tc_layout(const KmArgs &a)
@@ -106,7 +109,8 @@ TcLayout tc_layout(const KmArgs &a)
     L.b_bytes = bmax;
     L.x_stage = (size_t)nbm * kTile * 128;
     L.n2_off = L.b_bytes + 2 * L.x_stage;
-    L.bars_off = (L.n2_off + (size_t)(crm + 4) * 4 + 15) & ~size_t(15);
+    L.merge_off = (L.n2_off + (size_t)(crm + 4) * 4 + 15) & ~size_t(15);
+    L.bars_off = L.merge_off + (size_t)2 * kTile * 16;
     L.total = L.bars_off + sizeof(TcBars) + 16 + 1024;
     return L;
 }
@@ -115,7 +119,7 @@ struct TcParams {
     int TT;                 // token tiles per problem
     int Cpad;               // row stride of cent_bf / cn2p
     long long n_units;      // problems x TT
-    unsigned x_off, x_stage, n2_off, bars_off;   // shared-memory offsets
+    unsigned x_off, x_stage, n2_off, merge_off, bars_off;   // shared-memory offsets
 };
 
 // A bounded wait without the abort check, for draining copies and MMAs already issued.
@@ -125,13 +129,20 @@ __device__ __forceinline__ void drain_wait(uint64_t *b, uint32_t parity)
     while (!bar_test(b, parity) && global_ns() - t0 < kTcWaitNs) __nanosleep(64);
 }
 
-// Coefficient of |x| max|mu| in the bound on |score - S_c| for a window of ks MMA steps:
-// 2 x (bf16 split remainder 2^-16 + fp32 accumulation, taken as 2^-19 of sum |x_i mu_i|
-// per MMA step over the hi and the lo steps with a 1% allowance) + 4 x 2^-22 for the
-// rounding of the score itself.
-__device__ __forceinline__ float bound_coef(int ks)
+// Bound on |score - S_c| for a token of norm |x| <= xn, with M = max |mu_c|,
+// Rm = max |mu_c - hi_c - lo_c| and ks MMA steps per half:
+//   2 |x.r_c|                      <= 2 xn Rm               (Cauchy-Schwarz)
+//   2 x fp32 accumulation error     <= 2 (2 ks) 2^-21 sum |x_i hi_i| + |x_i lo_i|
+//                                   <= 4 ks 2^-21 (1 + 2^-7) xn M
+//   rounding of the score           <= 2^-21 xn M  (+ the |mu|^2 part, in the slack)
+//   |mu|^2 to fp32, reference sum   <= slack_max + 2^-40 xn^2
+// The accumulation term allows 4 units of 2^-23 of the running magnitude per MMA step;
+// the worst error measured on this hardware over 16 steps of random, wide-exponent and
+// cancelling operands was 11.2 units in total, against the 64 allowed.
+__device__ __forceinline__ float bound_E(int ks, float xn, float M, float Rm, float slack)
 {
-    return 2.f * (0x1p-16f + 2.02f * (float)ks * 0x1p-19f) + 4.f * 0x1p-22f;
+    const float coef = (4.f * (float)ks * 1.0079f + 1.f) * 0x1p-21f;
+    return fmaf(xn, fmaf(coef, M, 2.f * Rm), fmaf(0x1p-40f * xn, xn, slack));
 }
 
 __device__ __forceinline__ void bulk_copy(uint32_t dst, const void *src, uint32_t bytes, uint64_t *bar)
@@ -167,37 +178,48 @@ __global__ void __launch_bounds__(256) km_pack_kernel(KmArgs a, int Cpad)
         lo[idx] = __float2bfloat16(l);
     }
     float *n2 = a.cn2p + (size_t)p * (Cpad + 4);
-    double mx = 0.0;
+    double mx = 0.0, mr = 0.0;
     float msl = 0.f;
     for (int c = threadIdx.x; c < Cpad; c += blockDim.x) {
         if (c < R.C) {
             const double *mu = R.cent + ((size_t)bh * R.C + c) * a.d + R.ch0;
-            double s = 0.0;
-            for (int i = 0; i < R.dm; ++i) s += mu[i] * mu[i];
+            double s = 0.0, rr = 0.0;
+            for (int i = 0; i < R.dm; ++i) {
+                const double m = mu[i];
+                const double h = (double)__bfloat162float(__double2bfloat16(m));
+                const double rem = m - h;
+                const double res = rem - (double)__bfloat162float(__double2bfloat16(rem));  // exact
+                s += m * m;
+                rr += res * res;
+            }
             mx = fmax(mx, s);
+            mr = fmax(mr, rr);
             n2[c] = a.cnrm2[(size_t)p * a.Cs + c];
             msl = fmaxf(msl, a.cslack[(size_t)p * a.Cs + c]);
         } else {
             n2[c] = INFINITY;
         }
     }
-    __shared__ double smx[256];
+    __shared__ double smx[256], smr[256];
     __shared__ float ssl[256];
     smx[threadIdx.x] = mx;
+    smr[threadIdx.x] = mr;
     ssl[threadIdx.x] = msl;
     __syncthreads();
     for (int o = 128; o; o >>= 1) {
         if (threadIdx.x < o) {
             smx[threadIdx.x] = fmax(smx[threadIdx.x], smx[threadIdx.x + o]);
+            smr[threadIdx.x] = fmax(smr[threadIdx.x], smr[threadIdx.x + o]);
             ssl[threadIdx.x] = fmaxf(ssl[threadIdx.x], ssl[threadIdx.x + o]);
         }
         __syncthreads();
     }
     if (threadIdx.x == 0) {
-        // sqrt of the binary64 sum (itself within ~1e-14 of |mu|^2), rounded up, plus margin
+        // square roots of binary64 sums of squares (each within ~1e-14 of the exact
+        // value), rounded up with a margin: max |mu_c| and max |mu_c - hi_c - lo_c|
         n2[Cpad] = __double2float_ru(sqrt(smx[0]) * (1.0 + 0x1p-20));
         n2[Cpad + 1] = ssl[0];
-        n2[Cpad + 2] = 0.f;
+        n2[Cpad + 2] = __double2float_ru(sqrt(smr[0]) * (1.0 + 0x1p-20));
         n2[Cpad + 3] = 0.f;
     }
 }
@@ -222,12 +244,14 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     if (threadIdx.x == 0) {
         misc[0] = 0;
         bar_init(&bars->b_full, 1);
-        bar_init(&bars->b_empty, 1 + 4);
+        bar_init(&bars->b_empty, 1 + 8);
         for (int s = 0; s < 2; ++s) {
             bar_init(&bars->x_full[s], 1);
             bar_init(&bars->x_empty[s], 1 + 4);
             bar_init(&bars->acc_full[s], 1);
-            bar_init(&bars->acc_empty[s], 4);
+            bar_init(&bars->acc_empty[s], 8);
+            bar_init(&bars->mg_full[s], 4);
+            bar_init(&bars->mg_empty[s], 4);
         }
         bar_init(&bars->drain, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -335,14 +359,25 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
         }
         __syncwarp();
     } else {
-        // ------------------------------------------------------------ epilogue (warps 2-5)
+        // ------------------------------------------------------------ epilogue (warps 2-9)
+        // Two warpgroups share every chunk: warpgroup e takes the 16-column groups
+        // g = e, e+2, ... (two at a time, one TMEM wait per pair, one running minimum
+        // pair per group slot so consecutive columns do not form one dependency chain).
+        // Warpgroup 1 also computes the token norms and hands its (min, second min,
+        // winner, norm) per token to warpgroup 0 through a double-buffered slot; warpgroup
+        // 0 merges, certifies and writes the assignment.
+        const int e = (warp - 2) >> 2;                 // epilogue warpgroup
         const int q4 = warp & 3;                       // TMEM lane quarter of this warp
         const int row = q4 * 32 + lane;                // token row of the tile = TMEM lane
         const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
         const float *n2s = reinterpret_cast<const float *>(sm + t.n2_off);
+        float *mg_m1 = reinterpret_cast<float *>(sm + t.merge_off);   // [2][128]
+        float *mg_m2 = mg_m1 + 2 * kTile;
+        float *mg_xn = mg_m2 + 2 * kTile;
+        int *mg_ix = reinterpret_cast<int *>(mg_xn + 2 * kTile);
         int cur_p = -1;
         uint32_t nb = 0, xi = 0, g = 0;
-        float maxnm = 0.f, maxsl = 0.f;
+        float maxnm = 0.f, maxsl = 0.f, maxres = 0.f;
         for (long long u = ub; u < ue; ++u) {
             if (warp_aborted(abort_flag)) break;
             const int p = (int)(u / t.TT), tile = (int)(u % t.TT);
@@ -356,61 +391,78 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
                 cur_p = p;
                 maxnm = n2s[k.Cr];
                 maxsl = n2s[k.Cr + 1];
+                maxres = n2s[k.Cr + 2];
             }
             const int s = xi & 1;
-            if (!warp_wait(&bars->x_full[s], (xi >> 1) & 1, abort_flag, a.status)) break;
-            // |x|^2 over the role's channels, read from the 128-byte swizzled tile
-            const unsigned char *xt = sm + t.x_off + s * t.x_stage;
-            const int lo_c = R.ch0 - w.ws, hi_c = lo_c + R.dm;   // window-relative range
-            float ss = 0.f;
-            for (int j = lo_c >> 3; j <= (hi_c - 1) >> 3; ++j) {
-                const uint4 v = *reinterpret_cast<const uint4 *>(
-                    xt + (j >> 3) * (kTile * 128) + row * 128 + (((j & 7) ^ (row & 7)) << 4));
-                const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+            float xn = 0.f;
+            if (e == 1) {
+                if (!warp_wait(&bars->x_full[s], (xi >> 1) & 1, abort_flag, a.status)) break;
+                // |x| over the role's channels, read from the 128-byte swizzled tile
+                const unsigned char *xt = sm + t.x_off + s * t.x_stage;
+                const int lo_c = R.ch0 - w.ws, hi_c = lo_c + R.dm;   // window-relative range
+                float ss = 0.f;
+                for (int j = lo_c >> 3; j <= (hi_c - 1) >> 3; ++j) {
+                    const uint4 v = *reinterpret_cast<const uint4 *>(
+                        xt + (j >> 3) * (kTile * 128) + row * 128 + (((j & 7) ^ (row & 7)) << 4));
+                    const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const int c = j * 8 + e;
-                    const float x = __uint_as_float((e & 1) ? (wv[e >> 1] & 0xFFFF0000u) : (wv[e >> 1] << 16));
-                    if (c >= lo_c && c < hi_c) ss = fmaf(x, x, ss);
+                    for (int q = 0; q < 8; ++q) {
+                        const int c = j * 8 + q;
+                        const float x = __uint_as_float((q & 1) ? (wv[q >> 1] & 0xFFFF0000u) : (wv[q >> 1] << 16));
+                        if (c >= lo_c && c < hi_c) ss = fmaf(x, x, ss);
+                    }
                 }
+                __syncwarp();
+                if (lane == 0) bar_arrive(&bars->x_empty[s]);
+                xn = sqrtf(ss) * (1.0f + 0x1p-12f);
             }
-            __syncwarp();
-            if (lane == 0) bar_arrive(&bars->x_empty[s]);
             ++xi;
-            const float xn = sqrtf(ss) * (1.0f + 0x1p-12f);
-            const float E = fmaf(bound_coef(w.ks) * xn, maxnm, fmaf(0x1p-40f * xn, xn, maxsl));
-            float m1 = INFINITY, m2 = INFINITY;
-            int idx = 0;
+            // running (min, second min, winner) for the two group slots of this thread
+            float a1 = INFINITY, a2 = INFINITY, b1 = INFINITY, b2 = INFINITY;
+            int ai = 0, bi = 0;
             bool ok = true;
             for (int ch = 0; ch < k.nch; ++ch) {
                 const int n0 = ch * k.chunk0, nc = min(k.chunk0, k.Cr - n0);
+                const int ng = nc >> 4;                // 16-column groups in this chunk
                 const int buf = g & 1;
                 if (!warp_wait(&bars->acc_full[buf], (g >> 1) & 1, abort_flag, a.status)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                for (int c = 0; c < nc; c += 32) {
+                for (int gi = e; gi < ng; gi += 4) {
+                    const bool two = gi + 2 < ng;
                     float v[32];
-                    const uint32_t ta = tmem + lane_base + buf * kChunkMax + c;
-                    const bool two = c + 16 < nc;
+                    const uint32_t ta = tmem + lane_base + buf * kChunkMax + gi * 16;
                     tmem_ld16(ta, v);
-                    if (two) tmem_ld16(ta + 16, v + 16);
+                    if (two) tmem_ld16(ta + 32, v + 16);
                     tmem_wait_ld();
-                    const float4 *n4 = reinterpret_cast<const float4 *>(n2s + n0 + c);
+                    const int c0 = n0 + gi * 16;
+                    const float4 *na = reinterpret_cast<const float4 *>(n2s + c0);
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        if (q < 4 || two) {
-                            const float4 nn = n4[q];
+                    for (int q = 0; q < 4; ++q) {
+                        const float4 nn = na[q];
+                        const float nv[4] = {nn.x, nn.y, nn.z, nn.w};
+#pragma unroll
+                        for (int r = 0; r < 4; ++r) {
+                            const float A = fmaf(-2.f, v[4 * q + r], nv[r]);
+                            a2 = fminf(a2, fmaxf(a1, A));
+                            ai = A < a1 ? c0 + 4 * q + r : ai;
+                            a1 = fminf(a1, A);
+                        }
+                    }
+                    if (two) {
+                        const float4 *nb4 = reinterpret_cast<const float4 *>(n2s + c0 + 32);
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const float4 nn = nb4[q];
                             const float nv[4] = {nn.x, nn.y, nn.z, nn.w};
 #pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const float A = fmaf(-2.f, v[4 * q + e], nv[e]);
-                                m2 = fminf(m2, fmaxf(m1, A));
-                                if (A < m1) {
-                                    m1 = A;
-                                    idx = n0 + c + 4 * q + e;
-                                }
+                            for (int r = 0; r < 4; ++r) {
+                                const float A = fmaf(-2.f, v[16 + 4 * q + r], nv[r]);
+                                b2 = fminf(b2, fmaxf(b1, A));
+                                bi = A < b1 ? c0 + 32 + 4 * q + r : bi;
+                                b1 = fminf(b1, A);
                             }
                         }
                     }
@@ -425,10 +477,36 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
                 __syncwarp();
                 if (lane == 0) bar_arrive(&bars->b_empty);
             }
-            const int j = tile * kTile + row;
-            if (j < a.N) {
-                const bool sure = (m2 - m1) > (E + E) * (1.0f + 0x1p-20f);
-                R.assign[(size_t)bh * R.assign_bh + j] = sure ? (uint16_t)idx : kUnsureTc;
+            // merge the two slots (second smallest of a union = min of the second
+            // smallests and the larger of the smallests)
+            float m2 = fminf(fminf(a2, b2), fmaxf(a1, b1));
+            int idx = b1 < a1 ? bi : ai;
+            float m1 = fminf(a1, b1);
+            const uint32_t mi = (uint32_t)(u - ub), slot = mi & 1;
+            if (e == 1) {
+                if (!warp_wait(&bars->mg_empty[slot], ((mi >> 1) & 1) ^ 1, abort_flag, a.status)) break;
+                mg_m1[slot * kTile + row] = m1;
+                mg_m2[slot * kTile + row] = m2;
+                mg_xn[slot * kTile + row] = xn;
+                mg_ix[slot * kTile + row] = idx;
+                __syncwarp();
+                if (lane == 0) bar_arrive(&bars->mg_full[slot]);
+            } else {
+                if (!warp_wait(&bars->mg_full[slot], (mi >> 1) & 1, abort_flag, a.status)) break;
+                const float o1 = mg_m1[slot * kTile + row], o2 = mg_m2[slot * kTile + row];
+                xn = mg_xn[slot * kTile + row];
+                const int oi = mg_ix[slot * kTile + row];
+                __syncwarp();
+                if (lane == 0) bar_arrive(&bars->mg_empty[slot]);
+                m2 = fminf(fminf(m2, o2), fmaxf(m1, o1));
+                idx = o1 < m1 ? oi : idx;
+                m1 = fminf(m1, o1);
+                const int j = tile * kTile + row;
+                if (j < a.N) {
+                    const float E = bound_E(w.ks, xn, maxnm, maxres, maxsl);
+                    const bool sure = (m2 - m1) > (E + E) * (1.0f + 0x1p-20f);
+                    R.assign[(size_t)bh * R.assign_bh + j] = sure ? (uint16_t)idx : kUnsureTc;
+                }
             }
         }
     }
@@ -475,6 +553,7 @@ cudaError_t km_assign_tc(const KmArgs &a, int num_sms, cudaStream_t s)
     t.x_off = (unsigned)L.b_bytes;
     t.x_stage = (unsigned)L.x_stage;
     t.n2_off = (unsigned)L.n2_off;
+    t.merge_off = (unsigned)L.merge_off;
     t.bars_off = (unsigned)L.bars_off;
     // more than half of the SM's shared memory: one CTA (and one 512-column TMEM
     // allocation) per SM

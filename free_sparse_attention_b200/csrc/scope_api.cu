@@ -84,6 +84,7 @@ KmArgs km_base(const scope_params &p, const WsLayout &L, void *ws)
     a.d = p.d;
     a.is_bf16 = p.dtype == SCOPE_BF16;
     a.cent32 = at<float>(ws, L.cent32);
+    a.cent64T = at<double>(ws, L.cent64T);
     a.cnorm = at<float>(ws, L.cnorm);
     a.cnrm2 = at<float>(ws, L.cnrm2);
     a.cslack = at<float>(ws, L.cslack);
@@ -245,6 +246,7 @@ WsLayout ws_layout(const scope_params &p)
     L.status = take(sizeof(int32_t));
     L.counters = take(4 * sizeof(int32_t));
     L.cent32 = take(sizeof(float) * D.P * D.d * D.Cs);
+    L.cent64T = take(sizeof(double) * D.P * D.d * D.Cs);
     L.cnorm = take(sizeof(float) * D.P * D.Cs);
     L.cnrm2 = take(sizeof(float) * D.P * D.Cs);
     L.cslack = take(sizeof(float) * D.P * D.Cs);
