@@ -70,8 +70,10 @@ __global__ void __launch_bounds__(1024) attn_items_kernel(AttnArgs a)
 
 // Expands the selection bitmask of every (bh, cluster) that has queries into its
 // ascending list of selected key indices (the gather order of the attention kernel).
-// grid = BH*Cq units, 256 threads: one mask word per thread per chunk, block prefix sum
-// of the popcounts, then each thread writes its word's set bits.
+// grid = BH*Cq units, 256 threads.  Per chunk of 256 mask words: one word per thread,
+// a block prefix sum of the popcounts, then each warp writes its 32 words one word at
+// a time with lane l handling bit l, so consecutive selected keys go to consecutive
+// addresses (coalesced stores).
 __global__ void __launch_bounds__(256) attn_lists_kernel(AttnArgs a)
 {
     __shared__ int wsum[8];
@@ -81,6 +83,7 @@ __global__ void __launch_bounds__(256) attn_lists_kernel(AttnArgs a)
     if (off[c + 1] == off[c] || a.final_cnt[u] <= 0) return;
     const uint32_t *row = a.mask + (size_t)u * a.nw;
     int32_t *out = a.lists + (size_t)u * a.list_stride;
+    const uint32_t below = (1u << lane) - 1u;
     int base = 0;
     for (int w0 = 0; w0 < a.nw; w0 += 256) {
         const int w = w0 + tid;
@@ -102,10 +105,13 @@ __global__ void __launch_bounds__(256) attn_lists_kernel(AttnArgs a)
             before += k < w8 ? wsum[k] : 0;
             total += wsum[k];
         }
-        int pos = base + before + incl - pc;
-        while (bits) {
-            out[pos++] = w * 32 + __ffs(bits) - 1;
-            bits &= bits - 1;
+        const int excl = base + before + incl - pc;   // list position of this word's first key
+        const int wbase = (w0 + w8 * 32) * 32;        // key index of bit 0 of the warp's word 0
+#pragma unroll 4
+        for (int k = 0; k < 32; ++k) {
+            const uint32_t bk = __shfl_sync(0xffffffffu, bits, k);
+            const int pk = __shfl_sync(0xffffffffu, excl, k);
+            if ((bk >> lane) & 1u) out[pk + __popc(bk & below)] = wbase + k * 32 + lane;
         }
         base += total;
         __syncthreads();

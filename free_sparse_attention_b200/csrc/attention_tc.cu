@@ -5,7 +5,8 @@
 // review page, forward_implications[1]).  Queries are grouped by cluster, so one work
 // item = up to 256 queries of one (b, h, c) against the r_c keys of S_c.
 //
-// Per CTA (persistent, one per SM, static round-robin over the head-major work list):
+// Per CTA (persistent, one per SM; items of the head-major work list are handed out
+// dynamically, in order, through a global counter and a small shared-memory ring):
 //   warps 0-3 / 4-7  softmax + epilogue of Q tile 0 / 1 (thread r owns row r = TMEM lane r)
 //   warps 8-11       gather both Q tiles once per item and the selected K rows per key tile
 //   warps 12-13      gather the selected V rows per key tile
@@ -50,6 +51,8 @@ constexpr int kSoftmaxRegs = 192;  // 2 warpgroups x 128 threads x 192
 constexpr int kOtherRegs = 64;     //  + 2 warpgroups x 128 threads x 64 = 65536
 constexpr int kMaxStages = 8;
 constexpr uint32_t kTmemCols = 512;
+constexpr int kRing = 4;           // work items fetched ahead by the scheduler thread
+constexpr int kWarps = kThreads / 32;
 
 struct __align__(8) Bars {
     uint64_t q_full, q_empty;
@@ -59,6 +62,7 @@ struct __align__(8) Bars {
     uint64_t s_full[kQT][2], p_full[kQT][2], o_done[kQT][2];
     uint64_t o_free[kQT];  // epilogue has read O_q
     uint64_t turn[kQT];    // softmax warpgroups take turns: turn[q] = "Q tile q's softmax may run"
+    uint64_t item_full[kRing], item_empty[kRing];   // work-item ring (dynamic scheduler)
 };
 
 // Shared memory: two Q tiles, a K ring and a V ring (bf16, 128-byte swizzled, K-major).
@@ -118,6 +122,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             bar_init(&bars->o_free[q], 4);
             bar_init(&bars->turn[q], 4);
         }
+        for (int k = 0; k < kRing; ++k) {
+            bar_init(&bars->item_full[k], 1);
+            bar_init(&bars->item_empty[k], kWarps);
+        }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == 14) {
@@ -132,6 +140,34 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const int n_items = a.counter[0];
+    // Dynamic scheduler: one thread (lane 0 of warp 8) takes item indices from the global
+    // counter a.counter[1] in order and publishes them in a ring of kRing slots; every warp
+    // reads every slot (item k in slot k % kRing) and releases it.  -1 ends the work.
+    volatile int *ring = misc + 4;
+    auto fetch = [&](uint32_t k) -> bool {   // lane 0 of warp 8 only
+        const int slot = k % kRing;
+        if (!bar_wait(&bars->item_empty[slot], ((k / kRing) & 1) ^ 1, abort_flag, a.status)) return false;
+        const int it = atomicAdd(&a.counter[1], 1);
+        ring[slot] = it < n_items ? it : -1;
+        bar_arrive(&bars->item_full[slot]);
+        return true;
+    };
+    // item index k of this CTA for the calling warp; -1 = no more work or a failed wait
+    auto next_item = [&](uint32_t k) -> int {
+        const int slot = k % kRing;
+        if (!warp_wait(&bars->item_full[slot], (k / kRing) & 1, abort_flag, a.status)) return -1;
+        const int it = ring[slot];
+        __syncwarp();
+        if (lane == 0) bar_arrive(&bars->item_empty[slot]);
+        if (warp == 8 && it >= 0) {   // the scheduler thread fetches one item ahead
+            int ok = 1;
+            if (lane == 0) ok = fetch(k + 1) ? 1 : 0;
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) return -1;
+        }
+        return it;
+    };
+    if (warp == 8 && lane == 0) fetch(0);
 
     if (warp >= 8) {
     // warpgroups 2 and 3 give registers back (one setmaxnreg site for all their warps)
@@ -150,7 +186,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool active = lane < cnt * NB;
         const uint32_t kShareBytes = (uint32_t)cnt * 4 * D * 2;
         uint32_t stage_it = 0, q_it = 0;
-        for (int it = blockIdx.x; it < n_items && !warp_aborted(abort_flag); it += gridDim.x) {
+        for (uint32_t item_k = 0; !warp_aborted(abort_flag); ++item_k) {
+            const int it = next_item(item_k);
+            if (it < 0) break;
             const int4 item = a.items[it];
             const int bh = item.x, c = item.y, q0 = item.z, nq = item.w;
             const long long r = a.final_cnt[(size_t)bh * a.Cq + c];
@@ -229,7 +267,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (leader) mma_commit(b);
             __syncwarp();
         };
-        for (int it = blockIdx.x; it < n_items && !warp_aborted(abort_flag); it += gridDim.x) {
+        for (uint32_t item_k = 0; !warp_aborted(abort_flag); ++item_k) {
+            const int it = next_item(item_k);
+            if (it < 0) break;
             const int4 item = a.items[it];
             const long long r = a.final_cnt[(size_t)item.x * a.Cq + item.y];
             const int T = (int)((r + kBN - 1) / kBN);
@@ -306,7 +346,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float c = a.scale_log2;
         // parity of the o_done[q][j & 1] phase that completes when P(j) V(j) is done
         auto pv_parity = [&](int j) -> uint32_t { return ((o_par >> (j & 1)) + (uint32_t)(j >> 1)) & 1u; };
-        for (int it = blockIdx.x; it < n_items && !warp_aborted(abort_flag); it += gridDim.x) {
+        for (uint32_t item_k = 0; !warp_aborted(abort_flag); ++item_k) {
+            const int it = next_item(item_k);
+            if (it < 0) break;
             const int4 item = a.items[it];
             const int bh = item.x, cl = item.y, q0 = item.z, nq = item.w;
             if (q == 1 && nq <= kBM) continue;        // this Q tile is idle for the item
