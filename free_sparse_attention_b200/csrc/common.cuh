@@ -50,12 +50,16 @@ struct KmArgs {
     // tensor-core assignment (bf16 inputs): packed centroid operands, Cpad = Cs rounded up to 16
     __nv_bfloat16 *cent_bf;   // [P, 2 (hi, lo), Cpad, d] bf16 split of the centroids
     float *cn2p;              // [P, Cpad + 4] |mu|^2 (+inf padding), max |mu|, max slack
+    // tokens whose assignment the fast kernels could not certify, one list per launched
+    // role r: entries bh * N + j at unsure_list[r * BH * N ...], count unsure_count[r]
+    int32_t *unsure_list;     // [4, BH * N]
+    int32_t *unsure_count;    // [4], cleared before every assignment launch
 };
 
 // Workspace layout (byte offsets); computed identically by every entry point.
 struct WsLayout {
     size_t status, counters;
-    size_t cent32, cent64T, cnorm, cnrm2, cslack, perm, off, chunk_hist, cent_bf, cn2p;
+    size_t cent32, cent64T, cnorm, cnrm2, cslack, perm, off, chunk_hist, cent_bf, cn2p, unsure_list, unsure_count;
     size_t q_cent, q_assign, q_sizes, k_cent, k_codes, k_sizes;
     size_t topp, base, khead, final_cnt, mask, sel_state;
     size_t q_perm, q_off, q_hist, work_items, attn_counter, key_lists;
@@ -121,6 +125,19 @@ __device__ __forceinline__ float load_x(const void *X, long long idx, int is_bf1
 __device__ __forceinline__ void set_status(int32_t *status, int bits)
 {
     if (status) atomicOr(status, bits);
+}
+
+// Appends `value` for every lane with `take` to list[*count ...] with one atomic per
+// warp.  All 32 lanes of the warp must call it.
+__device__ __forceinline__ void warp_append(bool take, int32_t value, int32_t *list, int32_t *count)
+{
+    const unsigned m = __ballot_sync(0xffffffffu, take);
+    if (!m) return;
+    const int lane = threadIdx.x & 31, leader = __ffs(m) - 1;
+    int base = 0;
+    if (lane == leader) base = atomicAdd(count, __popc(m));
+    base = __shfl_sync(0xffffffffu, base, leader);
+    if (take) list[base + __popc(m & ((1u << lane) - 1u))] = value;
 }
 
 }  // namespace scope

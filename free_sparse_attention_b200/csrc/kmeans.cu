@@ -214,7 +214,9 @@ __global__ void __launch_bounds__(kAssignThreads) km_assign_fast_kernel(KmArgs a
             minU[t] = fminf(minU[t], oU);
         }
     }
-    // lane tx writes token ty*8 + tx for tx < 8
+    // lane tx writes token ty*8 + tx for tx < 8; undecided tokens go to the exact list
+    bool unsure = false;
+    int32_t entry = 0;
 #pragma unroll
     for (int t = 0; t < 8; ++t) {
         if (tx == t) {
@@ -222,75 +224,72 @@ __global__ void __launch_bounds__(kAssignThreads) km_assign_fast_kernel(KmArgs a
             if (j < a.N) {
                 bool sure = min2L[t] > minU[t];
                 R.assign[(size_t)bh * R.assign_bh + j] = sure ? (uint16_t)idxL[t] : kUnsure;
+                unsure = !sure;
+                entry = bh * a.N + j;
             }
         }
     }
+    warp_append(unsure, entry, a.unsure_list + (size_t)r * a.BH * a.N, a.unsure_count + r);
 }
 
 // ------------------------------------------------------------------------- exact assignment
-// One warp per group of 32 tokens (grid-stride); every unsure token is re-decided in
-// binary64 against all centroids.  The token's channels go to shared memory; lane l
-// takes centroids l, l+32, ... two at a time, reading the channel-major binary64 copy
-// (consecutive lanes, consecutive centroids), and sums the squared differences in
-// channel order with one rounding per operation, as the definition is evaluated.
+// One warp per listed unsure token (grid-stride over the list the fast kernels filled);
+// the token is re-decided in binary64 against all centroids.  The token's channels go
+// to shared memory; lane l takes centroids l, l+32, ... two at a time, reading the
+// channel-major binary64 copy (consecutive lanes, consecutive centroids), and sums the
+// squared differences in channel order with one rounding per operation, as the
+// definition is evaluated.
 constexpr int kExactWarps = 8;
 
 __global__ void __launch_bounds__(kExactWarps * 32) km_assign_exact_kernel(KmArgs a)
 {
     __shared__ double xs[kExactWarps][128];
     const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
-    const int ngroups = (a.N + 31) / 32;
-    const long long total = (long long)a.BH * a.nroles * ngroups;
-    const long long nwarps = (long long)gridDim.x * kExactWarps;
-    for (long long g = (long long)blockIdx.x * kExactWarps + wib; g < total; g += nwarps) {
-        const int p = (int)(g / ngroups);
-        int bh, r;
-        const RoleDesc &R = role_of(a, p, bh, r);
-        const int j = (int)(g % ngroups) * 32 + lane;
-        uint16_t *asg = R.assign + (size_t)bh * R.assign_bh;
-        bool unsure = j < a.N && asg[j] == kUnsure;
-        unsigned todo = __ballot_sync(0xffffffffu, unsure);
+    int cnt[4], total = 0;
+    for (int r = 0; r < a.nroles; ++r) total += (cnt[r] = a.unsure_count[r]);
+    for (int g = blockIdx.x * kExactWarps + wib; g < total; g += gridDim.x * kExactWarps) {
+        int r = 0, k = g;
+        while (k >= cnt[r]) k -= cnt[r++];
+        const int entry = a.unsure_list[(size_t)r * a.BH * a.N + k];
+        const int bh = entry / a.N, jj = entry - bh * a.N;
+        const int p = bh * a.nroles + r;
+        const RoleDesc &R = a.role[a.role0 + r];
         const double *muT = a.cent64T + (size_t)p * a.Cs * a.ds;
-        while (todo) {
-            const int src = __ffs(todo) - 1;
-            todo &= todo - 1;
-            const int jj = (int)(g % ngroups) * 32 + src;
-            const long long xrow = ((long long)bh * a.N + jj) * a.d + R.ch0;
-            for (int i = lane; i < R.dm; i += 32) xs[wib][i] = (double)load_x(R.X, xrow + i, a.is_bf16);
-            __syncwarp();
-            double best = INFINITY;
-            int bi = 0x7fffffff;
-            for (int c = lane; c < R.C; c += 64) {
-                const bool two = c + 32 < R.C;
-                const int c2 = two ? c + 32 : c;
-                double d0 = 0.0, d1 = 0.0;
-                for (int i = 0; i < R.dm; ++i) {
-                    const double x = xs[wib][i];
-                    const double e0 = __dsub_rn(x, muT[(size_t)i * a.Cs + c]);
-                    const double e1 = __dsub_rn(x, muT[(size_t)i * a.Cs + c2]);
-                    d0 = __dadd_rn(d0, __dmul_rn(e0, e0));
-                    d1 = __dadd_rn(d1, __dmul_rn(e1, e1));
-                }
-                if (d0 < best) {
-                    best = d0;
-                    bi = c;
-                }
-                if (two && d1 < best) {
-                    best = d1;
-                    bi = c2;
-                }
+        const long long xrow = ((long long)bh * a.N + jj) * a.d + R.ch0;
+        __syncwarp();
+        for (int i = lane; i < R.dm; i += 32) xs[wib][i] = (double)load_x(R.X, xrow + i, a.is_bf16);
+        __syncwarp();
+        double best = INFINITY;
+        int bi = 0x7fffffff;
+        for (int c = lane; c < R.C; c += 64) {
+            const bool two = c + 32 < R.C;
+            const int c2 = two ? c + 32 : c;
+            double d0 = 0.0, d1 = 0.0;
+            for (int i = 0; i < R.dm; ++i) {
+                const double x = xs[wib][i];
+                const double e0 = __dsub_rn(x, muT[(size_t)i * a.Cs + c]);
+                const double e1 = __dsub_rn(x, muT[(size_t)i * a.Cs + c2]);
+                d0 = __dadd_rn(d0, __dmul_rn(e0, e0));
+                d1 = __dadd_rn(d1, __dmul_rn(e1, e1));
             }
-            for (int off = 16; off; off >>= 1) {
-                double ob = __shfl_xor_sync(0xffffffffu, best, off);
-                int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-                if (ob < best || (ob == best && oi < bi)) {
-                    best = ob;
-                    bi = oi;
-                }
+            if (d0 < best) {
+                best = d0;
+                bi = c;
             }
-            if (lane == 0) asg[jj] = (uint16_t)bi;
-            __syncwarp();
+            if (two && d1 < best) {
+                best = d1;
+                bi = c2;
+            }
         }
+        for (int off = 16; off; off >>= 1) {
+            double ob = __shfl_xor_sync(0xffffffffu, best, off);
+            int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+            if (ob < best || (ob == best && oi < bi)) {
+                best = ob;
+                bi = oi;
+            }
+        }
+        if (lane == 0) R.assign[(size_t)bh * R.assign_bh + jj] = (uint16_t)bi;
     }
 }
 
@@ -411,42 +410,127 @@ __global__ void __launch_bounds__(128) sort_scatter_kernel(KmArgs a)
 }
 
 // ------------------------------------------------------------------------- update
-// grid (ceil(Cs/G), P), block 128: a group of dm threads per centroid sums its
-// members in token order (binary64) and divides by the count.
-__global__ void __launch_bounds__(128) km_update_kernel(KmArgs a)
+// grid (Cs, P), block kUpdThreads: one centroid per block.  Thread (s, g) sums channels
+// CH*g .. CH*g+CH-1 over segment s of the member list (members in token order, the list
+// split into S = kUpdThreads / (dm / CH) contiguous segments) in binary64, and records
+// the smallest ulp among its nonzero values and the sum of magnitudes.  Every input
+// value is an integer multiple of the smallest ulp u, so every partial sum in any order
+// is too; when the sum of magnitudes stays below 2^52 u (a factor 2 of margin under
+// 2^53 u), every partial sum is exactly representable and the segment sums add up (in
+// segment order) to exactly the in-order binary64 sum.  Otherwise, or for subnormal
+// inputs, that channel is summed again sequentially.  The mean is the sum divided by the
+// member count (one rounding).  bf16 inputs whose channel range starts and ends on an
+// even channel are read two channels (4 bytes) per load.
+constexpr int kUpdThreads = 256;
+constexpr int kUpdUnroll = 8;
+
+// Value and ulp exponent of one input element (bf16: 8 significant bits, fp32: 24); a
+// subnormal gives INT_MIN (no usable bound), 0 gives INT_MAX (no ulp).
+__device__ __forceinline__ void elem_bf16(uint32_t b16, double &x, int &e)
 {
+    x = (double)__uint_as_float(b16 << 16);
+    const int be = (b16 >> 7) & 0xFF;
+    e = (b16 & 0x7FFF) == 0 ? 0x7fffffff : (be == 0 ? (int)0x80000000 : be - 127 - 7);
+}
+
+__device__ __forceinline__ void elem_f32(uint32_t b32, double &x, int &e)
+{
+    x = (double)__uint_as_float(b32);
+    const int be = (b32 >> 23) & 0xFF;
+    e = (b32 & 0x7FFFFFFF) == 0 ? 0x7fffffff : (be == 0 ? (int)0x80000000 : be - 127 - 23);
+}
+
+template <int CH>
+__global__ void __launch_bounds__(kUpdThreads) km_update_kernel(KmArgs a)
+{
+    __shared__ double psum[kUpdThreads * CH], pabs[kUpdThreads * CH];
+    __shared__ int pexp[kUpdThreads * CH];
     int bh, r;
-    const int p = blockIdx.y;
+    const int p = blockIdx.y, c = blockIdx.x;
     const RoleDesc &R = role_of(a, p, bh, r);
-    const int dm = R.dm, G = max(1, 128 / dm);
-    const int g = threadIdx.x / dm, i = threadIdx.x % dm;
-    const int c = blockIdx.x * G + g;
-    const bool active = g < G && c < R.C;
+    const int dm = R.dm, dmc = dm / CH, S = kUpdThreads / dmc;
+    const int s = threadIdx.x / dmc, g = threadIdx.x - s * dmc;
+    const bool active = c < R.C;
     const int32_t *off = a.off + (size_t)p * (a.Cs + 1);
     const int32_t *perm = a.perm + (size_t)p * a.N;
-    const int beg = active ? off[c] : 0, end = active ? off[c + 1] : 0;
-    double *cent = R.cent + ((size_t)bh * R.C + c) * a.d + R.ch0;
-    if (active && end > beg) {
-        const long long base = (long long)bh * a.N * a.d + R.ch0 + i;
-        double acc = 0.0;
-        int m = beg;
-        for (; m + 4 <= end; m += 4) {
-            const int ja = perm[m], jb = perm[m + 1], jc = perm[m + 2], jd = perm[m + 3];
-            const double xa = (double)load_x(R.X, base + (long long)ja * a.d, a.is_bf16);
-            const double xb = (double)load_x(R.X, base + (long long)jb * a.d, a.is_bf16);
-            const double xc = (double)load_x(R.X, base + (long long)jc * a.d, a.is_bf16);
-            const double xd = (double)load_x(R.X, base + (long long)jd * a.d, a.is_bf16);
-            acc = __dadd_rn(acc, xa);
-            acc = __dadd_rn(acc, xb);
-            acc = __dadd_rn(acc, xc);
-            acc = __dadd_rn(acc, xd);
+    const int beg = active ? off[c] : 0, end = active ? off[c + 1] : 0, n = end - beg;
+    double *cent = R.cent + ((size_t)bh * R.C + (active ? c : 0)) * a.d + R.ch0;
+    const long long base = (long long)bh * a.N * a.d + R.ch0 + CH * g;   // element index
+    if (s < S && n > 0) {
+        const int m0 = beg + (int)((long long)n * s / S), m1 = beg + (int)((long long)n * (s + 1) / S);
+        double acc[CH], mag[CH];
+        int emin[CH];
+#pragma unroll
+        for (int h = 0; h < CH; ++h) {
+            acc[h] = 0.0;
+            mag[h] = 0.0;
+            emin[h] = 0x7fffffff;
         }
-        for (; m < end; ++m)
-            acc = __dadd_rn(acc, (double)load_x(R.X, base + (long long)perm[m] * a.d, a.is_bf16));
-        cent[i] = __ddiv_rn(acc, (double)(end - beg));
+        auto take = [&](uint32_t bits) {
+#pragma unroll
+            for (int h = 0; h < CH; ++h) {
+                double x;
+                int e;
+                if (CH == 2)
+                    elem_bf16(h ? bits >> 16 : bits & 0xFFFFu, x, e);
+                else if (a.is_bf16)
+                    elem_bf16(bits, x, e);
+                else
+                    elem_f32(bits, x, e);
+                acc[h] = __dadd_rn(acc[h], x);
+                mag[h] = __dadd_rn(mag[h], fabs(x));
+                emin[h] = min(emin[h], e);
+            }
+        };
+        auto load = [&](int tok) -> uint32_t {
+            const long long e = base + (long long)tok * a.d;
+            if (CH == 2) return *reinterpret_cast<const uint32_t *>(reinterpret_cast<const uint16_t *>(R.X) + e);
+            if (a.is_bf16) return reinterpret_cast<const uint16_t *>(R.X)[e];
+            return reinterpret_cast<const uint32_t *>(R.X)[e];
+        };
+        int m = m0;
+        for (; m + kUpdUnroll <= m1; m += kUpdUnroll) {
+            int tok[kUpdUnroll];
+#pragma unroll
+            for (int q = 0; q < kUpdUnroll; ++q) tok[q] = perm[m + q];
+            uint32_t bits[kUpdUnroll];
+#pragma unroll
+            for (int q = 0; q < kUpdUnroll; ++q) bits[q] = load(tok[q]);
+#pragma unroll
+            for (int q = 0; q < kUpdUnroll; ++q) take(bits[q]);
+        }
+        for (; m < m1; ++m) take(load(perm[m]));
+#pragma unroll
+        for (int h = 0; h < CH; ++h) {
+            psum[threadIdx.x * CH + h] = acc[h];
+            pabs[threadIdx.x * CH + h] = mag[h];
+            pexp[threadIdx.x * CH + h] = emin[h];
+        }
     }
     __syncthreads();
-    if (active) finalize_row(a, p, c, cent, dm, i);
+    if (s == 0 && active && n > 0) {
+#pragma unroll
+        for (int h = 0; h < CH; ++h) {
+            double sum = 0.0, mag = 0.0;
+            int emin = 0x7fffffff;
+            for (int q = 0; q < S; ++q) {
+                const int t = (q * dmc + g) * CH + h;
+                sum = __dadd_rn(sum, psum[t]);
+                mag = __dadd_rn(mag, pabs[t]);
+                emin = min(emin, pexp[t]);
+            }
+            const bool exact = emin == 0x7fffffff ||
+                               (emin != (int)0x80000000 && emin > -1000 && mag <= ldexp(1.0, 52 + emin));
+            if (!exact) {
+                sum = 0.0;
+                for (int m = beg; m < end; ++m)
+                    sum = __dadd_rn(sum, (double)load_x(R.X, base + h + (long long)perm[m] * a.d, a.is_bf16));
+            }
+            cent[CH * g + h] = __ddiv_rn(sum, (double)n);
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x < dm && active) finalize_row(a, p, c, cent, dm, threadIdx.x);
 }
 
 int max_blocks_for_groups(const KmArgs &a)
@@ -496,7 +580,12 @@ cudaError_t km_run(KmArgs a, int iters, cudaStream_t s)
     // assignment (kmeans_tc.cu); both paths certify their winners the same way and leave
     // the undecided tokens to the binary64 kernel.
     const bool tc = km_assign_tc_supported(a);
+    // two channels per 4-byte load when every launched channel range is even-aligned
+    bool upd2 = a.is_bf16 != 0;
+    for (int r = 0; r < a.nroles; ++r)
+        upd2 = upd2 && (a.role[a.role0 + r].ch0 % 2 == 0) && (a.role[a.role0 + r].dm % 2 == 0);
     for (int it = 0; it < iters; ++it) {
+        if (cudaMemsetAsync(a.unsure_count, 0, 4 * sizeof(int32_t), s) != cudaSuccess) return cudaGetLastError();
         if (tc) {
             cudaError_t e = km_pack(a, s);
             if (e == cudaSuccess) e = km_assign_tc(a, sms, s);
@@ -507,7 +596,10 @@ cudaError_t km_run(KmArgs a, int iters, cudaStream_t s)
         km_assign_exact_kernel<<<sms * 4, kExactWarps * 32, 0, s>>>(a);
         cudaError_t e = sort_by_cluster(a, s);
         if (e != cudaSuccess) return e;
-        km_update_kernel<<<dim3(gb, P), 128, 0, s>>>(a);
+        if (upd2)
+            km_update_kernel<2><<<dim3(a.Cs, P), kUpdThreads, 0, s>>>(a);
+        else
+            km_update_kernel<1><<<dim3(a.Cs, P), kUpdThreads, 0, s>>>(a);
     }
     return cudaGetLastError();
 }

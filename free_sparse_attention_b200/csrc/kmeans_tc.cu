@@ -502,11 +502,15 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
                 idx = o1 < m1 ? oi : idx;
                 m1 = fminf(m1, o1);
                 const int j = tile * kTile + row;
+                bool unsure = false;
                 if (j < a.N) {
                     const float E = bound_E(w.ks, xn, maxnm, maxres, maxsl);
                     const bool sure = (m2 - m1) > (E + E) * (1.0f + 0x1p-20f);
                     R.assign[(size_t)bh * R.assign_bh + j] = sure ? (uint16_t)idx : kUnsureTc;
+                    unsure = !sure;
                 }
+                const int r = p % a.nroles;
+                warp_append(unsure, bh * a.N + j, a.unsure_list + (size_t)r * a.BH * a.N, a.unsure_count + r);
             }
         }
     }

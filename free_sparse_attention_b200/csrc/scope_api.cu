@@ -93,6 +93,8 @@ KmArgs km_base(const scope_params &p, const WsLayout &L, void *ws)
     a.chunk_hist = at<int32_t>(ws, L.chunk_hist);
     a.cent_bf = at<__nv_bfloat16>(ws, L.cent_bf);
     a.cn2p = at<float>(ws, L.cn2p);
+    a.unsure_list = at<int32_t>(ws, L.unsure_list);
+    a.unsure_count = at<int32_t>(ws, L.unsure_count);
     a.nchunk = (int)D.nchunk;
     a.status = at<int32_t>(ws, L.status);
     return a;
@@ -256,6 +258,8 @@ WsLayout ws_layout(const scope_params &p)
     const long long Cpad = (D.Cs + 15) / 16 * 16;
     L.cent_bf = take(sizeof(__nv_bfloat16) * D.P * 2 * Cpad * D.d);
     L.cn2p = take(sizeof(float) * D.P * (Cpad + 4));
+    L.unsure_list = take(sizeof(int32_t) * D.P * D.N);
+    L.unsure_count = take(4 * sizeof(int32_t));
     L.q_cent = take(sizeof(double) * D.BH * p.Cq * p.d);
     L.q_assign = take(sizeof(uint16_t) * D.BH * D.N);
     L.q_sizes = take(sizeof(int32_t) * D.BH * p.Cq);
