@@ -61,7 +61,6 @@ struct __align__(8) Bars {
     // per Q tile and S buffer: S ready (MMA commit), P written (softmax), P V done (commit)
     uint64_t s_full[kQT][2], p_full[kQT][2], o_done[kQT][2];
     uint64_t o_free[kQT];  // epilogue has read O_q
-    uint64_t turn[kQT];    // softmax warpgroups take turns: turn[q] = "Q tile q's softmax may run"
     uint64_t item_full[kRing], item_empty[kRing];   // work-item ring (dynamic scheduler)
 };
 
@@ -120,7 +119,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 bar_init(&bars->o_done[q][b], 1);
             }
             bar_init(&bars->o_free[q], 4);
-            bar_init(&bars->turn[q], 4);
         }
         for (int k = 0; k < kRing; ++k) {
             bar_init(&bars->item_full[k], 1);
@@ -342,7 +340,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // bit b of s_par: parity of the next s_full[q][b] phase; bit b of o_par: parity of
         // the P V commits on o_done[q][b] before the current item (the softmax waits on
         // o_done only when it must, so it counts the phases per item instead)
-        uint32_t s_par = 0, o_par = 0, turn_cnt = 0;
+        uint32_t s_par = 0, o_par = 0;
         const float c = a.scale_log2;
         // parity of the o_done[q][j & 1] phase that completes when P(j) V(j) is done
         auto pv_parity = [&](int j) -> uint32_t { return ((o_par >> (j & 1)) + (uint32_t)(j >> 1)) & 1u; };
@@ -352,10 +350,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int4 item = a.items[it];
             const int bh = item.x, cl = item.y, q0 = item.z, nq = item.w;
             if (q == 1 && nq <= kBM) continue;        // this Q tile is idle for the item
-            // With both Q tiles active the two warpgroups take turns on the exponentials
-            // (tile 0 first), so one tile's exponentials overlap the other tile's MMAs
-            // instead of both competing for the special-function units at once.
-            const bool take_turns = nq > kBM;
             const long long r = a.final_cnt[(size_t)bh * a.Cq + cl];
             const int T = (int)((r + kBN - 1) / kBN);
             float m_run = -INFINITY, l = 0.f;
@@ -403,11 +397,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (need) l *= alpha;
                 }
                 if (need) m_run = mt;
-                if (take_turns) {
-                    ok = warp_wait(&bars->turn[q], (turn_cnt & 1) ^ (q == 0 ? 1u : 0u), abort_flag, a.status);
-                    if (!ok) break;
-                    ++turn_cnt;
-                }
                 // P = 2^(s*c - m) as bf16 pairs over the first kBN/2 columns of this S
                 // buffer; exponent arguments and row sums on packed fp32 pairs
                 const unsigned long long c2 = f2pack(c, c), nm2 = f2pack(-m_run, -m_run);
@@ -424,10 +413,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                         pk[e] = *reinterpret_cast<uint32_t *>(&hh);
                     }
                     tmem_st16(tmem + lane_base + sb_col + h * 16, pk);
-                }
-                if (take_turns) {
-                    __syncwarp();
-                    if (lane == 0) bar_arrive(&bars->turn[q ^ 1]);
                 }
                 const float2 la = f2unpack(ls2[0]), lb = f2unpack(ls2[1]);
                 float ls[4] = {la.x, la.y, lb.x, lb.y};

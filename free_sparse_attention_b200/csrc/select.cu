@@ -225,8 +225,10 @@ struct SelectOut {
 // Finds the first key of the ranking at which the cumulative weight reaches the target.
 // mass_mode: weight = softmax mass, target = rho * (total mass); else weight = 1 and
 // target = count (1 <= count <= N).  Called by all threads of the block.
+// umax_out (mass mode): the largest key weight, found in the first histogram pass.
 __device__ SelectOut block_select(const SelSmem &S, const Unit &u, bool mass_mode, double rho,
-                                  long long count, double smax, double smin, int32_t *status)
+                                  long long count, double smax, double smin, int32_t *status,
+                                  double *umax_out = nullptr)
 {
     Levels L;
     L.n = 0;
@@ -249,14 +251,16 @@ __device__ SelectOut block_select(const SelSmem &S, const Unit &u, bool mass_mod
             S.mlo[b] = 0;
         }
         __syncthreads();
-        double cmin = DBL_MAX, cmax = -DBL_MAX;
+        double cmin = DBL_MAX, cmax = -DBL_MAX, umx = 0.0;
         for (int j = tid; j < u.N; j += kSelThreads) {
             const double s = key_score(S, u, j);
             if (!in_candidates(L, s)) continue;
             const int b = L.jmode ? jbin(j, u.N) : vbin(s, hi, scale);
             atomicAdd(&S.cnt[b], 1);
             if (mass_mode) {
-                const unsigned long long W = key_mass(S, u, j);
+                const double uj = key_u(S, u, j);
+                umx = fmax(umx, uj);
+                const unsigned long long W = __double2ull_rn(fmin(__dmul_rn(uj, u.inv_umax), 1.0) * 9223372036854775808.0);
                 atomicAdd(&S.mhi[b], W >> 32);
                 atomicAdd(&S.mlo[b], W & 0xffffffffull);
             }
@@ -265,6 +269,7 @@ __device__ SelectOut block_select(const SelSmem &S, const Unit &u, bool mass_mod
         }
         cmin = block_min(cmin, S.red);
         cmax = block_max(cmax, S.red);
+        if (mass_mode && iter == 0 && umax_out) *umax_out = block_max(umx, S.red);
         if (!L.jmode && cmin == cmax) {
             // every candidate has the same logit: the ranking among them is by index
             L.jmode = true;
@@ -469,21 +474,35 @@ __global__ void __launch_bounds__(kSelThreads) sel_topp_kernel(SelArgs a)
     u.Cm = a.Cm;
     u.N = a.N;
     u.inv = a.inv_sqrt_d;
-    double smax = -DBL_MAX, smin = DBL_MAX, umax = 0.0;
-    for (int j = tid; j < a.N; j += kSelThreads) {
-        const double s = key_score(S, u, j);
-        smax = fmax(smax, s);
-        smin = fmin(smin, s);
-        umax = fmax(umax, key_u(S, u, j));
+    // Score bounds from the tables: rounded sums and the positive scale are monotone, so
+    // (1/sqrt d)((max P^T + max P^H) + max P^W) bounds every key's score from above (and
+    // likewise from below); they only set the range of the first histogram.
+    double tmax[3], tmin[3];
+    for (int m = 0; m < 3; ++m) {
+        double mx = -DBL_MAX, mn = DBL_MAX;
+        for (int z = tid; z < a.Cm; z += kSelThreads) {
+            mx = fmax(mx, S.lut[m * a.Cm + z]);
+            mn = fmin(mn, S.lut[m * a.Cm + z]);
+        }
+        tmax[m] = block_max(mx, S.red);
+        tmin[m] = block_min(mn, S.red);
     }
-    smax = block_max(smax, S.red);
-    smin = block_min(smin, S.red);
-    umax = block_max(umax, S.red);
-    u.inv_umax = 1.0 / umax;
+    const double smax = __dmul_rn(u.inv, __dadd_rn(__dadd_rn(tmax[0], tmax[1]), tmax[2]));
+    const double smin = __dmul_rn(u.inv, __dadd_rn(__dadd_rn(tmin[0], tmin[1]), tmin[2]));
+    // Key weights u_j = E^T E^H E^W <= 1 (each exponential table peaks at 1), so masses are
+    // quantised against 1: at most N 2^-64 of absolute error in total.  That stays below
+    // 1e-9 of the total mass Z >= max_j u_j unless the largest weight is tiny, in which
+    // case the selection runs again normalised by the largest weight itself.
+    u.inv_umax = 1.0;
     long long p = a.N;
     SelectOut so{smax, 0, 0};
     if (a.rho < 1.0) {
-        so = block_select(S, u, true, a.rho, 0, smax, smin, a.status);
+        double umax = 1.0;
+        so = block_select(S, u, true, a.rho, 0, smax, smin, a.status, &umax);
+        if (umax < (double)a.N * 0x1p-64 * 1e9 && umax > 0.0) {
+            u.inv_umax = 1.0 / umax;
+            so = block_select(S, u, true, a.rho, 0, smax, smin, a.status);
+        }
         p = so.rank + 1;
     }
     if (tid == 0) {
