@@ -35,7 +35,6 @@ sys.path.insert(0, ROOT)
 from free_sparse_attention_b200 import synth  # noqa: E402
 from free_sparse_attention_b200.workloads import ALL, HUNYUAN720  # noqa: E402
 
-FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12   # FMA pipes at the max SM clock
 METRIC = "SCOPE layer effective TFLOP/s (4*sum n_c*r_c*d / layer time) at 118800 tokens"
 
 
@@ -339,7 +338,9 @@ def run_scope(args, w):
                       "worklist": float(stage_ms[2]), "attention": attn_ms},
         "stage_fractions": {
             "clustering_hbm": clust_bytes / (stage_ms[0] * 1e-3) / 1e9 / pk["hbm_gbs"],
-            "clustering_fp32_alu": clust_flops / (stage_ms[0] * 1e-3) / 1e12 / FP32_ALU_TFLOPS,
+            # distance contractions 2 N C d_m per iteration (the tensor cores issue twice that
+            # for the bf16 hi/lo centroid split), against the measured bf16 peak
+            "clustering_tensor": clust_flops / (stage_ms[0] * 1e-3) / 1e12 / pk["bf16_sustained"],
             "selection_hbm": sel_bytes / (stage_ms[1] * 1e-3) / 1e9 / pk["hbm_gbs"]},
         "density": density, "effective_tflop_per_layer": flops / 1e12,
         "dense_sdpa_ms": dense_ms,
