@@ -143,3 +143,34 @@ def test_fp32_and_bf16_paths_agree_on_selection():
     for k in ("q_assign", "k_codes", "final_counts", "sel_mask", "k_head"):
         assert torch.equal(i16[k], i32[k]), k
     assert (O16.float() - O32).abs().max().item() <= 2e-2
+
+
+def _bf16_exact(a):
+    """Rounds float64 values to bf16 and returns them as float32 (exact copies)."""
+    return torch.from_numpy(np.ascontiguousarray(a, np.float32)).to(torch.bfloat16).float().numpy()
+
+
+@pytest.mark.parametrize("wide", [False, True])
+def test_member_sums_with_and_without_the_exact_parallel_path(wide):
+    """Centroid means of bf16 members are summed in parallel only when every partial sum is
+    exactly representable (sum |x| <= 2^52 * the smallest ulp among the members); otherwise
+    in token order.  With `wide`, half of the channels mix values near 2^40 and 2^-30 inside
+    one cluster, so those channels take the in-order path and the others the parallel one.
+    Either way the centroids must equal the oracle's in-order binary64 means bit for bit."""
+    w = Workload("sums", 1, 2, 4, 16, 16, 44, 42, 42, "bf16", 3, 5, seed=31)
+    rng = np.random.default_rng(5)
+    q = rng.standard_normal((w.H, w.N, w.d))
+    if wide:
+        big = rng.random((w.H, w.N)) < 0.05
+        q[:, :, 64:] = np.where(big[..., None], 2.0 ** 40, 2.0 ** -30) * (1.0 + rng.random((w.H, w.N, 64)))
+    q = _bf16_exact(q)
+    init = np.stack([rng.choice(w.N, w.Cq, replace=False) for _ in range(w.H)]).astype(np.int32)
+    Q = torch.from_numpy(q).reshape(w.B, w.H, w.N, w.d).to("cuda", torch.bfloat16)
+    p = capi.Params.from_workload(w)
+    qc, qa, qs = capi.cluster_queries(p, Q, init_idx=torch.from_numpy(init).reshape(w.B, w.H, w.Cq).cuda())
+    torch.cuda.synchronize()
+    for h in range(w.H):
+        ref = oracle.kmeans(q[h].astype(np.float32), 0, w.d, w.Cq, w.iters, init_idx=init[h])
+        np.testing.assert_array_equal(to_np(qa)[0, h], ref["assign"])
+        np.testing.assert_array_equal(to_np(qs)[0, h], ref["sizes"])
+        np.testing.assert_array_equal(to_np(qc)[0, h], ref["centroids"])
