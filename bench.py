@@ -132,7 +132,7 @@ def dist_setup():
 
 
 # ----------------------------------------------------------------------------- CPU oracle
-def oracle_sample(w, T_sample=6):
+def oracle_sample(w, T_sample=6, khead_off=False):
     """The oracle on a bounded sub-layer: head (0, 0) of the same workload with the
     grid cut to the first T_sample frames (N_s = T_sample*Hg*Wg tokens); every stage
     runs in full on it.  Each stage's cost is extrapolated to the whole layer by its
@@ -147,7 +147,7 @@ def oracle_sample(w, T_sample=6):
     rk = oracle.cluster_keys(k, (ws.d_t, ws.d_h, ws.d_w), ws.Cm, ws.iters, init_idx3=x["k_init"][0])
     t1 = time.perf_counter()
     sel = oracle.select(rq["centroids"], rq["sizes"], rk["centroids"], rk["codes"],
-                        (ws.d_t, ws.d_h, ws.d_w), ws.rho, ws.alpha)
+                        (ws.d_t, ws.d_h, ws.d_w), ws.rho, ws.alpha, khead_off=khead_off)
     t2 = time.perf_counter()
     oracle.attention(q, k, v, rq["assign"], sel["mask"])
     t3 = time.perf_counter()
@@ -176,11 +176,11 @@ def run_reference(args, w):
     if rank != 0:
         return 0
     for _ in range(args.warmup):
-        oracle_sample(w, T_sample=4)
+        oracle_sample(w, T_sample=4, khead_off=args.khead_off)
     times, desc, threads = [], "", 1
     flops = expected_layer_flops(w)
     for _ in range(args.steps):
-        s = oracle_sample(w, T_sample=4)
+        s = oracle_sample(w, T_sample=4, khead_off=args.khead_off)
         times.append(layer_seconds_from_sample(s, flops))
         desc, threads = s["desc"], s["threads"]
     sec = statistics.mean(times)
@@ -224,7 +224,7 @@ def run_scope(args, w):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=torch.device("cuda", local))
     capi.lib()
-    p = capi.Params.from_workload(w)
+    p = capi.Params.from_workload(w, khead_mode=capi.SCOPE_KHEAD_OFF if args.khead_off else capi.SCOPE_KHEAD_ONLINE)
     x = synth.layer_inputs(w)
     dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
     host = {n: torch.from_numpy(x[n]).reshape(w.B, w.H, w.N, w.d).to(dt).pin_memory() for n in "qkv"}
@@ -327,7 +327,8 @@ def run_scope(args, w):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded generator G: smooth field + noise, 3D RoPE)",
-        "config": {"workload": workload_desc(w), "global_batch": world * w.B, "seq_len": w.N,
+        "config": {"workload": workload_desc(w) + (" ablation: online k_head off (r_c = b_c)" if args.khead_off else ""),
+                   "global_batch": world * w.B, "seq_len": w.N,
                    "parallelism": f"{world} independent layers, one per GPU (no collective)",
                    "l2": "inputs larger than L2 (Q, K, V = 2.19 GB resident in HBM)"},
         "roofline": {"bound": "tensor", "kernel": "attn_tc_kernel (tcgen05 sparse attention)",
@@ -351,7 +352,7 @@ def run_scope(args, w):
         "clocks": clk,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        s = oracle_sample(w)
+        s = oracle_sample(w, khead_off=args.khead_off)
         sec = layer_seconds_from_sample(s, flops)
         line["cpu_baseline"] = {"value": flops / sec / 1e12, "unit": "TFLOP/s", "cores": s["threads"],
                                 "kind": "oracle", "sample": s["desc"]}
@@ -395,12 +396,18 @@ def main():
                     help="override the head count (small cases for profiling)")
     ap.add_argument("--profile-once", action="store_true",
                     help="run the layer once (after one warm-up) and exit; for ncu captures")
+    ap.add_argument("--rho", type=float, default=None,
+                    help="override the workload's Top-p threshold (rho sweeps)")
+    ap.add_argument("--khead-off", action="store_true",
+                    help="ablation: the online k_head disabled (r_c = b_c)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     w = ALL[args.workload]
     if args.heads:
         w = w.with_(H=args.heads)
+    if args.rho is not None:
+        w = w.with_(rho=args.rho)
     if args.profile_once:
         return profile_once(w)
     if args.impl == "reference":

@@ -32,12 +32,17 @@ class ScopeError(RuntimeError):
         self.code = code
 
 
+SCOPE_KHEAD_ONLINE = 0   # Eqs. 9-10: clusters topped up to k_head
+SCOPE_KHEAD_OFF = 1      # ablation: r_c = b_c
+
+
 class Params(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("T", ctypes.c_int),
                 ("Hg", ctypes.c_int), ("Wg", ctypes.c_int), ("d", ctypes.c_int),
                 ("d_t", ctypes.c_int), ("d_h", ctypes.c_int), ("d_w", ctypes.c_int),
                 ("Cq", ctypes.c_int), ("Cm", ctypes.c_int), ("iters", ctypes.c_int),
-                ("rho", ctypes.c_double), ("alpha", ctypes.c_double), ("dtype", ctypes.c_int)]
+                ("rho", ctypes.c_double), ("alpha", ctypes.c_double), ("dtype", ctypes.c_int),
+                ("khead_mode", ctypes.c_int)]
 
     @classmethod
     def from_workload(cls, w: Workload, **over) -> "Params":

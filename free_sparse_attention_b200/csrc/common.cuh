@@ -86,6 +86,7 @@ struct SelArgs {
     int BH, N, d, dt, dh, dw, Cq, Cm, nw;
     double rho, inv_sqrt_d;
     int kfix;
+    int khead_mode;           // SCOPE_KHEAD_ONLINE: r_c = max(b_c, k_head); SCOPE_KHEAD_OFF: r_c = b_c
     int32_t *status;
 };
 cudaError_t select_run(const SelArgs &a, cudaStream_t s);

@@ -32,6 +32,7 @@ scope_status validate(const scope_params *p)
     if (p->iters < 1 || p->iters > 64) return SCOPE_ERR_INVALID_ARGUMENT;
     if (!(p->rho > 0.0 && p->rho <= 1.0)) return SCOPE_ERR_INVALID_ARGUMENT;
     if (!(p->alpha >= 0.0 && p->alpha <= 1.0)) return SCOPE_ERR_INVALID_ARGUMENT;
+    if (p->khead_mode != SCOPE_KHEAD_ONLINE && p->khead_mode != SCOPE_KHEAD_OFF) return SCOPE_ERR_INVALID_ARGUMENT;
     if (p->dtype != SCOPE_F32 && p->dtype != SCOPE_BF16) return SCOPE_ERR_INVALID_ARGUMENT;
     return SCOPE_OK;
 }
@@ -190,6 +191,7 @@ SelArgs sel_args(const scope_params &p, const WsLayout &L, void *ws, const doubl
     a.inv_sqrt_d = 1.0 / std::sqrt((double)p.d);
     double kf = std::ceil(p.alpha * (double)D.N);
     a.kfix = kf < 0 ? 0 : (kf > (double)D.N ? (int)D.N : (int)kf);
+    a.khead_mode = p.khead_mode;
     a.status = at<int32_t>(ws, L.status);
     return a;
 }

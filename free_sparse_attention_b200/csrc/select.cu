@@ -519,7 +519,8 @@ __global__ void __launch_bounds__(kSelThreads) sel_topp_kernel(SelArgs a)
     }
 }
 
-// k_head (Eq. 9) and final counts r_c (Eq. 10).  grid BH.
+// k_head (Eq. 9) and final counts r_c (Eq. 10; with the online k_head switched off,
+// the ablation, r_c = b_c).  grid BH.
 __global__ void __launch_bounds__(256) sel_khead_kernel(SelArgs a)
 {
     __shared__ long long rn[8], rd[8];
@@ -553,7 +554,7 @@ __global__ void __launch_bounds__(256) sel_khead_kernel(SelArgs a)
     const long long kh = rn[0];
     for (int c = tid; c < a.Cq; c += 256) {
         const long long b = a.base[(size_t)bh * a.Cq + c];
-        a.final_cnt[(size_t)bh * a.Cq + c] = (int32_t)(b < kh ? kh : b);
+        a.final_cnt[(size_t)bh * a.Cq + c] = (int32_t)(b < kh && a.khead_mode == SCOPE_KHEAD_ONLINE ? kh : b);
     }
 }
 

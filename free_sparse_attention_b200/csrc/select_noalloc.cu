@@ -102,6 +102,7 @@ extern "C" scope_status scope_build_lut_and_select_noalloc(
     a.inv_sqrt_d = 1.0 / std::sqrt((double)p->d);
     const double kf = std::ceil(p->alpha * (double)N);
     a.kfix = kf < 0 ? 0 : (kf > (double)N ? (int)N : (int)kf);
+    a.khead_mode = p->khead_mode;
     a.status = status;
     return select_run(a, s) == cudaSuccess ? SCOPE_OK : SCOPE_ERR_CUDA;
 }

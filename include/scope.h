@@ -64,10 +64,17 @@ typedef enum { SCOPE_F32 = 0, SCOPE_BF16 = 1 } scope_dtype;
 #define SCOPE_DEV_BAD_ASSIGN     0x4   /* a cluster index >= C or a code >= Cm was supplied (clamped) */
 #define SCOPE_DEV_TIMEOUT        0x8   /* an on-chip pipeline wait gave up (~4 s); outputs invalid */
 
+/* k_head handling (scope_params.khead_mode).  ONLINE: Eqs. 9-10, every cluster is
+ * topped up to the head's k_head (the method).  OFF: the ablation the review page
+ * proposes (significance; forward_implications: "disable the online k_head"): k_head is
+ * still computed and reported, but r_c = b_c (hybrid Top-p / fixed Top-k only). */
+typedef enum { SCOPE_KHEAD_ONLINE = 0, SCOPE_KHEAD_OFF = 1 } scope_khead_mode;
+
 /* Shape and hyperparameters of one layer.  rho: Top-p threshold of Eq. 7 (the paper
  * does not report it; 0.9 is the usual choice).  alpha: fixed Top-k minimum as a
  * fraction of N, k_fix = ceil(alpha * N) (the paper gives alpha = 0.1).  iters: Lloyd
- * iterations of every k-means. */
+ * iterations of every k-means.  khead_mode: a scope_khead_mode (a zero-initialised
+ * struct gets the method, SCOPE_KHEAD_ONLINE). */
 typedef struct {
     int B, H;
     int T, Hg, Wg;
@@ -76,6 +83,7 @@ typedef struct {
     int iters;
     double rho, alpha;
     scope_dtype dtype;
+    int khead_mode;
 } scope_params;
 
 /* Optional intermediate outputs of scope_forward (device pointers; NULL = keep the

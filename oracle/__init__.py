@@ -52,7 +52,7 @@ def lib():
         L.oracle_select.restype = _int
         L.oracle_select.argtypes = [_f64p, _i32p, _f64p, _u16p, _i64, _int, _int, _int, _int,
                                     _int, _int, _dbl, _dbl, _vp, _i32p, _i32p, _i32p, _i32p,
-                                    _u32p, _vp]
+                                    _u32p, _vp, _int]
         L.oracle_attention.restype = _int
         L.oracle_attention.argtypes = [_f32p, _f32p, _f32p, _i64, _int, _u16p, _u32p, _int,
                                        _vp, _i64, _f64p]
@@ -96,8 +96,9 @@ def kmeans(X, ch0, dm, C, iters, init_idx=None, init_cent=None, logs=False):
     return out
 
 
-def select(qcent, qsizes, kcent, codes, d_split, rho, alpha, want_scores=False):
-    """Eqs. 6-10 for one head.  qcent [Cq, d], kcent [Cm, d], codes [3, N] uint16."""
+def select(qcent, qsizes, kcent, codes, d_split, rho, alpha, want_scores=False, khead_off=False):
+    """Eqs. 6-10 for one head.  qcent [Cq, d], kcent [Cm, d], codes [3, N] uint16.
+    khead_off: the review page's ablation (online k_head disabled): r_c = b_c."""
     qcent = np.ascontiguousarray(qcent, np.float64)
     kcent = np.ascontiguousarray(kcent, np.float64)
     qsizes = np.ascontiguousarray(qsizes, np.int32)
@@ -115,7 +116,8 @@ def select(qcent, qsizes, kcent, codes, d_split, rho, alpha, want_scores=False):
     mask = np.empty((Cq, nw), np.uint32)
     margin = np.empty(Cq, np.float64)
     rc = lib().oracle_select(qcent, qsizes, kcent, codes, N, d, dt, dh, dw, Cq, Cm, float(rho),
-                             float(alpha), _ptr(scores), p, b, kh, r, mask, _ptr(margin))
+                             float(alpha), _ptr(scores), p, b, kh, r, mask, _ptr(margin),
+                             1 if khead_off else 0)
     if rc:
         raise ValueError(f"oracle_select failed ({rc})")
     out = {"p": p, "b": b, "k_head": int(kh[0]), "r": r, "mask": mask, "topp_margin": margin}
@@ -168,12 +170,12 @@ def cluster_keys(K, d_split, Cm, iters, init_idx3=None, init_cent=None, logs=Fal
     return {"centroids": cent, "codes": codes, "sizes": sizes, "per_subspace": extra}
 
 
-def forward_head(q, k, v, wl, q_init, k_init, rows=None, logs=False, rho=None):
+def forward_head(q, k, v, wl, q_init, k_init, rows=None, logs=False, rho=None, khead_off=False):
     """The whole hot path for one head: clustering, selection, sparse attention."""
     rho = wl.rho if rho is None else rho
     qc = kmeans(q, 0, wl.d, wl.Cq, wl.iters, init_idx=q_init, logs=logs)
     kc = cluster_keys(k, (wl.d_t, wl.d_h, wl.d_w), wl.Cm, wl.iters, init_idx3=k_init, logs=logs)
     sel = select(qc["centroids"], qc["sizes"], kc["centroids"], kc["codes"],
-                 (wl.d_t, wl.d_h, wl.d_w), rho, wl.alpha)
+                 (wl.d_t, wl.d_h, wl.d_w), rho, wl.alpha, khead_off=khead_off)
     O = attention(q, k, v, qc["assign"], sel["mask"], rows=rows)
     return {"q": qc, "k": kc, "sel": sel, "O": O}

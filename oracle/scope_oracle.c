@@ -224,6 +224,8 @@ int64_t oracle_kfix(double alpha, int64_t N)
  *   Eq. 9: k_head = ceil( sum_c n_c b_c / sum_c n_c ), exact integer arithmetic.
  *   Eq. 10: r_c = max(b_c, k_head): only clusters below k_head take extra keys, the
  *     next ones in their ranking.  S_c = the first r_c keys of the ranking.
+ *   khead_off != 0 (the review page's ablation, significance: the online k_head
+ *     disabled): k_head is still computed and reported, r_c = b_c.
  * Outputs: p, b, r [Cq]; *khead; mask [Cq, ceil(N/32)] (bit j%32 of word j/32 set iff
  * key j is in S_c); optional scores [Cq, N]; optional topp_margin [Cq]
  * = min over r in {p_c - 1, p_c} of |mass_r - rho Z| / Z (the decision's closeness to
@@ -232,7 +234,8 @@ int64_t oracle_kfix(double alpha, int64_t N)
 int oracle_select(const double *qcent, const int32_t *qsizes, const double *kcent,
                   const uint16_t *codes, int64_t N, int d, int dt, int dh, int dw, int Cq, int Cm,
                   double rho, double alpha, double *scores, int32_t *p_out, int32_t *b_out,
-                  int32_t *khead_out, int32_t *r_out, uint32_t *mask, double *topp_margin)
+                  int32_t *khead_out, int32_t *r_out, uint32_t *mask, double *topp_margin,
+                  int khead_off)
 {
     if (dt + dh + dw != d || N <= 0 || Cq <= 0 || Cm <= 0 || !(rho > 0.0 && rho <= 1.0)
         || !(alpha >= 0.0 && alpha <= 1.0))
@@ -310,7 +313,7 @@ int oracle_select(const double *qcent, const int32_t *qsizes, const double *kcen
         #pragma omp for schedule(dynamic, 1)
         for (int c = 0; c < Cq; ++c) {
             if (!lut || !s || !order) continue;
-            int64_t r = b_out[c] < khead ? khead : b_out[c];
+            int64_t r = (b_out[c] < khead && !khead_off) ? khead : b_out[c];
             r_out[c] = (int32_t)r;
             proxy_scores(qcent + (size_t)c * d, kcent, codes, N, d, bounds, Cm, lut, s);
             rank_keys(s, N, order);

@@ -34,8 +34,11 @@ def _dev(w, x, q_init=None, k_init=None):
     return t
 
 
-def _forward_and_compare(w, x, t, q_init, k_init, rho=None):
-    p = capi.Params.from_workload(w, **({} if rho is None else {"rho": rho}))
+def _forward_and_compare(w, x, t, q_init, k_init, rho=None, khead_off=False):
+    over = {} if rho is None else {"rho": rho}
+    if khead_off:
+        over["khead_mode"] = capi.SCOPE_KHEAD_OFF
+    p = capi.Params.from_workload(w, **over)
     ws = capi.alloc_workspace(p)
     O, it = capi.forward(p, t["q"], t["k"], t["v"], t["qi"], t["ki"], ws=ws, intermediates=True)
     torch.cuda.synchronize()
@@ -43,12 +46,14 @@ def _forward_and_compare(w, x, t, q_init, k_init, rho=None):
     g = {k: to_np(v) for k, v in it.items()}
     O = O.float().cpu().numpy().reshape(w.B * w.H, w.N, w.d)
     for i in range(w.B * w.H):
-        ref = oracle.forward_head(x["q"][i], x["k"][i], x["v"][i], w, q_init[i], k_init[i], rho=rho)
+        ref = oracle.forward_head(x["q"][i], x["k"][i], x["v"][i], w, q_init[i], k_init[i], rho=rho,
+                                  khead_off=khead_off)
         np.testing.assert_array_equal(g["q_assign"][0, i], ref["q"]["assign"])
         np.testing.assert_array_equal(g["q_centroids"][0, i], ref["q"]["centroids"])
         np.testing.assert_array_equal(g["k_codes"][0, i], ref["k"]["codes"])
         np.testing.assert_array_equal(g["k_centroids"][0, i], ref["k"]["centroids"])
         np.testing.assert_array_equal(g["final_counts"][0, i], ref["sel"]["r"])
+        assert int(g["k_head"][0, i]) == ref["sel"]["k_head"]
         np.testing.assert_array_equal(g["sel_mask"][0, i].view(np.uint32), ref["sel"]["mask"])
         compare_attention(w, O[i], ref["O"])
     return g, O
@@ -174,3 +179,13 @@ def test_member_sums_with_and_without_the_exact_parallel_path(wide):
         np.testing.assert_array_equal(to_np(qa)[0, h], ref["assign"])
         np.testing.assert_array_equal(to_np(qs)[0, h], ref["sizes"])
         np.testing.assert_array_equal(to_np(qc)[0, h], ref["centroids"])
+
+
+def test_khead_off_ablation_matches_oracle():
+    """The review page's ablation with the online k_head disabled: the whole layer (r_c =
+    b_c, no top-up) against the oracle run with the same switch."""
+    w = W.with_(Cq=20, Cm=16)
+    x = synth.layer_inputs(w)
+    t = _dev(w, x)
+    g, _ = _forward_and_compare(w, x, t, x["q_init"], x["k_init"], khead_off=True)
+    np.testing.assert_array_equal(g["final_counts"], g["base_counts"])

@@ -203,6 +203,32 @@ def test_khead_is_exact_weighted_mean_ceiling_and_topup_invariants():
             np.testing.assert_array_equal(bits[c], expect_bits)
 
 
+def test_khead_off_ablation_keeps_the_hybrid_counts():
+    """The ablation with the online k_head disabled (review page, significance): p_c, b_c and
+    k_head are those of the method, r_c = b_c, and every S_c is the b_c-key prefix of the
+    cluster's ranking, so it sits inside the method's set (equal where b_c >= k_head)."""
+    rng = np.random.default_rng(18)
+    for trial in range(4):
+        qcent, qsizes, kcent, codes, split = _random_select_inputs(rng, N=160, Cq=11, Cm=6)
+        rho = [0.5, 0.8, 0.9, 0.97][trial]
+        on = oracle.select(qcent, qsizes, kcent, codes, split, rho, 0.1, want_scores=True)
+        off = oracle.select(qcent, qsizes, kcent, codes, split, rho, 0.1, want_scores=True, khead_off=True)
+        np.testing.assert_array_equal(off["p"], on["p"])
+        np.testing.assert_array_equal(off["b"], on["b"])
+        assert off["k_head"] == on["k_head"]
+        np.testing.assert_array_equal(off["r"], off["b"])
+        bon = np.unpackbits(on["mask"].view(np.uint8), bitorder="little").reshape(11, -1)[:, :160]
+        boff = np.unpackbits(off["mask"].view(np.uint8), bitorder="little").reshape(11, -1)[:, :160]
+        for c in range(11):
+            top = _ranking(off["scores"][c])[:off["b"][c]]
+            expect_bits = np.zeros(160, np.uint8)
+            expect_bits[top] = 1
+            np.testing.assert_array_equal(boff[c], expect_bits)
+            assert np.all(boff[c] <= bon[c])
+            if on["b"][c] >= on["k_head"]:
+                np.testing.assert_array_equal(boff[c], bon[c])
+
+
 def test_lossless_codebook_gives_exact_logits():
     """Keys whose subspace parts take at most Cm distinct values, clustered from those
     values, are reproduced exactly (k_hat = k), so the proxy is the true logit."""
