@@ -23,7 +23,8 @@ DEV_BAD_INIT_INDEX, DEV_SELECT_TIE, DEV_BAD_ASSIGN = 0x1, 0x2, 0x4
 
 EXPORTS = ("scope_workspace_bytes", "scope_cluster_queries", "scope_cluster_keys",
            "scope_build_lut_and_select", "scope_sparse_attention", "scope_forward",
-           "scope_status_string", "scope_get_device_status", "scope_build_lut_and_select_noalloc")
+           "scope_status_string", "scope_get_device_status", "scope_build_lut_and_select_noalloc",
+           "scope_selection_recall")
 
 
 class ScopeError(RuntimeError):
@@ -94,6 +95,9 @@ def lib() -> ctypes.CDLL:
                                     vp, sz, vp]
         L.scope_build_lut_and_select_noalloc.restype = i
         L.scope_build_lut_and_select_noalloc.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+        L.scope_selection_recall.restype = i
+        L.scope_selection_recall.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, i, ctypes.c_double,
+                                             vp, vp, vp, sz, vp]
         L.scope_status_string.restype = ctypes.c_char_p
         L.scope_status_string.argtypes = [i]
         L.scope_get_device_status.restype = i
@@ -236,6 +240,23 @@ def forward(p, Q, K, V, q_init_idx, k_init_idx, ws=None, out=None, intermediates
     if intermediates:
         return O, tensors
     return O
+
+
+def selection_recall(p, Q, K, q_assign, q_centroids, k_centroids, k_codes, sel_mask, samples, frac,
+                     scratch=None, stream=None):
+    """Proxy-ranking fidelity for the sampled queries (int64 indices (b*H + h)*N + i):
+    returns (recall_sel, recall_proxy), float64 [n_samples] each."""
+    dev = Q.device
+    n = samples.numel()
+    rs = torch.empty(n, dtype=torch.float64, device=dev)
+    rp = torch.empty(n, dtype=torch.float64, device=dev)
+    if scratch is None:
+        scratch = torch.empty(16 * p.N * min(max(n, 1), 148), dtype=torch.uint8, device=dev)
+    _check("scope_selection_recall", lib().scope_selection_recall(
+        ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(q_assign), _ptr(q_centroids), _ptr(k_centroids),
+        _ptr(k_codes), _ptr(sel_mask), _ptr(samples), n, float(frac), _ptr(rs), _ptr(rp),
+        _ptr(scratch), scratch.numel(), _stream(stream)))
+    return rs, rp
 
 
 def get_device_status(ws, stream=None) -> int:

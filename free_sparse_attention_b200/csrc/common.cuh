@@ -113,6 +113,26 @@ cudaError_t attention_run(const AttnArgs &a, cudaStream_t s);     // items + ker
 cudaError_t attention_items(const AttnArgs &a, cudaStream_t s);   // work list only
 cudaError_t attention_kernel(const AttnArgs &a, cudaStream_t s);  // kernel only
 cudaError_t attention_simt_run(const AttnArgs &a, cudaStream_t s);
+
+constexpr int kMaxFidCm = 1024;     // key centroids per subspace the fidelity kernel accepts
+struct FidArgs {
+    const void *Q, *K;
+    const uint16_t *q_assign;   // [BH, N]
+    const double *qcent;        // [BH, Cq, d]
+    const double *kcent;        // [BH, Cm, d]
+    const uint16_t *codes;      // [BH, 3, N]
+    const uint32_t *mask;       // [BH, Cq, nw]
+    const long long *samples;   // global query indices bh * N + i
+    int n_samples;
+    long long total;            // BH * N (samples outside [0, total) give NaN)
+    double *recall_sel, *recall_proxy;
+    double *scratch;            // [blocks, 2, N]
+    int blocks;
+    int N, d, dt, dh, dw, Cq, Cm, nw, is_bf16;
+    double inv_sqrt_d;
+    long long k;                // ceil(frac * N)
+};
+cudaError_t fidelity_run(const FidArgs &a, cudaStream_t s);
 size_t select_smem_bytes(int Cm, int d);
 
 // ---------------------------------------------------------------------------------

@@ -410,6 +410,60 @@ scope_status scope_sparse_attention(const scope_params *p, const void *Q, const 
     return cuda_status(attention_run(t, s));
 }
 
+scope_status scope_selection_recall(const scope_params *p, const void *Q, const void *K,
+                                    const uint16_t *q_assign, const double *q_centroids,
+                                    const double *k_centroids, const uint16_t *k_codes,
+                                    const uint32_t *sel_mask, const int64_t *samples, int n_samples,
+                                    double frac, double *recall_sel, double *recall_proxy,
+                                    void *scratch, size_t scratch_bytes, void *stream)
+{
+    scope_status st = validate(p);
+    if (st != SCOPE_OK) return st;
+    if (!ok_ptr(Q) || !ok_ptr(K) || !ok_ptr(q_assign) || !ok_ptr(q_centroids) || !ok_ptr(k_centroids) ||
+        !ok_ptr(k_codes) || !ok_ptr(sel_mask) || n_samples < 0 || (n_samples > 0 && !ok_ptr(samples)) ||
+        (n_samples > 0 && (!ok_ptr(recall_sel) || !ok_ptr(recall_proxy))) || !ok_ptr(scratch) ||
+        !(frac > 0.0 && frac <= 1.0))
+        return SCOPE_ERR_INVALID_ARGUMENT;
+    if (p->Cm > kMaxFidCm) return SCOPE_ERR_UNSUPPORTED;
+    const Dims D = dims_of(*p);
+    const size_t per = (size_t)16 * (size_t)D.N;
+    if (scratch_bytes < per) return SCOPE_ERR_WORKSPACE_TOO_SMALL;
+    if (n_samples == 0) return SCOPE_OK;
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return SCOPE_ERR_CUDA;
+    FidArgs a{};
+    a.Q = Q;
+    a.K = K;
+    a.q_assign = q_assign;
+    a.qcent = q_centroids;
+    a.kcent = k_centroids;
+    a.codes = k_codes;
+    a.mask = sel_mask;
+    a.samples = reinterpret_cast<const long long *>(samples);
+    a.n_samples = n_samples;
+    a.total = D.BH * D.N;
+    a.recall_sel = recall_sel;
+    a.recall_proxy = recall_proxy;
+    a.scratch = static_cast<double *>(scratch);
+    const size_t fit = scratch_bytes / per;
+    a.blocks = (int)(fit < (size_t)sms ? fit : (size_t)sms);
+    a.N = (int)D.N;
+    a.d = p->d;
+    a.dt = p->d_t;
+    a.dh = p->d_h;
+    a.dw = p->d_w;
+    a.Cq = p->Cq;
+    a.Cm = p->Cm;
+    a.nw = (int)D.nw;
+    a.is_bf16 = p->dtype == SCOPE_BF16;
+    a.inv_sqrt_d = 1.0 / std::sqrt((double)p->d);
+    const double kk = std::ceil(frac * (double)D.N);
+    a.k = kk < 1.0 ? 1 : (kk > (double)D.N ? D.N : (long long)kk);
+    return cuda_status(fidelity_run(a, static_cast<cudaStream_t>(stream)));
+}
+
 scope_status scope_forward(const scope_params *p, const void *Q, const void *K, const void *V,
                            const int32_t *q_init_idx, const int32_t *k_init_idx, void *O,
                            const scope_intermediates *inter, void *ws, size_t ws_bytes,

@@ -226,6 +226,29 @@ scope_status scope_build_lut_and_select_noalloc(const scope_params *p, const dou
                                                 int32_t *final_counts, uint32_t *sel_mask,
                                                 void *stream);
 
+/*
+ * Proxy-ranking fidelity (review page, falsifier and skeptic's concrete test: how many of
+ * a query's dominant keys the centroid-product proxy of Eq. 6 and the selected set keep).
+ * For every sampled query g = (b*H + h)*N + i of a layer that went through the stages
+ * above: T = its ceil(frac*N) keys of largest exact logit q_i.k_j (binary64, channels in
+ * order; ties to the lower key index); recall_sel[s] = |T n S_c| / |T|, S_c the selection
+ * of its cluster c = q_assign[g]; recall_proxy[s] = |T n P| / |T|, P the ceil(frac*N) keys
+ * of largest proxy logit of cluster c (Eq. 6, binary64; ties to the lower index).
+ * Inputs (device): Q, K [B,H,N,d] in params->dtype; q_assign [B,H,N]; q_centroids
+ * [B,H,Cq,d]; k_centroids [B,H,Cm,d]; k_codes [B,H,3,N]; sel_mask [B,H,Cq,ceil(N/32)];
+ * samples: n_samples int64 query indices.  Outputs (device): recall_sel, recall_proxy,
+ * n_samples doubles each (NaN for an index outside the layer).  scratch: caller-owned
+ * device memory, 16*N bytes per sample processed at once (at least 16*N; up to one sample
+ * per SM).  Requires 0 < frac <= 1 and Cm <= 1024; invalid arguments return an error
+ * before any launch.  Allocates nothing; enqueues on `stream`.
+ */
+scope_status scope_selection_recall(const scope_params *p, const void *Q, const void *K,
+                                    const uint16_t *q_assign, const double *q_centroids,
+                                    const double *k_centroids, const uint16_t *k_codes,
+                                    const uint32_t *sel_mask, const int64_t *samples, int n_samples,
+                                    double frac, double *recall_sel, double *recall_proxy,
+                                    void *scratch, size_t scratch_bytes, void *stream);
+
 /* Human-readable name of a status code (static storage). */
 const char *scope_status_string(scope_status s);
 

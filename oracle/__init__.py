@@ -20,6 +20,8 @@ from __future__ import annotations
 import ctypes
 import os
 
+import math
+
 import numpy as np
 
 from .build import build as _build
@@ -179,3 +181,24 @@ def forward_head(q, k, v, wl, q_init, k_init, rows=None, logs=False, rho=None, k
                  (wl.d_t, wl.d_h, wl.d_w), rho, wl.alpha, khead_off=khead_off)
     O = attention(q, k, v, qc["assign"], sel["mask"], rows=rows)
     return {"q": qc, "k": kc, "sel": sel, "O": O}
+
+
+def selection_recall(q, K, proxy, selected, frac):
+    """Proxy-ranking fidelity of one query (review page, falsifier and skeptic's concrete
+    test), from the definition: the query's exact logits l_j = q . k_j in binary64 with the
+    channels summed in order, T = its ceil(frac N) keys of largest logit (ties to the lower
+    index), P = the ceil(frac N) keys of largest proxy logit (ties to the lower index).
+    q [d], K [N, d], proxy [N] (Eq. 6 logits of the query's cluster), selected [N] bool.
+    Returns (|T n S| / |T|, |T n P| / |T|)."""
+    q = np.asarray(q, np.float64)
+    K = np.asarray(K, np.float64)
+    N = K.shape[0]
+    logit = np.zeros(N, np.float64)
+    for e in range(q.shape[0]):
+        logit = logit + q[e] * K[:, e]
+    k = min(max(int(math.ceil(frac * N)), 1), N)
+    idx = np.arange(N)
+    top_true = np.lexsort((idx, -logit))[:k]
+    top_proxy = np.lexsort((idx, -np.asarray(proxy, np.float64)))[:k]
+    sel = np.asarray(selected, bool)
+    return float(sel[top_true].sum()) / k, float(np.isin(top_true, top_proxy).sum()) / k

@@ -189,3 +189,41 @@ def test_khead_off_ablation_matches_oracle():
     t = _dev(w, x)
     g, _ = _forward_and_compare(w, x, t, x["q_init"], x["k_init"], khead_off=True)
     np.testing.assert_array_equal(g["final_counts"], g["base_counts"])
+
+
+def test_warm_start_from_previous_step_with_one_iteration():
+    """Warm start across denoising steps (review page, pith_inferences): the next step's
+    layer (the same inputs plus small noise) clusters from the previous step's centroids
+    with a single Lloyd iteration, then selects and attends through the stage entry
+    points; every stage equals the oracle run from the same centroids."""
+    w = W.with_(Cq=12, Cm=10)
+    x = synth.layer_inputs(w)
+    t = _dev(w, x)
+    p = capi.Params.from_workload(w)
+    _, it = capi.forward(p, t["q"], t["k"], t["v"], t["qi"], t["ki"], intermediates=True)
+    qc0, kc0 = it["q_centroids"].clone(), it["k_centroids"].clone()
+    rng = np.random.default_rng(9)
+    x2 = dict(x)
+    for n in "qkv":
+        x2[n] = _bf16_exact(x[n] + 0.05 * rng.standard_normal(x[n].shape))
+    t2 = _dev(w, x2)
+    p1 = capi.Params.from_workload(w, iters=1)
+    qc, qa, qs = capi.cluster_queries(p1, t2["q"], init_cent=qc0)
+    kc, kk = capi.cluster_keys(p1, t2["k"], init_cent=kc0)
+    sel = capi.build_lut_and_select(p, qc, qs, kc, kk)
+    O = capi.sparse_attention(p, t2["q"], t2["k"], t2["v"], qa, sel["sel_mask"], sel["final_counts"])
+    torch.cuda.synchronize()
+    O = O.float().cpu().numpy().reshape(w.H, w.N, w.d)
+    for h in range(w.H):
+        rq = oracle.kmeans(x2["q"][h], 0, w.d, w.Cq, 1, init_cent=to_np(qc0)[0, h])
+        rk = oracle.cluster_keys(x2["k"][h], (w.d_t, w.d_h, w.d_w), w.Cm, 1, init_cent=to_np(kc0)[0, h])
+        np.testing.assert_array_equal(to_np(qa)[0, h], rq["assign"])
+        np.testing.assert_array_equal(to_np(qc)[0, h], rq["centroids"])
+        np.testing.assert_array_equal(to_np(kk)[0, h], rk["codes"])
+        np.testing.assert_array_equal(to_np(kc)[0, h], rk["centroids"])
+        rs = oracle.select(rq["centroids"], rq["sizes"], rk["centroids"], rk["codes"],
+                           (w.d_t, w.d_h, w.d_w), w.rho, w.alpha)
+        np.testing.assert_array_equal(to_np(sel["final_counts"])[0, h], rs["r"])
+        np.testing.assert_array_equal(to_np(sel["sel_mask"])[0, h].view(np.uint32), rs["mask"])
+        ref = oracle.attention(x2["q"][h], x2["k"][h], x2["v"][h], rq["assign"], rs["mask"])
+        compare_attention(w, O[h], ref)

@@ -147,3 +147,32 @@ def test_forward_end_to_end(w):
             assert int(g["k_head"][b, h]) == sel["k_head"]
             np.testing.assert_array_equal(g["sel_mask"][b, h].view(np.uint32), sel["mask"])
             compare_attention(w, O[i], ref["O"])
+
+
+@pytest.mark.parametrize("w", [TINY, MID], ids=lambda w: w.name)
+def test_selection_recall_matches_oracle(w):
+    """Proxy-ranking fidelity of sampled queries through scope_selection_recall against the
+    oracle's definition (exact binary64 logits, Eq. 6 proxies, index tie-breaks)."""
+    x, t = _run(w)
+    p = capi.Params.from_workload(w)
+    ws = capi.alloc_workspace(p)
+    _, it = capi.forward(p, t["q"], t["k"], t["v"], t["q_init"], t["k_init"], ws=ws, intermediates=True)
+    rng = np.random.default_rng(12)
+    samples = np.sort(rng.choice(w.B * w.H * w.N, 23, replace=False)).astype(np.int64)
+    for frac in (0.1, 0.5):
+        rs, rp = capi.selection_recall(p, t["q"], t["k"], it["q_assign"], it["q_centroids"],
+                                       it["k_centroids"], it["k_codes"], it["sel_mask"],
+                                       torch.from_numpy(samples).cuda(), frac)
+        torch.cuda.synchronize()
+        rs, rp = to_np(rs), to_np(rp)
+        g = {k: to_np(v) for k, v in it.items()}
+        for s, gi in enumerate(samples):
+            bh, i = divmod(int(gi), w.N)
+            b, h = divmod(bh, w.H)
+            c = int(g["q_assign"][b, h, i])
+            sc = oracle.select(g["q_centroids"][b, h], g["q_sizes"][b, h], g["k_centroids"][b, h],
+                               g["k_codes"][b, h], (w.d_t, w.d_h, w.d_w), w.rho, w.alpha,
+                               want_scores=True)["scores"][c]
+            selected = mask_bits(g["sel_mask"][b, h, c], w.N).astype(bool)
+            ref = oracle.selection_recall(x["q"][bh][i], x["k"][bh], sc, selected, frac)
+            assert (rs[s], rp[s]) == ref, (s, rs[s], rp[s], ref)

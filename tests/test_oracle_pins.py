@@ -297,3 +297,41 @@ def test_tiny_forward_invariants():
     assert res["q"]["sizes"].sum() == TINY.N
     assert np.all(sel["r"] >= sel["k_head"]) and sel["k_head"] >= oracle.kfix(TINY.alpha, TINY.N)
     assert np.all(np.isfinite(res["O"]))
+
+
+def test_selection_recall_closed_forms_and_brute_force():
+    """Proxy-ranking fidelity (review page, falsifier): frac = 1 gives |S| / N and 1; a proxy
+    equal to the true logits recalls everything; selecting exactly the true top set recalls
+    everything; and a tiny case with tied logits against brute-force enumeration of the
+    ranking (value descending, index ascending)."""
+    rng = np.random.default_rng(21)
+    N, d = 97, 12
+    q = rng.standard_normal(d)
+    K = rng.standard_normal((N, d))
+    proxy = rng.standard_normal(N)
+    sel = rng.random(N) < 0.4
+    rs, rp = oracle.selection_recall(q, K, proxy, sel, 1.0)
+    assert rs == sel.sum() / N and rp == 1.0
+    exact = K @ q
+    for frac in (0.05, 0.1, 0.33, 0.7):
+        _, rp = oracle.selection_recall(q, K, exact, sel, frac)
+        assert rp == 1.0
+        k = math.ceil(frac * N)
+        top = np.argsort(-exact, kind="stable")[:k]
+        only = np.zeros(N, bool)
+        only[top] = True
+        rs, _ = oracle.selection_recall(q, K, exact, only, frac)
+        assert rs == 1.0
+    # ties: integer-valued keys so that many logits coincide exactly
+    Kt = rng.integers(-2, 3, size=(40, 3)).astype(np.float64)
+    qt = np.array([1.0, 1.0, 0.0])
+    pt = rng.integers(0, 4, size=40).astype(np.float64)
+    st = rng.random(40) < 0.5
+    for frac in (0.1, 0.25, 0.5):
+        k = math.ceil(frac * 40)
+        lt = [(-(qt @ Kt[j]), j) for j in range(40)]
+        T = {j for _, j in sorted(lt)[:k]}
+        P = {j for _, j in sorted((-pt[j], j) for j in range(40))[:k]}
+        rs, rp = oracle.selection_recall(qt, Kt, pt, st, frac)
+        assert rs == sum(st[j] for j in T) / k
+        assert rp == len(T & P) / k
