@@ -213,6 +213,25 @@ def traffic_from_profile(kernel_file):
     return p.get("dram_bytes_per_launch")
 
 
+def ablation_inputs(args, w, x):
+    """With --random-partition, the channels of q and k permuted alike (logits unchanged;
+    the key subspaces become random channel subsets)."""
+    if args.random_partition is not None:
+        perm = np.random.default_rng(args.random_partition).permutation(w.d)
+        x["q"] = np.ascontiguousarray(x["q"][..., perm])
+        x["k"] = np.ascontiguousarray(x["k"][..., perm])
+    return x
+
+
+def ablation_desc(args):
+    s = ""
+    if args.khead_off:
+        s += " ablation: online k_head off (r_c = b_c)"
+    if args.random_partition is not None:
+        s += f" ablation: random channel partition (seed {args.random_partition})"
+    return s
+
+
 def run_scope(args, w):
     import torch
     import torch.distributed as dist
@@ -225,7 +244,7 @@ def run_scope(args, w):
                                 device_id=torch.device("cuda", local))
     capi.lib()
     p = capi.Params.from_workload(w, khead_mode=capi.SCOPE_KHEAD_OFF if args.khead_off else capi.SCOPE_KHEAD_ONLINE)
-    x = synth.layer_inputs(w)
+    x = ablation_inputs(args, w, synth.layer_inputs(w))
     dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
     host = {n: torch.from_numpy(x[n]).reshape(w.B, w.H, w.N, w.d).to(dt).pin_memory() for n in "qkv"}
     host["qi"] = torch.from_numpy(x["q_init"]).reshape(w.B, w.H, w.Cq).pin_memory()
@@ -327,7 +346,7 @@ def run_scope(args, w):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded generator G: smooth field + noise, 3D RoPE)",
-        "config": {"workload": workload_desc(w) + (" ablation: online k_head off (r_c = b_c)" if args.khead_off else ""),
+        "config": {"workload": workload_desc(w) + ablation_desc(args),
                    "global_batch": world * w.B, "seq_len": w.N,
                    "parallelism": f"{world} independent layers, one per GPU (no collective)",
                    "l2": "inputs larger than L2 (Q, K, V = 2.19 GB resident in HBM)"},
@@ -470,7 +489,7 @@ def run_fidelity(args, w):
 
     capi.lib()
     p = capi.Params.from_workload(w, khead_mode=capi.SCOPE_KHEAD_OFF if args.khead_off else capi.SCOPE_KHEAD_ONLINE)
-    x = synth.layer_inputs(w)
+    x = ablation_inputs(args, w, synth.layer_inputs(w))
     dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
     Q, K, V = (torch.from_numpy(x[n]).reshape(w.B, w.H, w.N, w.d).to("cuda", dt) for n in "qkv")
     qi = torch.from_numpy(x["q_init"]).reshape(w.B, w.H, w.Cq).cuda()
@@ -495,7 +514,7 @@ def run_fidelity(args, w):
     density = float((n_c * it["final_counts"].double()).sum().item() / (w.B * w.H * w.N * w.N))
     print(json.dumps({
         "metric": "recall of each sampled query's true top 10 % keys (exact logits)",
-        "workload": workload_desc(w) + (" ablation: online k_head off" if args.khead_off else ""),
+        "workload": workload_desc(w) + ablation_desc(args),
         "samples": int(samples.size), "density": density,
         "recall_selection": {"mean": float(rs.mean()), "min": float(rs.min()), "p10": float(np.percentile(rs, 10))},
         "recall_proxy_top10": {"mean": float(rp.mean()), "min": float(rp.min()), "p10": float(np.percentile(rp, 10))},
@@ -520,6 +539,9 @@ def main():
                     help="override the workload's Top-p threshold (rho sweeps)")
     ap.add_argument("--khead-off", action="store_true",
                     help="ablation: the online k_head disabled (r_c = b_c)")
+    ap.add_argument("--random-partition", type=int, default=None, metavar="SEED",
+                    help="ablation: permute the channels of Q and K alike (seeded), so the key "
+                         "subspaces are random channel subsets")
     ap.add_argument("--fidelity", type=int, default=0, metavar="S",
                     help="proxy-ranking fidelity of S sampled queries per head (no timing run)")
     ap.add_argument("--warm-start", type=int, default=0, metavar="ITERS",

@@ -24,7 +24,7 @@ DEV_BAD_INIT_INDEX, DEV_SELECT_TIE, DEV_BAD_ASSIGN = 0x1, 0x2, 0x4
 EXPORTS = ("scope_workspace_bytes", "scope_cluster_queries", "scope_cluster_keys",
            "scope_build_lut_and_select", "scope_sparse_attention", "scope_forward",
            "scope_status_string", "scope_get_device_status", "scope_build_lut_and_select_noalloc",
-           "scope_selection_recall")
+           "scope_selection_recall", "scope_permute_channels")
 
 
 class ScopeError(RuntimeError):
@@ -98,6 +98,8 @@ def lib() -> ctypes.CDLL:
         L.scope_selection_recall.restype = i
         L.scope_selection_recall.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, i, ctypes.c_double,
                                              vp, vp, vp, sz, vp]
+        L.scope_permute_channels.restype = i
+        L.scope_permute_channels.argtypes = [P, vp, vp, vp, vp]
         L.scope_status_string.restype = ctypes.c_char_p
         L.scope_status_string.argtypes = [i]
         L.scope_get_device_status.restype = i
@@ -257,6 +259,14 @@ def selection_recall(p, Q, K, q_assign, q_centroids, k_centroids, k_codes, sel_m
         _ptr(k_codes), _ptr(sel_mask), _ptr(samples), n, float(frac), _ptr(rs), _ptr(rp),
         _ptr(scratch), scratch.numel(), _stream(stream)))
     return rs, rp
+
+
+def permute_channels(p, X, perm, out=None, stream=None):
+    """Y[..., e] = X[..., perm[e]] (perm: int32 [d] on the device)."""
+    Y = torch.empty_like(X) if out is None else out
+    _check("scope_permute_channels", lib().scope_permute_channels(
+        ctypes.byref(p), _ptr(X), _ptr(perm), _ptr(Y), _stream(stream)))
+    return Y
 
 
 def get_device_status(ws, stream=None) -> int:

@@ -133,6 +133,8 @@ struct FidArgs {
     long long k;                // ceil(frac * N)
 };
 cudaError_t fidelity_run(const FidArgs &a, cudaStream_t s);
+cudaError_t permute_channels_run(const void *X, const int32_t *perm, void *Y, long long rows, int d,
+                                 int is_bf16, int num_sms, cudaStream_t s);
 size_t select_smem_bytes(int Cm, int d);
 
 // ---------------------------------------------------------------------------------

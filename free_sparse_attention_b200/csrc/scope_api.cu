@@ -464,6 +464,21 @@ scope_status scope_selection_recall(const scope_params *p, const void *Q, const 
     return cuda_status(fidelity_run(a, static_cast<cudaStream_t>(stream)));
 }
 
+scope_status scope_permute_channels(const scope_params *p, const void *X, const int32_t *perm, void *Y,
+                                    void *stream)
+{
+    scope_status st = validate(p);
+    if (st != SCOPE_OK) return st;
+    if (!ok_ptr(X) || !ok_ptr(perm) || !ok_ptr(Y) || X == Y) return SCOPE_ERR_INVALID_ARGUMENT;
+    const Dims D = dims_of(*p);
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return SCOPE_ERR_CUDA;
+    return cuda_status(permute_channels_run(X, perm, Y, D.BH * D.N, p->d, p->dtype == SCOPE_BF16, sms,
+                                            static_cast<cudaStream_t>(stream)));
+}
+
 scope_status scope_forward(const scope_params *p, const void *Q, const void *K, const void *V,
                            const int32_t *q_init_idx, const int32_t *k_init_idx, void *O,
                            const scope_intermediates *inter, void *ws, size_t ws_bytes,

@@ -249,6 +249,18 @@ scope_status scope_selection_recall(const scope_params *p, const void *Q, const 
                                     double frac, double *recall_sel, double *recall_proxy,
                                     void *scratch, size_t scratch_bytes, void *stream);
 
+/*
+ * Channel permutation for the review page's ablation "random channel partition"
+ * (significance): Y[b,h,n,e] = X[b,h,n,perm[e]] for e < d.  One permutation applied to
+ * both Q and K leaves every logit q.k unchanged, so the layer run on the permuted Q and K
+ * (and the original V) is SCOPE with the key subspaces T, H, W made of the channel subsets
+ * perm[0 .. d_t), perm[d_t .. d_t+d_h), perm[d_t+d_h .. d) instead of the 3D-RoPE ranges.
+ * X, Y: [B,H,N,d] in params->dtype (device, distinct buffers); perm: d int32 (device), a
+ * permutation of 0 .. d-1 (entries outside [0, d) are clamped).  Enqueues on `stream`.
+ */
+scope_status scope_permute_channels(const scope_params *p, const void *X, const int32_t *perm, void *Y,
+                                    void *stream);
+
 /* Human-readable name of a status code (static storage). */
 const char *scope_status_string(scope_status s);
 

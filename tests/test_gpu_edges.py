@@ -227,3 +227,25 @@ def test_warm_start_from_previous_step_with_one_iteration():
         np.testing.assert_array_equal(to_np(sel["sel_mask"])[0, h].view(np.uint32), rs["mask"])
         ref = oracle.attention(x2["q"][h], x2["k"][h], x2["v"][h], rq["assign"], rs["mask"])
         compare_attention(w, O[h], ref)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_random_channel_partition_ablation(dtype):
+    """scope_permute_channels equals numpy indexing, and the layer run on Q and K permuted
+    alike (key subspaces = random channel subsets; review page, significance) equals the
+    oracle run on the same permuted inputs."""
+    w = W.with_(dtype=dtype, Cq=10, Cm=8)
+    x = synth.layer_inputs(w)
+    perm = np.random.default_rng(44).permutation(w.d).astype(np.int32)
+    t = _dev(w, x)
+    p = capi.Params.from_workload(w)
+    pd = torch.from_numpy(perm).cuda()
+    qp = capi.permute_channels(p, t["q"], pd)
+    kp = capi.permute_channels(p, t["k"], pd)
+    torch.cuda.synchronize()
+    xp = dict(x)
+    xp["q"] = np.ascontiguousarray(x["q"][..., perm])
+    xp["k"] = np.ascontiguousarray(x["k"][..., perm])
+    tp = _dev(w, xp)
+    assert torch.equal(qp, tp["q"]) and torch.equal(kp, tp["k"])
+    _forward_and_compare(w, xp, tp, x["q_init"], x["k_init"])

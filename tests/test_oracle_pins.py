@@ -335,3 +335,20 @@ def test_selection_recall_closed_forms_and_brute_force():
         rs, rp = oracle.selection_recall(qt, Kt, pt, st, frac)
         assert rs == sum(st[j] for j in T) / k
         assert rp == len(T & P) / k
+
+
+def test_common_channel_permutation_leaves_attention_unchanged():
+    """The random-channel-partition ablation permutes the channels of q and k alike: every
+    logit q.k, hence attention over any selection, is unchanged (up to summation order)."""
+    rng = np.random.default_rng(33)
+    N, d = 60, 16
+    q = rng.standard_normal((N, d)).astype(np.float32)
+    k = rng.standard_normal((N, d)).astype(np.float32)
+    v = rng.standard_normal((N, d)).astype(np.float32)
+    assign = rng.integers(0, 3, N).astype(np.uint16)
+    mask = rng.integers(0, 2 ** 32, size=(3, (N + 31) // 32), dtype=np.uint64).astype(np.uint32)
+    mask[:, 0] |= 1
+    perm = rng.permutation(d)
+    a = oracle.attention(q, k, v, assign, mask)
+    b = oracle.attention(np.ascontiguousarray(q[:, perm]), np.ascontiguousarray(k[:, perm]), v, assign, mask)
+    np.testing.assert_allclose(b, a, rtol=1e-12, atol=1e-14)
