@@ -522,6 +522,79 @@ def run_fidelity(args, w):
     return 0
 
 
+def run_schedule(args, w):
+    """The step before the path and the dense-prefix schedule (review page, major_comments:
+    "§4, Implementation details"), on pre-RoPE inputs resident in HBM:
+      rope      scope_rope3d of Q and K (HBM-bound: 2 reads + 2 writes of B*H*N*d elements);
+      dense     scope_dense_attention, the schedule's dense branch (4 N^2 d flops per head),
+                beside torch's scaled_dot_product_attention on the same tensors (library);
+      sparse    scope_attention_layer on a sparse (layer, step): RoPE + the SCOPE layer;
+      dense_l   scope_attention_layer on a dense (layer, step): RoPE + dense attention.
+    The schedule-weighted mean is the time of a layer >= 1 averaged over `n_steps` steps
+    of which the first `dense_steps` are dense."""
+    import torch
+    from free_sparse_attention_b200 import capi
+
+    capi.lib()
+    p = capi.Params.from_workload(w)
+    x = synth.layer_inputs(w, rope=False)
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    Q, K, V = (torch.from_numpy(x[n]).reshape(w.B, w.H, w.N, w.d).to("cuda", dt) for n in "qkv")
+    qi = torch.from_numpy(x["q_init"]).reshape(w.B, w.H, w.Cq).cuda()
+    ki = torch.from_numpy(x["k_init"]).reshape(w.B, w.H, 3, w.Cm).cuda()
+    del x
+    ws = capi.alloc_workspace(p)
+    Qr, Kr, O = torch.empty_like(Q), torch.empty_like(K), torch.empty_like(Q)
+    n_steps, dense_steps = 50, (5 if "hunyuan" in w.name else 10)
+    sparse_s = capi.Schedule(layer=1, step=dense_steps, dense_layers=1, dense_steps=dense_steps, rope=1,
+                             rope_base=10000.0)
+    dense_s = capi.Schedule(layer=0, step=dense_steps, dense_layers=1, dense_steps=dense_steps, rope=1,
+                            rope_base=10000.0)
+
+    def timed(fn, reps):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps
+
+    rope_ms = timed(lambda: capi.rope3d(p, Q, K, out_q=Qr, out_k=Kr), max(args.steps, 20))
+    capi.rope3d(p, Q, K, out_q=Qr, out_k=Kr)
+    dense_ms = timed(lambda: capi.dense_attention(p, Qr, Kr, V, ws=ws, out=O), args.steps)
+    sdpa_ms = timed(lambda: torch.nn.functional.scaled_dot_product_attention(Qr, Kr, V), args.steps)
+    sparse_ms = timed(lambda: capi.attention_layer(p, sparse_s, Q, K, V, qi, ki, ws=ws, out=O, out_q=Qr,
+                                                   out_k=Kr), args.steps)
+    dense_layer_ms = timed(lambda: capi.attention_layer(p, dense_s, Q, K, V, qi, ki, ws=ws, out=O, out_q=Qr,
+                                                        out_k=Kr), args.steps)
+    status = capi.get_device_status(ws)
+    pk = peaks()
+    elt = 2 if w.dtype == "bf16" else 4
+    rope_bytes = 4 * w.B * w.H * w.N * w.d * elt
+    rope_gbs = rope_bytes / (rope_ms * 1e-3) / 1e9
+    dense_flops = 4.0 * w.B * w.H * w.N * w.N * w.d
+    mean_ms = (dense_steps * dense_layer_ms + (n_steps - dense_steps) * sparse_ms) / n_steps
+    print(json.dumps({
+        "metric": "SCOPE layer under the dense-prefix schedule (ms, pre-RoPE inputs)",
+        "value": mean_ms, "unit": "ms", "higher_is_better": False, "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "dtype": w.dtype,
+        "config": {"workload": workload_desc(w), "n_steps": n_steps, "dense_steps": dense_steps,
+                   "dense_layers": 1, "rope_base": 10000.0,
+                   "l2": "inputs larger than L2 (Q, K, V resident in HBM)"},
+        "rope": {"ms": rope_ms, "bytes": rope_bytes, "achieved_gbs": rope_gbs, "peak_gbs": pk["hbm_gbs"],
+                 "frac": rope_gbs / pk["hbm_gbs"], "kernel": "rope3d_kernel (Q and K in one launch)"},
+        "dense_attention": {"ms": dense_ms, "tflops": dense_flops / (dense_ms * 1e-3) / 1e12,
+                            "frac": dense_flops / (dense_ms * 1e-3) / 1e12 / pk["bf16_sustained"],
+                            "torch_sdpa_ms": sdpa_ms},
+        "layer_sparse_ms": sparse_ms, "layer_dense_ms": dense_layer_ms,
+        "device_status": status}))
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -547,6 +620,9 @@ def main():
     ap.add_argument("--warm-start", type=int, default=0, metavar="ITERS",
                     help="time a next-step layer whose clustering starts from the previous "
                          "step's centroids with ITERS Lloyd iterations")
+    ap.add_argument("--schedule", action="store_true",
+                    help="pre-RoPE inputs: time 3D RoPE, the dense branch and the layer wrapper "
+                         "under the dense-prefix schedule (no main timing run)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -561,6 +637,8 @@ def main():
         return run_warm_start(args, w)
     if args.fidelity:
         return run_fidelity(args, w)
+    if args.schedule:
+        return run_schedule(args, w)
     if args.impl == "reference":
         return run_reference(args, w)
     return run_scope(args, w)

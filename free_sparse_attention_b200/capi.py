@@ -24,7 +24,8 @@ DEV_BAD_INIT_INDEX, DEV_SELECT_TIE, DEV_BAD_ASSIGN = 0x1, 0x2, 0x4
 EXPORTS = ("scope_workspace_bytes", "scope_cluster_queries", "scope_cluster_keys",
            "scope_build_lut_and_select", "scope_sparse_attention", "scope_forward",
            "scope_status_string", "scope_get_device_status", "scope_build_lut_and_select_noalloc",
-           "scope_selection_recall", "scope_permute_channels")
+           "scope_selection_recall", "scope_permute_channels", "scope_dense_attention",
+           "scope_rope3d", "scope_layer_is_dense", "scope_attention_layer")
 
 
 class ScopeError(RuntimeError):
@@ -60,6 +61,13 @@ class Params(ctypes.Structure):
     @property
     def nw(self) -> int:
         return (self.N + 31) // 32
+
+
+class Schedule(ctypes.Structure):
+    """scope_layer_schedule: the layer's place in the sampling loop and the dense-prefix
+    schedule (dense when layer < dense_layers or step < dense_steps)."""
+    _fields_ = [("layer", ctypes.c_int), ("step", ctypes.c_int), ("dense_layers", ctypes.c_int),
+                ("dense_steps", ctypes.c_int), ("rope", ctypes.c_int), ("rope_base", ctypes.c_double)]
 
 
 class Intermediates(ctypes.Structure):
@@ -100,6 +108,15 @@ def lib() -> ctypes.CDLL:
                                              vp, vp, vp, sz, vp]
         L.scope_permute_channels.restype = i
         L.scope_permute_channels.argtypes = [P, vp, vp, vp, vp]
+        L.scope_dense_attention.restype = i
+        L.scope_dense_attention.argtypes = [P, vp, vp, vp, vp, vp, sz, vp]
+        L.scope_rope3d.restype = i
+        L.scope_rope3d.argtypes = [P, ctypes.c_double, vp, vp, vp, vp, vp]
+        S = ctypes.POINTER(Schedule)
+        L.scope_layer_is_dense.restype = i
+        L.scope_layer_is_dense.argtypes = [S]
+        L.scope_attention_layer.restype = i
+        L.scope_attention_layer.argtypes = [P, S, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.scope_status_string.restype = ctypes.c_char_p
         L.scope_status_string.argtypes = [i]
         L.scope_get_device_status.restype = i
@@ -267,6 +284,49 @@ def permute_channels(p, X, perm, out=None, stream=None):
     _check("scope_permute_channels", lib().scope_permute_channels(
         ctypes.byref(p), _ptr(X), _ptr(perm), _ptr(Y), _stream(stream)))
     return Y
+
+
+def dense_attention(p, Q, K, V, ws=None, out=None, stream=None):
+    """Softmax attention of every query over all N keys (the schedule's dense branch)."""
+    ws = alloc_workspace(p, Q.device) if ws is None else ws
+    O = torch.empty_like(Q) if out is None else out
+    _check("scope_dense_attention", lib().scope_dense_attention(
+        ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(ws), ws.numel(), _stream(stream)))
+    return O
+
+
+def rope3d(p, Q, K=None, base=10000.0, out_q=None, out_k=None, stream=None):
+    """3D RoPE of pre-RoPE Q (and K); out_q / out_k may be Q / K (in place).
+    Returns (Qr, Kr) (Kr is None when K is None)."""
+    Qr = torch.empty_like(Q) if out_q is None else out_q
+    Kr = None if K is None else (torch.empty_like(K) if out_k is None else out_k)
+    _check("scope_rope3d", lib().scope_rope3d(
+        ctypes.byref(p), float(base), _ptr(Q), _ptr(K), _ptr(Qr), _ptr(Kr), _stream(stream)))
+    return Qr, Kr
+
+
+def layer_is_dense(sched: Schedule) -> bool:
+    """The schedule's decision, taken by the library on the host (no device needed)."""
+    r = int(lib().scope_layer_is_dense(ctypes.byref(sched)))
+    if r < 0:
+        raise ScopeError("scope_layer_is_dense", 1)
+    return bool(r)
+
+
+def attention_layer(p, sched: Schedule, Q, K, V, q_init_idx=None, k_init_idx=None, ws=None, out=None,
+                    out_q=None, out_k=None, stream=None):
+    """One layer under the dense-prefix schedule ([RoPE] then dense attention or SCOPE).
+    With sched.rope, the rotated Q and K go to out_q / out_k (new tensors when None)."""
+    ws = alloc_workspace(p, Q.device) if ws is None else ws
+    O = torch.empty_like(Q) if out is None else out
+    Qr = Kr = None
+    if sched.rope:
+        Qr = torch.empty_like(Q) if out_q is None else out_q
+        Kr = torch.empty_like(K) if out_k is None else out_k
+    _check("scope_attention_layer", lib().scope_attention_layer(
+        ctypes.byref(p), ctypes.byref(sched), _ptr(Q), _ptr(K), _ptr(V), _ptr(q_init_idx), _ptr(k_init_idx),
+        _ptr(O), _ptr(Qr), _ptr(Kr), _ptr(ws), ws.numel(), _stream(stream)))
+    return O
 
 
 def get_device_status(ws, stream=None) -> int:

@@ -210,6 +210,29 @@ cudaError_t attention_items(const AttnArgs &a, cudaStream_t s)
     return cudaGetLastError();
 }
 
+namespace {
+
+__global__ void dense_counts_kernel(int32_t *final_counts, long long BH, int N)
+{
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < BH; i += (long long)gridDim.x * blockDim.x)
+        final_counts[i] = N;
+}
+
+}  // namespace
+
+// Dense attention as one query cluster selecting every key: q_assign = 0, every mask bit
+// set (bits past N are ignored by the list kernel), r_0 = N.
+cudaError_t attention_dense_setup(uint16_t *q_assign, uint32_t *mask, int32_t *final_counts, long long BH,
+                                  long long N, long long nw, cudaStream_t s)
+{
+    cudaError_t e = cudaMemsetAsync(q_assign, 0, sizeof(uint16_t) * (size_t)(BH * N), s);
+    if (e != cudaSuccess) return e;
+    e = cudaMemsetAsync(mask, 0xFF, sizeof(uint32_t) * (size_t)(BH * nw), s);
+    if (e != cudaSuccess) return e;
+    dense_counts_kernel<<<(unsigned)((BH + 255) / 256), 256, 0, s>>>(final_counts, BH, (int)N);
+    return cudaGetLastError();
+}
+
 cudaError_t attention_simt_run(const AttnArgs &a, cudaStream_t s)
 {
     const long long warps = (long long)a.BH * a.N;

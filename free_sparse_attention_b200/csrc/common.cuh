@@ -133,6 +133,24 @@ struct FidArgs {
     long long k;                // ceil(frac * N)
 };
 cudaError_t fidelity_run(const FidArgs &a, cudaStream_t s);
+// 3D RoPE of up to two [rows, d] tensors (rope.cu).
+struct RopeArgs {
+    const void *X[2];
+    void *Y[2];
+    int n_tensors;
+    long long rows;   // B*H*N
+    int N, T, Hg, Wg;
+    int d, dt, dh, dw;
+    double base;
+    int is_bf16;
+};
+constexpr size_t kRopeMaxTableBytes = 192 * 1024;   // shared-memory cos/sin table limit
+size_t rope_table_bytes(int T, int Hg, int Wg, int dt, int dh, int dw);
+cudaError_t rope3d_run(const RopeArgs &a, int num_sms, cudaStream_t s);
+// Dense attention as the sparse kernel's special case: one query cluster that selects
+// every key (attention.cu).
+cudaError_t attention_dense_setup(uint16_t *q_assign, uint32_t *mask, int32_t *final_counts, long long BH,
+                                  long long N, long long nw, cudaStream_t s);
 cudaError_t permute_channels_run(const void *X, const int32_t *perm, void *Y, long long rows, int d,
                                  int is_bf16, int num_sms, cudaStream_t s);
 size_t select_smem_bytes(int Cm, int d);

@@ -381,6 +381,90 @@ scope_status scope_build_lut_and_select(const scope_params *p, const double *q_c
     return cuda_status(select_run(a, s));
 }
 
+namespace {
+
+// Groups the queries by cluster (stable counting sort of q_assign) and runs the attention
+// kernel; arguments already validated, status word already cleared.
+scope_status attention_impl(const scope_params &p, const WsLayout &L, void *ws, const void *Q, const void *K,
+                            const void *V, const uint16_t *q_assign, const uint32_t *sel_mask,
+                            const int32_t *final_counts, void *O, cudaStream_t s)
+{
+    KmArgs a = km_base(p, L, ws);
+    a.role0 = 0;
+    a.nroles = 1;
+    a.role[0] = query_role(p, Q, nullptr, const_cast<uint16_t *>(q_assign), at<int32_t>(ws, L.q_sizes), nullptr,
+                           nullptr);
+    a.Cs = p.Cq;
+    a.ds = p.d;
+    cudaError_t e = sort_by_cluster(a, s);
+    if (e != cudaSuccess) return SCOPE_ERR_CUDA;
+    const Dims D = dims_of(p);
+    AttnArgs t = attn_args(p, L, ws, Q, K, V, O, a.perm, D.N, a.off, p.Cq + 1, sel_mask, final_counts);
+    return cuda_status(attention_run(t, s));
+}
+
+// Dense attention: the layout of the one-cluster problem inside the caller's workspace
+// (never larger than the layout of `p` itself).
+scope_status dense_impl(const scope_params &p, void *ws, size_t ws_bytes, const void *Q, const void *K,
+                        const void *V, void *O, cudaStream_t s)
+{
+    scope_params p1 = p;
+    p1.Cq = 1;
+    const WsLayout L = ws_layout(p1);
+    if (ws_bytes < L.total) return SCOPE_ERR_WORKSPACE_TOO_SMALL;
+    const Dims D = dims_of(p1);
+    uint16_t *qa = at<uint16_t>(ws, L.q_assign);
+    uint32_t *mk = at<uint32_t>(ws, L.mask);
+    int32_t *fc = at<int32_t>(ws, L.final_cnt);
+    scope_status st = clear_status(ws, L, s);
+    if (st != SCOPE_OK) return st;
+    if (attention_dense_setup(qa, mk, fc, D.BH, D.N, D.nw, s) != cudaSuccess) return SCOPE_ERR_CUDA;
+    return attention_impl(p1, L, ws, Q, K, V, qa, mk, fc, O, s);
+}
+
+scope_status validate_rope(const scope_params &p, double base)
+{
+    if ((p.d_t & 1) || (p.d_h & 1) || (p.d_w & 1)) return SCOPE_ERR_INVALID_ARGUMENT;
+    if (!(base > 0.0) || !std::isfinite(base)) return SCOPE_ERR_INVALID_ARGUMENT;
+    if (rope_table_bytes(p.T, p.Hg, p.Wg, p.d_t, p.d_h, p.d_w) > kRopeMaxTableBytes) return SCOPE_ERR_UNSUPPORTED;
+    return SCOPE_OK;
+}
+
+scope_status rope_impl(const scope_params &p, double base, const void *Q, const void *K, void *Qr, void *Kr,
+                       cudaStream_t s)
+{
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return SCOPE_ERR_CUDA;
+    const Dims D = dims_of(p);
+    RopeArgs a{};
+    a.X[0] = Q;
+    a.Y[0] = Qr;
+    a.X[1] = K;
+    a.Y[1] = Kr;
+    a.n_tensors = K ? 2 : 1;
+    a.rows = D.BH * D.N;
+    a.N = (int)D.N;
+    a.T = p.T;
+    a.Hg = p.Hg;
+    a.Wg = p.Wg;
+    a.d = p.d;
+    a.dt = p.d_t;
+    a.dh = p.d_h;
+    a.dw = p.d_w;
+    a.base = base;
+    a.is_bf16 = p.dtype == SCOPE_BF16;
+    return cuda_status(rope3d_run(a, sms, s));
+}
+
+bool schedule_ok(const scope_layer_schedule *sc)
+{
+    return sc && sc->layer >= 0 && sc->step >= 0 && sc->dense_layers >= 0 && sc->dense_steps >= 0;
+}
+
+}  // namespace
+
 scope_status scope_sparse_attention(const scope_params *p, const void *Q, const void *K,
                                     const void *V, const uint16_t *q_assign,
                                     const uint32_t *sel_mask, const int32_t *final_counts,
@@ -394,20 +478,57 @@ scope_status scope_sparse_attention(const scope_params *p, const void *Q, const 
         !ok_ptr(final_counts) || !ok_ptr(O))
         return SCOPE_ERR_INVALID_ARGUMENT;
     if ((st = clear_status(ws, L, s)) != SCOPE_OK) return st;
-    // group the queries by cluster: stable counting sort of q_assign
-    KmArgs a = km_base(*p, L, ws);
-    a.role0 = 0;
-    a.nroles = 1;
-    a.role[0] = query_role(*p, Q, nullptr, const_cast<uint16_t *>(q_assign),
-                           at<int32_t>(ws, L.q_sizes), nullptr, nullptr);
-    a.Cs = p->Cq;
-    a.ds = p->d;
-    cudaError_t e = sort_by_cluster(a, s);
-    if (e != cudaSuccess) return SCOPE_ERR_CUDA;
-    const Dims D = dims_of(*p);
-    AttnArgs t = attn_args(*p, L, ws, Q, K, V, O, a.perm, D.N, a.off, p->Cq + 1, sel_mask,
-                           final_counts);
-    return cuda_status(attention_run(t, s));
+    return attention_impl(*p, L, ws, Q, K, V, q_assign, sel_mask, final_counts, O, s);
+}
+
+scope_status scope_dense_attention(const scope_params *p, const void *Q, const void *K, const void *V, void *O,
+                                   void *ws, size_t ws_bytes, void *stream)
+{
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    WsLayout L;
+    scope_status st = begin(p, ws, ws_bytes, L, s);
+    if (st != SCOPE_OK) return st;
+    if (!ok_ptr(Q) || !ok_ptr(K) || !ok_ptr(V) || !ok_ptr(O)) return SCOPE_ERR_INVALID_ARGUMENT;
+    return dense_impl(*p, ws, ws_bytes, Q, K, V, O, s);
+}
+
+scope_status scope_rope3d(const scope_params *p, double base, const void *Q, const void *K, void *Qr, void *Kr,
+                          void *stream)
+{
+    scope_status st = validate(p);
+    if (st != SCOPE_OK) return st;
+    if ((st = validate_rope(*p, base)) != SCOPE_OK) return st;
+    if (!ok_ptr(Q) || !ok_ptr(Qr) || !ok_opt(K) || !ok_opt(Kr) || (!K) != (!Kr)) return SCOPE_ERR_INVALID_ARGUMENT;
+    return rope_impl(*p, base, Q, K, Qr, Kr, static_cast<cudaStream_t>(stream));
+}
+
+int scope_layer_is_dense(const scope_layer_schedule *sc)
+{
+    if (!schedule_ok(sc)) return -1;
+    return (sc->layer < sc->dense_layers || sc->step < sc->dense_steps) ? 1 : 0;
+}
+
+scope_status scope_attention_layer(const scope_params *p, const scope_layer_schedule *sc, const void *Q,
+                                   const void *K, const void *V, const int32_t *q_init_idx,
+                                   const int32_t *k_init_idx, void *O, void *Qr, void *Kr, void *ws,
+                                   size_t ws_bytes, void *stream)
+{
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    WsLayout L;
+    scope_status st = begin(p, ws, ws_bytes, L, s);
+    if (st != SCOPE_OK) return st;
+    if (!schedule_ok(sc) || !ok_ptr(Q) || !ok_ptr(K) || !ok_ptr(V) || !ok_ptr(O)) return SCOPE_ERR_INVALID_ARGUMENT;
+    const bool dense = scope_layer_is_dense(sc) == 1;
+    if (!dense && (!ok_ptr(q_init_idx) || !ok_ptr(k_init_idx))) return SCOPE_ERR_INVALID_ARGUMENT;
+    if (sc->rope) {
+        if ((st = validate_rope(*p, sc->rope_base)) != SCOPE_OK) return st;
+        if (!ok_ptr(Qr) || !ok_ptr(Kr)) return SCOPE_ERR_INVALID_ARGUMENT;
+        if ((st = rope_impl(*p, sc->rope_base, Q, K, Qr, Kr, s)) != SCOPE_OK) return st;
+        Q = Qr;
+        K = Kr;
+    }
+    if (dense) return dense_impl(*p, ws, ws_bytes, Q, K, V, O, s);
+    return scope_forward(p, Q, K, V, q_init_idx, k_init_idx, O, nullptr, ws, ws_bytes, stream);
 }
 
 scope_status scope_selection_recall(const scope_params *p, const void *Q, const void *K,

@@ -14,7 +14,9 @@ Recipe, per (batch b, head h) and per tensor x in {q, k, v}, token (t, h, w):
 with a_i ~ N(0,1), omega_i uniform in {0..3}^3, phi_i ~ U[0, 2*pi),
 u_i ~ N(0, I_d)/sqrt(d) and eps ~ N(0, I_d).  q and k then get 3D rotary embedding
 (RoFormer pairs (2i, 2i+1) inside each of the temporal / height / width channel
-blocks, theta_i = 10000^(-2i/d_axis), integer positions t, h, w).  Values are built in
+blocks, theta_i = 10000^(-2i/d_axis), integer positions t, h, w), unless pre-RoPE
+inputs are asked for; that rotation is the generator's own, shared with neither the
+oracle nor the CUDA path, which each implement RoPE separately.  Values are built in
 float64, rounded to float32 (round-to-nearest-even) and, for bf16 workloads, to bf16
 (round-to-nearest-even).  Token index n = t*Hg*Wg + h*Wg + w.
 
@@ -74,8 +76,13 @@ def _rope3d_inplace(x: np.ndarray, w: Workload, pos) -> None:
         c0 += d_a
 
 
-def head_tensor(w: Workload, b: int, h: int, which: str) -> np.ndarray:
-    """One head's q, k or v as a float32 [N, d] array holding values of w.dtype."""
+def head_tensor(w: Workload, b: int, h: int, which: str, rope: bool = True,
+                raw: bool = False) -> np.ndarray:
+    """One head's q, k or v as a float32 [N, d] array holding values of w.dtype.
+
+    rope=False leaves q and k pre-RoPE (the same draws, no rotation): the inputs of the
+    layer variant that applies 3D RoPE on the device.  raw=True returns the float64
+    values before any rounding."""
     rng = _stream(w.seed, b, h, TENSOR_IDS[which])
     d, N = w.d, w.N
     a = rng.standard_normal(N_COMPONENTS)
@@ -88,8 +95,10 @@ def head_tensor(w: Workload, b: int, h: int, which: str) -> np.ndarray:
                          + np.outer(pw / w.Wg, omega[:, 2])) + phi[None, :]
     x = (a[None, :] * np.cos(arg)) @ u
     x += 0.5 * eps
-    if which in ("q", "k"):
+    if rope and which in ("q", "k"):
         _rope3d_inplace(x, w, (pt, ph, pw))
+    if raw:
+        return x
     x32 = x.astype(np.float32)
     if w.dtype == "bf16":
         x32 = round_to_bf16(x32)
@@ -103,8 +112,10 @@ def init_indices(w: Workload, b: int, h: int, role: int) -> np.ndarray:
     return rng.choice(w.N, size=C, replace=False).astype(np.int32)
 
 
-def layer_inputs(w: Workload, heads=None):
+def layer_inputs(w: Workload, heads=None, rope: bool = True):
     """Q, K, V as float32 [B, H', N, d] plus init indices, for the listed (b, h) heads.
+
+    rope=False gives pre-RoPE q and k (see head_tensor).
 
     ``heads`` is a list of (b, h); None means every head.  Returns a dict with
     "q", "k", "v" ([B*H' heads stacked as given], N, d), "q_init" [heads, Cq] and
@@ -118,7 +129,7 @@ def layer_inputs(w: Workload, heads=None):
 
     def fill(job):
         i, (b, h), name = job
-        out[name][i] = head_tensor(w, b, h, name)
+        out[name][i] = head_tensor(w, b, h, name, rope=rope)
 
     jobs = [(i, bh, name) for i, bh in enumerate(heads) for name in ("q", "k", "v")]
     # numpy's generators and ufuncs release the GIL, so threads overlap the draws

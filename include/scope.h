@@ -261,6 +261,74 @@ scope_status scope_selection_recall(const scope_params *p, const void *Q, const 
 scope_status scope_permute_channels(const scope_params *p, const void *X, const int32_t *perm, void *Y,
                                     void *stream);
 
+/*
+ * Dense attention, O_i = sum_j softmax_j(q_i . k_j / sqrt d) v_j over all N keys, on the
+ * same kernels as scope_sparse_attention (one query cluster that selects every key).  It is
+ * the dense branch of the dense-prefix schedule (review page, major_comments: "§4,
+ * Implementation details": the first attention layer runs dense at every denoising step,
+ * and every layer runs dense during the first 20 % (Wan2.1/2.2) or 10 % (HunyuanVideo) of
+ * the steps).
+ *   Q, K, V [B,H,N,d] dtype;  O out [B,H,N,d] dtype
+ *   ws      workspace of at least scope_workspace_bytes(p) bytes (p->Cq, p->Cm, p->iters,
+ *           p->rho, p->alpha and p->khead_mode are validated but not used)
+ */
+scope_status scope_dense_attention(const scope_params *p, const void *Q, const void *K, const void *V, void *O,
+                                   void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * 3D rotary position embedding (RoPE) of pre-RoPE queries and keys, the step before the
+ * path: SCOPE clusters post-RoPE q and k, whose channels split into the temporal, height and
+ * width ranges of 3D RoPE (SCOPE abstract; the rotation is RoFormer's, the page's reference
+ * [31]).  For token n = t*Hg*Wg + h*Wg + w and channel range a in {T, H, W} (start c_a, width
+ * d_a, position p_a = t, h, w), pair i = channels (c_a + 2i, c_a + 2i + 1) turns by
+ * phi = p_a * base^(-2i / d_a):
+ *   y[c_a+2i] = x[c_a+2i] cos phi - x[c_a+2i+1] sin phi
+ *   y[c_a+2i+1] = x[c_a+2i] sin phi + x[c_a+2i+1] cos phi
+ *   Q  [B,H,N,d] dtype, Qr out [B,H,N,d] dtype (Qr may be Q: in place)
+ *   K, Kr  the same for the keys, or both NULL to rotate Q only
+ *   base   > 0 (10000 for the usual RoPE)
+ * Arithmetic: angle, cos and sin in binary64, the two products and their sum each rounded
+ * to binary64 (no fused multiply-add), then one rounding to dtype.  Requires even d_t, d_h,
+ * d_w (else SCOPE_ERR_INVALID_ARGUMENT) and 16 * (T*d_t + Hg*d_h + Wg*d_w) / 2 <= 196608
+ * (the cos/sin table lives in shared memory; else SCOPE_ERR_UNSUPPORTED).  Input and output
+ * must be the same buffer or not overlap at all.  No workspace; allocates nothing.
+ */
+scope_status scope_rope3d(const scope_params *p, double base, const void *Q, const void *K, void *Qr, void *Kr,
+                          void *stream);
+
+/* Where a layer sits in the sampling loop, and the dense-prefix schedule (review page,
+ * major_comments: "§4, Implementation details"): a layer runs dense attention when
+ * layer < dense_layers (the paper: the first layer, dense_layers = 1) or step < dense_steps
+ * (the paper: the first 20 % of the denoising steps on Wan2.1/2.2, 10 % on HunyuanVideo;
+ * e.g. 10 or 5 of 50 steps), and SCOPE otherwise.  rope != 0: Q and K are pre-RoPE and get
+ * scope_rope3d with rope_base first. */
+typedef struct {
+    int layer;        /* attention layer index in the model, from 0 */
+    int step;         /* denoising step index, from 0 */
+    int dense_layers;
+    int dense_steps;
+    int rope;
+    double rope_base;
+} scope_layer_schedule;
+
+/* 1 when the schedule makes this layer dense, 0 when it runs SCOPE, -1 for a NULL
+ * schedule or a negative field.  Host only; touches no device. */
+int scope_layer_is_dense(const scope_layer_schedule *sched);
+
+/*
+ * One attention layer under the dense-prefix schedule: [3D RoPE of Q and K into Qr, Kr]
+ * then scope_dense_attention or scope_forward.
+ *   q_init_idx, k_init_idx  as for scope_forward (may be NULL on a dense layer)
+ *   Qr, Kr  [B,H,N,d] dtype outputs of the rotation when sched->rope (may be Q and K: in
+ *           place); ignored otherwise
+ *   ws      at least scope_workspace_bytes(p) bytes
+ * All arguments of both stages are validated before anything is enqueued.
+ */
+scope_status scope_attention_layer(const scope_params *p, const scope_layer_schedule *sched, const void *Q,
+                                   const void *K, const void *V, const int32_t *q_init_idx,
+                                   const int32_t *k_init_idx, void *O, void *Qr, void *Kr, void *ws,
+                                   size_t ws_bytes, void *stream);
+
 /* Human-readable name of a status code (static storage). */
 const char *scope_status_string(scope_status s);
 

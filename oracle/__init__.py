@@ -14,6 +14,12 @@ Parity status of each function (what pins it, in tests/test_oracle_pins.py):
                 lossless codebook.
   attention  -- pinned: torch scaled_dot_product_attention (float64, CPU) with the
                 selection as a boolean mask; rho=1 equals dense attention.
+  rope3d     -- pinned: closed-form angles (base^(-2i/d_a) at exact powers of ten) on unit
+                vectors per axis, identity at the origin token, pair norms, the relative-
+                position property, and the input generator's own post-RoPE tensors.
+  dense_attention -- pinned: torch scaled_dot_product_attention (float64, CPU).
+  layer      -- the schedule's choice between dense_attention and forward_head, after
+                rope3d; pinned through its parts.
 """
 from __future__ import annotations
 
@@ -202,3 +208,72 @@ def selection_recall(q, K, proxy, selected, frac):
     top_proxy = np.lexsort((idx, -np.asarray(proxy, np.float64)))[:k]
     sel = np.asarray(selected, bool)
     return float(sel[top_true].sum()) / k, float(np.isin(top_true, top_proxy).sum()) / k
+
+
+def rope3d(X, grid, d_split, base=10000.0, rows=None):
+    """3D rotary position embedding of one head's [N, d] tensor, binary64.
+
+    SCOPE clusters post-RoPE queries and keys whose channels fall into the temporal,
+    height and width ranges of 3D RoPE (SCOPE abstract; the rotation is RoFormer's, the
+    page's reference [31]).  Token n = t*Hg*Wg + h*Wg + w.  In channel range a (start c_a,
+    width d_a, position p_a in (t, h, w)), pair i = channels (c_a + 2i, c_a + 2i + 1) turns
+    counter-clockwise by phi = p_a * base**(-2i/d_a):
+        y0 = x0 cos(phi) - x1 sin(phi),   y1 = x0 sin(phi) + x1 cos(phi),
+    each product rounded to binary64, then the sum (no fused multiply-add).
+    grid = (T, Hg, Wg); d_split = (d_t, d_h, d_w), each even.  rows: the token index of
+    each row of X (all tokens in order when None)."""
+    X = np.asarray(X, np.float64)
+    T, Hg, Wg = grid
+    N, d = X.shape
+    n = np.arange(N) if rows is None else np.asarray(rows, np.int64)
+    positions = (n // (Hg * Wg), (n // Wg) % Hg, n % Wg)
+    Y = X.copy()
+    c_a = 0
+    for d_a, p_a in zip(d_split, positions):
+        for i in range(d_a // 2):
+            theta = base ** ((-2.0 * i) / d_a)
+            phi = p_a.astype(np.float64) * theta
+            cs, sn = np.cos(phi), np.sin(phi)
+            x0, x1 = X[:, c_a + 2 * i], X[:, c_a + 2 * i + 1]
+            Y[:, c_a + 2 * i] = x0 * cs - x1 * sn
+            Y[:, c_a + 2 * i + 1] = x0 * sn + x1 * cs
+        c_a += d_a
+    return Y
+
+
+def dense_attention(Q, K, V, rows=None):
+    """Softmax attention of the listed query rows over all N keys: the sparse attention
+    with one query cluster that keeps every key.  float64 [nrows, d]."""
+    N = np.asarray(Q).shape[0]
+    nw = (N + 31) // 32
+    mask = np.zeros((1, nw), np.uint32)
+    for j in range(N):
+        mask[0, j // 32] |= np.uint32(1 << (j % 32))
+    return attention(Q, K, V, np.zeros(N, np.uint16), mask, rows=rows)
+
+
+def layer_is_dense(layer, step, dense_layers, dense_steps):
+    """Dense-prefix schedule (review page, major_comments: "§4, Implementation details"):
+    the first dense_layers layers at every step, and every layer during the first
+    dense_steps denoising steps, run dense attention."""
+    return layer < dense_layers or step < dense_steps
+
+
+def layer(q, k, v, wl, q_init, k_init, dense, rope_base=None, rows=None, round_rope=None):
+    """One layer: [3D RoPE of q and k, then round_rope (the rounding to the path's element
+    type)], then dense attention or the SCOPE path.  Returns the forward_head dict (with
+    "O", plus "q", "k" post-RoPE when rope_base is given)."""
+    extra = {}
+    if rope_base is not None:
+        grid, split = (wl.T, wl.Hg, wl.Wg), (wl.d_t, wl.d_h, wl.d_w)
+        q = rope3d(q, grid, split, rope_base)
+        k = rope3d(k, grid, split, rope_base)
+        if round_rope is not None:
+            q, k = round_rope(q), round_rope(k)
+        extra = {"q_rot": q, "k_rot": k}
+    if dense:
+        out = {"O": dense_attention(q, k, v, rows=rows)}
+    else:
+        out = forward_head(q, k, v, wl, q_init, k_init, rows=rows)
+    out.update(extra)
+    return out

@@ -26,7 +26,7 @@ def L():
 def _declared_functions():
     text = open(os.path.join(ROOT, "include", "scope.h")).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(scope_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(scope_[a-z0-9_]+)\s*\(", text)))
 
 
 def test_every_declared_symbol_is_exported(L):
@@ -107,3 +107,56 @@ def test_missing_library_fails_loudly(monkeypatch):
     monkeypatch.setattr(capi, "LIB_PATH", "/nonexistent/libscope.so")
     with pytest.raises(RuntimeError):
         capi.lib()
+
+
+def test_layer_schedule_decision_matches_oracle(L):
+    """scope_layer_is_dense (host logic in the library) against the oracle's reading of
+    the dense-prefix schedule."""
+    import oracle
+    for layer in range(3):
+        for step in range(12):
+            for dense_layers in (0, 1, 2):
+                for dense_steps in (0, 5, 10):
+                    s = capi.Schedule(layer=layer, step=step, dense_layers=dense_layers,
+                                      dense_steps=dense_steps, rope=0, rope_base=10000.0)
+                    assert capi.layer_is_dense(s) == oracle.layer_is_dense(layer, step, dense_layers,
+                                                                            dense_steps)
+    assert L.scope_layer_is_dense(None) == -1
+    bad = capi.Schedule(layer=-1, step=0, dense_layers=1, dense_steps=0, rope=0, rope_base=1e4)
+    assert L.scope_layer_is_dense(ctypes.byref(bad)) == -1
+
+
+def test_rope_and_layer_rejections(L):
+    fake = ctypes.c_void_p(1 << 20)
+    p = capi.Params.from_workload(TINY)
+    # odd channel ranges, bad base, K without its output
+    odd = capi.Params.from_workload(TINY, d_t=TINY.d_t - 1, d_h=TINY.d_h + 1)
+    assert L.scope_rope3d(ctypes.byref(odd), 1e4, fake, fake, fake, fake, None) == 1
+    for base in (0.0, -2.0, float("nan"), float("inf")):
+        assert L.scope_rope3d(ctypes.byref(p), base, fake, fake, fake, fake, None) == 1
+    assert L.scope_rope3d(ctypes.byref(p), 1e4, fake, fake, fake, None, None) == 1
+    assert L.scope_rope3d(ctypes.byref(p), 1e4, None, None, fake, None, None) == 1
+    # a cos/sin table larger than shared memory allows: 16 B x (1*8 + 1*12 + 1100*12) pairs
+    wide = capi.Params.from_workload(TINY, T=1, Hg=1, Wg=1100)
+    assert L.scope_rope3d(ctypes.byref(wide), 1e4, fake, fake, fake, fake, None) == 2
+    # the layer: everything validated up front
+    need = capi.workspace_bytes(p)
+    sp = capi.Schedule(layer=3, step=20, dense_layers=1, dense_steps=5, rope=1, rope_base=1e4)
+    assert L.scope_attention_layer(ctypes.byref(p), ctypes.byref(sp), fake, fake, fake, fake, fake, fake,
+                                   None, fake, fake, need, None) == 1            # no Qr
+    assert L.scope_attention_layer(ctypes.byref(p), ctypes.byref(sp), fake, fake, fake, None, fake, fake,
+                                   fake, fake, fake, need, None) == 1            # sparse, no init
+    assert L.scope_attention_layer(ctypes.byref(p), ctypes.byref(sp), fake, fake, fake, fake, fake, fake,
+                                   fake, fake, fake, need - 256, None) == 3      # workspace
+    assert L.scope_attention_layer(ctypes.byref(p), None, fake, fake, fake, fake, fake, fake,
+                                   fake, fake, fake, need, None) == 1            # no schedule
+    assert L.scope_dense_attention(ctypes.byref(p), fake, fake, fake, fake, fake, need - 256, None) == 3
+    assert L.scope_dense_attention(ctypes.byref(p), fake, None, fake, fake, fake, need, None) == 1
+
+
+@pytest.mark.parametrize("name", sorted(ALL))
+def test_dense_layout_fits_the_layer_workspace(L, name):
+    """The dense branch carves a one-cluster layout out of the layer's workspace."""
+    p = capi.Params.from_workload(ALL[name])
+    p1 = capi.Params.from_workload(ALL[name], Cq=1)
+    assert 0 < capi.workspace_bytes(p1) <= capi.workspace_bytes(p)

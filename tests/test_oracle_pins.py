@@ -352,3 +352,100 @@ def test_common_channel_permutation_leaves_attention_unchanged():
     a = oracle.attention(q, k, v, assign, mask)
     b = oracle.attention(np.ascontiguousarray(q[:, perm]), np.ascontiguousarray(k[:, perm]), v, assign, mask)
     np.testing.assert_allclose(b, a, rtol=1e-12, atol=1e-14)
+
+
+# ----------------------------------------------------------------------------- 3D RoPE
+_GRID, _SPLIT = (3, 4, 6), (16, 56, 56)   # HunyuanVideo's channel split on a small grid
+
+
+def _token(t, h, w):
+    return (t * _GRID[1] + h) * _GRID[2] + w
+
+
+def test_rope3d_closed_form_angles_per_axis():
+    """RoFormer's rotation on unit vectors at angles with closed forms: with base 10000,
+    pair i of a range of width d_a turns by p * 10^(-8i/d_a).  t = 1 turns temporal pair 0
+    by exactly 1 rad and temporal pair 4 by 10^-2; h = 3 turns height pair 14 by 3*10^-2;
+    w = 5 turns width pair 7 by 5*10^-1; every other pair of the token stays put.  (1, 0)
+    goes to (cos, sin) and (0, 1) to (-sin, cos): the counter-clockwise sense."""
+    N, d = int(np.prod(_GRID)), sum(_SPLIT)
+    cases = [  # (token, first channel of the pair, angle in rad)
+        (_token(1, 0, 0), 0, 1.0),
+        (_token(1, 0, 0), 8, 0.01),
+        (_token(0, 3, 0), 16 + 28, 0.03),
+        (_token(0, 0, 5), 72 + 14, 0.5),
+    ]
+    # the printed decimal values of cos and sin at those angles
+    table = {1.0: (0.5403023058681398, 0.8414709848078965),
+             0.01: (0.9999500004166653, 0.009999833334166664),
+             0.03: (0.9995500337489875, 0.029995500202495664),
+             0.5: (0.8775825618903728, 0.479425538604203)}
+    for tok, c, ang in cases:
+        cs, sn = table[ang]
+        for x0, x1, e0, e1 in ((1.0, 0.0, cs, sn), (0.0, 1.0, -sn, cs)):
+            X = np.zeros((N, d))
+            X[tok, c], X[tok, c + 1] = x0, x1
+            Y = oracle.rope3d(X, _GRID, _SPLIT)
+            assert abs(Y[tok, c] - e0) < 1e-15 and abs(Y[tok, c + 1] - e1) < 1e-15, (tok, c)
+            # channels outside the pair and other tokens are untouched
+            Y[tok, c] = Y[tok, c + 1] = 0.0
+            assert not Y.any()
+
+
+def test_rope3d_origin_identity_and_pair_norms():
+    rng = np.random.default_rng(71)
+    N, d = int(np.prod(_GRID)), sum(_SPLIT)
+    X = rng.standard_normal((N, d))
+    Y = oracle.rope3d(X, _GRID, _SPLIT)
+    np.testing.assert_array_equal(Y[0], X[0])   # token (0, 0, 0): every angle is 0
+    nx = X[:, 0::2] ** 2 + X[:, 1::2] ** 2
+    ny = Y[:, 0::2] ** 2 + Y[:, 1::2] ** 2
+    np.testing.assert_allclose(ny, nx, rtol=1e-13, atol=1e-15)
+    assert np.abs(Y - X).max() > 0.5             # it does rotate
+
+
+def test_rope3d_relative_position_property():
+    """RoPE's defining property: the dot product of a rotated query and a rotated key
+    depends only on their displacement (dt, dh, dw), not on where the pair sits."""
+    rng = np.random.default_rng(72)
+    N, d = int(np.prod(_GRID)), sum(_SPLIT)
+    q, k = rng.standard_normal(d), rng.standard_normal(d)
+    Rq = oracle.rope3d(np.tile(q, (N, 1)), _GRID, _SPLIT)
+    Rk = oracle.rope3d(np.tile(k, (N, 1)), _GRID, _SPLIT)
+    for (a1, b1), (a2, b2) in [(((0, 0, 0), (1, 2, 3)), ((1, 1, 2), (2, 3, 5))),
+                               (((2, 3, 5), (0, 1, 1)), ((2, 2, 4), (0, 0, 0))),
+                               (((1, 0, 4), (1, 3, 0)), ((0, 0, 5), (0, 3, 1)))]:
+        s1 = Rq[_token(*a1)] @ Rk[_token(*b1)]
+        s2 = Rq[_token(*a2)] @ Rk[_token(*b2)]
+        assert abs(s1 - s2) < 1e-12 * (np.abs(q) @ np.abs(k))
+    # and the plain (unrotated) score is not what it gives off the diagonal
+    assert abs(Rq[_token(0, 0, 0)] @ Rk[_token(1, 2, 3)] - q @ k) > 1e-3
+
+
+@pytest.mark.parametrize("which", ["q", "k"])
+def test_rope3d_matches_generator_rotation(which):
+    """The generator rotates its own q and k (separate code, same RoFormer reading); the
+    oracle applied to the generator's pre-RoPE draws reproduces them in binary64."""
+    pre = synth.head_tensor(TINY, 0, 0, which, rope=False, raw=True)
+    post = synth.head_tensor(TINY, 0, 0, which, rope=True, raw=True)
+    got = oracle.rope3d(pre, (TINY.T, TINY.Hg, TINY.Wg), (TINY.d_t, TINY.d_h, TINY.d_w))
+    np.testing.assert_allclose(got, post, rtol=0, atol=1e-12)
+
+
+# ----------------------------------------------------------------------------- dense branch
+def test_dense_attention_equals_sdpa():
+    rng = np.random.default_rng(73)
+    N, d = 75, 32
+    Q, K, V = (rng.standard_normal((N, d)).astype(np.float32) for _ in range(3))
+    O = oracle.dense_attention(Q, K, V)
+    np.testing.assert_allclose(O, _sdpa64(Q, K, V, np.ones((N, N), bool)), rtol=1e-12, atol=1e-12)
+
+
+def test_dense_prefix_schedule_cases():
+    """The paper's schedule: the first layer dense at every step; every layer dense for the
+    first 20 % of 50 steps (Wan, 10 steps) or 10 % (HunyuanVideo, 5 steps)."""
+    for dense_steps in (10, 5):
+        for step in range(50):
+            for layer in range(4):
+                want = layer == 0 or step < dense_steps
+                assert oracle.layer_is_dense(layer, step, 1, dense_steps) == want
