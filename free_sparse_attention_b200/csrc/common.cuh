@@ -133,6 +133,10 @@ struct FidArgs {
     long long k;                // ceil(frac * N)
 };
 cudaError_t fidelity_run(const FidArgs &a, cudaStream_t s);
+// Divisor for x / d by multiply and shift (rope.cu).
+struct FastDiv {
+    unsigned m, l;
+};
 // 3D RoPE of up to two [rows, d] tensors (rope.cu).
 struct RopeArgs {
     const void *X[2];
@@ -143,6 +147,7 @@ struct RopeArgs {
     int d, dt, dh, dw;
     double base;
     int is_bf16;
+    FastDiv div_N, div_HW, div_Wg;   // filled by rope3d_run
 };
 constexpr size_t kRopeMaxTableBytes = 192 * 1024;   // shared-memory cos/sin table limit
 size_t rope_table_bytes(int T, int Hg, int Wg, int dt, int dh, int dw);

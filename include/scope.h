@@ -287,9 +287,10 @@ scope_status scope_dense_attention(const scope_params *p, const void *Q, const v
  *   Q  [B,H,N,d] dtype, Qr out [B,H,N,d] dtype (Qr may be Q: in place)
  *   K, Kr  the same for the keys, or both NULL to rotate Q only
  *   base   > 0 (10000 for the usual RoPE)
- * Arithmetic: angle, cos and sin in binary64, the two products and their sum each rounded
- * to binary64 (no fused multiply-add), then one rounding to dtype.  Requires even d_t, d_h,
- * d_w (else SCOPE_ERR_INVALID_ARGUMENT) and 16 * (T*d_t + Hg*d_h + Wg*d_w) / 2 <= 196608
+ * Result: angle, cos and sin in binary64, the two products and their sum each rounded
+ * to binary64 (no fused multiply-add), then one rounding to dtype (for bf16 a binary32
+ * evaluation is kept only where an error bound proves it rounds the same).  Requires even
+ * d_t, d_h, d_w (else SCOPE_ERR_INVALID_ARGUMENT) and 24 * (T*d_t + Hg*d_h + Wg*d_w) / 2 <= 196608
  * (the cos/sin table lives in shared memory; else SCOPE_ERR_UNSUPPORTED).  Input and output
  * must be the same buffer or not overlap at all.  No workspace; allocates nothing.
  */

@@ -136,7 +136,7 @@ def test_rope_and_layer_rejections(L):
         assert L.scope_rope3d(ctypes.byref(p), base, fake, fake, fake, fake, None) == 1
     assert L.scope_rope3d(ctypes.byref(p), 1e4, fake, fake, fake, None, None) == 1
     assert L.scope_rope3d(ctypes.byref(p), 1e4, None, None, fake, None, None) == 1
-    # a cos/sin table larger than shared memory allows: 16 B x (1*8 + 1*12 + 1100*12) pairs
+    # a cos/sin table larger than shared memory allows: 24 B x (1*8 + 1*12 + 1100*12) pairs
     wide = capi.Params.from_workload(TINY, T=1, Hg=1, Wg=1100)
     assert L.scope_rope3d(ctypes.byref(wide), 1e4, fake, fake, fake, fake, None) == 2
     # the layer: everything validated up front

@@ -165,3 +165,33 @@ def test_attention_layer_under_the_schedule(layer, step, rope):
             assert _check_rope(_np(Qr, w)[i], x["q"][i].astype(np.float64), w) == 0
             assert _check_rope(_np(Kr, w)[i], x["k"][i].astype(np.float64), w) == 0
         compare_attention(w, On[i], ref["O"])
+
+
+def test_rope3d_bf16_near_rounding_boundaries():
+    """Pairs whose rotated value lies within 2^-22 (|x0| + |x1|) of a bf16 rounding
+    boundary: the binary32 evaluation cannot decide them, so the kernel must fall back to
+    binary64 and still round like the oracle.  Temporal pair 0 of tokens with t = 1 turns
+    by exactly 1 rad."""
+    w = Workload("rope_edge", 1, 1, 2, 12, 10, 44, 42, 42, "bf16", 4, 4, seed=25)
+    rng = np.random.default_rng(9)
+    c, s = np.cos(1.0), np.sin(1.0)
+    found = []
+    while len(found) < 120:
+        e = rng.integers(-6, 6, size=(4096, 2))
+        m = rng.integers(128, 256, size=(4096, 2)) * rng.choice([-1, 1], size=(4096, 2))
+        x = np.ldexp(m.astype(np.float64), e - 7)            # bf16 values
+        S = np.abs(x).sum(axis=1)
+        for y in (x[:, 0] * c - x[:, 1] * s, x[:, 0] * s + x[:, 1] * c):
+            mid = _round(y, "bf16")
+            # nearest boundary: half a bf16 unit from the rounded value, on y's side
+            ulp = np.ldexp(1.0, np.frexp(np.abs(mid))[1] - 8)
+            dist = np.abs(np.abs(y - mid) - ulp / 2)
+            hit = np.nonzero(dist < S * 2.0 ** -22)[0]
+            found.extend(x[hit].tolist())
+    X = np.zeros((w.N, w.d), np.float32)
+    rows = np.arange(w.Hg * w.Wg, 2 * w.Hg * w.Wg)                  # tokens with t = 1
+    X[rows, 0:2] = np.asarray(found[:len(rows)], np.float32)
+    p = capi.Params.from_workload(w)
+    Qr, _ = capi.rope3d(p, _dev(w, X[None]), None)
+    torch.cuda.synchronize()
+    assert _check_rope(_np(Qr, w)[0], X.astype(np.float64), w) == 0
