@@ -223,8 +223,17 @@ def ablation_inputs(args, w, x):
     return x
 
 
+def ablation_params(args):
+    """scope_params switches of the ablations (the method when none is asked for)."""
+    from free_sparse_attention_b200 import capi
+    return {"khead_mode": capi.SCOPE_KHEAD_OFF if args.khead_off else capi.SCOPE_KHEAD_ONLINE,
+            "key_clustering": capi.SCOPE_KEYS_FULL if args.full_keys else capi.SCOPE_KEYS_SUBSPACES}
+
+
 def ablation_desc(args):
     s = ""
+    if args.full_keys:
+        s += " ablation: full-d key clustering (one k-means over all d channels)"
     if args.khead_off:
         s += " ablation: online k_head off (r_c = b_c)"
     if args.random_partition is not None:
@@ -243,7 +252,7 @@ def run_scope(args, w):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=torch.device("cuda", local))
     capi.lib()
-    p = capi.Params.from_workload(w, khead_mode=capi.SCOPE_KHEAD_OFF if args.khead_off else capi.SCOPE_KHEAD_ONLINE)
+    p = capi.Params.from_workload(w, **ablation_params(args))
     x = ablation_inputs(args, w, synth.layer_inputs(w))
     dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
     host = {n: torch.from_numpy(x[n]).reshape(w.B, w.H, w.N, w.d).to(dt).pin_memory() for n in "qkv"}
@@ -370,7 +379,7 @@ def run_scope(args, w):
         "device_status": status,
         "clocks": clk,
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.full_keys:
         s = oracle_sample(w, khead_off=args.khead_off)
         sec = layer_seconds_from_sample(s, flops)
         line["cpu_baseline"] = {"value": flops / sec / 1e12, "unit": "TFLOP/s", "cores": s["threads"],
@@ -488,7 +497,7 @@ def run_fidelity(args, w):
     from free_sparse_attention_b200 import capi
 
     capi.lib()
-    p = capi.Params.from_workload(w, khead_mode=capi.SCOPE_KHEAD_OFF if args.khead_off else capi.SCOPE_KHEAD_ONLINE)
+    p = capi.Params.from_workload(w, **ablation_params(args))
     x = ablation_inputs(args, w, synth.layer_inputs(w))
     dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
     Q, K, V = (torch.from_numpy(x[n]).reshape(w.B, w.H, w.N, w.d).to("cuda", dt) for n in "qkv")
@@ -620,6 +629,10 @@ def main():
     ap.add_argument("--warm-start", type=int, default=0, metavar="ITERS",
                     help="time a next-step layer whose clustering starts from the previous "
                          "step's centroids with ITERS Lloyd iterations")
+    ap.add_argument("--full-keys", action="store_true",
+                    help="ablation: one k-means of the keys over all d channels (cluster-level proxy)")
+    ap.add_argument("--cm", type=int, default=0,
+                    help="override the key centroid count Cm (e.g. 3 Cm with --full-keys)")
     ap.add_argument("--schedule", action="store_true",
                     help="pre-RoPE inputs: time 3D RoPE, the dense branch and the layer wrapper "
                          "under the dense-prefix schedule (no main timing run)")
@@ -631,6 +644,8 @@ def main():
         w = w.with_(H=args.heads)
     if args.rho is not None:
         w = w.with_(rho=args.rho)
+    if args.cm:
+        w = w.with_(Cm=args.cm)
     if args.profile_once:
         return profile_once(w)
     if args.warm_start:

@@ -36,6 +36,8 @@ class ScopeError(RuntimeError):
 
 SCOPE_KHEAD_ONLINE = 0   # Eqs. 9-10: clusters topped up to k_head
 SCOPE_KHEAD_OFF = 1      # ablation: r_c = b_c
+SCOPE_KEYS_SUBSPACES = 0  # the method: T / H / W key subspaces
+SCOPE_KEYS_FULL = 1       # ablation: one full-d key clustering (cluster-level proxy)
 
 
 class Params(ctypes.Structure):
@@ -44,7 +46,7 @@ class Params(ctypes.Structure):
                 ("d_t", ctypes.c_int), ("d_h", ctypes.c_int), ("d_w", ctypes.c_int),
                 ("Cq", ctypes.c_int), ("Cm", ctypes.c_int), ("iters", ctypes.c_int),
                 ("rho", ctypes.c_double), ("alpha", ctypes.c_double), ("dtype", ctypes.c_int),
-                ("khead_mode", ctypes.c_int)]
+                ("khead_mode", ctypes.c_int), ("key_clustering", ctypes.c_int)]
 
     @classmethod
     def from_workload(cls, w: Workload, **over) -> "Params":

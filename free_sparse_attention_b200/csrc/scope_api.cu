@@ -33,6 +33,8 @@ scope_status validate(const scope_params *p)
     if (!(p->rho > 0.0 && p->rho <= 1.0)) return SCOPE_ERR_INVALID_ARGUMENT;
     if (!(p->alpha >= 0.0 && p->alpha <= 1.0)) return SCOPE_ERR_INVALID_ARGUMENT;
     if (p->khead_mode != SCOPE_KHEAD_ONLINE && p->khead_mode != SCOPE_KHEAD_OFF) return SCOPE_ERR_INVALID_ARGUMENT;
+    if (p->key_clustering != SCOPE_KEYS_SUBSPACES && p->key_clustering != SCOPE_KEYS_FULL)
+        return SCOPE_ERR_INVALID_ARGUMENT;
     if (p->dtype != SCOPE_F32 && p->dtype != SCOPE_BF16) return SCOPE_ERR_INVALID_ARGUMENT;
     return SCOPE_OK;
 }
@@ -121,15 +123,32 @@ RoleDesc query_role(const scope_params &p, const void *Q, double *cent, uint16_t
     return r;
 }
 
+// Number of key k-means problems per head: three channel ranges, or one over all d.
+int key_roles(const scope_params &p)
+{
+    return p.key_clustering == SCOPE_KEYS_FULL ? 1 : 3;
+}
+
+// Channel range m of the key clustering: (start, width).
+void key_range(const scope_params &p, int m, int &ch0, int &dm)
+{
+    if (p.key_clustering == SCOPE_KEYS_FULL) {
+        ch0 = 0;
+        dm = p.d;
+        return;
+    }
+    const int bnd[4] = {0, p.d_t, p.d_t + p.d_h, p.d};
+    ch0 = bnd[m];
+    dm = bnd[m + 1] - bnd[m];
+}
+
 RoleDesc key_role(const scope_params &p, int m, const void *K, double *cent, uint16_t *codes,
                   int32_t *sizes3, const int32_t *init_idx, const double *init_cent)
 {
     const long long N = (long long)p.T * p.Hg * p.Wg;
-    const int bnd[4] = {0, p.d_t, p.d_t + p.d_h, p.d};
     RoleDesc r{};
     r.X = K;
-    r.ch0 = bnd[m];
-    r.dm = bnd[m + 1] - bnd[m];
+    key_range(p, m, r.ch0, r.dm);
     r.C = p.Cm;
     r.cent = cent;
     r.assign = codes + m * N;
@@ -140,6 +159,27 @@ RoleDesc key_role(const scope_params &p, int m, const void *K, double *cent, uin
     r.init_bh = 3ll * p.Cm;
     r.init_cent = init_cent;
     return r;
+}
+
+// With one full-d key clustering, code rows 1 and 2 of every head are zero.
+cudaError_t zero_unused_codes(const scope_params &p, uint16_t *codes, cudaStream_t s)
+{
+    if (p.key_clustering != SCOPE_KEYS_FULL) return cudaSuccess;
+    const size_t N = (size_t)p.T * p.Hg * p.Wg, BH = (size_t)p.B * p.H;
+    return cudaMemset2DAsync(codes + N, 3 * N * sizeof(uint16_t), 0, 2 * N * sizeof(uint16_t), BH, s);
+}
+
+// Subspace split the selection and the fidelity kernels read the codes with.
+void code_split(const scope_params &p, int &dt, int &dh, int &dw)
+{
+    if (p.key_clustering == SCOPE_KEYS_FULL) {
+        dt = p.d;
+        dh = dw = 0;
+    } else {
+        dt = p.d_t;
+        dh = p.d_h;
+        dw = p.d_w;
+    }
 }
 
 scope_status cuda_status(cudaError_t e)
@@ -181,9 +221,7 @@ SelArgs sel_args(const scope_params &p, const WsLayout &L, void *ws, const doubl
     a.BH = (int)D.BH;
     a.N = (int)D.N;
     a.d = p.d;
-    a.dt = p.d_t;
-    a.dh = p.d_h;
-    a.dw = p.d_w;
+    code_split(p, a.dt, a.dh, a.dw);
     a.Cq = p.Cq;
     a.Cm = p.Cm;
     a.nw = (int)D.nw;
@@ -351,13 +389,15 @@ scope_status scope_cluster_keys(const scope_params *p, const void *K, const int3
     if ((st = clear_status(ws, L, s)) != SCOPE_OK) return st;
     KmArgs a = km_base(*p, L, ws);
     a.role0 = 1;
-    a.nroles = 3;
-    for (int m = 0; m < 3; ++m)
+    a.nroles = key_roles(*p);
+    for (int m = 0; m < a.nroles; ++m)
         a.role[1 + m] = key_role(*p, m, K, k_centroids, k_codes, at<int32_t>(ws, L.k_sizes),
                                  init_idx, init_cent);
     a.Cs = p->Cm;
-    a.ds = std::max(p->d_t, std::max(p->d_h, p->d_w));
-    return cuda_status(km_run(a, p->iters, s));
+    a.ds = p->key_clustering == SCOPE_KEYS_FULL ? p->d : std::max(p->d_t, std::max(p->d_h, p->d_w));
+    cudaError_t e = km_run(a, p->iters, s);
+    if (e == cudaSuccess) e = zero_unused_codes(*p, k_codes, s);
+    return cuda_status(e);
 }
 
 scope_status scope_build_lut_and_select(const scope_params *p, const double *q_centroids,
@@ -572,9 +612,7 @@ scope_status scope_selection_recall(const scope_params *p, const void *Q, const 
     a.blocks = (int)(fit < (size_t)sms ? fit : (size_t)sms);
     a.N = (int)D.N;
     a.d = p->d;
-    a.dt = p->d_t;
-    a.dh = p->d_h;
-    a.dw = p->d_w;
+    code_split(*p, a.dt, a.dh, a.dw);
     a.Cq = p->Cq;
     a.Cm = p->Cm;
     a.nw = (int)D.nw;
@@ -638,13 +676,14 @@ scope_status scope_forward(const scope_params *p, const void *Q, const void *K, 
     // stage 1: query clustering and the three key-subspace clusterings, one launch set
     KmArgs a = km_base(*p, L, ws);
     a.role0 = 0;
-    a.nroles = 4;
+    a.nroles = 1 + key_roles(*p);
     a.role[0] = query_role(*p, Q, qc, qa, qs, q_init_idx, nullptr);
-    for (int m = 0; m < 3; ++m)
+    for (int m = 0; m + 1 < a.nroles; ++m)
         a.role[1 + m] = key_role(*p, m, K, kc, kk, at<int32_t>(ws, L.k_sizes), k_init_idx, nullptr);
     a.Cs = std::max(p->Cq, p->Cm);
     a.ds = p->d;
     cudaError_t e = km_run(a, p->iters, s);
+    if (e == cudaSuccess) e = zero_unused_codes(*p, kk, s);
     if (e != cudaSuccess || mark(1) != cudaSuccess) return SCOPE_ERR_CUDA;
 
     // stage 2: LUT, proxy logits, Top-p, k_head, top-up, masks
@@ -654,7 +693,7 @@ scope_status scope_forward(const scope_params *p, const void *Q, const void *K, 
 
     // stage 3: attention; the last clustering iteration already grouped the queries
     const Dims D = dims_of(*p);
-    AttnArgs t = attn_args(*p, L, ws, Q, K, V, O, a.perm, 4 * D.N, a.off, 4 * (a.Cs + 1), mk, fc);
+    AttnArgs t = attn_args(*p, L, ws, Q, K, V, O, a.perm, a.nroles * D.N, a.off, a.nroles * (a.Cs + 1), mk, fc);
     e = attention_items(t, s);
     if (e != cudaSuccess || mark(3) != cudaSuccess) return SCOPE_ERR_CUDA;
     e = attention_kernel(t, s);

@@ -92,9 +92,10 @@ extern "C" scope_status scope_build_lut_and_select_noalloc(
     a.BH = (int)BH;
     a.N = (int)N;
     a.d = p->d;
-    a.dt = p->d_t;
-    a.dh = p->d_h;
-    a.dw = p->d_w;
+    const bool full = p->key_clustering == SCOPE_KEYS_FULL;   // one subspace of all d channels
+    a.dt = full ? p->d : p->d_t;
+    a.dh = full ? 0 : p->d_h;
+    a.dw = full ? 0 : p->d_w;
     a.Cq = p->Cq;
     a.Cm = p->Cm;
     a.nw = (int)((N + 31) / 32);

@@ -70,11 +70,20 @@ typedef enum { SCOPE_F32 = 0, SCOPE_BF16 = 1 } scope_dtype;
  * still computed and reported, but r_c = b_c (hybrid Top-p / fixed Top-k only). */
 typedef enum { SCOPE_KHEAD_ONLINE = 0, SCOPE_KHEAD_OFF = 1 } scope_khead_mode;
 
+/* Key clustering (scope_params.key_clustering).  SUBSPACES: the method, three k-means over
+ * the temporal / height / width channel ranges.  FULL: the ablation the review page asks
+ * for (significance; falsifier: "full-dimensional cluster scoring"): one k-means of the
+ * keys over all d channels into Cm centroids, so that the proxy of Eq. 6 becomes the
+ * cluster-level s~_cj = q_c . mu_{z_j} / sqrt d.  k_codes row 0 then holds z_j and rows 1
+ * and 2 are zero; selection reads it as a one-subspace product code with split (d, 0, 0),
+ * where the two empty subspaces contribute exact zeros. */
+typedef enum { SCOPE_KEYS_SUBSPACES = 0, SCOPE_KEYS_FULL = 1 } scope_key_clustering;
+
 /* Shape and hyperparameters of one layer.  rho: Top-p threshold of Eq. 7 (the paper
  * does not report it; 0.9 is the usual choice).  alpha: fixed Top-k minimum as a
  * fraction of N, k_fix = ceil(alpha * N) (the paper gives alpha = 0.1).  iters: Lloyd
- * iterations of every k-means.  khead_mode: a scope_khead_mode (a zero-initialised
- * struct gets the method, SCOPE_KHEAD_ONLINE). */
+ * iterations of every k-means.  khead_mode: a scope_khead_mode, key_clustering: a
+ * scope_key_clustering (a zero-initialised struct gets the method in both). */
 typedef struct {
     int B, H;
     int T, Hg, Wg;
@@ -84,6 +93,7 @@ typedef struct {
     double rho, alpha;
     scope_dtype dtype;
     int khead_mode;
+    int key_clustering;
 } scope_params;
 
 /* Optional intermediate outputs of scope_forward (device pointers; NULL = keep the

@@ -153,13 +153,24 @@ def attention(Q, K, V, qassign, mask, rows=None):
     return O
 
 
-def cluster_keys(K, d_split, Cm, iters, init_idx3=None, init_cent=None, logs=False):
+def cluster_keys(K, d_split, Cm, iters, init_idx3=None, init_cent=None, logs=False, full=False):
     """The three subspace k-means of one head's keys.
 
     Returns centroids [Cm, d] (subspace m's centroid in m's channel range), codes
     [3, N] uint16 and per-subspace logs.  init_idx3 is [3, Cm]; init_cent is [Cm, d].
+    full=True: the review page's ablation (full-dimensional cluster scoring): one k-means
+    over all d channels (initial indices init_idx3[0]); codes row 0 holds the clusters and
+    rows 1, 2 are zero, to be read with the split (d, 0, 0) (see key_split).
     """
     N, d = K.shape
+    if full:
+        res = kmeans(K, 0, d, Cm, iters, init_idx=None if init_idx3 is None else init_idx3[0],
+                     init_cent=init_cent, logs=logs)
+        codes = np.zeros((3, N), np.uint16)
+        codes[0] = res["assign"]
+        sizes = np.zeros((3, Cm), np.int32)
+        sizes[0] = res["sizes"]
+        return {"centroids": res["centroids"], "codes": codes, "sizes": sizes, "per_subspace": [res]}
     bounds = [0, d_split[0], d_split[0] + d_split[1], d]
     cent = np.zeros((Cm, d), np.float64)
     codes = np.empty((3, N), np.uint16)
@@ -178,13 +189,21 @@ def cluster_keys(K, d_split, Cm, iters, init_idx3=None, init_cent=None, logs=Fal
     return {"centroids": cent, "codes": codes, "sizes": sizes, "per_subspace": extra}
 
 
-def forward_head(q, k, v, wl, q_init, k_init, rows=None, logs=False, rho=None, khead_off=False):
+def key_split(wl, full=False):
+    """Channel split the proxy of Eq. 6 reads the key codes with: the three RoPE ranges,
+    or, for full-d key clustering, one subspace of all d channels and two empty ones."""
+    return (wl.d, 0, 0) if full else (wl.d_t, wl.d_h, wl.d_w)
+
+
+def forward_head(q, k, v, wl, q_init, k_init, rows=None, logs=False, rho=None, khead_off=False,
+                 key_full=False):
     """The whole hot path for one head: clustering, selection, sparse attention."""
     rho = wl.rho if rho is None else rho
     qc = kmeans(q, 0, wl.d, wl.Cq, wl.iters, init_idx=q_init, logs=logs)
-    kc = cluster_keys(k, (wl.d_t, wl.d_h, wl.d_w), wl.Cm, wl.iters, init_idx3=k_init, logs=logs)
+    kc = cluster_keys(k, (wl.d_t, wl.d_h, wl.d_w), wl.Cm, wl.iters, init_idx3=k_init, logs=logs,
+                      full=key_full)
     sel = select(qc["centroids"], qc["sizes"], kc["centroids"], kc["codes"],
-                 (wl.d_t, wl.d_h, wl.d_w), rho, wl.alpha, khead_off=khead_off)
+                 key_split(wl, key_full), rho, wl.alpha, khead_off=khead_off)
     O = attention(q, k, v, qc["assign"], sel["mask"], rows=rows)
     return {"q": qc, "k": kc, "sel": sel, "O": O}
 

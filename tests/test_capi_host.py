@@ -62,6 +62,7 @@ BAD = [
     dict(rho=0.0), dict(rho=1.5), dict(rho=float("nan")),
     dict(alpha=-0.1), dict(alpha=1.1),
     dict(iters=0), dict(B=0), dict(T=0), dict(dtype=7),
+    dict(khead_mode=2), dict(key_clustering=2), dict(key_clustering=-1),
 ]
 
 

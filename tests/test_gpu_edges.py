@@ -34,10 +34,12 @@ def _dev(w, x, q_init=None, k_init=None):
     return t
 
 
-def _forward_and_compare(w, x, t, q_init, k_init, rho=None, khead_off=False):
+def _forward_and_compare(w, x, t, q_init, k_init, rho=None, khead_off=False, key_full=False):
     over = {} if rho is None else {"rho": rho}
     if khead_off:
         over["khead_mode"] = capi.SCOPE_KHEAD_OFF
+    if key_full:
+        over["key_clustering"] = capi.SCOPE_KEYS_FULL
     p = capi.Params.from_workload(w, **over)
     ws = capi.alloc_workspace(p)
     O, it = capi.forward(p, t["q"], t["k"], t["v"], t["qi"], t["ki"], ws=ws, intermediates=True)
@@ -47,7 +49,7 @@ def _forward_and_compare(w, x, t, q_init, k_init, rho=None, khead_off=False):
     O = O.float().cpu().numpy().reshape(w.B * w.H, w.N, w.d)
     for i in range(w.B * w.H):
         ref = oracle.forward_head(x["q"][i], x["k"][i], x["v"][i], w, q_init[i], k_init[i], rho=rho,
-                                  khead_off=khead_off)
+                                  khead_off=khead_off, key_full=key_full)
         np.testing.assert_array_equal(g["q_assign"][0, i], ref["q"]["assign"])
         np.testing.assert_array_equal(g["q_centroids"][0, i], ref["q"]["centroids"])
         np.testing.assert_array_equal(g["k_codes"][0, i], ref["k"]["codes"])
@@ -249,3 +251,17 @@ def test_random_channel_partition_ablation(dtype):
     tp = _dev(w, xp)
     assert torch.equal(qp, tp["q"]) and torch.equal(kp, tp["k"])
     _forward_and_compare(w, xp, tp, x["q_init"], x["k_init"])
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_full_d_key_clustering_ablation(dtype):
+    """The review page's full-dimensional cluster scoring (significance; falsifier): one
+    k-means of the keys over all d channels; code rows 1 and 2 are zero and the proxy is
+    the cluster-level dot product.  Whole layer against the oracle, at Cm and at 3 Cm
+    (the same number of key centroids as the three subspaces)."""
+    for Cm in (W.Cm, 3 * W.Cm):
+        w = W.with_(dtype=dtype, Cm=Cm)
+        x = synth.layer_inputs(w)
+        t = _dev(w, x)
+        g, _ = _forward_and_compare(w, x, t, x["q_init"], x["k_init"], key_full=True)
+        assert not g["k_codes"][:, :, 1:].any()

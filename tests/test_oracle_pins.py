@@ -449,3 +449,29 @@ def test_dense_prefix_schedule_cases():
             for layer in range(4):
                 want = layer == 0 or step < dense_steps
                 assert oracle.layer_is_dense(layer, step, 1, dense_steps) == want
+
+
+# ----------------------------------------------------------------------------- full-d keys
+def test_full_d_key_proxy_is_the_cluster_level_dot_product():
+    """Full-d key clustering read as a one-subspace code with split (d, 0, 0): the Eq. 6
+    proxy reduces to q_c . mu_{z_j} / sqrt d (numpy matmul), the empty subspaces adding
+    nothing; with every key its own centroid the selection ranks the exact logits."""
+    rng = np.random.default_rng(81)
+    N, d, Cq, Cm = 70, 24, 3, 9
+    K = rng.standard_normal((N, d)).astype(np.float32)
+    qcent = rng.standard_normal((Cq, d))
+    kc = oracle.cluster_keys(K, (8, 8, 8), Cm, 3, init_idx3=np.tile(np.arange(Cm, dtype=np.int32), (3, 1)),
+                             full=True)
+    assert not kc["codes"][1:].any()
+    ref = oracle.kmeans(K, 0, d, Cm, 3, init_idx=np.arange(Cm, dtype=np.int32))
+    np.testing.assert_array_equal(kc["codes"][0], ref["assign"])
+    sel = oracle.select(qcent, np.full(Cq, N // Cq, np.int32), kc["centroids"], kc["codes"], (d, 0, 0), 0.9, 0.1,
+                        want_scores=True)
+    want = (qcent @ kc["centroids"].T)[:, kc["codes"][0]] / math.sqrt(d)
+    np.testing.assert_allclose(sel["scores"], want, rtol=1e-12, atol=1e-12)
+    # lossless: Cm = N, centroid j = key j
+    codes = np.zeros((3, N), np.uint16)
+    codes[0] = np.arange(N)
+    sel = oracle.select(qcent, np.full(Cq, 10, np.int32), K.astype(np.float64), codes, (d, 0, 0), 0.9, 0.1,
+                        want_scores=True)
+    np.testing.assert_allclose(sel["scores"], qcent @ K.astype(np.float64).T / math.sqrt(d), rtol=1e-12, atol=1e-12)
