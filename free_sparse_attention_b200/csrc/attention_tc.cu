@@ -10,8 +10,9 @@
 //   warps 0-3 / 4-7  softmax + epilogue of Q tile 0 / 1 (thread r owns row r = TMEM lane r)
 //   warps 8-11       gather both Q tiles once per item and the selected K rows per key tile
 //   warps 12-13      gather the selected V rows per key tile
-//   warps 14 / 15    issue the MMAs of Q tile 0 / 1 (one thread each; warp 14 also
-//                    allocates TMEM)
+//   warps 14 / 15    issue the MMAs of Q tile 0 / 1 (lane 0 alone, with single-thread
+//                    mbarrier waits: warp-wide waits and broadcasts on this critical path
+//                    cost ~11 % of the kernel's time; warp 14 also allocates TMEM)
 // A TMA gather4 stream sustains ~15 GB/s per issuing warp, so each tile is split over
 // four (K) or two (V) warps; every warp signals its own share with arrive.expect_tx.
 // Registers are rebalanced per warpgroup with setmaxnreg: the softmax warpgroups hold a
@@ -247,88 +248,83 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // ------------------------------------------------------------ MMA issuers (warps 14, 15)
-        // Warp 14 + q issues Q tile q's products.  S is double-buffered: S_q(j) goes to
-        // buffer j & 1, so S_q(t+1) is ready while the softmax still works on S_q(t).  The
-        // order per tile is S(0), S(1), then for every t: O += P(t) V(t), S(t+2).  S(t+2)
-        // reuses the buffer whose first columns hold P(t); issuing it after P(t) V(t) from
-        // the same thread keeps the in-order tensor pipe from overwriting P(t) early.  Both
-        // warps consume every K and V stage in the same order (an idle Q tile only waits
-        // for the data and releases the stage), so the ring phases advance in step.
-        const int q = warp - 14;
-        constexpr uint32_t idesc_qk = f16_idesc(kBM, kBN, false);
-        constexpr uint32_t idesc_pv = f16_idesc(kBM, D, true);
-        uint32_t k_it = 0, v_it = 0, q_it = 0, o_items = 0;
-        uint32_t p_par = 0;   // bit b: parity of the next p_full[q][b] phase
-        const bool leader = lane == 0;
-        const uint64_t qd = sw128_desc(sbase + L::kQ + q * L::kQTile, 16, 1024);
-        auto release = [&](uint64_t *b) {
-            if (leader) mma_commit(b);
-            __syncwarp();
-        };
-        for (uint32_t item_k = 0; !warp_aborted(abort_flag); ++item_k) {
-            const int it = next_item(item_k);
-            if (it < 0) break;
-            const int4 item = a.items[it];
-            const long long r = a.final_cnt[(size_t)item.x * a.Cq + item.y];
-            const int T = (int)((r + kBN - 1) / kBN);
-            const bool active = q == 0 || item.w > kBM;   // Q tile 1 idles on items of <= 128 queries
-            if (!warp_wait(&bars->q_full, q_it & 1, abort_flag, a.status)) break;
-            ++q_it;
-            // S_q(j) = Q_q K(j)^T into buffer j & 1
-            auto qk_step = [&](int j) -> bool {
-                const int ks = k_it % L::kKS;
-                if (!warp_wait(&bars->k_full[ks], (k_it / L::kKS) & 1, abort_flag, a.status)) return false;
-                tc_fence_after();
-                if (active && leader) {
-                    const uint64_t kd = sw128_desc(sbase + L::kK + ks * L::kKVTile, 16, 1024);
-                    const uint32_t dst = tmem + q * 128 + (j & 1) * kBN;
+        // Lane 0 of warp 14 + q issues Q tile q's products alone (lanes 1-31 wait at the end):
+        // S(0), S(1), then for every t: O += P(t) V(t), S(t+2).  S(t+2) reuses the buffer
+        // whose first columns hold P(t); issuing it after P(t) V(t) from the same thread keeps
+        // the in-order tensor pipe from overwriting P(t) early.  Both issuers consume every K
+        // and V stage in the same order (an idle Q tile only waits for the data and releases
+        // the stage), so the ring phases advance in step.
+        if (lane == 0) {
+            const int q = warp - 14;
+            constexpr uint32_t idesc_qk = f16_idesc(kBM, kBN, false);
+            constexpr uint32_t idesc_pv = f16_idesc(kBM, D, true);
+            uint32_t k_it = 0, v_it = 0, q_it = 0, o_items = 0;
+            uint32_t p_par = 0;   // bit b: parity of the next p_full[q][b] phase
+            const uint64_t qd = sw128_desc(sbase + L::kQ + q * L::kQTile, 16, 1024);
+            for (uint32_t item_k = 0; !*abort_flag; ++item_k) {
+                const int slot = item_k % kRing;
+                if (!bar_wait(&bars->item_full[slot], (item_k / kRing) & 1, abort_flag, a.status)) break;
+                const int it = ring[slot];
+                bar_arrive(&bars->item_empty[slot]);
+                if (it < 0) break;
+                const int4 item = a.items[it];
+                const long long r = a.final_cnt[(size_t)item.x * a.Cq + item.y];
+                const int T = (int)((r + kBN - 1) / kBN);
+                const bool active = q == 0 || item.w > kBM;   // Q tile 1 idles on items of <= 128 queries
+                if (!bar_wait(&bars->q_full, q_it & 1, abort_flag, a.status)) break;
+                ++q_it;
+                // S_q(j) = Q_q K(j)^T into buffer j & 1
+                auto qk_step = [&](int j) -> bool {
+                    const int ks = k_it % L::kKS;
+                    if (!bar_wait(&bars->k_full[ks], (k_it / L::kKS) & 1, abort_flag, a.status)) return false;
+                    tc_fence_after();
+                    if (active) {
+                        const uint64_t kd = sw128_desc(sbase + L::kK + ks * L::kKVTile, 16, 1024);
+                        const uint32_t dst = tmem + q * 128 + (j & 1) * kBN;
 #pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint64_t offa = (uint64_t)(((kk >> 2) * (kBM * 128) + (kk & 3) * 32) >> 4);
-                        const uint64_t offb = (uint64_t)(((kk >> 2) * (kBN * 128) + (kk & 3) * 32) >> 4);
-                        mma_bf16(dst, qd + offa, kd + offb, idesc_qk, kk > 0);
+                        for (int kk = 0; kk < D / 16; ++kk) {
+                            const uint64_t offa = (uint64_t)(((kk >> 2) * (kBM * 128) + (kk & 3) * 32) >> 4);
+                            const uint64_t offb = (uint64_t)(((kk >> 2) * (kBN * 128) + (kk & 3) * 32) >> 4);
+                            mma_bf16(dst, qd + offa, kd + offb, idesc_qk, kk > 0);
+                        }
+                        mma_commit(&bars->s_full[q][j & 1]);
                     }
-                    mma_commit(&bars->s_full[q][j & 1]);
-                }
-                __syncwarp();
-                release(&bars->k_empty[ks]);
-                if (j == T - 1) release(&bars->q_empty);
-                ++k_it;
-                return true;
-            };
-            bool ok = qk_step(0);
-            if (ok && T > 1) ok = qk_step(1);
-            for (int t = 0; t < T && ok; ++t) {
-                const int vs = v_it % L::kVS;
-                const int b = t & 1;
-                ok = warp_wait(&bars->v_full[vs], (v_it / L::kVS) & 1, abort_flag, a.status);
-                if (ok && active) {
-                    ok = warp_wait(&bars->p_full[q][b], (p_par >> b) & 1u, abort_flag, a.status);
-                    if (ok && t == 0) ok = warp_wait(&bars->o_free[q], (o_items & 1) ^ 1, abort_flag, a.status);
-                    if (ok) {
-                        p_par ^= 1u << b;
-                        tc_fence_after();
-                        // O_q += P_q(t) V(t), P_q(t) from TMEM (columns q*128 + b*64 + [0, 32))
-                        if (leader) {
+                    mma_commit(&bars->k_empty[ks]);
+                    if (j == T - 1) mma_commit(&bars->q_empty);
+                    ++k_it;
+                    return true;
+                };
+                bool ok = qk_step(0);
+                if (ok && T > 1) ok = qk_step(1);
+                for (int t = 0; t < T && ok; ++t) {
+                    const int vs = v_it % L::kVS;
+                    const int b = t & 1;
+                    ok = bar_wait(&bars->v_full[vs], (v_it / L::kVS) & 1, abort_flag, a.status);
+                    if (ok && active) {
+                        ok = bar_wait(&bars->p_full[q][b], (p_par >> b) & 1u, abort_flag, a.status);
+                        if (ok && t == 0) ok = bar_wait(&bars->o_free[q], (o_items & 1) ^ 1, abort_flag, a.status);
+                        if (ok) {
+                            p_par ^= 1u << b;
+                            tc_fence_after();
+                            // O_q += P_q(t) V(t), P_q(t) from TMEM (columns q*128 + b*64 + [0, 32))
                             const uint64_t vd = sw128_desc(sbase + L::kV + vs * L::kKVTile, kBN * 128, 1024);
 #pragma unroll
                             for (int kk = 0; kk < kBN / 16; ++kk)
                                 mma_bf16_ts(tmem + 256 + q * D, tmem + q * 128 + b * kBN + kk * 8,
-                                            vd + (uint64_t)(kk * 2048 >> 4), idesc_pv,
-                                            (t > 0 || kk > 0) ? 1u : 0u);
+                                            vd + (uint64_t)(kk * 2048 >> 4), idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
                             mma_commit(&bars->o_done[q][b]);
                         }
-                        __syncwarp();
                     }
+                    if (!ok) break;
+                    mma_commit(&bars->v_empty[vs]);
+                    ++v_it;
+                    if (t + 2 < T) ok = qk_step(t + 2);
                 }
                 if (!ok) break;
-                release(&bars->v_empty[vs]);
-                ++v_it;
-                if (t + 2 < T) ok = qk_step(t + 2);
+                if (active) ++o_items;
             }
-            if (!ok) break;
-            if (active) ++o_items;
         }
+        __syncwarp();
     }
     } else {
         // ------------------------------------------------------------ softmax + epilogue
