@@ -492,7 +492,8 @@ def run_fidelity(args, w):
     """Proxy-ranking fidelity (review page, falsifier / skeptic's concrete test) of the layer
     the bench times: `args.fidelity` seeded queries per head, the fraction of each query's
     true top 10 % keys (exact logits) kept by its cluster's selection and by the proxy
-    ranking's own top 10 %."""
+    ranking's own top 10 %, and Spearman's rho of the proxy with the exact logits for the
+    first 4 of them per head."""
     import torch
     from free_sparse_attention_b200 import capi
 
@@ -518,7 +519,16 @@ def run_fidelity(args, w):
                                    it["k_codes"], it["sel_mask"], smp, frac)
     e1.record()
     torch.cuda.synchronize()
+    recall_ms = e0.elapsed_time(e1)
     rs, rp = rs.cpu().numpy(), rp.cpu().numpy()
+    # Spearman's rho of the proxy with the exact logits, the first 4 sampled queries per head
+    sub = torch.from_numpy(samples.reshape(w.B * w.H, -1)[:, :4].reshape(-1).copy()).cuda()
+    e0.record()
+    rho = capi.rank_correlation(p, Q, K, it["q_assign"], it["q_centroids"], it["k_centroids"], it["k_codes"], sub)
+    e1.record()
+    torch.cuda.synchronize()
+    rank_ms = e0.elapsed_time(e1)
+    rho = rho.cpu().numpy()
     n_c = it["q_sizes"].double()
     density = float((n_c * it["final_counts"].double()).sum().item() / (w.B * w.H * w.N * w.N))
     print(json.dumps({
@@ -527,7 +537,9 @@ def run_fidelity(args, w):
         "samples": int(samples.size), "density": density,
         "recall_selection": {"mean": float(rs.mean()), "min": float(rs.min()), "p10": float(np.percentile(rs, 10))},
         "recall_proxy_top10": {"mean": float(rp.mean()), "min": float(rp.min()), "p10": float(np.percentile(rp, 10))},
-        "kernel_ms": e0.elapsed_time(e1), "device_status": capi.get_device_status(ws)}))
+        "spearman_proxy_vs_logits": {"samples": int(rho.size), "mean": float(rho.mean()), "min": float(rho.min()),
+                                     "max": float(rho.max()), "kernel_ms": rank_ms},
+        "kernel_ms": recall_ms, "device_status": capi.get_device_status(ws)}))
     return 0
 
 

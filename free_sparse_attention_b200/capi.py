@@ -25,7 +25,8 @@ EXPORTS = ("scope_workspace_bytes", "scope_cluster_queries", "scope_cluster_keys
            "scope_build_lut_and_select", "scope_sparse_attention", "scope_forward",
            "scope_status_string", "scope_get_device_status", "scope_build_lut_and_select_noalloc",
            "scope_selection_recall", "scope_permute_channels", "scope_dense_attention",
-           "scope_rope3d", "scope_layer_is_dense", "scope_attention_layer")
+           "scope_rope3d", "scope_layer_is_dense", "scope_attention_layer",
+           "scope_rank_correlation_scratch_bytes", "scope_rank_correlation")
 
 
 class ScopeError(RuntimeError):
@@ -108,6 +109,10 @@ def lib() -> ctypes.CDLL:
         L.scope_selection_recall.restype = i
         L.scope_selection_recall.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, i, ctypes.c_double,
                                              vp, vp, vp, sz, vp]
+        L.scope_rank_correlation_scratch_bytes.restype = sz
+        L.scope_rank_correlation_scratch_bytes.argtypes = [P, i]
+        L.scope_rank_correlation.restype = i
+        L.scope_rank_correlation.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, i, vp, vp, sz, vp]
         L.scope_permute_channels.restype = i
         L.scope_permute_channels.argtypes = [P, vp, vp, vp, vp]
         L.scope_dense_attention.restype = i
@@ -278,6 +283,23 @@ def selection_recall(p, Q, K, q_assign, q_centroids, k_centroids, k_codes, sel_m
         _ptr(k_codes), _ptr(sel_mask), _ptr(samples), n, float(frac), _ptr(rs), _ptr(rp),
         _ptr(scratch), scratch.numel(), _stream(stream)))
     return rs, rp
+
+
+def rank_correlation(p, Q, K, q_assign, q_centroids, k_centroids, k_codes, samples, stream=None):
+    """Spearman's rho between each sampled query's exact logits and its cluster's Eq. 6
+    proxy logits over all keys (int64 samples (b*H + h)*N + i): float64 [n_samples]."""
+    n = samples.numel()
+    out = torch.empty(n, dtype=torch.float64, device=Q.device)
+    if n == 0:
+        return out
+    need = int(lib().scope_rank_correlation_scratch_bytes(ctypes.byref(p), n))
+    if need == 0:
+        raise ScopeError("scope_rank_correlation_scratch_bytes", 2)
+    scratch = torch.empty(need, dtype=torch.uint8, device=Q.device)
+    _check("scope_rank_correlation", lib().scope_rank_correlation(
+        ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(q_assign), _ptr(q_centroids), _ptr(k_centroids), _ptr(k_codes),
+        _ptr(samples), n, _ptr(out), _ptr(scratch), scratch.numel(), _stream(stream)))
+    return out
 
 
 def permute_channels(p, X, perm, out=None, stream=None):

@@ -133,6 +133,9 @@ struct FidArgs {
     long long k;                // ceil(frac * N)
 };
 cudaError_t fidelity_run(const FidArgs &a, cudaStream_t s);
+// Spearman's rho of each sample's exact logits with its proxy logits (rankcorr.cu).
+size_t rank_corr_scratch_bytes(int N, int n_samples);
+cudaError_t rank_corr_run(const FidArgs &a, double *spearman, void *scratch, int num_sms, cudaStream_t s);
 // Divisor for x / d by multiply and shift (rope.cu).
 struct FastDiv {
     unsigned m, l;

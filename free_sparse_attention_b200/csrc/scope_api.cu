@@ -623,6 +623,57 @@ scope_status scope_selection_recall(const scope_params *p, const void *Q, const 
     return cuda_status(fidelity_run(a, static_cast<cudaStream_t>(stream)));
 }
 
+size_t scope_rank_correlation_scratch_bytes(const scope_params *p, int n_samples)
+{
+    if (validate(p) != SCOPE_OK || n_samples < 1) return 0;
+    const long long N = (long long)p->T * p->Hg * p->Wg;
+    if (2ll * n_samples * N >= (1ll << 31)) return 0;
+    return rank_corr_scratch_bytes((int)N, n_samples);
+}
+
+scope_status scope_rank_correlation(const scope_params *p, const void *Q, const void *K, const uint16_t *q_assign,
+                                    const double *q_centroids, const double *k_centroids, const uint16_t *k_codes,
+                                    const int64_t *samples, int n_samples, double *spearman, void *scratch,
+                                    size_t scratch_bytes, void *stream)
+{
+    scope_status st = validate(p);
+    if (st != SCOPE_OK) return st;
+    if (!ok_ptr(Q) || !ok_ptr(K) || !ok_ptr(q_assign) || !ok_ptr(q_centroids) || !ok_ptr(k_centroids) ||
+        !ok_ptr(k_codes) || n_samples < 0 || (n_samples > 0 && (!ok_ptr(samples) || !ok_ptr(spearman))) ||
+        !ok_ptr(scratch))
+        return SCOPE_ERR_INVALID_ARGUMENT;
+    if (p->Cm > kMaxFidCm) return SCOPE_ERR_UNSUPPORTED;
+    if (n_samples == 0) return SCOPE_OK;
+    const Dims D = dims_of(*p);
+    if (2ll * n_samples * D.N >= (1ll << 31)) return SCOPE_ERR_UNSUPPORTED;
+    const size_t need = scope_rank_correlation_scratch_bytes(p, n_samples);
+    if (need == 0) return SCOPE_ERR_CUDA;
+    if (scratch_bytes < need) return SCOPE_ERR_WORKSPACE_TOO_SMALL;
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return SCOPE_ERR_CUDA;
+    FidArgs a{};
+    a.Q = Q;
+    a.K = K;
+    a.q_assign = q_assign;
+    a.qcent = q_centroids;
+    a.kcent = k_centroids;
+    a.codes = k_codes;
+    a.samples = reinterpret_cast<const long long *>(samples);
+    a.n_samples = n_samples;
+    a.total = D.BH * D.N;
+    a.N = (int)D.N;
+    a.d = p->d;
+    code_split(*p, a.dt, a.dh, a.dw);
+    a.Cq = p->Cq;
+    a.Cm = p->Cm;
+    a.nw = (int)D.nw;
+    a.is_bf16 = p->dtype == SCOPE_BF16;
+    a.inv_sqrt_d = 1.0 / std::sqrt((double)p->d);
+    return cuda_status(rank_corr_run(a, spearman, scratch, sms, static_cast<cudaStream_t>(stream)));
+}
+
 scope_status scope_permute_channels(const scope_params *p, const void *X, const int32_t *perm, void *Y,
                                     void *stream)
 {

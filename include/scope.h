@@ -260,6 +260,24 @@ scope_status scope_selection_recall(const scope_params *p, const void *Q, const 
                                     void *scratch, size_t scratch_bytes, void *stream);
 
 /*
+ * Rank correlation of the proxy with the true logits (review page, the skeptic's concrete
+ * test: "the rank correlation between Eq. (6) proxy logits and true logits").  For every
+ * sampled query g = (b*H + h)*N + i: spearman[s] = Spearman's rho over the N keys of head
+ * (b, h) between x_j = q_i . k_j (exact, binary64, channels in order) and y_j = s~_{c,j}, the
+ * Eq. 6 proxy logits of its cluster c = q_assign[g]: the Pearson correlation of the two
+ * vectors of average ranks (tied values share the mean of their 1-based ranks).  NaN for an
+ * index outside the layer.  Inputs as for scope_selection_recall; scratch: caller-owned
+ * device memory of at least scope_rank_correlation_scratch_bytes(p, n_samples) bytes (about
+ * 64 * N bytes per sample plus the sort's temporary storage); requires Cm <= 1024 and
+ * 2 * n_samples * N < 2^31.  Allocates nothing; enqueues on `stream`.
+ */
+size_t scope_rank_correlation_scratch_bytes(const scope_params *p, int n_samples);
+scope_status scope_rank_correlation(const scope_params *p, const void *Q, const void *K, const uint16_t *q_assign,
+                                    const double *q_centroids, const double *k_centroids, const uint16_t *k_codes,
+                                    const int64_t *samples, int n_samples, double *spearman, void *scratch,
+                                    size_t scratch_bytes, void *stream);
+
+/*
  * Channel permutation for the review page's ablation "random channel partition"
  * (significance): Y[b,h,n,e] = X[b,h,n,perm[e]] for e < d.  One permutation applied to
  * both Q and K leaves every logit q.k unchanged, so the layer run on the permuted Q and K

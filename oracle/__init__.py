@@ -18,6 +18,8 @@ Parity status of each function (what pins it, in tests/test_oracle_pins.py):
                 vectors per axis, identity at the origin token, pair norms, the relative-
                 position property, and the input generator's own post-RoPE tensors.
   dense_attention -- pinned: torch scaled_dot_product_attention (float64, CPU).
+  rank_correlation -- pinned: scipy.stats.spearmanr, +-1 for monotone maps, a hand-worked
+                case with ties, invariance under a common permutation of the keys.
   layer      -- the schedule's choice between dense_attention and forward_head, after
                 rope3d; pinned through its parts.
 """
@@ -296,3 +298,34 @@ def layer(q, k, v, wl, q_init, k_init, dense, rope_base=None, rows=None, round_r
         out = forward_head(q, k, v, wl, q_init, k_init, rows=rows)
     out.update(extra)
     return out
+
+
+def average_ranks(v):
+    """1-based ranks of v in ascending order; tied values share the mean of their ranks."""
+    v = np.asarray(v, np.float64)
+    order = np.argsort(v, kind="stable")
+    sv = v[order]
+    ranks = np.empty(v.shape[0], np.float64)
+    lo = 0
+    n = v.shape[0]
+    while lo < n:
+        hi = lo + 1
+        while hi < n and sv[hi] == sv[lo]:
+            hi += 1
+        ranks[order[lo:hi]] = 0.5 * (lo + 1 + hi)
+        lo = hi
+    return ranks
+
+
+def rank_correlation(q, K, proxy):
+    """Spearman's rho of one query's exact logits (binary64, channels summed in order) with
+    the Eq. 6 proxy logits of its cluster (review page, the skeptic's concrete test): the
+    Pearson correlation of the two vectors of average ranks."""
+    q = np.asarray(q, np.float64)
+    K = np.asarray(K, np.float64)
+    logit = np.zeros(K.shape[0], np.float64)
+    for e in range(q.shape[0]):
+        logit = logit + q[e] * K[:, e]
+    rx = average_ranks(logit) - 0.5 * (K.shape[0] + 1)
+    ry = average_ranks(proxy) - 0.5 * (K.shape[0] + 1)
+    return float((rx @ ry) / math.sqrt((rx @ rx) * (ry @ ry)))

@@ -217,8 +217,14 @@ def test_warm_start_from_previous_step_with_one_iteration():
     torch.cuda.synchronize()
     O = O.float().cpu().numpy().reshape(w.H, w.N, w.d)
     for h in range(w.H):
-        rq = oracle.kmeans(x2["q"][h], 0, w.d, w.Cq, 1, init_cent=to_np(qc0)[0, h])
-        rk = oracle.cluster_keys(x2["k"][h], (w.d_t, w.d_h, w.d_w), w.Cm, 1, init_cent=to_np(kc0)[0, h])
+        # step A by the oracle itself (equal to the GPU's, whose centroids started step B)
+        qa0 = oracle.kmeans(x["q"][h], 0, w.d, w.Cq, w.iters, init_idx=x["q_init"][h])["centroids"]
+        ka0 = oracle.cluster_keys(x["k"][h], (w.d_t, w.d_h, w.d_w), w.Cm, w.iters,
+                                  init_idx3=x["k_init"][h])["centroids"]
+        np.testing.assert_array_equal(to_np(qc0)[0, h], qa0)
+        np.testing.assert_array_equal(to_np(kc0)[0, h], ka0)
+        rq = oracle.kmeans(x2["q"][h], 0, w.d, w.Cq, 1, init_cent=qa0)
+        rk = oracle.cluster_keys(x2["k"][h], (w.d_t, w.d_h, w.d_w), w.Cm, 1, init_cent=ka0)
         np.testing.assert_array_equal(to_np(qa)[0, h], rq["assign"])
         np.testing.assert_array_equal(to_np(qc)[0, h], rq["centroids"])
         np.testing.assert_array_equal(to_np(kk)[0, h], rk["codes"])

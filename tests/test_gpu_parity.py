@@ -149,30 +149,62 @@ def test_forward_end_to_end(w):
             compare_attention(w, O[i], ref["O"])
 
 
+def _oracle_scores(w, x, bh, cache):
+    """The oracle's own clustering and Eq. 6 proxy scores for head bh (no GPU values)."""
+    if bh not in cache:
+        qc = oracle.kmeans(x["q"][bh], 0, w.d, w.Cq, w.iters, init_idx=x["q_init"][bh])
+        kc = oracle.cluster_keys(x["k"][bh], (w.d_t, w.d_h, w.d_w), w.Cm, w.iters, init_idx3=x["k_init"][bh])
+        sel = oracle.select(qc["centroids"], qc["sizes"], kc["centroids"], kc["codes"], (w.d_t, w.d_h, w.d_w),
+                            w.rho, w.alpha, want_scores=True)
+        cache[bh] = (qc["assign"], sel["scores"], sel["mask"])
+    return cache[bh]
+
+
 @pytest.mark.parametrize("w", [TINY, MID], ids=lambda w: w.name)
 def test_selection_recall_matches_oracle(w):
     """Proxy-ranking fidelity of sampled queries through scope_selection_recall against the
-    oracle's definition (exact binary64 logits, Eq. 6 proxies, index tie-breaks)."""
+    oracle's definition (exact binary64 logits, Eq. 6 proxies, index tie-breaks), the
+    oracle running its own clustering and selection."""
     x, t = _run(w)
     p = capi.Params.from_workload(w)
     ws = capi.alloc_workspace(p)
     _, it = capi.forward(p, t["q"], t["k"], t["v"], t["q_init"], t["k_init"], ws=ws, intermediates=True)
     rng = np.random.default_rng(12)
     samples = np.sort(rng.choice(w.B * w.H * w.N, 23, replace=False)).astype(np.int64)
+    cache = {}
     for frac in (0.1, 0.5):
         rs, rp = capi.selection_recall(p, t["q"], t["k"], it["q_assign"], it["q_centroids"],
                                        it["k_centroids"], it["k_codes"], it["sel_mask"],
                                        torch.from_numpy(samples).cuda(), frac)
         torch.cuda.synchronize()
         rs, rp = to_np(rs), to_np(rp)
-        g = {k: to_np(v) for k, v in it.items()}
         for s, gi in enumerate(samples):
             bh, i = divmod(int(gi), w.N)
-            b, h = divmod(bh, w.H)
-            c = int(g["q_assign"][b, h, i])
-            sc = oracle.select(g["q_centroids"][b, h], g["q_sizes"][b, h], g["k_centroids"][b, h],
-                               g["k_codes"][b, h], (w.d_t, w.d_h, w.d_w), w.rho, w.alpha,
-                               want_scores=True)["scores"][c]
-            selected = mask_bits(g["sel_mask"][b, h, c], w.N).astype(bool)
-            ref = oracle.selection_recall(x["q"][bh][i], x["k"][bh], sc, selected, frac)
+            assign, scores, mask = _oracle_scores(w, x, bh, cache)
+            c = int(assign[i])
+            selected = mask_bits(mask[c], w.N).astype(bool)
+            ref = oracle.selection_recall(x["q"][bh][i], x["k"][bh], scores[c], selected, frac)
             assert (rs[s], rp[s]) == ref, (s, rs[s], rp[s], ref)
+
+
+@pytest.mark.parametrize("w", [TINY, MID], ids=lambda w: w.name)
+def test_rank_correlation_matches_oracle(w):
+    """Spearman's rho of sampled queries' exact logits with their cluster's Eq. 6 proxy
+    logits (scope_rank_correlation) against the oracle's average-rank definition."""
+    x, t = _run(w)
+    p = capi.Params.from_workload(w)
+    ws = capi.alloc_workspace(p)
+    _, it = capi.forward(p, t["q"], t["k"], t["v"], t["q_init"], t["k_init"], ws=ws, intermediates=True)
+    rng = np.random.default_rng(13)
+    samples = np.sort(rng.choice(w.B * w.H * w.N, 17, replace=False)).astype(np.int64)
+    samples = np.concatenate([samples, [-1, w.B * w.H * w.N]]).astype(np.int64)   # two outside the layer
+    rho = to_np(capi.rank_correlation(p, t["q"], t["k"], it["q_assign"], it["q_centroids"], it["k_centroids"],
+                                      it["k_codes"], torch.from_numpy(samples).cuda()))
+    torch.cuda.synchronize()
+    assert np.isnan(rho[-1]) and np.isnan(rho[-2])
+    cache = {}
+    for s, gi in enumerate(samples[:-2]):
+        bh, i = divmod(int(gi), w.N)
+        assign, scores, _ = _oracle_scores(w, x, bh, cache)
+        ref = oracle.rank_correlation(x["q"][bh][i], x["k"][bh], scores[int(assign[i])])
+        assert abs(rho[s] - ref) < 1e-9, (s, rho[s], ref)

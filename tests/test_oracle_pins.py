@@ -475,3 +475,28 @@ def test_full_d_key_proxy_is_the_cluster_level_dot_product():
     sel = oracle.select(qcent, np.full(Cq, 10, np.int32), K.astype(np.float64), codes, (d, 0, 0), 0.9, 0.1,
                         want_scores=True)
     np.testing.assert_allclose(sel["scores"], qcent @ K.astype(np.float64).T / math.sqrt(d), rtol=1e-12, atol=1e-12)
+
+
+# ----------------------------------------------------------------------------- rank correlation
+def test_rank_correlation_pins():
+    """Spearman's rho: scipy's spearmanr (average ranks for ties), +-1 under monotone maps,
+    a hand-worked case with ties, and invariance under a common permutation of the keys."""
+    import scipy.stats
+    rng = np.random.default_rng(91)
+    N, d = 200, 16
+    q = rng.standard_normal(d).astype(np.float32)
+    K = rng.standard_normal((N, d)).astype(np.float32)
+    logit = K.astype(np.float64) @ q.astype(np.float64)
+    proxy = np.round(logit + 0.8 * rng.standard_normal(N), 1)          # with many ties
+    rho = oracle.rank_correlation(q, K, proxy)
+    assert abs(rho - scipy.stats.spearmanr(logit, proxy).statistic) < 1e-12
+    assert abs(oracle.rank_correlation(q, K, np.exp(logit)) - 1.0) < 1e-12
+    assert abs(oracle.rank_correlation(q, K, -logit ** 3) + 1.0) < 1e-12
+    perm = rng.permutation(N)
+    assert abs(oracle.rank_correlation(q, K[perm], proxy[perm]) - rho) < 1e-12
+    # hand-worked: ranks (1, 2.5, 2.5, 4) and (1, 3, 2, 4), centred (-1.5, 0, 0, 1.5) and
+    # (-1.5, 0.5, -0.5, 1.5): rho = 4.5 / sqrt(4.5 * 5)
+    np.testing.assert_array_equal(oracle.average_ranks([1.0, 2.0, 2.0, 3.0]), [1.0, 2.5, 2.5, 4.0])
+    q1 = np.ones(1, np.float32)
+    K1 = np.array([[1.0], [2.0], [2.0], [3.0]], np.float32)
+    assert abs(oracle.rank_correlation(q1, K1, np.array([1.0, 3.0, 2.0, 4.0])) - 4.5 / math.sqrt(22.5)) < 1e-15
