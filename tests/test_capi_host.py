@@ -161,3 +161,22 @@ def test_dense_layout_fits_the_layer_workspace(L, name):
     p = capi.Params.from_workload(ALL[name])
     p1 = capi.Params.from_workload(ALL[name], Cq=1)
     assert 0 < capi.workspace_bytes(p1) <= capi.workspace_bytes(p)
+
+
+def test_rank_correlation_rejections(L):
+    """Validation of scope_rank_correlation happens before any device work."""
+    fake = ctypes.c_void_p(1 << 20)
+    p = capi.Params.from_workload(TINY)
+    args = [fake] * 6
+    # no samples: nothing to do
+    assert L.scope_rank_correlation(ctypes.byref(p), *args, None, 0, None, fake, 0, None) == 0
+    assert L.scope_rank_correlation(ctypes.byref(p), *args, fake, -1, fake, fake, 1 << 30, None) == 1
+    assert L.scope_rank_correlation(ctypes.byref(p), *args, None, 3, fake, fake, 1 << 30, None) == 1   # no samples
+    assert L.scope_rank_correlation(ctypes.byref(p), *args, fake, 3, None, fake, 1 << 30, None) == 1   # no output
+    assert L.scope_rank_correlation(ctypes.byref(p), ctypes.c_void_p((1 << 20) + 4), *args[1:], fake, 3, fake,
+                                    fake, 1 << 30, None) == 1   # misaligned Q
+    big = capi.Params.from_workload(TINY, Cm=1100, T=8, Hg=16, Wg=16)
+    assert L.scope_rank_correlation(ctypes.byref(big), *args, fake, 3, fake, fake, 1 << 30, None) == 2
+    assert L.scope_rank_correlation_scratch_bytes(ctypes.byref(p), 0) == 0
+    bad = capi.Params.from_workload(TINY, rho=2.0)
+    assert L.scope_rank_correlation_scratch_bytes(ctypes.byref(bad), 4) == 0
