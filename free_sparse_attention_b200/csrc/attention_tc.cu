@@ -55,6 +55,14 @@ constexpr uint32_t kTmemCols = 512;
 constexpr int kRing = 4;           // work items fetched ahead by the scheduler thread
 constexpr int kWarps = kThreads / 32;
 
+// max(a, b, c) in one instruction (the three-input form of max.f32 on sm_100)
+__device__ __forceinline__ float fmax3(float a, float b, float c)
+{
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
 struct __align__(8) Bars {
     uint64_t q_full, q_empty;
     uint64_t k_full[kMaxStages], k_empty[kMaxStages];
@@ -367,13 +375,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int j = 0; j < kBN; ++j)
                         if (j >= nvalid) s[j] = -INFINITY;
                 }
+                // row maximum with three-input max (half the instructions of a pairwise tree)
                 float m8[8];
 #pragma unroll
                 for (int k = 0; k < 8; ++k) m8[k] = s[k];
 #pragma unroll
-                for (int j = 8; j < kBN; ++j) m8[j & 7] = fmaxf(m8[j & 7], s[j]);
-                const float mt = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                                       fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) * c;
+                for (int j = 8; j < kBN; j += 16) {
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) m8[k] = fmax3(m8[k], s[j + k], s[j + 8 + k]);
+                }
+                const float mt = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7])) * c;
                 const bool need = mt > m_run + 8.f;
                 if (t > 0 && __any_sync(0xffffffffu, need)) {
                     // rescaling O needs every earlier P V done; the last one is P(t-1) V(t-1)

@@ -85,28 +85,66 @@ struct Unit {
     double inv_umax;     // mass normalisation
 };
 
-// Codes are clamped to [0, Cm) so that a malformed caller-supplied code cannot read
+// Keys are visited kBatch at a time per thread (keys j0 + k * kSelThreads + tid): the codes
+// and table entries of the batch are all loaded before any of them is used, so a thread
+// keeps 3 kBatch independent shared-memory loads in flight instead of one key's chain.
+constexpr int kBatch = 2;
+
+// Codes of one batch, clamped to [0, Cm) so that a malformed caller-supplied code cannot read
 // outside the tables (sel_check_kernel reports such codes in the status word).
-__device__ __forceinline__ double key_score(const SelSmem &S, const Unit &u, int j)
+struct KeyBatch {
+    int zt[kBatch], zh[kBatch], zw[kBatch];
+    bool v[kBatch];
+};
+
+__device__ __forceinline__ KeyBatch load_batch(const Unit &u, int j0)
 {
-    const int zt = min((int)u.zt[j], u.Cm - 1), zh = min((int)u.zh[j], u.Cm - 1),
-              zw = min((int)u.zw[j], u.Cm - 1);
-    const double a = S.lut[zt], b = S.lut[u.Cm + zh], c = S.lut[2 * u.Cm + zw];
-    return __dmul_rn(u.inv, __dadd_rn(__dadd_rn(a, b), c));
+    KeyBatch kb;
+#pragma unroll
+    for (int k = 0; k < kBatch; ++k) {
+        const int j = j0 + k * kSelThreads + (int)threadIdx.x;
+        kb.v[k] = j < u.N;
+        const int jj = kb.v[k] ? j : 0;
+        kb.zt[k] = min((int)u.zt[jj], u.Cm - 1);
+        kb.zh[k] = min((int)u.zh[jj], u.Cm - 1);
+        kb.zw[k] = min((int)u.zw[jj], u.Cm - 1);
+    }
+    return kb;
 }
 
-__device__ __forceinline__ double key_u(const SelSmem &S, const Unit &u, int j)
+// s_j of Eq. 6 for every key of the batch
+__device__ __forceinline__ void batch_scores(const SelSmem &S, const Unit &u, const KeyBatch &kb, double (&s)[kBatch])
 {
-    const int zt = min((int)u.zt[j], u.Cm - 1), zh = min((int)u.zh[j], u.Cm - 1),
-              zw = min((int)u.zw[j], u.Cm - 1);
-    return __dmul_rn(__dmul_rn(S.E[zt], S.E[u.Cm + zh]), S.E[2 * u.Cm + zw]);
+    double a[kBatch], b[kBatch], c[kBatch];
+#pragma unroll
+    for (int k = 0; k < kBatch; ++k) {
+        a[k] = S.lut[kb.zt[k]];
+        b[k] = S.lut[u.Cm + kb.zh[k]];
+        c[k] = S.lut[2 * u.Cm + kb.zw[k]];
+    }
+#pragma unroll
+    for (int k = 0; k < kBatch; ++k) s[k] = __dmul_rn(u.inv, __dadd_rn(__dadd_rn(a[k], b[k]), c[k]));
 }
 
-// fixed-point mass in units of 2^-63, clamped to [0, 2^63]
-__device__ __forceinline__ unsigned long long key_mass(const SelSmem &S, const Unit &u, int j)
+// key weights u_j = E^T E^H E^W for every key of the batch
+__device__ __forceinline__ void batch_weights(const SelSmem &S, const Unit &u, const KeyBatch &kb,
+                                              double (&w)[kBatch])
 {
-    double w = fmin(__dmul_rn(key_u(S, u, j), u.inv_umax), 1.0);
-    return __double2ull_rn(w * 9223372036854775808.0);
+    double a[kBatch], b[kBatch], c[kBatch];
+#pragma unroll
+    for (int k = 0; k < kBatch; ++k) {
+        a[k] = S.E[kb.zt[k]];
+        b[k] = S.E[u.Cm + kb.zh[k]];
+        c[k] = S.E[2 * u.Cm + kb.zw[k]];
+    }
+#pragma unroll
+    for (int k = 0; k < kBatch; ++k) w[k] = __dmul_rn(__dmul_rn(a[k], b[k]), c[k]);
+}
+
+// fixed-point mass of weight w in units of 2^-63, clamped to [0, 2^63]
+__device__ __forceinline__ unsigned long long weight_mass(double w, const Unit &u)
+{
+    return __double2ull_rn(fmin(__dmul_rn(w, u.inv_umax), 1.0) * 9223372036854775808.0);
 }
 
 __device__ __forceinline__ double mass_to_double(unsigned long long hi, unsigned long long lo)
@@ -252,20 +290,27 @@ __device__ SelectOut block_select(const SelSmem &S, const Unit &u, bool mass_mod
         }
         __syncthreads();
         double cmin = DBL_MAX, cmax = -DBL_MAX, umx = 0.0;
-        for (int j = tid; j < u.N; j += kSelThreads) {
-            const double s = key_score(S, u, j);
-            if (!in_candidates(L, s)) continue;
-            const int b = L.jmode ? jbin(j, u.N) : vbin(s, hi, scale);
-            atomicAdd(&S.cnt[b], 1);
-            if (mass_mode) {
-                const double uj = key_u(S, u, j);
-                umx = fmax(umx, uj);
-                const unsigned long long W = __double2ull_rn(fmin(__dmul_rn(uj, u.inv_umax), 1.0) * 9223372036854775808.0);
-                atomicAdd(&S.mhi[b], W >> 32);
-                atomicAdd(&S.mlo[b], W & 0xffffffffull);
+        for (int j0 = 0; j0 < u.N; j0 += kBatch * kSelThreads) {
+            const KeyBatch kb = load_batch(u, j0);
+            double sc[kBatch], uw[kBatch];
+            batch_scores(S, u, kb, sc);
+            if (mass_mode) batch_weights(S, u, kb, uw);
+#pragma unroll
+            for (int k = 0; k < kBatch; ++k) {
+                const double s = sc[k];
+                if (!kb.v[k] || !in_candidates(L, s)) continue;
+                const int j = j0 + k * kSelThreads + tid;
+                const int b = L.jmode ? jbin(j, u.N) : vbin(s, hi, scale);
+                atomicAdd(&S.cnt[b], 1);
+                if (mass_mode) {
+                    umx = fmax(umx, uw[k]);
+                    const unsigned long long W = weight_mass(uw[k], u);
+                    atomicAdd(&S.mhi[b], W >> 32);
+                    atomicAdd(&S.mlo[b], W & 0xffffffffull);
+                }
+                cmin = fmin(cmin, s);
+                cmax = fmax(cmax, s);
             }
-            cmin = fmin(cmin, s);
-            cmax = fmax(cmax, s);
         }
         cmin = block_min(cmin, S.red);
         cmax = block_max(cmax, S.red);
@@ -340,16 +385,27 @@ __device__ SelectOut block_select(const SelSmem &S, const Unit &u, bool mass_mod
             // gather the crossing bin's keys
             if (tid == 0) S.misc[1] = 0;
             __syncthreads();
-            for (int j = tid; j < u.N; j += kSelThreads) {
-                const double s = key_score(S, u, j);
-                if (!in_candidates(L, s)) continue;
-                const int b = L.jmode ? jbin(j, u.N) : vbin(s, hi, scale);
-                if (b != bstar) continue;
-                const int slot = atomicAdd(&S.misc[1], 1);
-                if (slot < kCap) {
-                    S.cs[slot] = s;
-                    S.cj[slot] = j;
-                    if (mass_mode) S.cw[slot] = key_mass(S, u, j);
+            for (int j0 = 0; j0 < u.N; j0 += kBatch * kSelThreads) {
+                const KeyBatch kb = load_batch(u, j0);
+                double sc[kBatch];
+                batch_scores(S, u, kb, sc);
+#pragma unroll
+                for (int k = 0; k < kBatch; ++k) {
+                    const double s = sc[k];
+                    if (!kb.v[k] || !in_candidates(L, s)) continue;
+                    const int j = j0 + k * kSelThreads + tid;
+                    const int b = L.jmode ? jbin(j, u.N) : vbin(s, hi, scale);
+                    if (b != bstar) continue;
+                    const int slot = atomicAdd(&S.misc[1], 1);
+                    if (slot < kCap) {
+                        S.cs[slot] = s;
+                        S.cj[slot] = j;
+                        if (mass_mode) {
+                            const double w = __dmul_rn(__dmul_rn(S.E[kb.zt[k]], S.E[u.Cm + kb.zh[k]]),
+                                                       S.E[2 * u.Cm + kb.zw[k]]);
+                            S.cw[slot] = weight_mass(w, u);
+                        }
+                    }
                 }
             }
             __syncthreads();
@@ -595,15 +651,20 @@ __global__ void __launch_bounds__(kSelThreads) sel_mask_kernel(SelArgs a)
         s_star = so.s;
         j_star = so.j;
     }
-    for (int w = warp; w < a.nw; w += kSelThreads / 32) {
-        const int j = w * 32 + lane;
-        bool sel = false;
-        if (j < a.N) {
-            const double s = key_score(S, u, j);
-            sel = (s > s_star) || (s == s_star && j <= j_star);
+    // word w of the row holds keys 32 w .. 32 w + 31; a batch covers kBatch x 16 words, word
+    // j0 / 32 + k * 16 + warp of batch j0 from warp `warp`
+    for (int j0 = 0; j0 < a.N; j0 += kBatch * kSelThreads) {
+        const KeyBatch kb = load_batch(u, j0);
+        double sc[kBatch];
+        batch_scores(S, u, kb, sc);
+#pragma unroll
+        for (int k = 0; k < kBatch; ++k) {
+            const int j = j0 + k * kSelThreads + tid;
+            const bool sel = kb.v[k] && ((sc[k] > s_star) || (sc[k] == s_star && j <= j_star));
+            const unsigned bits = __ballot_sync(0xffffffffu, sel);
+            const int w = (j0 + k * kSelThreads) / 32 + warp;
+            if (lane == 0 && w < a.nw) row[w] = bits;
         }
-        const unsigned bits = __ballot_sync(0xffffffffu, sel);
-        if (lane == 0) row[w] = bits;
     }
 }
 
