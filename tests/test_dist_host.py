@@ -54,3 +54,27 @@ def test_max_over_ranks_and_rank_roles_with_gloo():
 def test_single_process_max_is_identity():
     import bench
     assert bench.max_over_ranks(3.5) == 3.5
+
+
+def test_attention_traffic_record_follows_the_kernel_source(tmp_path):
+    """The roofline's DRAM traffic comes from the committed ncu record only while the
+    attention kernel's source is the one it was captured from; any edit voids it."""
+    import hashlib
+    import json
+    import bench
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    src = os.path.join(root, "free_sparse_attention_b200", "csrc", "attention_tc.cu")
+    with open(os.path.join(root, "profiles", "attn_tc_hunyuan720p.json")) as f:
+        rec = json.load(f)
+    # per launch = captured bytes scaled from the captured heads to the 24-head layer
+    assert rec["dram_bytes_per_launch"] == rec["dram_bytes_captured"] * 24 / rec["captured_heads"]
+    with open(src, "rb") as f:
+        body = f.read()
+    got = bench.traffic_from_profile(src)
+    if hashlib.sha256(body).hexdigest() == rec["kernel_sha256"]:
+        assert got == rec["dram_bytes_per_launch"]
+    else:
+        assert got is None
+    changed = tmp_path / "attention_tc.cu"
+    changed.write_bytes(body + b"\n")
+    assert bench.traffic_from_profile(str(changed)) is None
