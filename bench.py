@@ -303,28 +303,78 @@ def run_scope(args, w):
     ms = max_over_ranks(ms, device="cuda")
     status |= capi.get_device_status(ws)
 
-    # end to end through the C ABI with host buffers: H2D inputs, layer, D2H output
-    Oh = torch.empty(O.shape, dtype=O.dtype, pin_memory=True)
+    # end to end through the C ABI with host buffers: every step copies its inputs H2D from
+    # pinned host memory and reads its output back D2H, all inside the timed region.
+    O_dev = O.clone()
+    Oh = [torch.empty(O.shape, dtype=O.dtype, pin_memory=True) for _ in range(2)]
     h2d = sum(host[n].numel() * host[n].element_size() for n in host)
-    d2h = Oh.numel() * Oh.element_size()
+    d2h = Oh[0].numel() * Oh[0].element_size()
+    comp = torch.cuda.current_stream()
 
-    def e2e_step():
+    # serial form: copies, layer and read-back one after another on one stream
+    def e2e_serial_step():
         for n in host:
             dev[n].copy_(host[n], non_blocking=True)
         capi.forward(p, dev["q"], dev["k"], dev["v"], dev["qi"], dev["ki"], ws=ws, out=O)
-        Oh.copy_(O, non_blocking=True)
+        Oh[0].copy_(O, non_blocking=True)
 
     for _ in range(max(1, min(args.warmup, 2))):
-        e2e_step()
+        e2e_serial_step()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     e0.record()
     for _ in range(args.steps):
-        e2e_step()
+        e2e_serial_step()
     e1.record()
     torch.cuda.synchronize()
+    e2e_serial_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, device="cuda")
+
+    # pipelined form: two device input/output sets; step i+1's H2D (copy stream s_in) and step
+    # i-1's D2H (copy stream s_out) run under step i's layer, events guard every buffer reuse
+    dev2 = [dev, {n: torch.empty_like(t) for n, t in dev.items()}]
+    O2 = [O, torch.empty_like(O)]
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+
+    def e2e_pipelined(n_steps, start_ev):
+        in_ready = [torch.cuda.Event() for _ in range(n_steps)]
+        done = [torch.cuda.Event() for _ in range(n_steps)]
+        read = [torch.cuda.Event() for _ in range(n_steps)]
+        s_in.wait_event(start_ev)
+        for i in range(n_steps):
+            b = i % 2
+            with torch.cuda.stream(s_in):
+                if i >= 2:
+                    s_in.wait_event(done[i - 2])     # layer i-2 has consumed input set b
+                for n in host:
+                    dev2[b][n].copy_(host[n], non_blocking=True)
+                in_ready[i].record(s_in)
+            comp.wait_event(in_ready[i])
+            if i >= 2:
+                comp.wait_event(read[i - 2])          # output set b has been read back
+            capi.forward(p, dev2[b]["q"], dev2[b]["k"], dev2[b]["v"], dev2[b]["qi"], dev2[b]["ki"],
+                         ws=ws, out=O2[b], stream=comp)
+            done[i].record(comp)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(done[i])
+                Oh[b].copy_(O2[b], non_blocking=True)
+                read[i].record(s_out)
+        comp.wait_event(read[n_steps - 1])
+
+    warm = torch.cuda.Event()
+    warm.record(comp)
+    e2e_pipelined(2, warm)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0.record(comp)
+    e2e_pipelined(args.steps, e0)
+    e1.record(comp)
+    torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, device="cuda")
+    # every step computes the same layer: its read-back output equals the device-resident run
+    e2e_match = bool(torch.equal(Oh[0], Oh[1]) and torch.equal(Oh[0].cuda(), O_dev))
+    del dev2, O2, O_dev
 
     # dense attention on the same shape (library comparator, not part of the path)
     dense_ms = None
@@ -374,7 +424,11 @@ def run_scope(args, w):
         "density": density, "effective_tflop_per_layer": flops / 1e12,
         "dense_sdpa_ms": dense_ms,
         "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
-                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
+                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+                "pipelining": "two device buffer sets; step i+1's H2D and step i-1's D2H on their own "
+                              "copy streams under step i's layer",
+                "output_matches_device_run": e2e_match,
+                "serial": {"value": world * flops / (e2e_serial_ms * 1e-3) / 1e12, "ms_per_step": e2e_serial_ms}},
         "gpu_launches": kernels_per_forward(w.iters) * args.steps,
         "device_status": status,
         "clocks": clk,
