@@ -180,3 +180,57 @@ def test_rank_correlation_rejections(L):
     assert L.scope_rank_correlation_scratch_bytes(ctypes.byref(p), 0) == 0
     bad = capi.Params.from_workload(TINY, rho=2.0)
     assert L.scope_rank_correlation_scratch_bytes(ctypes.byref(bad), 4) == 0
+
+
+def test_cluster_keys_rejections(L):
+    p = capi.Params.from_workload(TINY)
+    need = capi.workspace_bytes(p)
+    fake = ctypes.c_void_p(1 << 20)
+    # workspace too small, misaligned workspace, no initial centroids, misaligned K
+    assert L.scope_cluster_keys(ctypes.byref(p), fake, fake, None, fake, fake, fake, need - 256, None) == 3
+    assert L.scope_cluster_keys(ctypes.byref(p), fake, fake, None, fake, fake,
+                                ctypes.c_void_p((1 << 20) + 8), need, None) == 1
+    assert L.scope_cluster_keys(ctypes.byref(p), fake, None, None, fake, fake, fake, need, None) == 1
+    assert L.scope_cluster_keys(ctypes.byref(p), ctypes.c_void_p((1 << 20) + 2), fake, None, fake, fake,
+                                fake, need, None) == 1
+    bad = capi.Params.from_workload(TINY, key_clustering=3)
+    assert L.scope_cluster_keys(ctypes.byref(bad), fake, fake, None, fake, fake, fake, need, None) == 1
+
+
+def test_permute_channels_rejections(L):
+    p = capi.Params.from_workload(TINY)
+    fake, other = ctypes.c_void_p(1 << 20), ctypes.c_void_p(1 << 21)
+    assert L.scope_permute_channels(ctypes.byref(p), fake, fake, fake, None) == 1        # in place
+    assert L.scope_permute_channels(ctypes.byref(p), fake, None, other, None) == 1       # no permutation
+    assert L.scope_permute_channels(ctypes.byref(p), ctypes.c_void_p((1 << 20) + 4), fake, other, None) == 1
+    bad = capi.Params.from_workload(TINY, d_t=10)
+    assert L.scope_permute_channels(ctypes.byref(bad), fake, fake, other, None) == 1
+
+
+def test_selection_recall_rejections(L):
+    p = capi.Params.from_workload(TINY)
+    fake = ctypes.c_void_p(1 << 20)
+    f = L.scope_selection_recall
+
+    def call(params, n, frac, scratch_bytes, samples=fake):
+        return f(ctypes.byref(params), fake, fake, fake, fake, fake, fake, fake, samples, n,
+                 ctypes.c_double(frac), fake, fake, fake, scratch_bytes, None)
+
+    per = 16 * TINY.N                       # scratch bytes the recall pass needs
+    for frac in (0.0, -0.5, 1.5, float("nan")):
+        assert call(p, 1, frac, per) == 1
+    assert call(p, -1, 0.1, per) == 1
+    assert call(p, 1, 0.1, per, samples=None) == 1
+    assert call(p, 0, 0.1, per - 16) == 3   # scratch too small
+    assert call(p, 0, 0.1, per) == 0        # nothing to do: no launch
+    # a valid layer with more key centroids than the fidelity kernels hold
+    from free_sparse_attention_b200.workloads import COGVIDEOX
+    big = capi.Params.from_workload(COGVIDEOX, Cm=1500)
+    assert capi.workspace_bytes(big) > 0
+    assert call(big, 1, 0.1, 16 * COGVIDEOX.N) == 2
+
+
+def test_device_status_rejections(L):
+    out = ctypes.c_int32(0)
+    assert L.scope_get_device_status(None, None, ctypes.byref(out)) == 1
+    assert L.scope_get_device_status(ctypes.c_void_p(1 << 20), None, None) == 1
