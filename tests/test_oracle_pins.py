@@ -500,3 +500,34 @@ def test_rank_correlation_pins():
     q1 = np.ones(1, np.float32)
     K1 = np.array([[1.0], [2.0], [2.0], [3.0]], np.float32)
     assert abs(oracle.rank_correlation(q1, K1, np.array([1.0, 3.0, 2.0, 4.0])) - 4.5 / math.sqrt(22.5)) < 1e-15
+
+
+def test_equal_scores_rank_by_ascending_index():
+    """The ranking is (proxy descending, key index ascending): with every key on the same
+    code triple all proxies are equal, so S_c is exactly keys 0 .. r_c - 1; with two code
+    groups, the higher-scoring group comes first and each group is cut in index order."""
+    N, Cq, Cm, d = 300, 3, 2, 16
+    rng = np.random.default_rng(21)
+    qcent = rng.standard_normal((Cq, d))
+    kcent = rng.standard_normal((Cm, d))
+    codes = np.zeros((3, N), np.uint16)
+    sel = oracle.select(qcent, np.full(Cq, 5, np.int32), kcent, codes, (4, 6, 6), 0.5, 0.0)
+    bits = np.unpackbits(sel["mask"].view(np.uint8), bitorder="little").reshape(Cq, -1)[:, :N]
+    for c in range(Cq):
+        r = int(sel["r"][c])
+        assert np.all(bits[c, :r] == 1) and np.all(bits[c, r:] == 0), c
+    # two groups of keys, interleaved: even keys on centroid 0, odd keys on centroid 1
+    codes2 = np.zeros((3, N), np.uint16)
+    codes2[:, 1::2] = 1
+    sel2 = oracle.select(qcent, np.full(Cq, 5, np.int32), kcent, codes2, (4, 6, 6), 0.5, 0.0,
+                         want_scores=True)
+    bits2 = np.unpackbits(sel2["mask"].view(np.uint8), bitorder="little").reshape(Cq, -1)[:, :N]
+    for c in range(Cq):
+        s = sel2["scores"][c]
+        assert s[0] != s[1]
+        hi = 0 if s[0] > s[1] else 1          # the group whose proxy is larger
+        order = np.concatenate([np.arange(hi, N, 2), np.arange(1 - hi, N, 2)])
+        r = int(sel2["r"][c])
+        expect = np.zeros(N, np.uint8)
+        expect[order[:r]] = 1
+        assert np.array_equal(bits2[c], expect), c
