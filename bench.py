@@ -597,6 +597,15 @@ def run_fidelity(args, w):
     return 0
 
 
+def dense_prefix_schedule(name, n_steps=50):
+    """(dense_layers, dense_steps) of the dense-prefix schedule the pages print (review page,
+    major_comments: "§4, Implementation details"): the first attention layer dense at every
+    denoising step, and every layer dense for the first 10 % of the steps on HunyuanVideo and
+    20 % on Wan2.1 / Wan2.2 (the other shapes take the Wan share)."""
+    frac = 0.10 if "hunyuan" in name else 0.20
+    return 1, round(frac * n_steps)
+
+
 def run_schedule(args, w):
     """The step before the path and the dense-prefix schedule (review page, major_comments:
     "§4, Implementation details"), on pre-RoPE inputs resident in HBM:
@@ -620,10 +629,11 @@ def run_schedule(args, w):
     del x
     ws = capi.alloc_workspace(p)
     Qr, Kr, O = torch.empty_like(Q), torch.empty_like(K), torch.empty_like(Q)
-    n_steps, dense_steps = 50, (5 if "hunyuan" in w.name else 10)
-    sparse_s = capi.Schedule(layer=1, step=dense_steps, dense_layers=1, dense_steps=dense_steps, rope=1,
+    n_steps = 50
+    dense_layers, dense_steps = dense_prefix_schedule(w.name, n_steps)
+    sparse_s = capi.Schedule(layer=dense_layers, step=dense_steps, dense_layers=dense_layers, dense_steps=dense_steps, rope=1,
                              rope_base=10000.0)
-    dense_s = capi.Schedule(layer=0, step=dense_steps, dense_layers=1, dense_steps=dense_steps, rope=1,
+    dense_s = capi.Schedule(layer=0, step=dense_steps, dense_layers=dense_layers, dense_steps=dense_steps, rope=1,
                             rope_base=10000.0)
 
     def timed(fn, reps):
@@ -658,7 +668,7 @@ def run_schedule(args, w):
         "value": mean_ms, "unit": "ms", "higher_is_better": False, "n_gpus": 1,
         "steps": args.steps, "warmup": args.warmup, "dtype": w.dtype,
         "config": {"workload": workload_desc(w), "n_steps": n_steps, "dense_steps": dense_steps,
-                   "dense_layers": 1, "rope_base": 10000.0,
+                   "dense_layers": dense_layers, "rope_base": 10000.0,
                    "l2": "inputs larger than L2 (Q, K, V resident in HBM)"},
         "rope": {"ms": rope_ms, "bytes": rope_bytes, "achieved_gbs": rope_gbs, "peak_gbs": pk["hbm_gbs"],
                  "frac": rope_gbs / pk["hbm_gbs"], "kernel": "rope3d_kernel (Q and K in one launch)"},
