@@ -631,10 +631,10 @@ def run_schedule(args, w):
     Qr, Kr, O = torch.empty_like(Q), torch.empty_like(K), torch.empty_like(Q)
     n_steps = 50
     dense_layers, dense_steps = dense_prefix_schedule(w.name, n_steps)
-    sparse_s = capi.Schedule(layer=dense_layers, step=dense_steps, dense_layers=dense_layers, dense_steps=dense_steps, rope=1,
-                             rope_base=10000.0)
-    dense_s = capi.Schedule(layer=0, step=dense_steps, dense_layers=dense_layers, dense_steps=dense_steps, rope=1,
-                            rope_base=10000.0)
+    sparse_s = capi.Schedule(layer=dense_layers, step=dense_steps, dense_layers=dense_layers,
+                             dense_steps=dense_steps, rope=1, rope_base=10000.0)
+    dense_s = capi.Schedule(layer=0, step=dense_steps, dense_layers=dense_layers,
+                            dense_steps=dense_steps, rope=1, rope_base=10000.0)
 
     def timed(fn, reps):
         for _ in range(args.warmup):
