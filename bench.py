@@ -49,10 +49,24 @@ def peaks():
     return {"hbm_gbs": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "source": "fallback"}
 
 
+def per_clock_frac(achieved, clk, pk):
+    """Achieved TFLOP/s per SM MHz (median clock sampled during the timed region) against
+    the sustained bf16 matmul's TFLOP/s per MHz at the median clock it ran at."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if not clk or not os.path.exists(path):
+        return None
+    with open(path) as f:
+        peak_mhz = json.load(f).get("clocks_under_load", {}).get("sm_mhz_median")
+    if not peak_mhz or not clk.get("sm_mhz"):
+        return None
+    return (achieved / clk["sm_mhz"]) / (pk["bf16_sustained"] / peak_mhz)
+
+
 def kernels_per_forward(iters: int) -> int:
-    # clustering: init + iters x (fast assign, exact assign, hist, scan, scatter, update)
-    # selection: check, top-p, k_head, mask; attention: items, zero-fill, attention
-    return 1 + 6 * iters + 4 + 3
+    # clustering: init + iters x (pack, tensor-core assign, exact assign, hist, scan,
+    # scatter, update); selection: check, top-p, k_head, mask; attention: items, zero-fill,
+    # attention
+    return 1 + 7 * iters + 4 + 3
 
 
 def workload_desc(w):
@@ -132,12 +146,15 @@ def dist_setup():
 
 
 # ----------------------------------------------------------------------------- CPU oracle
-def oracle_sample(w, T_sample=6, khead_off=False):
+ORACLE_SAMPLE_FRAMES = 4   # both CPU legs (cpu_baseline and --impl reference) use this sample
+
+
+def oracle_sample(w, T_sample=ORACLE_SAMPLE_FRAMES, khead_off=False):
     """The oracle on a bounded sub-layer: head (0, 0) of the same workload with the
     grid cut to the first T_sample frames (N_s = T_sample*Hg*Wg tokens); every stage
-    runs in full on it.  Each stage's cost is extrapolated to the whole layer by its
+    runs in full on it.  Each stage's cost is EXTRAPOLATED to the whole layer by its
     complexity (clustering and selection linear in N per head, attention by its
-    effective FLOPs).  Returns (layer seconds, description, threads)."""
+    effective FLOPs); the sample's own realised density estimates the layer's."""
     import oracle
     ws = w.with_(T=T_sample, H=1, B=1)
     x = synth.layer_inputs(ws)
@@ -151,24 +168,36 @@ def oracle_sample(w, T_sample=6, khead_off=False):
     t2 = time.perf_counter()
     oracle.attention(q, k, v, rq["assign"], sel["mask"])
     t3 = time.perf_counter()
-    eff = 4.0 * float(np.dot(rq["sizes"].astype(np.float64), sel["r"].astype(np.float64))) * ws.d
+    nr = float(np.dot(rq["sizes"].astype(np.float64), sel["r"].astype(np.float64)))
+    eff = 4.0 * nr * ws.d
+    density = nr / (ws.N * ws.N)
     scale = (w.N / ws.N) * w.H * w.B
-    desc = (f"oracle on head (0,0) cut to the first {T_sample} frames (N_s={ws.N}): clustering "
-            f"{t1 - t0:.2f}s, selection {t2 - t1:.2f}s, attention {t3 - t2:.2f}s "
-            f"({eff / (t3 - t2) / 1e9:.2f} GFLOP/s); clustering and selection scaled by "
-            f"N/N_s x heads, attention by the layer's effective FLOPs")
+    desc = (f"EXTRAPOLATED from the oracle on head (0,0) cut to the first {T_sample} frames "
+            f"(N_s={ws.N}): clustering {t1 - t0:.2f}s, selection {t2 - t1:.2f}s, attention {t3 - t2:.2f}s "
+            f"({eff / (t3 - t2) / 1e9:.2f} GFLOP/s, sample density {density:.4f}); clustering and "
+            f"selection scaled by N/N_s x heads, attention by the layer's effective FLOPs")
     return {"clust_s": (t1 - t0) * scale, "sel_s": (t2 - t1) * scale, "attn_rate": eff / (t3 - t2),
-            "desc": desc, "threads": oracle.num_threads()}
+            "desc": desc, "threads": oracle.num_threads(), "density": density,
+            "sample_s": t3 - t0}
 
 
 def layer_seconds_from_sample(s, flops):
     return s["clust_s"] + s["sel_s"] + flops / s["attn_rate"]
 
 
-def expected_layer_flops(w):
-    """Effective FLOPs of the layer when r_c is unknown (reference arm): dense x 0.89,
-    the realised density the oracle measures on this generator at rho = 0.9."""
-    return 4.0 * w.B * w.H * w.N * w.N * w.d * 0.89
+def sample_layer_flops(w, s):
+    """Effective FLOPs of the whole layer estimated by the oracle alone: dense FLOPs times
+    the realised density of its own sample (no GPU value enters the CPU legs)."""
+    return 4.0 * w.B * w.H * w.N * w.N * w.d * s["density"]
+
+
+def oracle_baseline(w, khead_off=False):
+    """The CPU leg both arms report: the extrapolated oracle layer time and its metric."""
+    s = oracle_sample(w, khead_off=khead_off)
+    flops = sample_layer_flops(w, s)
+    sec = layer_seconds_from_sample(s, flops)
+    return {"value": flops / sec / 1e12, "unit": "TFLOP/s", "cores": s["threads"], "kind": "oracle",
+            "extrapolated": True, "sample": s["desc"], "layer_s": sec}
 
 
 def run_reference(args, w):
@@ -176,14 +205,14 @@ def run_reference(args, w):
     if rank != 0:
         return 0
     for _ in range(args.warmup):
-        oracle_sample(w, T_sample=4, khead_off=args.khead_off)
-    times, desc, threads = [], "", 1
-    flops = expected_layer_flops(w)
+        oracle_sample(w, khead_off=args.khead_off)
+    times, desc, threads, flops = [], "", 1, 0.0
     for _ in range(args.steps):
-        s = oracle_sample(w, T_sample=4, khead_off=args.khead_off)
+        s = oracle_sample(w, khead_off=args.khead_off)
+        flops = sample_layer_flops(w, s)
         times.append(layer_seconds_from_sample(s, flops))
         desc, threads = s["desc"], s["threads"]
-    sec = statistics.mean(times)
+    sec = statistics.median(times)
     value = flops / sec / 1e12
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
@@ -191,7 +220,7 @@ def run_reference(args, w):
             "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded generator G)",
             "config": {"workload": workload_desc(w), "parallelism": "oracle, OpenMP threads"},
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-                             "sample": desc + "; effective FLOPs taken at density 0.89"},
+                             "extrapolated": True, "sample": desc},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -270,6 +299,10 @@ def run_scope(args, w):
     r_c = it["final_counts"].double()
     flops = float(4.0 * (n_c * r_c).sum().item() * w.d)
     density = float((n_c * r_c).sum().item() / (w.B * w.H * w.N * w.N))
+    kh = it["k_head"].double()
+    khead_stats = {"min": int(kh.min().item()), "mean": float(kh.mean().item()), "max": int(kh.max().item()),
+                   "clusters_topped_up": int((it["final_counts"] > it["base_counts"]).sum().item()),
+                   "clusters": int(it["final_counts"].numel())}
     del it
 
     def mk_events():
@@ -297,10 +330,15 @@ def run_scope(args, w):
     if world > 1:
         dist.barrier()
     clk = clocks.stop()
-    ms = e0.elapsed_time(e1) / args.steps
+    ms_mean = e0.elapsed_time(e1) / args.steps
+    # per-step layer times from each step's first stage event to the next step's (the last
+    # to the closing event); the step time reported is their median
+    starts = [ev[0] for ev in stage_evs] + [e1]
+    step_ms = [starts[i].elapsed_time(starts[i + 1]) for i in range(args.steps)]
     st = np.array([[ev[i].elapsed_time(ev[i + 1]) for i in range(4)] for ev in stage_evs])
-    stage_ms = st.mean(axis=0)
-    ms = max_over_ranks(ms, device="cuda")
+    stage_ms = np.median(st, axis=0)
+    ms = max_over_ranks(statistics.median(step_ms), device="cuda")
+    ms_mean = max_over_ranks(ms_mean, device="cuda")
     status |= capi.get_device_status(ws)
 
     # end to end through the C ABI with host buffers: every step copies its inputs H2D from
@@ -410,9 +448,11 @@ def run_scope(args, w):
                    "parallelism": f"{world} independent layers, one per GPU (no collective)",
                    "l2": "inputs larger than L2 (Q, K, V = 2.19 GB resident in HBM)"},
         "roofline": {"bound": "tensor", "kernel": "attn_tc_kernel (tcgen05 sparse attention)",
-                     "achieved": achieved, "peak": pk["bf16_sustained"], "unit": "TFLOP/s",
-                     "frac": achieved / pk["bf16_sustained"], "traffic": traffic,
-                     "peak_source": f"{pk['source']} bf16 sustained (kernel timed inside the step)"},
+                     "achieved": achieved, "peak": pk["bf16"], "unit": "TFLOP/s",
+                     "frac": achieved / pk["bf16"], "traffic": traffic,
+                     "peak_source": f"{pk['source']} bf16 burst",
+                     "frac_of_sustained": achieved / pk["bf16_sustained"],
+                     "frac_per_clock": per_clock_frac(achieved, clk, pk)},
         "stages_ms": {"clustering": float(stage_ms[0]), "selection": float(stage_ms[1]),
                       "worklist": float(stage_ms[2]), "attention": attn_ms},
         "stage_fractions": {
@@ -422,6 +462,7 @@ def run_scope(args, w):
             "clustering_tensor": clust_flops / (stage_ms[0] * 1e-3) / 1e12 / pk["bf16_sustained"],
             "selection_hbm": sel_bytes / (stage_ms[1] * 1e-3) / 1e9 / pk["hbm_gbs"]},
         "density": density, "effective_tflop_per_layer": flops / 1e12,
+        "ms_per_step_mean": ms_mean, "k_head": khead_stats,
         "dense_sdpa_ms": dense_ms,
         "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
@@ -434,10 +475,7 @@ def run_scope(args, w):
         "clocks": clk,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.full_keys:
-        s = oracle_sample(w, khead_off=args.khead_off)
-        sec = layer_seconds_from_sample(s, flops)
-        line["cpu_baseline"] = {"value": flops / sec / 1e12, "unit": "TFLOP/s", "cores": s["threads"],
-                                "kind": "oracle", "sample": s["desc"]}
+        line["cpu_baseline"] = oracle_baseline(w, khead_off=args.khead_off)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -18,7 +18,8 @@ LIB_PATH = os.path.join(HERE, "libscope.so")
 
 SCOPE_F32, SCOPE_BF16 = 0, 1
 STATUS = {0: "SCOPE_OK", 1: "SCOPE_ERR_INVALID_ARGUMENT", 2: "SCOPE_ERR_UNSUPPORTED",
-          3: "SCOPE_ERR_WORKSPACE_TOO_SMALL", 4: "SCOPE_ERR_CUDA", 5: "SCOPE_ERR_DEVICE_CHECK"}
+          3: "SCOPE_ERR_WORKSPACE_TOO_SMALL", 4: "SCOPE_ERR_CUDA", 5: "SCOPE_ERR_DEVICE_CHECK",
+          6: "SCOPE_ERR_TIMEOUT"}
 DEV_BAD_INIT_INDEX, DEV_SELECT_TIE, DEV_BAD_ASSIGN = 0x1, 0x2, 0x4
 
 EXPORTS = ("scope_workspace_bytes", "scope_cluster_queries", "scope_cluster_keys",
@@ -26,7 +27,8 @@ EXPORTS = ("scope_workspace_bytes", "scope_cluster_queries", "scope_cluster_keys
            "scope_status_string", "scope_get_device_status", "scope_build_lut_and_select_noalloc",
            "scope_selection_recall", "scope_permute_channels", "scope_dense_attention",
            "scope_rope3d", "scope_layer_is_dense", "scope_attention_layer",
-           "scope_rank_correlation_scratch_bytes", "scope_rank_correlation")
+           "scope_rank_correlation_scratch_bytes", "scope_rank_correlation", "scope_check_wait_timeout",
+           "scope_tc_accumulation_probe")
 
 
 class ScopeError(RuntimeError):
@@ -128,6 +130,10 @@ def lib() -> ctypes.CDLL:
         L.scope_status_string.argtypes = [i]
         L.scope_get_device_status.restype = i
         L.scope_get_device_status.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_int32)]
+        L.scope_check_wait_timeout.restype = i
+        L.scope_check_wait_timeout.argtypes = [P, ctypes.c_uint64, vp, sz, vp]
+        L.scope_tc_accumulation_probe.restype = i
+        L.scope_tc_accumulation_probe.argtypes = [vp, vp, i, i, vp, vp]
         _lib = L
     return _lib
 
@@ -353,9 +359,35 @@ def attention_layer(p, sched: Schedule, Q, K, V, q_init_idx=None, k_init_idx=Non
     return O
 
 
+def check_wait_timeout(p, wait_limit_ns, ws=None, stream=None):
+    """Runs the attention kernel with its scheduler held so every first wait gives up after
+    wait_limit_ns (the device-side timeout path); returns the workspace used."""
+    ws = alloc_workspace(p) if ws is None else ws
+    _check("scope_check_wait_timeout", lib().scope_check_wait_timeout(
+        ctypes.byref(p), int(wait_limit_ns), _ptr(ws), ws.numel(), _stream(stream)))
+    return ws
+
+
+def tc_accumulation_probe(A, B, stream=None):
+    """The tensor core's fp32 result of A @ B^T (A [128, K], B [N, K] bf16 on the device) as
+    one chain of K/16 tcgen05.mma steps."""
+    K, N = A.shape[1], B.shape[0]
+    D = torch.empty((128, N), dtype=torch.float32, device=A.device)
+    _check("scope_tc_accumulation_probe", lib().scope_tc_accumulation_probe(
+        _ptr(A), _ptr(B), int(K), int(N), _ptr(D), _stream(stream)))
+    return D
+
+
+def device_status_code(ws, stream=None):
+    """(return code of scope_get_device_status, status word)."""
+    out = ctypes.c_int32(0)
+    code = lib().scope_get_device_status(_ptr(ws), _stream(stream), ctypes.byref(out))
+    return int(code), int(out.value)
+
+
 def get_device_status(ws, stream=None) -> int:
     out = ctypes.c_int32(0)
     code = lib().scope_get_device_status(_ptr(ws), _stream(stream), ctypes.byref(out))
-    if code not in (0, 5):
+    if code not in (0, 5, 6):
         raise ScopeError("scope_get_device_status", code)
     return int(out.value)

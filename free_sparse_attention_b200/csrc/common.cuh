@@ -11,7 +11,8 @@ namespace scope {
 
 constexpr int kMaxC = 2048;         // max centroids per problem (LUT and histogram sizes)
 constexpr int kSortChunk = 512;     // tokens per warp in the stable counting sort
-constexpr int kAttnTile = 256;      // queries per attention work item (two 128-row tiles)
+constexpr int kAttnTile = 128;      // queries per attention work item (one 128-row tile)
+constexpr unsigned long long kTcWaitDefaultNs = 4000000000ull;   // pipeline wait limit (4 s)
 
 // ---------------------------------------------------------------------------------
 // Clustering problems.  Role 0 = queries (all d channels, C = Cq); roles 1..3 = the
@@ -61,8 +62,8 @@ struct WsLayout {
     size_t status, counters;
     size_t cent32, cent64T, cnorm, cnrm2, cslack, perm, off, chunk_hist, cent_bf, cn2p, unsure_list, unsure_count;
     size_t q_cent, q_assign, q_sizes, k_cent, k_codes, k_sizes;
-    size_t topp, base, khead, final_cnt, mask, sel_state;
-    size_t q_perm, q_off, q_hist, work_items, attn_counter, key_lists;
+    size_t topp, base, khead, final_cnt, mask, sel_state, sel_hist;
+    size_t q_perm, q_off, q_hist, work_items, unit_pos, head_pair, attn_counter;
     size_t total;
 };
 
@@ -83,6 +84,7 @@ struct SelArgs {
     int32_t *topp, *base, *khead, *final_cnt;
     uint32_t *mask;           // [BH, Cq, nw]
     double *state;            // [BH*Cq, 8] per-unit selection state
+    int32_t *hist;            // [BH*Cq, 2048] level-0 key counts of the Top-p pass (or NULL)
     int BH, N, d, dt, dh, dw, Cq, Cm, nw;
     double rho, inv_sqrt_d;
     int kfix;
@@ -99,15 +101,17 @@ struct AttnArgs {
     long long perm_bh, off_bh;
     const uint32_t *mask;     // [BH, Cq, nw]
     const int32_t *final_cnt; // [BH, Cq]
-    int4 *items;              // work list (bh, c, q0, nq)
-    int32_t *lists;           // selected key indices of unit u at lists[u*list_stride ...], ascending
-    long long list_stride;    // N rounded up to a multiple of 4
-    int32_t *counter;         // [2]: item count, dynamic scheduler
+    int4 *items;              // work list: pair p = items[2p], items[2p+1], each (bh, c, q0, nq)
+    int32_t *unit_pos;        // [BH*Cq + 1] scratch of the work-list builder
+    int32_t *head_pair;       // [BH] scratch of the work-list builder
+    int32_t *counter;         // [2]: pair count, dynamic scheduler
     int BH, N, d, Cq, nw, is_bf16;
     int use_tc;               // bf16 on the tensor cores (else CUDA cores)
     float scale_log2;         // log2(e)/sqrt(d)
     int32_t *status;
     int num_sms;
+    unsigned long long wait_ns;   // limit of every pipeline wait of the tensor-core kernel
+    int hold_items;           // nonzero: the kernel's scheduler publishes no item (timeout check)
 };
 cudaError_t attention_run(const AttnArgs &a, cudaStream_t s);     // items + kernel
 cudaError_t attention_items(const AttnArgs &a, cudaStream_t s);   // work list only
@@ -162,6 +166,7 @@ cudaError_t attention_dense_setup(uint16_t *q_assign, uint32_t *mask, int32_t *f
 cudaError_t permute_channels_run(const void *X, const int32_t *perm, void *Y, long long rows, int d,
                                  int is_bf16, int num_sms, cudaStream_t s);
 size_t select_smem_bytes(int Cm, int d);
+constexpr int kSelBins = 2048;      // histogram bins of the selection passes
 
 // ---------------------------------------------------------------------------------
 __device__ __forceinline__ float load_x(const void *X, long long idx, int is_bf16)

@@ -7,13 +7,14 @@
 // non-empty centroid moves to the mean of its members.
 //
 // Design (B200): the assignment is a [tokens x dm] x [dm x C] contraction followed by
-// an argmin.  For bf16 inputs it runs on the tensor cores (kmeans_tc.cu); otherwise
+// an argmin.  For bf16 inputs it runs on the tensor cores (kmeans_tc.cu, whose error
+// bound rests on a measured model of the tensor core's accumulation); otherwise
 // (fp32 inputs, or centroid sets too large for shared memory) on the fp32 FMA pipes
-// with centroids staged in shared memory (km_assign_fast_kernel below);
-// each distance carries a rigorous error bound, and a token whose best and runner-up
-// cannot be told apart under that bound is re-decided in binary64 with the channels
-// summed in order (one rounding per operation).  Hence the assignment equals a
-// binary64 evaluation of the definition exactly.  The update sums each centroid's
+// with centroids staged in shared memory (km_assign_fast_kernel below), where each
+// distance carries an error bound proven from IEEE binary32 arithmetic.  A token whose
+// best and runner-up cannot be told apart under its bound is re-decided in binary64
+// with the channels summed in order (one rounding per operation).  Hence the assignment
+// equals a binary64 evaluation of the definition exactly.  The update sums each centroid's
 // members in increasing token order in binary64: a stable counting sort by cluster
 // gives every (centroid, channel) pair its member list, so the sum is sequential and
 // the means are bit-identical to an in-order binary64 evaluation.

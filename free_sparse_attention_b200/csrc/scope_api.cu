@@ -218,6 +218,7 @@ SelArgs sel_args(const scope_params &p, const WsLayout &L, void *ws, const doubl
     a.final_cnt = fin;
     a.mask = mask;
     a.state = at<double>(ws, L.sel_state);
+    a.hist = at<int32_t>(ws, L.sel_hist);
     a.BH = (int)D.BH;
     a.N = (int)D.N;
     a.d = p.d;
@@ -252,8 +253,8 @@ AttnArgs attn_args(const scope_params &p, const WsLayout &L, void *ws, const voi
     a.mask = mask;
     a.final_cnt = fin;
     a.items = at<int4>(ws, L.work_items);
-    a.lists = at<int32_t>(ws, L.key_lists);
-    a.list_stride = (D.N + 3) / 4 * 4;
+    a.unit_pos = at<int32_t>(ws, L.unit_pos);
+    a.head_pair = at<int32_t>(ws, L.head_pair);
     a.counter = at<int32_t>(ws, L.counters);
     a.BH = (int)D.BH;
     a.N = (int)D.N;
@@ -268,6 +269,8 @@ AttnArgs attn_args(const scope_params &p, const WsLayout &L, void *ws, const voi
     cudaGetDevice(&dev);
     a.num_sms = 148;
     cudaDeviceGetAttribute(&a.num_sms, cudaDevAttrMultiProcessorCount, dev);
+    a.wait_ns = kTcWaitDefaultNs;
+    a.hold_items = 0;
     return a;
 }
 
@@ -312,8 +315,10 @@ WsLayout ws_layout(const scope_params &p)
     L.final_cnt = take(sizeof(int32_t) * D.BH * p.Cq);
     L.mask = take(sizeof(uint32_t) * D.BH * p.Cq * D.nw);
     L.sel_state = take(sizeof(double) * 8 * D.BH * p.Cq);
-    L.work_items = take(sizeof(int4) * D.BH * ((D.N + kAttnTile - 1) / kAttnTile + p.Cq));
-    L.key_lists = take(sizeof(int32_t) * D.BH * p.Cq * ((D.N + 3) / 4 * 4));
+    L.sel_hist = take(sizeof(int32_t) * kSelBins * D.BH * p.Cq);
+    L.work_items = take(sizeof(int4) * D.BH * ((D.N + kAttnTile - 1) / kAttnTile + p.Cq + 2));
+    L.unit_pos = take(sizeof(int32_t) * (D.BH * p.Cq + 1));
+    L.head_pair = take(sizeof(int32_t) * (D.BH + 1));
     L.total = o;
     return L;
 }
@@ -337,6 +342,7 @@ const char *scope_status_string(scope_status s)
     case SCOPE_ERR_WORKSPACE_TOO_SMALL: return "SCOPE_ERR_WORKSPACE_TOO_SMALL";
     case SCOPE_ERR_CUDA: return "SCOPE_ERR_CUDA";
     case SCOPE_ERR_DEVICE_CHECK: return "SCOPE_ERR_DEVICE_CHECK";
+    case SCOPE_ERR_TIMEOUT: return "SCOPE_ERR_TIMEOUT";
     }
     return "SCOPE_ERR_UNKNOWN";
 }
@@ -350,6 +356,7 @@ scope_status scope_get_device_status(const void *ws, void *stream, int32_t *out)
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);
     if (e != cudaSuccess) return SCOPE_ERR_CUDA;
     *out = v;
+    if (v & SCOPE_DEV_TIMEOUT) return SCOPE_ERR_TIMEOUT;
     return v ? SCOPE_ERR_DEVICE_CHECK : SCOPE_OK;
 }
 
@@ -687,6 +694,24 @@ scope_status scope_permute_channels(const scope_params *p, const void *X, const 
         return SCOPE_ERR_CUDA;
     return cuda_status(permute_channels_run(X, perm, Y, D.BH * D.N, p->d, p->dtype == SCOPE_BF16, sms,
                                             static_cast<cudaStream_t>(stream)));
+}
+
+scope_status scope_check_wait_timeout(const scope_params *p, uint64_t wait_limit_ns, void *ws, size_t ws_bytes,
+                                      void *stream)
+{
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    WsLayout L;
+    scope_status st = begin(p, ws, ws_bytes, L, s);
+    if (st != SCOPE_OK) return st;
+    if (p->dtype != SCOPE_BF16) return SCOPE_ERR_UNSUPPORTED;
+    if (wait_limit_ns < 1 || wait_limit_ns > 10000000000ull) return SCOPE_ERR_INVALID_ARGUMENT;
+    if ((st = clear_status(ws, L, s)) != SCOPE_OK) return st;
+    if (cudaMemsetAsync(at<char>(ws, L.counters), 0, 4 * sizeof(int32_t), s) != cudaSuccess) return SCOPE_ERR_CUDA;
+    // no tensor is read: the held scheduler never hands out an item
+    AttnArgs t = attn_args(*p, L, ws, nullptr, nullptr, nullptr, nullptr, nullptr, 0, nullptr, 0, nullptr, nullptr);
+    t.wait_ns = wait_limit_ns;
+    t.hold_items = 1;
+    return cuda_status(attention_kernel(t, s));
 }
 
 scope_status scope_forward(const scope_params *p, const void *Q, const void *K, const void *V,

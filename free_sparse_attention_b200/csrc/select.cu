@@ -15,12 +15,19 @@
 // most 2048 keys, otherwise it is binned again over its own value range; keys with
 // identical logits are binned by index instead.
 //
-// The softmax mass of key j is exp(s_j - max s) up to the factorisation
-//   exp(s_j) = exp(P^T/sqrt d) exp(P^H/sqrt d) exp(P^W/sqrt d),
-// i.e. three table lookups and two products instead of an exponential per key
-// (relative error ~1e-15).  Masses are accumulated as fixed-point integers
-// (2^-63 units, split 32/32 bits), so every sum is exact and independent of order:
-// results are deterministic run to run.
+// The softmax mass of key j is w_j = exp(s_j - s_ref), s_ref an upper bound of every
+// logit: t = (s_j - s_ref) log2 e in binary64 is split into n + f (n an integer, f in
+// [0, 1)) and w_j = 2^n 2^f with 2^f from the fp32 ex2 instruction (relative error of w_j
+// below 3e-7, no table lookup).  Masses are accumulated as fixed-point integers (2^-63
+// units, split 32/32 bits), so every sum is exact and independent of order: results are
+// deterministic run to run, and a Top-p count can differ from a binary64 evaluation only
+// where the mass of a prefix is within ~3e-7 (relative) of rho times the total, inside the
+// 1e-6 band in which the oracle logs a near tie.
+//
+// The Top-p kernel saves the count histogram of its first (full-range) pass; the mask
+// kernel uses it to find the bin where the r_c-th key of the ranking lies, so that one
+// pass over the keys writes the selected set (keys of higher bins set directly, the keys
+// of that bin ranked exactly in shared memory).
 #include "common.cuh"
 
 #include <cfloat>
@@ -30,13 +37,13 @@ namespace scope {
 namespace {
 
 constexpr int kSelThreads = 512;
-constexpr int kBins = 2048;
+constexpr int kBins = kSelBins;
 constexpr int kCap = 2048;
 constexpr int kMaxLevels = 6;
 constexpr int kBinsPerThread = kBins / kSelThreads;
 
 struct SelSmem {
-    double *lut, *E, *qc;
+    double *lut, *qc;
     int *cnt;
     unsigned long long *mhi, *mlo;
     double *cs;
@@ -50,7 +57,7 @@ struct SelSmem {
 
 __host__ __device__ size_t sel_smem_bytes(int Cm, int d)
 {
-    return sizeof(double) * (6 * (size_t)Cm + d) + sizeof(int) * kBins +
+    return sizeof(double) * (3 * (size_t)Cm + d) + sizeof(int) * kBins +
            2 * sizeof(unsigned long long) * kBins + sizeof(double) * kCap + sizeof(int) * kCap +
            sizeof(unsigned long long) * kCap + sizeof(int) * kCap + sizeof(double) * 32 +
            sizeof(unsigned long long) * 96 + sizeof(int) * 8;
@@ -61,8 +68,7 @@ __device__ SelSmem carve(char *base, int Cm, int d)
     SelSmem s;
     double *dp = reinterpret_cast<double *>(base);
     s.lut = dp;
-    s.E = dp + 3 * Cm;
-    s.qc = dp + 6 * Cm;
+    s.qc = dp + 3 * Cm;
     s.cs = s.qc + d;
     s.red = s.cs + kCap;
     unsigned long long *up = reinterpret_cast<unsigned long long *>(s.red + 32);
@@ -82,6 +88,7 @@ struct Unit {
     const uint16_t *zt, *zh, *zw;
     int Cm, N;
     double inv;          // 1/sqrt(d)
+    double sref;         // logit reference of the weights (>= every logit)
     double inv_umax;     // mass normalisation
 };
 
@@ -126,19 +133,23 @@ __device__ __forceinline__ void batch_scores(const SelSmem &S, const Unit &u, co
     for (int k = 0; k < kBatch; ++k) s[k] = __dmul_rn(u.inv, __dadd_rn(__dadd_rn(a[k], b[k]), c[k]));
 }
 
-// key weights u_j = E^T E^H E^W for every key of the batch
-__device__ __forceinline__ void batch_weights(const SelSmem &S, const Unit &u, const KeyBatch &kb,
-                                              double (&w)[kBatch])
+// Softmax weight of a key of logit s: exp(s - sref) = 2^n 2^f with t = (s - sref) log2 e
+// = n + f (binary64; t - n is exact) and 2^f from ex2.approx.f32 (at most 2 ulp).
+__device__ __forceinline__ double key_weight(double s, const Unit &u)
 {
-    double a[kBatch], b[kBatch], c[kBatch];
+    const double t = __dmul_rn(__dsub_rn(s, u.sref), 1.4426950408889634);
+    const double n = floor(t);
+    if (n < -1000.0) return 0.0;
+    float p;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(p) : "f"((float)(t - n)));
+    return __dmul_rn((double)p, __hiloint2double(((int)n + 1023) << 20, 0));
+}
+
+// key weights for every key of the batch (from its logit)
+__device__ __forceinline__ void batch_weights(const Unit &u, const double (&s)[kBatch], double (&w)[kBatch])
+{
 #pragma unroll
-    for (int k = 0; k < kBatch; ++k) {
-        a[k] = S.E[kb.zt[k]];
-        b[k] = S.E[u.Cm + kb.zh[k]];
-        c[k] = S.E[2 * u.Cm + kb.zw[k]];
-    }
-#pragma unroll
-    for (int k = 0; k < kBatch; ++k) w[k] = __dmul_rn(__dmul_rn(a[k], b[k]), c[k]);
+    for (int k = 0; k < kBatch; ++k) w[k] = key_weight(s[k], u);
 }
 
 // fixed-point mass of weight w in units of 2^-63, clamped to [0, 2^63]
@@ -266,7 +277,7 @@ struct SelectOut {
 // umax_out (mass mode): the largest key weight, found in the first histogram pass.
 __device__ SelectOut block_select(const SelSmem &S, const Unit &u, bool mass_mode, double rho,
                                   long long count, double smax, double smin, int32_t *status,
-                                  double *umax_out = nullptr)
+                                  double *umax_out = nullptr, int32_t *save_hist = nullptr)
 {
     Levels L;
     L.n = 0;
@@ -294,7 +305,7 @@ __device__ SelectOut block_select(const SelSmem &S, const Unit &u, bool mass_mod
             const KeyBatch kb = load_batch(u, j0);
             double sc[kBatch], uw[kBatch];
             batch_scores(S, u, kb, sc);
-            if (mass_mode) batch_weights(S, u, kb, uw);
+            if (mass_mode) batch_weights(u, sc, uw);
 #pragma unroll
             for (int k = 0; k < kBatch; ++k) {
                 const double s = sc[k];
@@ -315,6 +326,8 @@ __device__ SelectOut block_select(const SelSmem &S, const Unit &u, bool mass_mod
         cmin = block_min(cmin, S.red);
         cmax = block_max(cmax, S.red);
         if (mass_mode && iter == 0 && umax_out) *umax_out = block_max(umx, S.red);
+        if (iter == 0 && save_hist && !(cmin == cmax))   // the full-range counts, for the mask kernel
+            for (int b = tid; b < kBins; b += kSelThreads) save_hist[b] = S.cnt[b];
         if (!L.jmode && cmin == cmax) {
             // every candidate has the same logit: the ranking among them is by index
             L.jmode = true;
@@ -400,11 +413,7 @@ __device__ SelectOut block_select(const SelSmem &S, const Unit &u, bool mass_mod
                     if (slot < kCap) {
                         S.cs[slot] = s;
                         S.cj[slot] = j;
-                        if (mass_mode) {
-                            const double w = __dmul_rn(__dmul_rn(S.E[kb.zt[k]], S.E[u.Cm + kb.zh[k]]),
-                                                       S.E[2 * u.Cm + kb.zw[k]]);
-                            S.cw[slot] = weight_mass(w, u);
-                        }
+                        if (mass_mode) S.cw[slot] = weight_mass(key_weight(s, u), u);
                     }
                 }
             }
@@ -476,8 +485,8 @@ __device__ SelectOut block_select(const SelSmem &S, const Unit &u, bool mass_mod
     return out;
 }
 
-// Builds the LUT (and, with want_E, the per-subspace exponential tables) for unit c.
-__device__ void build_tables(const SelArgs &a, const SelSmem &S, int bh, int c, bool want_E)
+// Builds the LUT of unit c: P^m[c, z] for the three subspaces m and every code z.
+__device__ void build_tables(const SelArgs &a, const SelSmem &S, int bh, int c)
 {
     const int tid = threadIdx.x, Cm = a.Cm, d = a.d;
     const double *qc = a.qcent + ((size_t)bh * a.Cq + c) * d;
@@ -493,15 +502,6 @@ __device__ void build_tables(const SelArgs &a, const SelSmem &S, int bh, int c, 
         S.lut[idx] = acc;
     }
     __syncthreads();
-    if (!want_E) return;
-    for (int m = 0; m < 3; ++m) {
-        double mx = -DBL_MAX;
-        for (int z = tid; z < Cm; z += kSelThreads) mx = fmax(mx, S.lut[m * Cm + z]);
-        mx = block_max(mx, S.red);
-        for (int z = tid; z < Cm; z += kSelThreads)
-            S.E[m * Cm + z] = exp(__dmul_rn(__dsub_rn(S.lut[m * Cm + z], mx), a.inv_sqrt_d));
-        __syncthreads();
-    }
 }
 
 // ------------------------------------------------------------------------- kernels
@@ -522,7 +522,7 @@ __global__ void __launch_bounds__(kSelThreads) sel_topp_kernel(SelArgs a)
     extern __shared__ __align__(16) char smem_raw[];
     const SelSmem S = carve(smem_raw, a.Cm, a.d);
     const int c = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
-    build_tables(a, S, bh, c, true);
+    build_tables(a, S, bh, c);
     Unit u;
     u.zt = a.codes + (size_t)bh * 3 * a.N;
     u.zh = u.zt + a.N;
@@ -549,20 +549,25 @@ __global__ void __launch_bounds__(kSelThreads) sel_topp_kernel(SelArgs a)
     // quantised against 1: at most N 2^-64 of absolute error in total.  That stays below
     // 1e-9 of the total mass Z >= max_j u_j unless the largest weight is tiny, in which
     // case the selection runs again normalised by the largest weight itself.
+    u.sref = smax;
     u.inv_umax = 1.0;
     long long p = a.N;
     SelectOut so{smax, 0, 0};
+    const size_t unit = (size_t)bh * a.Cq + c;
+    int32_t *hist = a.hist ? a.hist + unit * kBins : nullptr;
     if (a.rho < 1.0) {
         double umax = 1.0;
-        so = block_select(S, u, true, a.rho, 0, smax, smin, a.status, &umax);
+        so = block_select(S, u, true, a.rho, 0, smax, smin, a.status, &umax, hist);
         if (umax < (double)a.N * 0x1p-64 * 1e9 && umax > 0.0) {
             u.inv_umax = 1.0 / umax;
             so = block_select(S, u, true, a.rho, 0, smax, smin, a.status);
         }
         p = so.rank + 1;
     }
+    // rho = 1 selects every key: no pass ran, so the level-0 counts are only saved when a
+    // count-based selection will need them (never: r = N then)
+    const bool saved = hist && a.rho < 1.0 && smax > smin;
     if (tid == 0) {
-        const size_t unit = (size_t)bh * a.Cq + c;
         const long long b = p > a.kfix ? p : a.kfix;
         if (a.topp) a.topp[unit] = (int32_t)p;
         a.base[unit] = (int32_t)b;
@@ -572,6 +577,7 @@ __global__ void __launch_bounds__(kSelThreads) sel_topp_kernel(SelArgs a)
         st[2] = so.s;
         st[3] = (double)so.j;
         st[4] = (double)p;
+        st[5] = saved ? 1.0 : 0.0;
     }
 }
 
@@ -631,7 +637,7 @@ __global__ void __launch_bounds__(kSelThreads) sel_mask_kernel(SelArgs a)
         }
         return;
     }
-    build_tables(a, S, bh, c, false);
+    build_tables(a, S, bh, c);
     Unit u;
     u.zt = a.codes + (size_t)bh * 3 * a.N;
     u.zh = u.zt + a.N;
@@ -639,18 +645,59 @@ __global__ void __launch_bounds__(kSelThreads) sel_mask_kernel(SelArgs a)
     u.Cm = a.Cm;
     u.N = a.N;
     u.inv = a.inv_sqrt_d;
+    u.sref = a.state[unit * 8];
     u.inv_umax = 1.0;
     const double *st = a.state + unit * 8;
-    double s_star;
-    int j_star;
+    const double hi = st[0], lo = st[1];
+    const double scale = (hi > lo) ? (double)kBins / (hi - lo) : 0.0;
+    // Either the exact last selected key (s*, j*) is known -- the Top-p boundary when r_c =
+    // p_c, or a count-based select -- or the level-0 counts saved by the Top-p kernel give the
+    // bin b* that holds the r_c-th key: every key of a lower bin (higher logits) is selected,
+    // and the keys of b* are gathered in this same pass and ranked afterwards.
+    double s_star = 0.0;
+    int j_star = 0, bstar = -1;
+    long long before = 0;
     if ((long long)st[4] == r) {
         s_star = st[2];
         j_star = (int)st[3];
     } else {
-        const SelectOut so = block_select(S, u, false, 0.0, r, st[0], st[1], a.status);
-        s_star = so.s;
-        j_star = so.j;
+        if (st[5] != 0.0) {
+            const int32_t *h = a.hist + unit * kBins;
+            unsigned long long z0 = 0, z1 = 0, tc = 0;
+            const int b0 = tid * kBinsPerThread;
+            int cnt[kBinsPerThread];
+            for (int q = 0; q < kBinsPerThread; ++q) {
+                cnt[q] = h[b0 + q];
+                tc += (unsigned long long)cnt[q];
+            }
+            unsigned long long tot[3];
+            block_excl_scan3(z0, z1, tc, S.ured, tot);
+            if (tid == 0) S.misc[0] = -1;
+            __syncthreads();
+            long long ec = (long long)tc;
+            for (int q = 0; q < kBinsPerThread; ++q) {
+                if (ec < r && ec + cnt[q] >= r) {
+                    S.misc[0] = b0 + q;
+                    S.misc[1] = cnt[q];
+                    reinterpret_cast<long long *>(S.ured)[3] = ec;
+                }
+                ec += cnt[q];
+            }
+            __syncthreads();
+            if (S.misc[0] >= 0 && S.misc[1] <= kCap) {
+                bstar = S.misc[0];
+                before = reinterpret_cast<long long *>(S.ured)[3];
+            }
+            __syncthreads();
+        }
+        if (bstar < 0) {   // no saved counts, or a crossing bin too large to gather
+            const SelectOut so = block_select(S, u, false, 0.0, r, hi, lo, a.status);
+            s_star = so.s;
+            j_star = so.j;
+        }
     }
+    if (tid == 0) S.misc[2] = 0;
+    __syncthreads();
     // word w of the row holds keys 32 w .. 32 w + 31; a batch covers kBatch x 16 words, word
     // j0 / 32 + k * 16 + warp of batch j0 from warp `warp`
     for (int j0 = 0; j0 < a.N; j0 += kBatch * kSelThreads) {
@@ -660,11 +707,46 @@ __global__ void __launch_bounds__(kSelThreads) sel_mask_kernel(SelArgs a)
 #pragma unroll
         for (int k = 0; k < kBatch; ++k) {
             const int j = j0 + k * kSelThreads + tid;
-            const bool sel = kb.v[k] && ((sc[k] > s_star) || (sc[k] == s_star && j <= j_star));
+            bool sel;
+            if (bstar < 0) {
+                sel = kb.v[k] && ((sc[k] > s_star) || (sc[k] == s_star && j <= j_star));
+            } else {
+                const int b = kb.v[k] ? vbin(sc[k], hi, scale) : kBins;
+                sel = b < bstar;
+                if (b == bstar) {
+                    const int slot = atomicAdd(&S.misc[2], 1);
+                    if (slot < kCap) {
+                        S.cs[slot] = sc[k];
+                        S.cj[slot] = j;
+                    }
+                }
+            }
             const unsigned bits = __ballot_sync(0xffffffffu, sel);
             const int w = (j0 + k * kSelThreads) / 32 + warp;
             if (lane == 0 && w < a.nw) row[w] = bits;
         }
+    }
+    if (bstar < 0) return;
+    // rank the keys of b* (logit descending, index ascending) and add the first r - before
+    __threadfence_block();
+    __syncthreads();
+    const int n = min(S.misc[2], kCap);
+    if (n != S.misc[1] && tid == 0) set_status(a.status, SCOPE_DEV_SELECT_TIE);   // counts disagree
+    for (int i = tid; i < n; i += kSelThreads) {
+        const double si = S.cs[i];
+        const int ji = S.cj[i];
+        int rk = 0;
+        for (int k = 0; k < n; ++k) {
+            const double sk = S.cs[k];
+            rk += (sk > si) || (sk == si && S.cj[k] < ji);
+        }
+        S.order[rk] = i;
+    }
+    __syncthreads();
+    const long long need = r - before;
+    for (long long q = tid; q < need && q < n; q += kSelThreads) {
+        const int j = S.cj[S.order[q]];
+        atomicOr(&row[j >> 5], 1u << (j & 31));
     }
 }
 

@@ -14,7 +14,6 @@
 #include "common.cuh"
 
 #include <cmath>
-#include <mutex>
 
 namespace scope {
 
@@ -26,26 +25,16 @@ constexpr size_t kNoAllocStateBytes = (size_t)SCOPE_NOALLOC_MAX_UNITS * 8 * size
 // Every GPU that loads the library holds this array until the process exits.
 static __device__ __align__(256) unsigned char g_select_scratch[kNoAllocStatusBytes + kNoAllocStateBytes];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_setup_mutex;
-void *g_scratch_ptr[kMaxDevices] = {};
-
-// Device address of g_select_scratch on the current device (looked up once per device;
-// host code must not use the symbol itself as a device address).
+// Device address of g_select_scratch on the current device, looked up on every call (host
+// code must not use the symbol itself as a device address).  The lookup allocates nothing
+// and enqueues nothing; not caching it keeps the address right after a device reset, which
+// gives the array a new address in the new context.
 cudaError_t scratch_address(void **out)
 {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    void *p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_select_scratch);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    std::lock_guard<std::mutex> lock(g_setup_mutex);
-    if (!g_scratch_ptr[dev]) {
-        void *p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_select_scratch);
-        if (e != cudaSuccess) return e;
-        g_scratch_ptr[dev] = p;
-    }
-    *out = g_scratch_ptr[dev];
+    *out = p;
     return cudaSuccess;
 }
 

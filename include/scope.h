@@ -20,9 +20,9 @@
  *    channels [0, d_t) / [d_t, d_t+d_h) / [d_t+d_h, d) are the temporal / height /
  *    width subspaces.  Element type of Q, K, V, O is params->dtype.
  *  - The caller owns every buffer, including the workspace `ws` of at least
- *    scope_workspace_bytes(params) bytes (256-byte aligned).  The workspace is
- *    dominated by the attention gather lists, 4 * B*H*Cq*N bytes (3.4 GB for 24 heads
- *    of 118800 tokens and Cq = 300).  The library allocates
+ *    scope_workspace_bytes(params) bytes (256-byte aligned): the clustering scratch,
+ *    the intermediates of scope_forward and the selection masks (318 MiB for 24 heads of
+ *    118800 tokens, Cq = 300, Cm = 333).  The library allocates
  *    no device memory, keeps no state between calls and never synchronises the
  *    stream, except scope_get_device_status.  Calls on one workspace must not overlap.
  *  - `stream` is a cudaStream_t (NULL = legacy default stream).  Work is enqueued;
@@ -53,7 +53,8 @@ typedef enum {
     SCOPE_ERR_UNSUPPORTED = 2,
     SCOPE_ERR_WORKSPACE_TOO_SMALL = 3,
     SCOPE_ERR_CUDA = 4,
-    SCOPE_ERR_DEVICE_CHECK = 5
+    SCOPE_ERR_DEVICE_CHECK = 5,
+    SCOPE_ERR_TIMEOUT = 6
 } scope_status;
 
 typedef enum { SCOPE_F32 = 0, SCOPE_BF16 = 1 } scope_dtype;
@@ -63,6 +64,8 @@ typedef enum { SCOPE_F32 = 0, SCOPE_BF16 = 1 } scope_dtype;
 #define SCOPE_DEV_SELECT_TIE     0x2   /* a selection boundary could not be resolved exactly */
 #define SCOPE_DEV_BAD_ASSIGN     0x4   /* a cluster index >= C or a code >= Cm was supplied (clamped) */
 #define SCOPE_DEV_TIMEOUT        0x8   /* an on-chip pipeline wait gave up (~4 s); outputs invalid */
+#define SCOPE_DEV_BAD_COUNTS     0x10  /* a selection mask row holds fewer keys than its r_c; the
+                                          missing keys were taken as key 0 */
 
 /* k_head handling (scope_params.khead_mode).  ONLINE: Eqs. 9-10, every cluster is
  * topped up to the head's k_head (the method).  OFF: the ablation the review page
@@ -219,8 +222,10 @@ scope_status scope_forward(const scope_params *p, const void *Q, const void *K, 
  * (256 B + 1 MiB, held by every GPU that loads the library until the process exits).
  *  - B*H*Cq must not exceed SCOPE_NOALLOC_MAX_UNITS; larger layers are rejected with
  *    SCOPE_ERR_UNSUPPORTED before anything is enqueued.
- *  - The first call on a device looks up the array's device address on that device
- *    (cudaGetSymbolAddress); make that first call before any stream capture.
+ *  - Every call looks up the array's device address on the current device
+ *    (cudaGetSymbolAddress: no allocation, no stream operation), so the address stays right
+ *    after a device reset; the first call on a device also loads the library's device code
+ *    there, so make that first call before any stream capture.
  *  - Every call shares the array and it keeps the last call's contents; each call clears
  *    the status word it needs.  Calls whose work overlaps on the GPU (other streams, or
  *    other host threads on the same device) race on the array: serialise them.
@@ -358,11 +363,48 @@ scope_status scope_attention_layer(const scope_params *p, const scope_layer_sche
                                    const int32_t *k_init_idx, void *O, void *Qr, void *Kr, void *ws,
                                    size_t ws_bytes, void *stream);
 
+/*
+ * Check of the device-side wait limit (failure detection; the paper has no counterpart).
+ * Every pipeline wait of the tensor-core kernels gives up after a limit, sets
+ * SCOPE_DEV_TIMEOUT in the status word and lets the kernel drain and return, so that a lost
+ * signal ends in an error status instead of a hung GPU.  This entry point makes such a wait
+ * run out on purpose: it launches the bf16 attention kernel with its work-item scheduler
+ * held back (no item is ever published), so the first wait of every warp gives up after
+ * wait_limit_ns, before any copy or tensor-core product is issued.  Afterwards
+ * scope_get_device_status(ws) returns SCOPE_ERR_TIMEOUT with SCOPE_DEV_TIMEOUT set, and the
+ * context stays usable for the next call.
+ *   p              a valid bf16 layer (else SCOPE_ERR_UNSUPPORTED); its tensors are not read
+ *   wait_limit_ns  1 .. 10^10 (else SCOPE_ERR_INVALID_ARGUMENT)
+ *   ws             workspace of at least scope_workspace_bytes(p) bytes (its status word
+ *                  and scheduler counters are written)
+ * Allocates nothing; enqueues one kernel on `stream`.
+ */
+scope_status scope_check_wait_timeout(const scope_params *p, uint64_t wait_limit_ns, void *ws, size_t ws_bytes,
+                                      void *stream);
+
+/*
+ * Accumulation check of the tensor-core products (a diagnostic; the paper has no
+ * counterpart).  The certified k-means assignment bounds the fp32 error of its
+ * tcgen05.mma scores with an allowance per 16-channel step for the sum the tensor core
+ * forms of its exact bf16 products and the accumulator, which NVIDIA does not document.
+ * This runs that instruction form (kind::f16, M = 128, bf16 operands in 128-byte swizzled
+ * K-major shared memory, fp32 accumulator in TMEM) as one chain of K/16 steps:
+ *   D[i][j] = sum_k A[i][k] B[j][k]   (the tensor core's own fp32 result)
+ *   A  [128, K] bf16, B [N, K] bf16, D out [128, N] float (device, 16-byte aligned)
+ *   64 <= K <= 512 with K % 64 == 0; 16 <= N <= 256 with N % 16 == 0; the operands must fit
+ *   in shared memory: (K/64) * (128 + N) * 128 bytes <= 231 KB (else SCOPE_ERR_UNSUPPORTED).
+ * One CTA; allocates nothing; enqueues on `stream`.
+ */
+scope_status scope_tc_accumulation_probe(const void *A, const void *B, int K, int N, float *D, void *stream);
+
 /* Human-readable name of a status code (static storage). */
 const char *scope_status_string(scope_status s);
 
 /* Synchronises `stream` and returns the device status word of the last call that used
- * `ws` in *out (0 = clean; SCOPE_DEV_* bits otherwise). */
+ * `ws` in *out (0 = clean; SCOPE_DEV_* bits otherwise).  Returns SCOPE_OK for a clean word,
+ * SCOPE_ERR_TIMEOUT when SCOPE_DEV_TIMEOUT is set (a pipeline wait gave up; the outputs of
+ * that call are invalid, the context stays usable), SCOPE_ERR_DEVICE_CHECK for any other
+ * bit, SCOPE_ERR_CUDA if the copy or the synchronisation failed. */
 scope_status scope_get_device_status(const void *ws, void *stream, int32_t *out);
 
 #ifdef __cplusplus

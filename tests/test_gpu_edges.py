@@ -271,3 +271,26 @@ def test_full_d_key_clustering_ablation(dtype):
         t = _dev(w, x)
         g, _ = _forward_and_compare(w, x, t, x["q_init"], x["k_init"], key_full=True)
         assert not g["k_codes"][:, :, 1:].any()
+
+
+def test_wait_timeout_is_reported_and_the_context_survives():
+    """Failure detection without a GPU fault: scope_check_wait_timeout holds the attention
+    kernel's scheduler back, so the first wait of every warp runs out after 2 ms, before
+    any copy or tensor-core product is issued.  The kernel returns with SCOPE_DEV_TIMEOUT in
+    the status word (scope_get_device_status: SCOPE_ERR_TIMEOUT), and the next layer on the
+    same workspace runs normally and matches the oracle."""
+    x = synth.layer_inputs(W)
+    t = _dev(W, x)
+    p = capi.Params.from_workload(W)
+    ws = capi.alloc_workspace(p)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    capi.check_wait_timeout(p, 2_000_000, ws=ws)
+    e1.record()
+    code, word = capi.device_status_code(ws)
+    assert code == 6 and word == 0x8, (code, word)          # SCOPE_ERR_TIMEOUT, SCOPE_DEV_TIMEOUT only
+    assert 2.0 <= e0.elapsed_time(e1) < 1000.0               # gave up after the limit, not hung
+    O = capi.forward(p, t["q"], t["k"], t["v"], t["qi"], t["ki"], ws=ws)
+    assert capi.device_status_code(ws) == (0, 0)             # the same workspace, clean again
+    g, O2 = _forward_and_compare(W, x, t, x["q_init"], x["k_init"])
+    np.testing.assert_array_equal(O.float().cpu().numpy().reshape(O2.shape), O2)

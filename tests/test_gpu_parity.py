@@ -12,8 +12,7 @@ import oracle
 from free_sparse_attention_b200 import capi, synth
 from free_sparse_attention_b200.workloads import TINY, COGVIDEOX, Workload
 
-from gpu_common import (compare_attention, device_inputs, mask_bits, oracle_head, to_np,
-                        NEAR_TIE)
+from gpu_common import (check_selection, compare_attention, device_inputs, mask_bits, oracle_head, to_np)
 
 pytestmark = pytest.mark.gpu
 
@@ -81,15 +80,15 @@ def test_selection_matches_oracle_stagewise(w):
     torch.cuda.synchronize()
     assert capi.get_device_status(ws) == 0
     g = {k: to_np(v).reshape((BH,) + tuple(v.shape[2:])) for k, v in out.items()}
+    ties = 0
     for i, sel in enumerate(refs):
-        bad = np.nonzero(g["topp_counts"][i] != sel["p"])[0]
-        assert all(sel["topp_margin"][c] < NEAR_TIE for c in bad), (i, bad)
-        if len(bad):
-            continue   # a logged near tie changed p_c; downstream values legitimately differ
-        np.testing.assert_array_equal(g["base_counts"][i], sel["b"])
-        assert int(g["k_head"][i]) == sel["k_head"]
-        np.testing.assert_array_equal(g["final_counts"][i], sel["r"])
-        np.testing.assert_array_equal(g["sel_mask"][i].view(np.uint32), sel["mask"])
+        gi = {k: g[k][i] for k in g}
+        rerun = lambda i=i: oracle.select(qcs[i], qss[i], kcs[i], kks[i], (w.d_t, w.d_h, w.d_w), w.rho,
+                                          w.alpha, want_scores=True)
+        ties += check_selection(w, gi, sel, qss[i], rerun)
+    # the committed seeds give no near tie; a nonzero count (every value still validated
+    # above) means a change of input or arithmetic reached one
+    assert ties == 0, f"{ties} clusters took the near-tie branch"
 
 
 @pytest.mark.parametrize("w", CONFIGS + [COG2], ids=lambda w: w.name)
@@ -140,13 +139,13 @@ def test_forward_end_to_end(w):
         np.testing.assert_array_equal(g["k_codes"][b, h], ref["k"]["codes"])
         np.testing.assert_array_equal(g["k_centroids"][b, h], ref["k"]["centroids"])
         sel = ref["sel"]
-        bad = np.nonzero(g["topp_counts"][b, h] != sel["p"])[0]
-        assert all(sel["topp_margin"][c] < NEAR_TIE for c in bad)
-        if len(bad) == 0:
-            np.testing.assert_array_equal(g["final_counts"][b, h], sel["r"])
-            assert int(g["k_head"][b, h]) == sel["k_head"]
-            np.testing.assert_array_equal(g["sel_mask"][b, h].view(np.uint32), sel["mask"])
-            compare_attention(w, O[i], ref["O"])
+        gi = {k: g[k][b, h] for k in ("topp_counts", "base_counts", "final_counts", "k_head", "sel_mask")}
+        rerun = lambda ref=ref: oracle.select(ref["q"]["centroids"], ref["q"]["sizes"], ref["k"]["centroids"],
+                                              ref["k"]["codes"], (w.d_t, w.d_h, w.d_w), w.rho, w.alpha,
+                                              want_scores=True)
+        ties = check_selection(w, gi, sel, ref["q"]["sizes"], rerun)
+        assert ties == 0, f"head {i}: {ties} clusters took the near-tie branch"
+        compare_attention(w, O[i], ref["O"])
 
 
 def _oracle_scores(w, x, bh, cache):

@@ -4,7 +4,7 @@ scope_build_lut_and_select_noalloc exists for callers that cannot call cudaMallo
 host application that owns every device allocation, or a loop that must not let
 cudaMalloc / cudaFree synchronise the device): it keeps its scratch in a fixed device
 array of the library.  This file is collected last on purpose, and it must pass both in
-a fresh process (the first call on the device looks up the array's address) and after
+a fresh process (the first call on the device also loads the device code there) and after
 the other tests.  Two calls in a row check that the array's leftover contents from the
 previous call do not leak into the next one.
 """
