@@ -15,95 +15,106 @@ cudaError_t attention_tc_run(const AttnArgs &a, cudaStream_t s);
 
 namespace {
 
-// Exclusive prefix sum of one value per thread over the 1024-thread block; `carry` (shared)
-// holds the running total of earlier calls and is advanced by this block's total.
-__device__ int block_scan_excl(int v, int *wsum, int *carry)
-{
-    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
-    int incl = v;
-    for (int o = 1; o < 32; o <<= 1) {
-        const int n = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += n;
-    }
-    if (lane == 31) wsum[w] = incl;
-    __syncthreads();
-    if (w == 0) {
-        int t = wsum[lane];
-        for (int o = 1; o < 32; o <<= 1) {
-            const int n = __shfl_up_sync(0xffffffffu, t, o);
-            if (lane >= o) t += n;
-        }
-        wsum[lane] = t;
-    }
-    __syncthreads();
-    const int r = *carry + incl - v + (w ? wsum[w - 1] : 0);
-    __syncthreads();
-    if (tid == 0) *carry += wsum[31];
-    __syncthreads();
-    return r;
-}
-
-// Work list of the tensor-core kernel: the queries of every (bh, cluster) that selects keys
-// are cut into chunks of up to kAttnTile in cluster order, and the chunks of each head are
-// paired in order (chunk 2k with chunk 2k+1 of the same head; an odd last chunk is paired
-// with an empty one): pair p is items[2p], items[2p+1], each (bh, c, q0, nq).  Pairs are
-// head-major.  Single block; counter[0] = number of pairs, counter[1] = 0 (scheduler).
+// Work list: one item per kAttnTile queries of one (bh, cluster), head-major.
+// Single block; counter[0] = number of items, counter[1] = 0 (scheduler).
 __global__ void __launch_bounds__(1024) attn_items_kernel(AttnArgs a)
 {
     __shared__ int wsum[32];
     __shared__ int carry;
-    const int tid = threadIdx.x;
-    const int units = a.BH * a.Cq;
-    auto chunks_of = [&](int u, int &q0, int &nq) {
-        const int bh = u / a.Cq, c = u - bh * a.Cq;
-        const int32_t *off = a.off + (size_t)bh * a.off_bh;
-        q0 = off[c];
-        nq = off[c + 1] - q0;
-        if (a.final_cnt[u] <= 0) nq = 0;   // nothing selected: output written as zeros
-        return (nq + kAttnTile - 1) / kAttnTile;
-    };
-    // chunk position of every unit's first chunk (unit order = head-major)
+    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+    const int total = a.BH * a.Cq;
     if (tid == 0) carry = 0;
     __syncthreads();
-    for (int base = 0; base < units; base += 1024) {
+    for (int base = 0; base < total; base += 1024) {
         const int u = base + tid;
-        int q0 = 0, nq = 0;
-        const int n = u < units ? chunks_of(u, q0, nq) : 0;
-        const int pos = block_scan_excl(n, wsum, &carry);
-        if (u < units) a.unit_pos[u] = pos;
-    }
-    if (tid == 0) a.unit_pos[units] = carry;
-    __syncthreads();
-    // first pair of every head
-    if (tid == 0) carry = 0;
-    __syncthreads();
-    for (int base = 0; base < a.BH; base += 1024) {
-        const int h = base + tid;
-        const int np = h < a.BH ? (a.unit_pos[(h + 1) * a.Cq] - a.unit_pos[h * a.Cq] + 1) / 2 : 0;
-        const int ps = block_scan_excl(np, wsum, &carry);
-        if (h < a.BH) a.head_pair[h] = ps;
-    }
-    __syncthreads();
-    // chunk k of head h goes to items[2 * head_pair[h] + k]
-    for (int u = tid; u < units; u += 1024) {
-        int q0 = 0, nq = 0;
-        const int n = chunks_of(u, q0, nq);
-        if (!n) continue;
-        const int bh = u / a.Cq, c = u - bh * a.Cq;
-        const int k0 = a.unit_pos[u] - a.unit_pos[bh * a.Cq];
-        int4 *dst = a.items + 2 * (size_t)a.head_pair[bh] + k0;
-        for (int t = 0; t < n; ++t) {
-            const int qs = q0 + t * kAttnTile;
-            dst[t] = make_int4(bh, c, qs, min(kAttnTile, q0 + nq - qs));
+        int nq = 0, q0 = 0, bh = 0, c = 0;
+        if (u < total) {
+            bh = u / a.Cq;
+            c = u - bh * a.Cq;
+            const int32_t *off = a.off + (size_t)bh * a.off_bh;
+            q0 = off[c];
+            nq = off[c + 1] - q0;
+            if (a.final_cnt[u] <= 0) nq = 0;   // nothing selected: output written as zeros below
         }
-    }
-    for (int h = tid; h < a.BH; h += 1024) {
-        const int nch = a.unit_pos[(h + 1) * a.Cq] - a.unit_pos[h * a.Cq];
-        if (nch & 1) a.items[2 * (size_t)a.head_pair[h] + nch] = make_int4(h, 0, 0, 0);
+        const int tiles = (nq + kAttnTile - 1) / kAttnTile;
+        int v = tiles;
+        for (int o = 1; o < 32; o <<= 1) {
+            int n = __shfl_up_sync(0xffffffffu, v, o);
+            if (lane >= o) v += n;
+        }
+        if (lane == 31) wsum[w] = v;
+        __syncthreads();
+        if (w == 0) {
+            int s = wsum[lane];
+            for (int o = 1; o < 32; o <<= 1) {
+                int n = __shfl_up_sync(0xffffffffu, s, o);
+                if (lane >= o) s += n;
+            }
+            wsum[lane] = s;
+        }
+        __syncthreads();
+        int pos = carry + v - tiles + (w ? wsum[w - 1] : 0);
+        for (int t = 0; t < tiles; ++t) {
+            const int qs = q0 + t * kAttnTile;
+            a.items[pos + t] = make_int4(bh, c, qs, min(kAttnTile, q0 + nq - qs));
+        }
+        __syncthreads();
+        if (tid == 0) carry += wsum[31];
+        __syncthreads();
     }
     if (tid == 0) {
         a.counter[0] = carry;
         a.counter[1] = 0;
+    }
+}
+
+// Expands the selection bitmask of every (bh, cluster) that has queries into its
+// ascending list of selected key indices (the gather order of the attention kernel).
+// grid = BH*Cq units, 256 threads.  Per chunk of 256 mask words: one word per thread,
+// a block prefix sum of the popcounts, then each warp writes its 32 words one word at
+// a time with lane l handling bit l, so consecutive selected keys go to consecutive
+// addresses (coalesced stores).
+__global__ void __launch_bounds__(256) attn_lists_kernel(AttnArgs a)
+{
+    __shared__ int wsum[8];
+    const int u = blockIdx.x, tid = threadIdx.x, lane = tid & 31, w8 = tid >> 5;
+    const int bh = u / a.Cq, c = u - bh * a.Cq;
+    const int32_t *off = a.off + (size_t)bh * a.off_bh;
+    if (off[c + 1] == off[c] || a.final_cnt[u] <= 0) return;
+    const uint32_t *row = a.mask + (size_t)u * a.nw;
+    int32_t *out = a.lists + (size_t)u * a.list_stride;
+    const uint32_t below = (1u << lane) - 1u;
+    int base = 0;
+    for (int w0 = 0; w0 < a.nw; w0 += 256) {
+        const int w = w0 + tid;
+        uint32_t bits = 0;
+        if (w < a.nw) {
+            bits = row[w];
+            if (w == a.nw - 1 && (a.N & 31)) bits &= (1u << (a.N & 31)) - 1u;
+        }
+        const int pc = __popc(bits);
+        int incl = pc;
+        for (int o = 1; o < 32; o <<= 1) {
+            const int t = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += t;
+        }
+        if (lane == 31) wsum[w8] = incl;
+        __syncthreads();
+        int before = 0, total = 0;
+        for (int k = 0; k < 8; ++k) {
+            before += k < w8 ? wsum[k] : 0;
+            total += wsum[k];
+        }
+        const int excl = base + before + incl - pc;   // list position of this word's first key
+        const int wbase = (w0 + w8 * 32) * 32;        // key index of bit 0 of the warp's word 0
+#pragma unroll 4
+        for (int k = 0; k < 32; ++k) {
+            const uint32_t bk = __shfl_sync(0xffffffffu, bits, k);
+            const int pk = __shfl_sync(0xffffffffu, excl, k);
+            if ((bk >> lane) & 1u) out[pk + __popc(bk & below)] = wbase + k * 32 + lane;
+        }
+        base += total;
+        __syncthreads();
     }
 }
 
@@ -195,6 +206,7 @@ cudaError_t attention_items(const AttnArgs &a, cudaStream_t s)
 {
     attn_items_kernel<<<1, 1024, 0, s>>>(a);
     attn_zero_empty_kernel<<<a.BH * a.Cq, 128, 0, s>>>(a);
+    if (a.is_bf16 && a.use_tc) attn_lists_kernel<<<a.BH * a.Cq, 256, 0, s>>>(a);
     return cudaGetLastError();
 }
 
@@ -209,7 +221,7 @@ __global__ void dense_counts_kernel(int32_t *final_counts, long long BH, int N)
 }  // namespace
 
 // Dense attention as one query cluster selecting every key: q_assign = 0, every mask bit
-// set (bits past N are ignored by the attention kernels), r_0 = N.
+// set (bits past N are ignored by the list kernel), r_0 = N.
 cudaError_t attention_dense_setup(uint16_t *q_assign, uint32_t *mask, int32_t *final_counts, long long BH,
                                   long long N, long long nw, cudaStream_t s)
 {

@@ -1,92 +1,78 @@
-// Sparse attention on the Blackwell tensor cores (tcgen05, sm_100a), bf16.
+// Gathered sparse attention on the Blackwell tensor cores (tcgen05, sm_100a), bf16.
 //
 // SCOPE computes exact softmax attention of every query over the ORIGINAL keys and
-// values its query cluster selected (arXiv 2608.12780, abstract; review page,
-// forward_implications[1]):  O_i = sum_{j in S_c} softmax_j(q_i . k_j / sqrt d) v_j.
+// values its query cluster selected (arXiv 2608.12780, abstract;
+// review page, forward_implications[1]).  Queries are grouped by cluster, so one work
+// item = up to 256 queries of one (b, h, c) against the r_c keys of S_c.
 //
-// Every cluster of a head draws its keys from the same N rows of K and V, so this kernel
-// streams the head's keys in their own order, in blocks of 128 consecutive rows, and
-// applies each cluster's selection as a mask inside the softmax (an unselected logit is
-// -inf, its P exactly 0): the keys travel as plain 2-D TMA tiles, and a block that no
-// query tile of the CTA selects is skipped without being loaded.  A work unit is a PAIR of
-// 128-query chunks of the same head (two query tiles, possibly of two clusters), so every
-// K/V block serves 256 queries.
-//
-// Per CTA (persistent, one per SM; pairs handed out in order by a global counter and a
-// small shared-memory ring):
-//   warps 0-3 / 4-7  softmax of query tile 0 / 1: thread r owns row r (TMEM lane r), masks
-//                    and exponentiates its 128 logits, writes bf16 P over its S buffer,
-//                    keeps the running maximum and row sum, and writes the output rows
-//   warp 8           loads: the pair's Q rows (tile::gather4, in cluster order) and, per
-//                    selected block, the K and V tiles (128 rows x 64 columns per box);
-//                    it walks both clusters' masks and publishes each step's block index
-//                    and mask words in a shared-memory ring; it also runs the scheduler
-//   warp 9           issues the MMAs (one thread) and owns the TMEM allocation
-// TMEM (512 columns): S_0, S_1 (128 fp32 columns each; P_q as bf16 pairs over the first
-// 64 columns of S_q), O_0, O_1 (D columns each).  Per step (block s) the issuing thread
-// runs, in one in-order stream,  P_0(s) V(s), S_0(s+1), P_1(s) V(s), S_1(s+1):  S_q(s+1)
-// overwrites P_q(s) only after the tensor core has read it, and the softmax of one tile
-// overlaps the other tile's products.
-//   S_q = Q_q K^T     tcgen05.mma kind::f16, M=128, N=128 keys, K=d, fp32 in TMEM
-//   O_q += P_q V      M=128, N=d, K=128 keys, P_q bf16 from TMEM (TS form), V from smem
-// The softmax rescales O_q (TMEM load/store) only when its running maximum grows by more
-// than 2^8, so P <= 256 and the final O / l is exact softmax arithmetic.  Every mbarrier
-// wait gives up after a limit (4 s by default), sets a status bit and lets the CTA drain:
-// the loader waits for its own copies, the issuing thread for its own products, and only
-// then is TMEM freed.
+// Per CTA (persistent, one per SM; items of the head-major work list are handed out
+// dynamically, in order, through a global counter and a small shared-memory ring):
+//   warps 0-3 / 4-7  softmax + epilogue of Q tile 0 / 1 (thread r owns row r = TMEM lane r)
+//   warps 8-11       gather both Q tiles once per item and the selected K rows per key tile
+//   warps 12-13      gather the selected V rows per key tile
+//   warps 14 / 15    issue the MMAs of Q tile 0 / 1 (lane 0 alone, with single-thread
+//                    mbarrier waits: warp-wide waits and broadcasts on this critical path
+//                    cost ~11 % of the kernel's time; warp 14 also allocates TMEM)
+// A TMA gather4 stream sustains ~15 GB/s per issuing warp, so each tile is split over
+// four (K) or two (V) warps; every warp signals its own share with arrive.expect_tx.
+// Registers are rebalanced per warpgroup with setmaxnreg: the softmax warpgroups hold a
+// row of logits (192 registers), the gather / MMA warpgroups need 64.
+// Each cluster's selected key indices are expanded once from the bitmask into an
+// ascending list (attn_lists_kernel).  Rows are gathered with TMA tile::gather4 (four
+// arbitrary rows of one 64-column, 128-byte box per instruction, each lane issuing its
+// own four rows) straight into the 128B-swizzled K-major layout the tensor core reads.
+//   S_q  = Q_q K^T     tcgen05.mma kind::f16, M=128, N=64 keys, K=d, fp32 in TMEM
+//   O_q += P_q V       M=128, N=d, K=64, P_q bf16 written by the softmax over the first
+//                      columns of its own S buffer (A operand from TMEM), V from smem
+// Both Q tiles reuse every gathered K/V tile.  S is double-buffered per Q tile (two
+// 64-column buffers; 2 x (2 x 64 + 128) = 512 TMEM columns at d = 128): the MMA thread
+// of tile q issues S(0), S(1), then P(t) V(t) followed by S(t+2) into the buffer P(t)
+// occupied, so the softmax of step t+1 runs while the tensor core works on step t.  A
+// thread's tcgen05.commit costs it roughly one pipe latency before its next MMA starts,
+// which is why each Q tile has its own issuing thread.  The softmax keeps a running row
+// maximum and rescales O (TMEM load/store) only when the maximum grows by more than
+// 2^8, so P stays <= 256 and the final O / l is exact softmax arithmetic.  Every
+// mbarrier wait gives up after ~4 s, sets a status bit and lets the CTA drain and free
+// its TMEM; on that path every warp first waits (bounded) for the copies and products it
+// issued.
 #include "tc_common.cuh"
 
 namespace scope {
 
 namespace {
 
-constexpr int kBM = 128;           // queries per tile (TMEM lanes)
-constexpr int kBK = 128;           // keys per block (one S buffer)
-constexpr int kWords = kBK / 32;   // selection-mask words per block
-constexpr int kRing = 4;           // work pairs fetched ahead by the scheduler thread
-constexpr int kSteps = 8;          // step ring (block index and mask words)
+constexpr int kBM = 128;           // queries per Q tile (TMEM lanes)
+constexpr int kQT = 2;             // Q tiles per CTA, both against every gathered K/V tile
+constexpr int kBN = 64;            // keys per K/V tile (one S buffer)
 constexpr int kThreads = 512;      // 16 warps = 4 warpgroups
+constexpr int kKWarps = 4;         // K (and Q) gather warps
+constexpr int kVWarps = 2;         // V gather warps
+constexpr int kMmaWarps = 2;       // one MMA-issuing warp per Q tile
 constexpr int kLaunchRegs = 128;   // 65536 / 512; the setmaxnreg split below sums to it
 constexpr int kSoftmaxRegs = 192;  // 2 warpgroups x 128 threads x 192
 constexpr int kOtherRegs = 64;     //  + 2 warpgroups x 128 threads x 64 = 65536
-constexpr int kWLoad = 8, kWIssue = 9;
-constexpr int kItemWarps = 10;     // warps 0-9 read every work pair
+constexpr int kMaxStages = 8;
 constexpr uint32_t kTmemCols = 512;
-constexpr int kSmemLimit = 232448;
-constexpr int kEnd = -1;           // step-ring block index that ends a pair
+constexpr int kRing = 4;           // work items fetched ahead by the scheduler thread
+constexpr int kWarps = kThreads / 32;
+
+// max(a, b, c) in one instruction (the three-input form of max.f32 on sm_100)
+__device__ __forceinline__ float fmax3(float a, float b, float c)
+{
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
 
 struct __align__(8) Bars {
     uint64_t q_full, q_empty;
-    uint64_t k_full[4], v_full[4], kv_empty[4];   // per K/V stage
-    uint64_t s_full[2], p_full[2];                // per query tile
-    uint64_t o_free;                              // the epilogue has read O_0 and O_1
-    uint64_t item_full[kRing], item_empty[kRing];
-    uint64_t drain;
-};
-
-struct Step {
-    int block;                   // key block index, or kEnd
-    uint32_t w[2][kWords];       // the two tiles' mask words for the block
-};
-
-// Shared memory: Q_0, Q_1, the K and V stages (bf16, 128-byte swizzled, K-major, 64-column
-// boxes of 128 rows), the step ring and the barriers.
-template <int D>
-struct Lay {
-    static constexpr int kTile = 128 * D * 2;                // one Q tile or one K/V block
-    static constexpr int kStages = D == 128 ? 2 : 3;
-    static constexpr int kQ = 0;
-    static constexpr int kK = kQ + 2 * kTile;
-    static constexpr int kV = kK + kStages * kTile;
-    static constexpr int kRingOff = kV + kStages * kTile;
-    static constexpr int kBars = kRingOff + kSteps * (int)sizeof(Step);
-    static constexpr int kMisc = kBars + (int)sizeof(Bars);
-    static constexpr int kBytes = kMisc + 64;
-    // more than half of the SM's shared memory, so one CTA (and one 512-column TMEM
-    // allocation) per SM; 1 KB of room to align the base
-    static constexpr int kAlloc = kBytes + 1024 > kSmemLimit / 2 + 1024 ? kBytes + 1024 : kSmemLimit / 2 + 1024;
-    static_assert(kAlloc <= kSmemLimit, "shared memory budget");
-    static_assert(kStages <= 4, "stage barriers");
+    uint64_t k_full[kMaxStages], k_empty[kMaxStages];
+    uint64_t v_full[kMaxStages], v_empty[kMaxStages];
+    // per Q tile and S buffer: S ready (MMA commit), P written (softmax), P V done (commit)
+    uint64_t s_full[kQT][2], p_full[kQT][2], o_done[kQT][2];
+    uint64_t o_free[kQT];  // epilogue has read O_q
+    uint64_t item_full[kRing], item_empty[kRing];   // work-item ring (dynamic scheduler)
+    uint64_t drain[kQT];                            // the issuing threads' last products
 };
 
 struct Waiter {
@@ -95,8 +81,7 @@ struct Waiter {
     unsigned long long limit_ns;
 };
 
-// Bounded wait by one thread: test, then poll with a short sleep; on the kernel's limit it
-// sets the CTA abort flag and the device status.
+// Bounded wait by one thread (as bar_wait in tc_common.cuh, with the launch's limit).
 __device__ __forceinline__ bool wait1(uint64_t *b, uint32_t parity, const Waiter &w)
 {
     if (bar_test(b, parity)) return true;
@@ -132,61 +117,71 @@ __device__ __forceinline__ void drain_wait(uint64_t *b, uint32_t parity, unsigne
     while (!bar_test(b, parity) && global_ns() - t0 < limit_ns) __nanosleep(64);
 }
 
-// max(a, b, c) in one instruction (the three-input form of max.f32 on sm_100)
-__device__ __forceinline__ float fmax3(float a, float b, float c)
-{
-    float d;
-    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
-    return d;
-}
-
-// Tensor maps of one launch: row gathers of Q (64 x 1 boxes, tile::gather4) and 64 x 128
-// tiles of K and V.
-struct Maps {
-    CUtensorMap qg, kt, vt;
+// Shared memory: two Q tiles, a K ring and a V ring (bf16, 128-byte swizzled, K-major).
+// TMEM: two S buffers per Q tile (fp32, 64 columns each; P bf16 pairs over the first 32
+// columns of its own buffer) at q*128 + b*64, O_q (fp32, D columns) at 256 + q*D.
+template <int D>
+struct Smem {
+    static constexpr int kKS = D == 128 ? 5 : 8;       // K ring depth
+    static constexpr int kVS = D == 128 ? 5 : 8;       // V ring depth
+    static constexpr int kQTile = kBM * D * 2;
+    static constexpr int kKVTile = kBN * D * 2;
+    static constexpr int kQ = 0;
+    static constexpr int kK = kQ + kQT * kQTile;
+    static constexpr int kV = kK + kKS * kKVTile;
+    static constexpr int kBars = kV + kVS * kKVTile;
+    static constexpr int kMisc = kBars + (int)sizeof(Bars);
+    static constexpr int kBytes = kMisc + 64;
+    static constexpr int kAlloc = kBytes + 1024;       // room to align the base to 1 KB
+    static_assert(kAlloc <= 232448, "shared memory budget");
+    static_assert(kKS <= kMaxStages && kVS <= kMaxStages, "ring depth");
+    static_assert(kAlloc > 232448 / 2, "one CTA (and its 512 TMEM columns) per SM");
 };
 
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_constant__ Maps maps, AttnArgs a)
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, AttnArgs a)
 {
-    using L = Lay<D>;
-    constexpr int NB = D / 64;        // 64-column boxes per row
-    constexpr int KS = L::kStages;
+    using L = Smem<D>;
+    constexpr int NB = D / 64;     // 64-column boxes per row
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char *sm = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     Bars *bars = reinterpret_cast<Bars *>(sm + L::kBars);
-    Step *steps = reinterpret_cast<Step *>(sm + L::kRingOff);
     int *misc = reinterpret_cast<int *>(sm + L::kMisc);
     volatile int *abort_flag = misc;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(misc + 1);
-    volatile int *ring = misc + 4;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t sbase = smem_u32(sm);
     const Waiter W{abort_flag, a.status, a.wait_ns};
 
     if (threadIdx.x == 0) {
         misc[0] = 0;
-        bar_init(&bars->q_full, 1);
-        bar_init(&bars->q_empty, 1);
-        for (int s = 0; s < 4; ++s) {
-            bar_init(&bars->k_full[s], 1);
-            bar_init(&bars->v_full[s], 1);
-            bar_init(&bars->kv_empty[s], 1);
+        bar_init(&bars->q_full, kKWarps);
+        bar_init(&bars->q_empty, kMmaWarps);
+        for (int s = 0; s < kMaxStages; ++s) {
+            bar_init(&bars->k_full[s], kKWarps);
+            bar_init(&bars->v_full[s], kVWarps);
+            bar_init(&bars->k_empty[s], kMmaWarps);
+            bar_init(&bars->v_empty[s], kMmaWarps);
         }
-        for (int q = 0; q < 2; ++q) {
-            bar_init(&bars->s_full[q], 1);
-            bar_init(&bars->p_full[q], 4);
+        for (int q = 0; q < kQT; ++q) {
+            for (int b = 0; b < 2; ++b) {
+                bar_init(&bars->s_full[q][b], 1);
+                bar_init(&bars->p_full[q][b], 4);
+                bar_init(&bars->o_done[q][b], 1);
+            }
+            bar_init(&bars->o_free[q], 4);
         }
-        bar_init(&bars->o_free, 8);
         for (int k = 0; k < kRing; ++k) {
             bar_init(&bars->item_full[k], 1);
-            bar_init(&bars->item_empty[k], kItemWarps);
+            bar_init(&bars->item_empty[k], kWarps);
         }
-        bar_init(&bars->drain, 1);
+        for (int q = 0; q < kQT; ++q) bar_init(&bars->drain[q], 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    if (warp == kWIssue) {
+    if (warp == 14) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                          smem_u32(tmem_slot)),
                      "r"(kTmemCols)
@@ -197,25 +192,27 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const int n_pairs = a.counter[0];
-    // Dynamic scheduler: one thread (lane 0 of the load warp) takes pair indices from the
-    // global counter a.counter[1] in order and publishes them in a ring of kRing slots;
-    // warps 0-9 read every slot (pair k in slot k % kRing) and release it.  -1 ends the work.
-    auto fetch = [&](uint32_t k) -> bool {
+    const int n_items = a.counter[0];
+    // Dynamic scheduler: one thread (lane 0 of warp 8) takes item indices from the global
+    // counter a.counter[1] in order and publishes them in a ring of kRing slots; every warp
+    // reads every slot (item k in slot k % kRing) and releases it.  -1 ends the work.
+    volatile int *ring = misc + 4;
+    auto fetch = [&](uint32_t k) -> bool {   // lane 0 of warp 8 only
         const int slot = k % kRing;
         if (!wait1(&bars->item_empty[slot], ((k / kRing) & 1) ^ 1, W)) return false;
         const int it = atomicAdd(&a.counter[1], 1);
-        ring[slot] = it < n_pairs ? it : -1;
+        ring[slot] = it < n_items ? it : -1;
         bar_arrive(&bars->item_full[slot]);
         return true;
     };
-    auto next_pair = [&](uint32_t k) -> int {   // a whole warp
+    // item index k of this CTA for the calling warp; -1 = no more work or a failed wait
+    auto next_item = [&](uint32_t k) -> int {
         const int slot = k % kRing;
         if (!waitw(&bars->item_full[slot], (k / kRing) & 1, W)) return -1;
         const int it = ring[slot];
         __syncwarp();
         if (lane == 0) bar_arrive(&bars->item_empty[slot]);
-        if (warp == kWLoad && it >= 0) {   // the scheduler thread fetches one pair ahead
+        if (warp == 8 && it >= 0) {   // the scheduler thread fetches one item ahead
             int ok = 1;
             if (lane == 0) ok = fetch(k + 1) ? 1 : 0;
             ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -223,387 +220,350 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         }
         return it;
     };
-    auto next_pair1 = [&](uint32_t k) -> int {   // one thread
-        const int slot = k % kRing;
-        if (!wait1(&bars->item_full[slot], (k / kRing) & 1, W)) return -1;
-        const int it = ring[slot];
-        bar_arrive(&bars->item_empty[slot]);
-        return it;
-    };
     // a.hold_items: the scheduler publishes nothing, so every first wait runs out (the
     // check of the timeout path: no copy or product is ever issued)
-    if (warp == kWLoad && lane == 0 && !a.hold_items) fetch(0);
-    const int NBK = (a.N + kBK - 1) / kBK;   // key blocks per head
+    if (warp == 8 && lane == 0 && !a.hold_items) fetch(0);
 
     if (warp >= 8) {
     // warpgroups 2 and 3 give registers back (one setmaxnreg site for all their warps)
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kOtherRegs));
-    if (warp == kWLoad) {
-        // ------------------------------------------------------------ loads + mask walk
-        uint32_t step = 0, q_it = 0;
-        bool ok = true;
-        for (uint32_t pk = 0; ok && !warp_aborted(abort_flag); ++pk) {
-            const int pr = next_pair(pk);
-            if (pr < 0) break;
-            const int4 A = a.items[2 * pr], B = a.items[2 * pr + 1];
-            const int bh = A.x, rowbase = bh * a.N;
-            const bool hasB = B.w > 0;
-            const uint32_t *mA = a.mask + ((size_t)bh * a.Cq + A.y) * a.nw;
-            const uint32_t *mB = a.mask + ((size_t)bh * a.Cq + B.y) * a.nw;
-            // the Q rows of both tiles, perm[q0 ..] in cluster order (rows beyond a chunk's
-            // nq repeat its last query): 32 gather4 of 4 rows per box and tile
-            if (!(ok = waitw(&bars->q_empty, (q_it & 1) ^ 1, W))) break;
-            if (lane == 0) bar_expect_tx(&bars->q_full, (uint32_t)(hasB ? 2 : 1) * L::kTile);
-            __syncwarp();
-            for (int q = 0; q < (hasB ? 2 : 1); ++q) {
-                const int4 I = q ? B : A;
-                const int32_t *perm = a.perm + (size_t)bh * a.perm_bh + I.z;
-                for (int g = lane; g < 32 * NB; g += 32) {
-                    const int r0 = 4 * (g & 31), box = g >> 5;
+    if (warp < 14) {
+        // ------------------------------------------------------------ gather warps
+        const bool is_k = warp < 12;
+        const int gw = is_k ? warp - 8 : warp - 12;   // this warp's share of each tile
+        const CUtensorMap *tm = is_k ? &tmK : &tmV;
+        const int NS = is_k ? L::kKS : L::kVS;
+        // K/V tile: kBN/4 groups of 4 rows x NB boxes, split evenly over the K (or V) warps
+        constexpr int kGroups = kBN / 4;
+        const int per = is_k ? kGroups / kKWarps : kGroups / kVWarps, g_lo = gw * per,
+                  cnt = min(per, kGroups - g_lo);
+        const int grp = g_lo + lane / NB, blk = lane % NB;
+        const bool active = lane < cnt * NB;
+        const uint32_t kShareBytes = (uint32_t)cnt * 4 * D * 2;
+        uint32_t stage_it = 0, q_it = 0;
+        for (uint32_t item_k = 0; !warp_aborted(abort_flag); ++item_k) {
+            const int it = next_item(item_k);
+            if (it < 0) break;
+            const int4 item = a.items[it];
+            const int bh = item.x, c = item.y, q0 = item.z, nq = item.w;
+            const long long r = a.final_cnt[(size_t)bh * a.Cq + c];
+            const int T = (int)((r + kBN - 1) / kBN);
+            const int rowbase = bh * a.N;
+            if (is_k) {
+                // both Q tiles: rows perm[q0 .. q0+nq); rows beyond nq repeat the last query.
+                // 64 groups of 4 rows over the two tiles; warp gw takes groups 16*gw .. +15.
+                if (!waitw(&bars->q_empty, (q_it & 1) ^ 1, W)) break;
+                if (lane == 0) bar_expect_tx(&bars->q_full, 16 * 4 * D * 2);
+                __syncwarp();
+                if (lane < 16) {
+                    const int32_t *perm = a.perm + (size_t)bh * a.perm_bh + q0;
+                    const int g = gw * 16 + lane, q = g >> 5, r0 = (g & 31) * 4;
                     int rr[4];
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) rr[k] = rowbase + perm[min(r0 + k, I.w - 1)];
-                    tma_gather4(sbase + L::kQ + q * L::kTile + box * (kBM * 128) + r0 * 128, &maps.qg, box * 64,
-                                rr[0], rr[1], rr[2], rr[3], &bars->q_full);
-                }
-            }
-            ++q_it;
-            // the selected blocks in order, 32 at a time: lane l reads the words of block b0 + l
-            for (int b0 = 0; b0 < NBK && ok; b0 += 32) {
-                const int b = b0 + lane;
-                uint32_t wa[kWords], wb[kWords];
-                bool any = false;
+                    for (int k = 0; k < 4; ++k) rr[k] = rowbase + perm[min(q * kBM + r0 + k, nq - 1)];
 #pragma unroll
-                for (int k = 0; k < kWords; ++k) {
-                    const int wi = b * kWords + k;
-                    wa[k] = (b < NBK && wi < a.nw) ? mA[wi] : 0u;
-                    wb[k] = (b < NBK && wi < a.nw && hasB) ? mB[wi] : 0u;
-                    any |= (wa[k] | wb[k]) != 0u;
+                    for (int b = 0; b < NB; ++b)
+                        tma_gather4(sbase + L::kQ + q * L::kQTile + b * (kBM * 128) + r0 * 128, &tmQ, b * 64,
+                                    rr[0], rr[1], rr[2], rr[3], &bars->q_full);
                 }
-                unsigned bal = __ballot_sync(0xffffffffu, any);
-                while (bal) {
-                    const int l = __ffs(bal) - 1;
-                    bal &= bal - 1;
-                    const int st = step % KS;
-                    if (!(ok = waitw(&bars->kv_empty[st], ((step / KS) & 1) ^ 1, W))) break;
-                    Step *e = steps + step % kSteps;
-#pragma unroll
-                    for (int k = 0; k < kWords; ++k) {
-                        const uint32_t x = __shfl_sync(0xffffffffu, wa[k], l), y = __shfl_sync(0xffffffffu, wb[k], l);
-                        if (lane == 0) {
-                            e->w[0][k] = x;
-                            e->w[1][k] = y;
-                        }
-                    }
-                    if (lane == 0) {
-                        e->block = b0 + l;
-                        const int y = rowbase + (b0 + l) * kBK;
-                        bar_expect_tx(&bars->k_full[st], L::kTile);
-                        for (int x = 0; x < NB; ++x)
-                            tma_tile2d(sbase + L::kK + st * L::kTile + x * (kBK * 128), &maps.kt, 64 * x, y,
-                                       &bars->k_full[st]);
-                        bar_expect_tx(&bars->v_full[st], L::kTile);
-                        for (int x = 0; x < NB; ++x)
-                            tma_tile2d(sbase + L::kV + st * L::kTile + x * (kBK * 128), &maps.vt, 64 * x, y,
-                                       &bars->v_full[st]);
-                    }
-                    __syncwarp();
-                    ++step;
+                ++q_it;
+            }
+            const int32_t *list = a.lists + ((size_t)bh * a.Cq + c) * a.list_stride;
+            // this lane's four keys of tile t; keys past r_c (last tile) load key 0 and are
+            // masked by the softmax.  Indices are loaded two tiles ahead of their gathers.
+            auto keys_of = [&](int t) {
+                const long long j0 = (long long)t * kBN + 4 * grp;
+                int4 v;
+                if (j0 + 3 < r) {
+                    v = *reinterpret_cast<const int4 *>(list + j0);
+                } else {
+                    v.x = j0 < r ? list[j0] : 0;
+                    v.y = j0 + 1 < r ? list[j0 + 1] : 0;
+                    v.z = j0 + 2 < r ? list[j0 + 2] : 0;
+                    v.w = 0;
                 }
+                return v;
+            };
+            int4 g0 = keys_of(0), g1 = T > 1 ? keys_of(1) : make_int4(0, 0, 0, 0);
+            for (int t = 0; t < T; ++t) {
+                const int s = stage_it % NS;
+                if (!waitw(is_k ? &bars->k_empty[s] : &bars->v_empty[s], ((stage_it / NS) & 1) ^ 1, W))
+                    break;
+                uint64_t *full = is_k ? &bars->k_full[s] : &bars->v_full[s];
+                if (lane == 0) bar_expect_tx(full, kShareBytes);
+                __syncwarp();
+                if (active)
+                    tma_gather4(sbase + (is_k ? L::kK : L::kV) + s * L::kKVTile + blk * (kBN * 128) + grp * 512,
+                                tm, blk * 64, rowbase + g0.x, rowbase + g0.y, rowbase + g0.z,
+                                rowbase + g0.w, full);
+                g0 = g1;
+                if (t + 2 < T) g1 = keys_of(t + 2);
+                ++stage_it;
             }
-            if (!ok) break;
-            // the pair's end: a step with no block (no copy; both barriers arrive plainly)
-            const int st = step % KS;
-            if (!(ok = waitw(&bars->kv_empty[st], ((step / KS) & 1) ^ 1, W))) break;
-            if (lane == 0) {
-                steps[step % kSteps].block = kEnd;
-                bar_arrive(&bars->k_full[st]);
-                bar_arrive(&bars->v_full[st]);
-            }
-            __syncwarp();
-            ++step;
         }
-        // copies already issued land before the CTA exits
+        // loads already issued land before the CTA exits (bounded: on an abort another
+        // warp's share of a stage may never come, but this warp's own copies have landed)
         if (lane == 0) {
-            for (uint32_t v = step > (uint32_t)KS ? step - KS : 0; v < step; ++v) {
-                drain_wait(&bars->k_full[v % KS], (v / KS) & 1, W.limit_ns);
-                drain_wait(&bars->v_full[v % KS], (v / KS) & 1, W.limit_ns);
-            }
-            if (q_it > 0) drain_wait(&bars->q_full, (q_it - 1) & 1, W.limit_ns);
+            uint64_t *fb = is_k ? bars->k_full : bars->v_full;
+            for (uint32_t v = stage_it > (uint32_t)NS ? stage_it - NS : 0; v < stage_it; ++v)
+                drain_wait(&fb[v % NS], (v / NS) & 1, W.limit_ns);
+            if (is_k && q_it > 0) drain_wait(&bars->q_full, (q_it - 1) & 1, W.limit_ns);
         }
         __syncwarp();
-    } else if (warp == kWIssue) {
-        // ------------------------------------------------------------ MMA issue (one thread)
-        // Per pair: S_q(e0) for the first step, then per block step e:
-        //   P_0(e) V(e), S_0(e+1), commit s_full[0];  P_1(e) V(e), S_1(e+1), commit s_full[1];
-        //   commit kv_empty[e]
-        // (S_q(e+1) only when step e+1 is a block).  s_full[q] completes once per step of
-        // the pair, the end step included (then it means "O_q final").
+    } else {
+        // ------------------------------------------------------------ MMA issuers (warps 14, 15)
+        // Lane 0 of warp 14 + q issues Q tile q's products alone (lanes 1-31 wait at the end):
+        // S(0), S(1), then for every t: O += P(t) V(t), S(t+2).  S(t+2) reuses the buffer
+        // whose first columns hold P(t); issuing it after P(t) V(t) from the same thread keeps
+        // the in-order tensor pipe from overwriting P(t) early.  Both issuers consume every K
+        // and V stage in the same order (an idle Q tile only waits for the data and releases
+        // the stage), so the ring phases advance in step.
         if (lane == 0) {
-            constexpr uint32_t idesc_qk = f16_idesc(kBM, kBK, false);
+            const int q = warp - 14;
+            constexpr uint32_t idesc_qk = f16_idesc(kBM, kBN, false);
             constexpr uint32_t idesc_pv = f16_idesc(kBM, D, true);
-            uint32_t step = 0, q_it = 0, o_items = 0, pcnt[2] = {0, 0};
+            uint32_t k_it = 0, v_it = 0, q_it = 0, o_items = 0;
+            uint32_t p_par = 0;   // bit b: parity of the next p_full[q][b] phase
             bool issued = false;
-            auto qk = [&](int q, int st) {   // S_q = Q_q K(stage st)^T
-                const uint64_t qd = sw128_desc(sbase + L::kQ + q * L::kTile, 16, 1024);
-                const uint64_t kd = sw128_desc(sbase + L::kK + st * L::kTile, 16, 1024);
-#pragma unroll 1
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint64_t off = (uint64_t)(((kk >> 2) * (128 * 128) + (kk & 3) * 32) >> 4);
-                    mma_bf16(tmem + q * 128, qd + off, kd + off, idesc_qk, kk > 0);
-                }
-            };
-            auto pv = [&](int q, int st, bool first) {   // O_q += P_q V(stage st)
-                const uint64_t vd = sw128_desc(sbase + L::kV + st * L::kTile, kBK * 128, 1024);
-#pragma unroll 1
-                for (int kk = 0; kk < kBK / 16; ++kk)
-                    mma_bf16_ts(tmem + 256 + q * D, tmem + q * 128 + kk * 8, vd + (uint64_t)(kk * 2048 >> 4), idesc_pv,
-                                (!first || kk > 0) ? 1u : 0u);
-            };
-            bool ok = true;
-            for (uint32_t pk = 0; ok && !*abort_flag; ++pk) {
-                const int pr = next_pair1(pk);
-                if (pr < 0) break;
-                const int nt = a.items[2 * pr + 1].w > 0 ? 2 : 1;
-                if (!(ok = wait1(&bars->q_full, q_it & 1, W))) break;
+            const uint64_t qd = sw128_desc(sbase + L::kQ + q * L::kQTile, 16, 1024);
+            for (uint32_t item_k = 0; !*abort_flag; ++item_k) {
+                const int slot = item_k % kRing;
+                if (!wait1(&bars->item_full[slot], (item_k / kRing) & 1, W)) break;
+                const int it = ring[slot];
+                bar_arrive(&bars->item_empty[slot]);
+                if (it < 0) break;
+                const int4 item = a.items[it];
+                const long long r = a.final_cnt[(size_t)item.x * a.Cq + item.y];
+                const int T = (int)((r + kBN - 1) / kBN);
+                const bool active = q == 0 || item.w > kBM;   // Q tile 1 idles on items of <= 128 queries
+                if (!wait1(&bars->q_full, q_it & 1, W)) break;
                 ++q_it;
-                uint32_t e = step;
-                if (!(ok = wait1(&bars->k_full[e % KS], (e / KS) & 1, W))) break;
-                int blk = steps[e % kSteps].block;
-                tc_fence_after();
-                // both tiles take part in every step's handshakes; an idle tile (a pair with
-                // one chunk) only skips its products
-                for (int q = 0; q < 2; ++q) {
-                    if (blk != kEnd && q < nt) qk(q, e % KS);
-                    mma_commit(&bars->s_full[q]);   // S_q(e0) ready (or, for an empty pair, "O_q final")
-                }
-                issued = true;
-                bool first = true;
-                while (blk != kEnd) {
-                    const uint32_t e1 = e + 1;
-                    if (!(ok = wait1(&bars->k_full[e1 % KS], (e1 / KS) & 1, W))) break;
-                    const int nblk = steps[e1 % kSteps].block;
-                    if (!(ok = wait1(&bars->v_full[e % KS], (e / KS) & 1, W))) break;
-                    if (first && !(ok = wait1(&bars->o_free, (o_items & 1) ^ 1, W))) break;
-                    for (int q = 0; q < 2 && ok; ++q) {
-                        if (!(ok = wait1(&bars->p_full[q], pcnt[q] & 1, W))) break;
-                        ++pcnt[q];
-                        tc_fence_after();
-                        if (q < nt) {
-                            pv(q, e % KS, first);
-                            if (nblk != kEnd) qk(q, e1 % KS);
+                // S_q(j) = Q_q K(j)^T into buffer j & 1
+                auto qk_step = [&](int j) -> bool {
+                    const int ks = k_it % L::kKS;
+                    if (!wait1(&bars->k_full[ks], (k_it / L::kKS) & 1, W)) return false;
+                    tc_fence_after();
+                    if (active) {
+                        const uint64_t kd = sw128_desc(sbase + L::kK + ks * L::kKVTile, 16, 1024);
+                        const uint32_t dst = tmem + q * 128 + (j & 1) * kBN;
+#pragma unroll
+                        for (int kk = 0; kk < D / 16; ++kk) {
+                            const uint64_t offa = (uint64_t)(((kk >> 2) * (kBM * 128) + (kk & 3) * 32) >> 4);
+                            const uint64_t offb = (uint64_t)(((kk >> 2) * (kBN * 128) + (kk & 3) * 32) >> 4);
+                            mma_bf16(dst, qd + offa, kd + offb, idesc_qk, kk > 0);
                         }
-                        mma_commit(&bars->s_full[q]);
+                        mma_commit(&bars->s_full[q][j & 1]);
+                    }
+                    mma_commit(&bars->k_empty[ks]);
+                    if (j == T - 1) mma_commit(&bars->q_empty);
+                    ++k_it;
+                    return true;
+                };
+                issued = true;
+                bool ok = qk_step(0);
+                if (ok && T > 1) ok = qk_step(1);
+                for (int t = 0; t < T && ok; ++t) {
+                    const int vs = v_it % L::kVS;
+                    const int b = t & 1;
+                    ok = wait1(&bars->v_full[vs], (v_it / L::kVS) & 1, W);
+                    if (ok && active) {
+                        ok = wait1(&bars->p_full[q][b], (p_par >> b) & 1u, W);
+                        if (ok && t == 0) ok = wait1(&bars->o_free[q], (o_items & 1) ^ 1, W);
+                        if (ok) {
+                            p_par ^= 1u << b;
+                            tc_fence_after();
+                            // O_q += P_q(t) V(t), P_q(t) from TMEM (columns q*128 + b*64 + [0, 32))
+                            const uint64_t vd = sw128_desc(sbase + L::kV + vs * L::kKVTile, kBN * 128, 1024);
+#pragma unroll
+                            for (int kk = 0; kk < kBN / 16; ++kk)
+                                mma_bf16_ts(tmem + 256 + q * D, tmem + q * 128 + b * kBN + kk * 8,
+                                            vd + (uint64_t)(kk * 2048 >> 4), idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
+                            mma_commit(&bars->o_done[q][b]);
+                        }
                     }
                     if (!ok) break;
-                    mma_commit(&bars->kv_empty[e % KS]);
-                    first = false;
-                    e = e1;
-                    blk = nblk;
+                    mma_commit(&bars->v_empty[vs]);
+                    ++v_it;
+                    if (t + 2 < T) ok = qk_step(t + 2);
                 }
                 if (!ok) break;
-                mma_commit(&bars->kv_empty[e % KS]);   // the end step's stage
-                mma_commit(&bars->q_empty);
-                step = e + 1;
-                ++o_items;
+                if (active) ++o_items;
             }
             // every product issued completes before TMEM is freed
             if (issued) {
-                mma_commit(&bars->drain);
-                drain_wait(&bars->drain, 0, W.limit_ns);
+                mma_commit(&bars->drain[q]);
+                drain_wait(&bars->drain[q], 0, W.limit_ns);
             }
         }
         __syncwarp();
     }
-    // warps 10-15 have no role
     } else {
         // ------------------------------------------------------------ softmax + epilogue
         asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
-        const int q = warp >> 2;                       // query tile of this warpgroup
-        const int row = (warp & 3) * 32 + lane;        // 0..127 = TMEM lane
+        const int q = warp >> 2;                       // Q tile of this warpgroup
+        const int row = threadIdx.x - q * kBM;         // 0..127 = TMEM lane
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
         const uint32_t s_col = q * 128, o_col = 256 + q * D;
+        // bit b of s_par: parity of the next s_full[q][b] phase; bit b of o_par: parity of
+        // the P V commits on o_done[q][b] before the current item (the softmax waits on
+        // o_done only when it must, so it counts the phases per item instead)
+        uint32_t s_par = 0, o_par = 0;
         const float c = a.scale_log2;
-        uint32_t step = 0, scnt = 0;
-        for (uint32_t pk = 0; !warp_aborted(abort_flag); ++pk) {
-            const int pr = next_pair(pk);
-            if (pr < 0) break;
-            const int4 A = a.items[2 * pr], B = a.items[2 * pr + 1];
-            const int4 I = q ? B : A;
-            const bool active = q == 0 || B.w > 0;
+        // parity of the o_done[q][j & 1] phase that completes when P(j) V(j) is done
+        auto pv_parity = [&](int j) -> uint32_t { return ((o_par >> (j & 1)) + (uint32_t)(j >> 1)) & 1u; };
+        for (uint32_t item_k = 0; !warp_aborted(abort_flag); ++item_k) {
+            const int it = next_item(item_k);
+            if (it < 0) break;
+            const int4 item = a.items[it];
+            const int bh = item.x, cl = item.y, q0 = item.z, nq = item.w;
+            if (q == 1 && nq <= kBM) continue;        // this Q tile is idle for the item
+            const long long r = a.final_cnt[(size_t)bh * a.Cq + cl];
+            const int T = (int)((r + kBN - 1) / kBN);
             float m_run = -INFINITY, l = 0.f;
-            bool have = false, ok = true;
-            uint32_t e = step;
-            while (true) {
-                // step e: its S_q (or, at the end step, O_q final), and its ring entry; an
-                // idle tile takes part in the handshakes only
-                if (!(ok = waitw(&bars->s_full[q], scnt & 1, W))) break;
-                ++scnt;
-                if (!(ok = waitw(&bars->k_full[e % KS], (e / KS) & 1, W))) break;
-                const Step *se = steps + e % kSteps;
-                const int blk = se->block;
-                if (blk == kEnd) break;
-                ++e;
-                if (!active) {
-                    __syncwarp();
-                    if (lane == 0) bar_arrive(&bars->p_full[q]);
-                    continue;
-                }
-                uint32_t wq[kWords];
-#pragma unroll
-                for (int k = 0; k < kWords; ++k) wq[k] = se->w[q][k];
-                const int nvalid = min(kBK, a.N - blk * kBK);
-                bool full = nvalid == kBK, none = true;
-#pragma unroll
-                for (int k = 0; k < kWords; ++k) {
-                    full = full && wq[k] == 0xffffffffu;
-                    none = none && wq[k] == 0u;
-                }
+            bool ok = true;
+            for (int t = 0; t < T; ++t) {
+                const int b = t & 1;
+                ok = waitw(&bars->s_full[q][b], (s_par >> b) & 1u, W);
+                if (!ok) break;
+                s_par ^= 1u << b;
                 tc_fence_after();
-                if (none) {
-                    // nothing of this tile's cluster in the block: P = 0
-                    uint32_t z[16];
+                const uint32_t sb_col = s_col + b * kBN;
+                float s[kBN];
 #pragma unroll
-                    for (int k = 0; k < 16; ++k) z[k] = 0u;
+                for (int h = 0; h < kBN / 32; ++h) tmem_ld32(tmem + lane_base + sb_col + h * 32, s + h * 32);
+                tmem_wait_ld();
+                const int nvalid = (int)min((long long)kBN, r - (long long)t * kBN);
+                if (nvalid < kBN) {
 #pragma unroll
-                    for (int h = 0; h < kBK / 32; ++h) tmem_st16(tmem + lane_base + s_col + h * 16, z);
-                } else {
-                    // two passes over the 128 logits in 32-column chunks (chunk h = mask word
-                    // h), so that a thread holds 32 of them at a time: the row maximum, then
-                    // P = 2^(s*c - m) as bf16 pairs; P chunk h (columns 16h .. 16h+15) only
-                    // overwrites logits already read
-                    auto load_chunk = [&](int h, float (&v)[32]) {
-                        tmem_ld32(tmem + lane_base + s_col + h * 32, v);
-                        tmem_wait_ld();
-                        if (!full) {
-                            const uint32_t wk = wq[h];
-#pragma unroll
-                            for (int j = 0; j < 32; ++j)
-                                if (!((wk >> j) & 1u) || h * 32 + j >= nvalid) v[j] = -INFINITY;
-                        }
-                    };
-                    float mx = -INFINITY;
-#pragma unroll 1
-                    for (int h = 0; h < kBK / 32; ++h) {
-                        float v[32];
-                        load_chunk(h, v);
-                        float m8[8];
-#pragma unroll
-                        for (int k = 0; k < 8; ++k) m8[k] = fmax3(v[k], v[8 + k], v[16 + k]);
-#pragma unroll
-                        for (int k = 0; k < 8; ++k) m8[k] = fmaxf(m8[k], v[24 + k]);
-                        mx = fmax3(mx, fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], fmax3(m8[5], m8[6], m8[7])));
-                    }
-                    const float mt = mx * c;
-                    const bool need = mt > m_run + 8.f;
-                    const bool rescale = have && __any_sync(0xffffffffu, need);
-                    const float alpha = (have && need) ? fast_exp2(m_run - mt) : 1.f;
-                    if (need) m_run = mt;
-                    const unsigned long long c2 = f2pack(c, c), nm2 = f2pack(-m_run, -m_run);
-                    unsigned long long ls2[2] = {0ull, 0ull};
-#pragma unroll 1
-                    for (int h = 0; h < kBK / 32; ++h) {
-                        float v[32];
-                        load_chunk(h, v);
-                        uint32_t pkd[16];
-#pragma unroll
-                        for (int k = 0; k < 16; ++k) {
-                            const float2 av = f2unpack(f2fma(f2pack(v[2 * k], v[2 * k + 1]), c2, nm2));
-                            const float p0 = fast_exp2(av.x), p1 = fast_exp2(av.y);
-                            ls2[k & 1] = f2add(ls2[k & 1], f2pack(p0, p1));
-                            __nv_bfloat162 hh = __floats2bfloat162_rn(p0, p1);
-                            pkd[k] = *reinterpret_cast<uint32_t *>(&hh);
-                        }
-                        tmem_st16(tmem + lane_base + s_col + h * 16, pkd);
-                    }
-                    const float2 la = f2unpack(ls2[0]), lb = f2unpack(ls2[1]);
-                    l = fmaf(l, alpha, (la.x + la.y) + (lb.x + lb.y));
-                    if (rescale) {
-                        // O_q *= alpha before P_q V of this step adds to it; O_q is current:
-                        // this step's s_full commit followed P_q V of the last step
-#pragma unroll 1
-                        for (int h = 0; h < D / 32; ++h) {
-                            float o[32];
-                            tmem_ld32(tmem + lane_base + o_col + h * 32, o);
-                            tmem_wait_ld();
-#pragma unroll
-                            for (int k = 0; k < 32; ++k) o[k] *= alpha;
-                            tmem_st32(tmem + lane_base + o_col + h * 32, o);
-                        }
-                    }
-                    have = true;
+                    for (int j = 0; j < kBN; ++j)
+                        if (j >= nvalid) s[j] = -INFINITY;
                 }
+                // row maximum with three-input max (half the instructions of a pairwise tree)
+                float m8[8];
+#pragma unroll
+                for (int k = 0; k < 8; ++k) m8[k] = s[k];
+#pragma unroll
+                for (int j = 8; j < kBN; j += 16) {
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) m8[k] = fmax3(m8[k], s[j + k], s[j + 8 + k]);
+                }
+                const float mt = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7])) * c;
+                const bool need = mt > m_run + 8.f;
+                if (t > 0 && __any_sync(0xffffffffu, need)) {
+                    // rescaling O needs every earlier P V done; the last one is P(t-1) V(t-1)
+                    ok = waitw(&bars->o_done[q][(t - 1) & 1], pv_parity(t - 1), W);
+                    if (!ok) break;
+                    tc_fence_after();
+                    const float alpha = need ? fast_exp2(m_run - mt) : 1.f;
+#pragma unroll 1
+                    for (int h = 0; h < D / 32; ++h) {
+                        float o[32];
+                        tmem_ld32(tmem + lane_base + o_col + h * 32, o);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) o[e] *= alpha;
+                        tmem_st32(tmem + lane_base + o_col + h * 32, o);
+                    }
+                    if (need) l *= alpha;
+                }
+                if (need) m_run = mt;
+                // P = 2^(s*c - m) as bf16 pairs over the first kBN/2 columns of this S
+                // buffer; exponent arguments and row sums on packed fp32 pairs
+                const unsigned long long c2 = f2pack(c, c), nm2 = f2pack(-m_run, -m_run);
+                unsigned long long ls2[2] = {0ull, 0ull};
+#pragma unroll
+                for (int h = 0; h < kBN / 32; ++h) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const float2 av = f2unpack(f2fma(f2pack(s[h * 32 + 2 * e], s[h * 32 + 2 * e + 1]), c2, nm2));
+                        const float p0 = fast_exp2(av.x), p1 = fast_exp2(av.y);
+                        ls2[e & 1] = f2add(ls2[e & 1], f2pack(p0, p1));
+                        __nv_bfloat162 hh = __floats2bfloat162_rn(p0, p1);
+                        pk[e] = *reinterpret_cast<uint32_t *>(&hh);
+                    }
+                    tmem_st16(tmem + lane_base + sb_col + h * 16, pk);
+                }
+                const float2 la = f2unpack(ls2[0]), lb = f2unpack(ls2[1]);
+                float ls[4] = {la.x, la.y, lb.x, lb.y};
+                l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) bar_arrive(&bars->p_full[q]);
+                if (lane == 0) bar_arrive(&bars->p_full[q][b]);
             }
             if (!ok) break;
-            step = e + 1;   // past the end step
-            if (active) {
-                // epilogue: O_q / l for the valid rows (the end step's s_full wait made O_q final)
-                tc_fence_after();
-                const float inv = l > 0.f ? 1.f / l : 0.f;
-                const bool valid = row < I.w;
-                __nv_bfloat16 *dst = nullptr;
-                if (valid) {
-                    const int tok = a.perm[(size_t)I.x * a.perm_bh + I.z + row];
-                    dst = reinterpret_cast<__nv_bfloat16 *>(a.O) + ((size_t)I.x * a.N + tok) * D;
-                }
+            // epilogue: O / l for the valid rows of this Q tile, once P(T-1) V(T-1) is done
+            if (!waitw(&bars->o_done[q][(T - 1) & 1], pv_parity(T - 1), W)) break;
+            o_par ^= (uint32_t)(((T + 1) >> 1) & 1) | ((uint32_t)((T >> 1) & 1) << 1);
+            tc_fence_after();
+            const float inv = l > 0.f ? 1.f / l : 0.f;
+            const bool valid = q * kBM + row < nq;
+            __nv_bfloat16 *dst = nullptr;
+            if (valid) {
+                const int tok = a.perm[(size_t)bh * a.perm_bh + q0 + q * kBM + row];
+                dst = reinterpret_cast<__nv_bfloat16 *>(a.O) + ((size_t)bh * a.N + tok) * D;
+            }
 #pragma unroll 1
-                for (int h = 0; h < D / 32; ++h) {
-                    float o[32];
-                    tmem_ld32(tmem + lane_base + o_col + h * 32, o);
-                    tmem_wait_ld();
-                    if (valid) {
+            for (int h = 0; h < D / 32; ++h) {
+                float o[32];
+                tmem_ld32(tmem + lane_base + o_col + h * 32, o);
+                tmem_wait_ld();
+                if (valid) {
 #pragma unroll
-                        for (int k = 0; k < 32; k += 8) {
-                            uint32_t pkd[4];
+                    for (int e = 0; e < 32; e += 8) {
+                        uint32_t pk[4];
 #pragma unroll
-                            for (int t = 0; t < 4; ++t) {
-                                const float y0 = l > 0.f ? o[k + 2 * t] * inv : 0.f;
-                                const float y1 = l > 0.f ? o[k + 2 * t + 1] * inv : 0.f;
-                                __nv_bfloat162 hh = __floats2bfloat162_rn(y0, y1);
-                                pkd[t] = *reinterpret_cast<uint32_t *>(&hh);
-                            }
-                            *reinterpret_cast<uint4 *>(dst + h * 32 + k) = make_uint4(pkd[0], pkd[1], pkd[2], pkd[3]);
+                        for (int k = 0; k < 4; ++k) {
+                            __nv_bfloat162 hh = __floats2bfloat162_rn(o[e + 2 * k] * inv, o[e + 2 * k + 1] * inv);
+                            pk[k] = *reinterpret_cast<uint32_t *>(&hh);
                         }
+                        *reinterpret_cast<uint4 *>(dst + h * 32 + e) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
                     }
                 }
-                tc_fence_before();
             }
+            tc_fence_before();
             __syncwarp();
-            if (lane == 0) bar_arrive(&bars->o_free);
+            if (lane == 0) bar_arrive(&bars->o_free[q]);
         }
     }
-    // drain (every role has waited for its own copies and products) and free TMEM
+    // drain and free TMEM
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == kWIssue)
+    if (warp == 14)
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
                      : "memory");
+}
+
+}  // namespace
+
+namespace {
+
+// [rows, D] bf16 row-major; box = 64 columns x 1 row (tile::gather4), 128-byte swizzle.
+bool row_gather_map(CUtensorMap *m, const void *base, long long rows, int D)
+{
+    return bf16_tile_map(m, base, rows, D, 64, 1);
 }
 
 template <int D>
 cudaError_t launch_tc(const AttnArgs &a, cudaStream_t s)
 {
+    CUtensorMap tq, tk, tv;
+    const long long rows = (long long)a.BH * a.N;
+    // without tensors (the held-scheduler check) the maps are never used: any valid address
+    const void *q = a.Q ? a.Q : a.status, *k = a.K ? a.K : a.status, *v = a.V ? a.V : a.status;
+    if (!row_gather_map(&tq, q, a.Q ? rows : 1, D) || !row_gather_map(&tk, k, a.K ? rows : 1, D) ||
+        !row_gather_map(&tv, v, a.V ? rows : 1, D))
+        return cudaErrorInvalidValue;
     // setmaxnreg moves registers between warpgroups inside the block's launch allocation;
     // the split only adds up if the kernel was compiled to exactly kLaunchRegs
     cudaFuncAttributes fa;
     if (cudaFuncGetAttributes(&fa, attn_tc_kernel<D>) != cudaSuccess || fa.numRegs != kLaunchRegs)
         return cudaErrorInvalidDeviceFunction;
-    Maps m;
-    const long long rows = (long long)a.BH * a.N;
-    // without tensors (the held-scheduler check) the maps are never used: any valid address
-    const void *q = a.Q ? a.Q : a.status, *k = a.K ? a.K : a.status, *v = a.V ? a.V : a.status;
-    const long long qrows = a.Q ? rows : kBK, krows = a.K ? rows : kBK, vrows = a.V ? rows : kBK;
-    if (!bf16_tile_map(&m.qg, q, qrows, D, 64, 1) || !bf16_tile_map(&m.kt, k, krows, D, 64, kBK) ||
-        !bf16_tile_map(&m.vt, v, vrows, D, 64, kBK))
-        return cudaErrorInvalidValue;
-    const int smem = Lay<D>::kAlloc;
+    const int smem = Smem<D>::kAlloc;
     cudaFuncSetAttribute(attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    attn_tc_kernel<D><<<a.num_sms, kThreads, smem, s>>>(m, a);
+    attn_tc_kernel<D><<<a.num_sms, kThreads, smem, s>>>(tq, tk, tv, a);
     return cudaGetLastError();
 }
 

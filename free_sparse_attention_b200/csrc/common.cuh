@@ -11,7 +11,7 @@ namespace scope {
 
 constexpr int kMaxC = 2048;         // max centroids per problem (LUT and histogram sizes)
 constexpr int kSortChunk = 512;     // tokens per warp in the stable counting sort
-constexpr int kAttnTile = 128;      // queries per attention work item (one 128-row tile)
+constexpr int kAttnTile = 256;      // queries per attention work item (two 128-row tiles)
 constexpr unsigned long long kTcWaitDefaultNs = 4000000000ull;   // pipeline wait limit (4 s)
 
 // ---------------------------------------------------------------------------------
@@ -63,7 +63,7 @@ struct WsLayout {
     size_t cent32, cent64T, cnorm, cnrm2, cslack, perm, off, chunk_hist, cent_bf, cn2p, unsure_list, unsure_count;
     size_t q_cent, q_assign, q_sizes, k_cent, k_codes, k_sizes;
     size_t topp, base, khead, final_cnt, mask, sel_state, sel_hist;
-    size_t q_perm, q_off, q_hist, work_items, unit_pos, head_pair, attn_counter;
+    size_t q_perm, q_off, q_hist, work_items, attn_counter, key_lists;
     size_t total;
 };
 
@@ -101,10 +101,10 @@ struct AttnArgs {
     long long perm_bh, off_bh;
     const uint32_t *mask;     // [BH, Cq, nw]
     const int32_t *final_cnt; // [BH, Cq]
-    int4 *items;              // work list: pair p = items[2p], items[2p+1], each (bh, c, q0, nq)
-    int32_t *unit_pos;        // [BH*Cq + 1] scratch of the work-list builder
-    int32_t *head_pair;       // [BH] scratch of the work-list builder
-    int32_t *counter;         // [2]: pair count, dynamic scheduler
+    int4 *items;              // work list (bh, c, q0, nq)
+    int32_t *lists;           // selected key indices of unit u at lists[u*list_stride ...], ascending
+    long long list_stride;    // N rounded up to a multiple of 4
+    int32_t *counter;         // [2]: item count, dynamic scheduler
     int BH, N, d, Cq, nw, is_bf16;
     int use_tc;               // bf16 on the tensor cores (else CUDA cores)
     float scale_log2;         // log2(e)/sqrt(d)

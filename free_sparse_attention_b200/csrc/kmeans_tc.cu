@@ -155,6 +155,28 @@ __device__ __forceinline__ float bound_E(int ks, float xn, float M, float Rm, fl
     return fmaf(xn, fmaf(coef, M, 2.f * Rm), fmaf(0x1p-40f * xn, xn, slack));
 }
 
+__device__ __forceinline__ float fmin3f(float a, float b, float c)
+{
+    float d;
+    asm("min.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// Scores of centroids i and i+1 from their products v0, v1 and norms n0, n1, folded into a
+// running (smallest m1, second smallest m2, index of the smallest mi).  The second smallest
+// of {m1, m2} and {lo, hi} is min(m2, hi, max(m1, lo)); on equal scores the index of the
+// pair's first element is kept (ties are never certified: they are re-decided exactly).
+__device__ __forceinline__ void pair_update(float v0, float v1, float n0, float n1, int i, float &m1, float &m2,
+                                            int &mi)
+{
+    const float2 A = f2unpack(f2fma(f2pack(-2.f, -2.f), f2pack(v0, v1), f2pack(n0, n1)));
+    const float lo = fminf(A.x, A.y), hi = fmaxf(A.x, A.y);
+    const int li = A.y < A.x ? i + 1 : i;
+    m2 = fmin3f(m2, hi, fmaxf(m1, lo));
+    mi = lo < m1 ? li : mi;
+    m1 = fminf(m1, lo);
+}
+
 __device__ __forceinline__ void bulk_copy(uint32_t dst, const void *src, uint32_t bytes, uint64_t *bar)
 {
     asm volatile(
@@ -448,32 +470,23 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
                     if (two) tmem_ld16(ta + 32, v + 16);
                     tmem_wait_ld();
                     const int c0 = n0 + gi * 16;
+                    // scores two at a time: A = |mu|^2 - 2 x.mu on packed pairs, then the
+                    // smaller and larger of the pair update (min, second min, winner) with
+                    // three-input min / max
                     const float4 *na = reinterpret_cast<const float4 *>(n2s + c0);
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
                         const float4 nn = na[q];
-                        const float nv[4] = {nn.x, nn.y, nn.z, nn.w};
-#pragma unroll
-                        for (int r = 0; r < 4; ++r) {
-                            const float A = fmaf(-2.f, v[4 * q + r], nv[r]);
-                            a2 = fminf(a2, fmaxf(a1, A));
-                            ai = A < a1 ? c0 + 4 * q + r : ai;
-                            a1 = fminf(a1, A);
-                        }
+                        pair_update(v[4 * q], v[4 * q + 1], nn.x, nn.y, c0 + 4 * q, a1, a2, ai);
+                        pair_update(v[4 * q + 2], v[4 * q + 3], nn.z, nn.w, c0 + 4 * q + 2, a1, a2, ai);
                     }
                     if (two) {
                         const float4 *nb4 = reinterpret_cast<const float4 *>(n2s + c0 + 32);
 #pragma unroll
                         for (int q = 0; q < 4; ++q) {
                             const float4 nn = nb4[q];
-                            const float nv[4] = {nn.x, nn.y, nn.z, nn.w};
-#pragma unroll
-                            for (int r = 0; r < 4; ++r) {
-                                const float A = fmaf(-2.f, v[16 + 4 * q + r], nv[r]);
-                                b2 = fminf(b2, fmaxf(b1, A));
-                                bi = A < b1 ? c0 + 32 + 4 * q + r : bi;
-                                b1 = fminf(b1, A);
-                            }
+                            pair_update(v[16 + 4 * q], v[16 + 4 * q + 1], nn.x, nn.y, c0 + 32 + 4 * q, b1, b2, bi);
+                            pair_update(v[16 + 4 * q + 2], v[16 + 4 * q + 3], nn.z, nn.w, c0 + 32 + 4 * q + 2, b1, b2, bi);
                         }
                     }
                 }

@@ -253,8 +253,8 @@ AttnArgs attn_args(const scope_params &p, const WsLayout &L, void *ws, const voi
     a.mask = mask;
     a.final_cnt = fin;
     a.items = at<int4>(ws, L.work_items);
-    a.unit_pos = at<int32_t>(ws, L.unit_pos);
-    a.head_pair = at<int32_t>(ws, L.head_pair);
+    a.lists = at<int32_t>(ws, L.key_lists);
+    a.list_stride = (D.N + 3) / 4 * 4;
     a.counter = at<int32_t>(ws, L.counters);
     a.BH = (int)D.BH;
     a.N = (int)D.N;
@@ -316,9 +316,8 @@ WsLayout ws_layout(const scope_params &p)
     L.mask = take(sizeof(uint32_t) * D.BH * p.Cq * D.nw);
     L.sel_state = take(sizeof(double) * 8 * D.BH * p.Cq);
     L.sel_hist = take(sizeof(int32_t) * kSelBins * D.BH * p.Cq);
-    L.work_items = take(sizeof(int4) * D.BH * ((D.N + kAttnTile - 1) / kAttnTile + p.Cq + 2));
-    L.unit_pos = take(sizeof(int32_t) * (D.BH * p.Cq + 1));
-    L.head_pair = take(sizeof(int32_t) * (D.BH + 1));
+    L.work_items = take(sizeof(int4) * D.BH * ((D.N + kAttnTile - 1) / kAttnTile + p.Cq));
+    L.key_lists = take(sizeof(int32_t) * D.BH * p.Cq * ((D.N + 3) / 4 * 4));
     L.total = o;
     return L;
 }

@@ -20,9 +20,9 @@
  *    channels [0, d_t) / [d_t, d_t+d_h) / [d_t+d_h, d) are the temporal / height /
  *    width subspaces.  Element type of Q, K, V, O is params->dtype.
  *  - The caller owns every buffer, including the workspace `ws` of at least
- *    scope_workspace_bytes(params) bytes (256-byte aligned): the clustering scratch,
- *    the intermediates of scope_forward and the selection masks (318 MiB for 24 heads of
- *    118800 tokens, Cq = 300, Cm = 333).  The library allocates
+ *    scope_workspace_bytes(params) bytes (256-byte aligned).  The workspace is
+ *    dominated by the attention gather lists, 4 * B*H*Cq*N bytes (3.4 GB for 24 heads
+ *    of 118800 tokens and Cq = 300).  The library allocates
  *    no device memory, keeps no state between calls and never synchronises the
  *    stream, except scope_get_device_status.  Calls on one workspace must not overlap.
  *  - `stream` is a cudaStream_t (NULL = legacy default stream).  Work is enqueued;

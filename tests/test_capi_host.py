@@ -50,10 +50,9 @@ def test_workspace_bytes_for_every_workload(L, name):
 
 
 def test_workspace_fits_hbm_at_118800_tokens(L):
-    # the attention kernel reads the selection bitmask directly (no per-key index lists):
-    # clustering scratch, intermediates and masks only
+    # dominated by the attention gather lists: 4 B x B*H*Cq*N (3.4 GB here)
     n = capi.workspace_bytes(capi.Params.from_workload(HUNYUAN720))
-    assert n < 512 * 1024 ** 2
+    assert n < 5 * 1024 ** 3
 
 
 BAD = [
