@@ -51,6 +51,7 @@ struct KmArgs {
     // tensor-core assignment (bf16 inputs): packed centroid operands, Cpad = Cs rounded up to 16
     __nv_bfloat16 *cent_bf;   // [P, 2 (hi, lo), Cpad, d] bf16 split of the centroids
     float *cn2p;              // [P, Cpad + 4] |mu|^2 (+inf padding), max |mu|, max slack
+    float *xnorm;             // [P, N] |x| over the role's channels, rounded up (per run)
     // tokens whose assignment the fast kernels could not certify, one list per launched
     // role r: entries bh * N + j at unsure_list[r * BH * N ...], count unsure_count[r]
     int32_t *unsure_list;     // [4, BH * N]
@@ -60,7 +61,8 @@ struct KmArgs {
 // Workspace layout (byte offsets); computed identically by every entry point.
 struct WsLayout {
     size_t status, counters;
-    size_t cent32, cent64T, cnorm, cnrm2, cslack, perm, off, chunk_hist, cent_bf, cn2p, unsure_list, unsure_count;
+    size_t cent32, cent64T, cnorm, cnrm2, cslack, perm, off, chunk_hist, cent_bf, cn2p, xnorm, unsure_list,
+        unsure_count;
     size_t q_cent, q_assign, q_sizes, k_cent, k_codes, k_sizes;
     size_t topp, base, khead, final_cnt, mask, sel_state, sel_hist;
     size_t q_perm, q_off, q_hist, work_items, attn_counter, key_lists;
@@ -74,6 +76,7 @@ cudaError_t km_run(KmArgs a, int iters, cudaStream_t s);
 cudaError_t sort_by_cluster(KmArgs a, cudaStream_t s);  // stable counting sort, all problems
 bool km_assign_tc_supported(const KmArgs &a);            // bf16 and the operands fit on chip
 cudaError_t km_pack(const KmArgs &a, cudaStream_t s);     // centroids -> cent_bf, cn2p
+cudaError_t km_norms(const KmArgs &a, cudaStream_t s);    // token norms -> xnorm (once per run)
 cudaError_t km_assign_tc(const KmArgs &a, int num_sms, cudaStream_t s);
 
 struct SelArgs {

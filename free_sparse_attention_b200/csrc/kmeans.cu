@@ -324,6 +324,8 @@ __global__ void __launch_bounds__(128) sort_hist_kernel(KmArgs a)
 }
 
 // Per problem: prefix over chunks for every cluster, sizes, and cluster offsets.
+constexpr int kScanBatch = 16;
+
 __global__ void __launch_bounds__(1024) sort_scan_kernel(KmArgs a)
 {
     __shared__ int wsum[32];
@@ -338,9 +340,22 @@ __global__ void __launch_bounds__(1024) sort_scan_kernel(KmArgs a)
         int c = threadIdx.x * per + q;
         int run = 0;
         if (c < C) {
+            // the column's chunk counts are read kScanBatch at a time (independent loads in
+            // flight), then replaced by their exclusive prefix
             int32_t *col = a.chunk_hist + (size_t)p * a.nchunk * a.Cs + c;
-            for (int k = 0; k < a.nchunk; ++k) {
-                int h = col[(size_t)k * a.Cs];
+            int k = 0;
+            for (; k + kScanBatch <= a.nchunk; k += kScanBatch) {
+                int h[kScanBatch];
+#pragma unroll
+                for (int q = 0; q < kScanBatch; ++q) h[q] = col[(size_t)(k + q) * a.Cs];
+#pragma unroll
+                for (int q = 0; q < kScanBatch; ++q) {
+                    col[(size_t)(k + q) * a.Cs] = run;
+                    run += h[q];
+                }
+            }
+            for (; k < a.nchunk; ++k) {
+                const int h = col[(size_t)k * a.Cs];
                 col[(size_t)k * a.Cs] = run;
                 run += h;
             }
@@ -585,6 +600,10 @@ cudaError_t km_run(KmArgs a, int iters, cudaStream_t s)
     bool upd2 = a.is_bf16 != 0;
     for (int r = 0; r < a.nroles; ++r)
         upd2 = upd2 && (a.role[a.role0 + r].ch0 % 2 == 0) && (a.role[a.role0 + r].dm % 2 == 0);
+    if (tc) {
+        cudaError_t e = km_norms(a, s);
+        if (e != cudaSuccess) return e;
+    }
     for (int it = 0; it < iters; ++it) {
         if (cudaMemsetAsync(a.unsure_count, 0, 4 * sizeof(int32_t), s) != cudaSuccess) return cudaGetLastError();
         if (tc) {

@@ -29,8 +29,9 @@
 //   warp 0     TMA producer: the problem's centroid matrix (hi, lo) and |mu|^2 row once
 //              per problem, the token tile into a 2-deep ring
 //   warp 1     TMEM allocation and MMA issue (one thread)
-//   warps 2-9  epilogue, two warpgroups splitting every chunk's columns: token norms
-//              from the shared-memory tile, TMEM loads, running minima, certification
+//   warps 2-9  epilogue, two warpgroups splitting every chunk's columns: TMEM loads,
+//              running minima, certification against the token norms that
+//              km_norms_kernel computes once per clustering run
 // The centroids are split in chunks of at most 256 columns, double-buffered in TMEM
 // (2 x 256 columns), so the epilogue of one chunk overlaps the MMAs of the next.
 // Every mbarrier wait gives up after ~4 s, sets a status bit and lets the CTA drain.
@@ -43,7 +44,11 @@ namespace scope {
 namespace {
 
 constexpr int kTile = 128;             // tokens per unit (TMEM lanes)
-constexpr int kThreadsTc = 320;        // 10 warps
+#ifndef SCOPE_KM_EPI_WG
+#define SCOPE_KM_EPI_WG 2
+#endif
+constexpr int kEpiWG = SCOPE_KM_EPI_WG;  // epilogue warpgroups
+constexpr int kThreadsTc = 64 + 128 * kEpiWG;   // producer warp, MMA warp, epilogue
 constexpr int kChunkMax = 256;         // centroid columns per TMEM buffer
 constexpr uint32_t kTmemColsTc = 512;  // two accumulator buffers
 constexpr uint16_t kUnsureTc = 0xFFFF;
@@ -114,7 +119,7 @@ TcLayout tc_layout(const KmArgs &a)
     L.x_stage = (size_t)nbm * kTile * 128;
     L.n2_off = L.b_bytes + 2 * L.x_stage;
     L.merge_off = (L.n2_off + (size_t)(crm + 4) * 4 + 15) & ~size_t(15);
-    L.bars_off = L.merge_off + (size_t)2 * kTile * 16;
+    L.bars_off = L.merge_off + (size_t)(kEpiWG - 1) * 2 * 3 * kTile * 4;   // [wg-1][slot][m1, m2, ix][128]
     L.total = L.bars_off + sizeof(TcBars) + 16 + 1024;
     return L;
 }
@@ -134,10 +139,16 @@ __device__ __forceinline__ void drain_wait(uint64_t *b, uint32_t parity)
 }
 
 // Bound on |score - S_c| for a token of norm |x| <= xn, with M = max |mu_c|,
-// Rm = max |mu_c - hi_c - lo_c| and ks MMA steps per half:
+// Rm = max |mu_c - hi_c - lo_c| and ks MMA steps per half (|hi| <= (1 + 2^-8) |mu|,
+// |lo| <= 2^-8 (1 + 2^-8) |mu|):
 //   2 |x.r_c|                      <= 2 xn Rm               (Cauchy-Schwarz)
-//   2 x fp32 accumulation error     <= 2 (2 ks) 18 2^-23 sum |x_i hi_i| + |x_i lo_i|
-//                                   <= 18 ks 2^-21 (1 + 2^-7) xn M
+//   2 x fp32 accumulation error     <= 2 x 18 2^-23 x (sum over steps of the largest
+//                                      magnitude the step holds); the ks lo steps run
+//                                      first and hold at most sum |x_i lo_i| <= 2^-8 (1 + 2^-8)
+//                                      xn M each, the ks hi steps at most sum |x_i lo_i| +
+//                                      sum |x_i hi_i| <= (1 + 2^-7 + 2^-16) xn M each, so
+//                                   <= 9 ks 2^-21 (1 + 2^-7 + 2^-8 + 2^-15) xn M
+//                                   <= 9 ks 2^-21 1.012 xn M
 //   rounding of the score           <= 2^-21 xn M  (+ the |mu|^2 part, in the slack)
 //   |mu|^2 to fp32, reference sum   <= slack_max + 2^-40 xn^2
 // Accumulation model (Fasi, Higham, Mikaitis, Pranesh, "Numerical behavior of NVIDIA
@@ -151,7 +162,7 @@ __device__ __forceinline__ void drain_wait(uint64_t *b, uint32_t parity)
 // operands.
 __device__ __forceinline__ float bound_E(int ks, float xn, float M, float Rm, float slack)
 {
-    const float coef = (18.f * (float)ks * 1.0079f + 1.f) * 0x1p-21f;
+    const float coef = (9.f * (float)ks * 1.012f + 1.f) * 0x1p-21f;
     return fmaf(xn, fmaf(coef, M, 2.f * Rm), fmaf(0x1p-40f * xn, xn, slack));
 }
 
@@ -186,18 +197,24 @@ __device__ __forceinline__ void bulk_copy(uint32_t dst, const void *src, uint32_
 }
 
 // ------------------------------------------------------------------------- pack
-// One block per problem: the bf16 hi / lo split of every centroid row over all d channels
-// (zero outside the role's channel range and for padded rows), |mu|^2 in fp32 with +inf
-// for padded rows, then max |mu| (rounded up) and the largest slack term.
+// grid (P, kPackSplit), block 256: block (p, y) handles the centroid rows c = y mod kPackSplit
+// of problem p: the bf16 hi / lo split of every row over all d channels (zero outside the
+// role's channel range and for padded rows), |mu|^2 in fp32 with +inf for padded rows, and
+// (one warp per row) the block's largest |mu|^2, split remainder and slack term, folded into
+// the problem's maxima with integer atomicMax on the non-negative float bits (the launcher
+// zeroes them first): max |mu| (rounded up), the largest slack term, max |mu - hi - lo|.
+constexpr int kPackSplit = 8;
+
 __global__ void __launch_bounds__(256) km_pack_kernel(KmArgs a, int Cpad)
 {
-    const int p = blockIdx.x;
+    const int p = blockIdx.x, part = blockIdx.y;
     const int r = p % a.nroles, bh = p / a.nroles;
     const RoleDesc &R = a.role[a.role0 + r];
     __nv_bfloat16 *hi = a.cent_bf + (size_t)p * 2 * Cpad * a.d;
     __nv_bfloat16 *lo = hi + (size_t)Cpad * a.d;
-    for (int idx = threadIdx.x; idx < Cpad * a.d; idx += blockDim.x) {
-        const int c = idx / a.d, i = idx - c * a.d;
+    const int rows = (Cpad - part + kPackSplit - 1) / kPackSplit;
+    for (int k = threadIdx.x; k < rows * a.d; k += blockDim.x) {
+        const int c = part + (k / a.d) * kPackSplit, i = k % a.d;
         float h = 0.f, l = 0.f;
         if (c < R.C && i >= R.ch0 && i < R.ch0 + R.dm) {
             const double m = R.cent[((size_t)bh * R.C + c) * a.d + i];
@@ -206,17 +223,18 @@ __global__ void __launch_bounds__(256) km_pack_kernel(KmArgs a, int Cpad)
             h = __bfloat162float(hb);
             l = __bfloat162float(__double2bfloat16(rem));
         }
-        hi[idx] = __float2bfloat16(h);
-        lo[idx] = __float2bfloat16(l);
+        hi[(size_t)c * a.d + i] = __float2bfloat16(h);
+        lo[(size_t)c * a.d + i] = __float2bfloat16(l);
     }
     float *n2 = a.cn2p + (size_t)p * (Cpad + 4);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     double mx = 0.0, mr = 0.0;
     float msl = 0.f;
-    for (int c = threadIdx.x; c < Cpad; c += blockDim.x) {
+    for (int c = part + warp * kPackSplit; c < Cpad; c += 8 * kPackSplit) {
         if (c < R.C) {
             const double *mu = R.cent + ((size_t)bh * R.C + c) * a.d + R.ch0;
             double s = 0.0, rr = 0.0;
-            for (int i = 0; i < R.dm; ++i) {
+            for (int i = lane; i < R.dm; i += 32) {
                 const double m = mu[i];
                 const double h = (double)__bfloat162float(__double2bfloat16(m));
                 const double rem = m - h;
@@ -224,39 +242,112 @@ __global__ void __launch_bounds__(256) km_pack_kernel(KmArgs a, int Cpad)
                 s += m * m;
                 rr += res * res;
             }
+            for (int o = 16; o; o >>= 1) {
+                s += __shfl_xor_sync(0xffffffffu, s, o);
+                rr += __shfl_xor_sync(0xffffffffu, rr, o);
+            }
             mx = fmax(mx, s);
             mr = fmax(mr, rr);
-            n2[c] = a.cnrm2[(size_t)p * a.Cs + c];
-            msl = fmaxf(msl, a.cslack[(size_t)p * a.Cs + c]);
-        } else {
+            if (lane == 0) {
+                n2[c] = a.cnrm2[(size_t)p * a.Cs + c];
+                msl = fmaxf(msl, a.cslack[(size_t)p * a.Cs + c]);
+            }
+        } else if (lane == 0) {
             n2[c] = INFINITY;
         }
     }
-    __shared__ double smx[256], smr[256];
-    __shared__ float ssl[256];
-    smx[threadIdx.x] = mx;
-    smr[threadIdx.x] = mr;
-    ssl[threadIdx.x] = msl;
-    __syncthreads();
-    for (int o = 128; o; o >>= 1) {
-        if (threadIdx.x < o) {
-            smx[threadIdx.x] = fmax(smx[threadIdx.x], smx[threadIdx.x + o]);
-            smr[threadIdx.x] = fmax(smr[threadIdx.x], smr[threadIdx.x + o]);
-            ssl[threadIdx.x] = fmaxf(ssl[threadIdx.x], ssl[threadIdx.x + o]);
-        }
-        __syncthreads();
+    __shared__ double smx[8], smr[8];
+    __shared__ float ssl[8];
+    if (lane == 0) {
+        smx[warp] = mx;
+        smr[warp] = mr;
+        ssl[warp] = msl;
     }
+    __syncthreads();
     if (threadIdx.x == 0) {
+        for (int w = 1; w < 8; ++w) {
+            mx = fmax(mx, smx[w]);
+            mr = fmax(mr, smr[w]);
+            msl = fmaxf(msl, ssl[w]);
+        }
         // square roots of binary64 sums of squares (each within ~1e-14 of the exact
         // value), rounded up with a margin: max |mu_c| and max |mu_c - hi_c - lo_c|
-        n2[Cpad] = __double2float_ru(sqrt(smx[0]) * (1.0 + 0x1p-20));
-        n2[Cpad + 1] = ssl[0];
-        n2[Cpad + 2] = __double2float_ru(sqrt(smr[0]) * (1.0 + 0x1p-20));
-        n2[Cpad + 3] = 0.f;
+        int *n2i = reinterpret_cast<int *>(n2);
+        atomicMax(n2i + Cpad, __float_as_int(__double2float_ru(sqrt(mx) * (1.0 + 0x1p-20))));
+        atomicMax(n2i + Cpad + 1, __float_as_int(msl));
+        atomicMax(n2i + Cpad + 2, __float_as_int(__double2float_ru(sqrt(mr) * (1.0 + 0x1p-20))));
     }
 }
 
+// ------------------------------------------------------------------------- token norms
+// grid (ceil(N / 256), P), block 256: thread j of problem p computes |x_j| over the role's
+// channels, summing x_i^2 in fp32 with one fma per channel in channel order, and stores
+// sqrt(sum) (1 + 2^-12): an upper bound of the binary64 norm (the fp32 sum of dm squares is
+// within dm 2^-24 of it, the square root within 2^-24).  The inputs do not change between
+// Lloyd iterations, so this runs once per clustering run.
+__global__ void __launch_bounds__(256) km_norms_kernel(KmArgs a)
+{
+    const int p = blockIdx.y, j = blockIdx.x * blockDim.x + threadIdx.x;
+    if (j >= a.N) return;
+    const int bh = p / a.nroles;
+    const RoleDesc &R = a.role[a.role0 + p % a.nroles];
+    const uint4 *row = reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(R.X) +
+                                                       ((size_t)bh * a.N + j) * a.d);
+    const int lo_c = R.ch0, hi_c = R.ch0 + R.dm;
+    float ss = 0.f;
+    for (int q8 = lo_c >> 3; q8 <= (hi_c - 1) >> 3; ++q8) {
+        const uint4 v = row[q8];
+        const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            const int c = q8 * 8 + q;
+            const float x = __uint_as_float((q & 1) ? (wv[q >> 1] & 0xFFFF0000u) : (wv[q >> 1] << 16));
+            if (c >= lo_c && c < hi_c) ss = fmaf(x, x, ss);
+        }
+    }
+    a.xnorm[(size_t)p * a.N + j] = sqrtf(ss) * (1.0f + 0x1p-12f);
+}
+
 // ------------------------------------------------------------------------- assignment
+// The 2 KS products of one chunk: x . lo over the KS 16-channel steps, then x . hi (the order
+// bound_E assumes), into one TMEM accumulator.  The step offsets are compile-time constants
+// added to the low word of the descriptors (the start address field; no carry out of it for
+// shared-memory addresses), so the issuing thread spends a few instructions per product.
+// bstride16 = the centroid box stride (Cr rows of 128 bytes) in 16-byte units.
+template <int KS>
+__device__ __forceinline__ void issue_chunk_ks(uint32_t dst, uint64_t ad, uint64_t bd_lo, uint64_t bd_hi,
+                                               uint32_t bstride16, uint32_t idesc)
+{
+    const uint32_t ahi = (uint32_t)(ad >> 32), alo = (uint32_t)ad;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const uint64_t bd = h == 0 ? bd_lo : bd_hi;
+        const uint32_t bhi = (uint32_t)(bd >> 32), blo = (uint32_t)bd;
+#pragma unroll
+        for (int kk = 0; kk < KS; ++kk) {
+            const uint32_t oa = (uint32_t)(((kk >> 2) * (kTile * 128) + (kk & 3) * 32) >> 4);
+            const uint32_t ob = (uint32_t)(kk >> 2) * bstride16 + (uint32_t)((kk & 3) * 2);
+            mma_bf16(dst, ((uint64_t)ahi << 32) | (alo + oa), ((uint64_t)bhi << 32) | (blo + ob), idesc,
+                     (h | kk) != 0 ? 1u : 0u);
+        }
+    }
+}
+
+__device__ __forceinline__ void issue_chunk(int ks, uint32_t dst, uint64_t ad, uint64_t bd_lo, uint64_t bd_hi,
+                                            uint32_t bstride16, uint32_t idesc)
+{
+    switch (ks) {
+    case 1: issue_chunk_ks<1>(dst, ad, bd_lo, bd_hi, bstride16, idesc); break;
+    case 2: issue_chunk_ks<2>(dst, ad, bd_lo, bd_hi, bstride16, idesc); break;
+    case 3: issue_chunk_ks<3>(dst, ad, bd_lo, bd_hi, bstride16, idesc); break;
+    case 4: issue_chunk_ks<4>(dst, ad, bd_lo, bd_hi, bstride16, idesc); break;
+    case 5: issue_chunk_ks<5>(dst, ad, bd_lo, bd_hi, bstride16, idesc); break;
+    case 6: issue_chunk_ks<6>(dst, ad, bd_lo, bd_hi, bstride16, idesc); break;
+    case 7: issue_chunk_ks<7>(dst, ad, bd_lo, bd_hi, bstride16, idesc); break;
+    default: issue_chunk_ks<8>(dst, ad, bd_lo, bd_hi, bstride16, idesc); break;
+    }
+}
+
 __global__ void __launch_bounds__(kThreadsTc, 1)
     km_assign_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmB, KmArgs a, TcParams t)
@@ -276,13 +367,13 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     if (threadIdx.x == 0) {
         misc[0] = 0;
         bar_init(&bars->b_full, 1);
-        bar_init(&bars->b_empty, 1 + 8);
+        bar_init(&bars->b_empty, 1 + 4 * kEpiWG);
         for (int s = 0; s < 2; ++s) {
             bar_init(&bars->x_full[s], 1);
-            bar_init(&bars->x_empty[s], 1 + 4);
+            bar_init(&bars->x_empty[s], 1);
             bar_init(&bars->acc_full[s], 1);
-            bar_init(&bars->acc_empty[s], 8);
-            bar_init(&bars->mg_full[s], 4);
+            bar_init(&bars->acc_empty[s], 4 * kEpiWG);
+            bar_init(&bars->mg_full[s], 4 * (kEpiWG - 1));
             bar_init(&bars->mg_empty[s], 4);
         }
         bar_init(&bars->drain, 1);
@@ -344,12 +435,19 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
         if (lane == 0) {
             int cur_p = -1;
             uint32_t nb = 0, xi = 0, g = 0;
+            // the unit's (problem, tile) advance incrementally; role constants change per problem
+            int p = (int)(ub / t.TT), tile = (int)(ub % t.TT);
+            int ks = 1, nbox = 1, nch = 1, chunk0 = 16, Cr = 16;
             for (long long u = ub; u < ue && !*abort_flag; ++u) {
-                const int p = (int)(u / t.TT);
-                const RoleDesc &R = a.role[a.role0 + p % a.nroles];
-                const Window w = window_of(R.ch0, R.dm);
-                const Chunks k = chunks_of(R.C);
                 if (p != cur_p) {
+                    const RoleDesc &R = a.role[a.role0 + p % a.nroles];
+                    const Window w = window_of(R.ch0, R.dm);
+                    const Chunks k = chunks_of(R.C);
+                    ks = w.ks;
+                    nbox = w.nbox;
+                    nch = k.nch;
+                    chunk0 = k.chunk0;
+                    Cr = k.Cr;
                     if (!bar_wait(&bars->b_full, nb & 1, abort_flag, a.status)) break;
                     ++nb;
                     cur_p = p;
@@ -357,33 +455,31 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
                 const int s = xi & 1;
                 if (!bar_wait(&bars->x_full[s], (xi >> 1) & 1, abort_flag, a.status)) break;
                 tc_fence_after();
-                const uint32_t xa = sbase + t.x_off + s * t.x_stage;
+                const uint64_t ad0 = sw128_desc(sbase + t.x_off + s * t.x_stage, 16, 1024);
                 bool ok = true;
-                for (int ch = 0; ch < k.nch; ++ch) {
-                    const int n0 = ch * k.chunk0, nc = min(k.chunk0, k.Cr - n0);
+                for (int ch = 0; ch < nch; ++ch) {
+                    const int n0 = ch * chunk0, nc = min(chunk0, Cr - n0);
                     const int buf = g & 1;
                     if (!bar_wait(&bars->acc_empty[buf], ((g >> 1) & 1) ^ 1, abort_flag, a.status)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t idesc = f16_idesc(kTile, nc, false);
-                    const uint32_t dst = tmem + buf * kChunkMax;
-                    for (int sp = 0; sp < 2; ++sp)
-                        for (int kk = 0; kk < w.ks; ++kk) {
-                            const uint64_t ad = sw128_desc(xa + (kk >> 2) * (kTile * 128) + (kk & 3) * 32, 16, 1024);
-                            const uint64_t bd = sw128_desc(
-                                sbase + ((sp * w.nbox + (kk >> 2)) * k.Cr + n0) * 128 + (kk & 3) * 32, 16, 1024);
-                            mma_bf16(dst, ad, bd, idesc, (sp | kk) != 0 ? 1u : 0u);
-                        }
+                    issue_chunk(ks, tmem + buf * kChunkMax, ad0, sw128_desc(sbase + (nbox * Cr + n0) * 128, 16, 1024),
+                                sw128_desc(sbase + n0 * 128, 16, 1024), (uint32_t)(Cr * 128) >> 4,
+                                f16_idesc(kTile, nc, false));
                     mma_commit(&bars->acc_full[buf]);
                     ++g;
                 }
                 if (!ok) break;
                 mma_commit(&bars->x_empty[s]);
                 ++xi;
+                if (++tile == t.TT) {
+                    tile = 0;
+                    ++p;
+                }
                 // the CTA's last unit of this problem releases the centroids
-                if (u + 1 == ue || (int)((u + 1) / t.TT) != p) mma_commit(&bars->b_empty);
+                if (u + 1 == ue || tile == 0) mma_commit(&bars->b_empty);
             }
             // every issued MMA completes before TMEM is freed
             mma_commit(&bars->drain);
@@ -391,33 +487,38 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
         }
         __syncwarp();
     } else {
-        // ------------------------------------------------------------ epilogue (warps 2-9)
-        // Two warpgroups share every chunk: warpgroup e takes the 16-column groups
-        // g = e, e+2, ... (two at a time, one TMEM wait per pair, one running minimum
+        // ------------------------------------------------------------ epilogue (warps 2-)
+        // kEpiWG warpgroups share every chunk: warpgroup e takes the 16-column groups
+        // g = e, e + kEpiWG, ... (two at a time, one TMEM wait per pair, one running minimum
         // pair per group slot so consecutive columns do not form one dependency chain).
-        // Warpgroup 1 also computes the token norms and hands its (min, second min,
-        // winner, norm) per token to warpgroup 0 through a double-buffered slot; warpgroup
-        // 0 merges, certifies and writes the assignment.
+        // Warpgroups 1.. hand their (min, second min, winner) per token to warpgroup 0
+        // through a double-buffered slot; warpgroup 0 merges, certifies (with the token's
+        // norm, computed once per run by km_norms_kernel) and writes the assignment.
         const int e = (warp - 2) >> 2;                 // epilogue warpgroup
         const int q4 = warp & 3;                       // TMEM lane quarter of this warp
         const int row = q4 * 32 + lane;                // token row of the tile = TMEM lane
         const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
         const float *n2s = reinterpret_cast<const float *>(sm + t.n2_off);
-        float *mg_m1 = reinterpret_cast<float *>(sm + t.merge_off);   // [2][128]
-        float *mg_m2 = mg_m1 + 2 * kTile;
-        float *mg_xn = mg_m2 + 2 * kTile;
-        int *mg_ix = reinterpret_cast<int *>(mg_xn + 2 * kTile);
+        float *mg = reinterpret_cast<float *>(sm + t.merge_off);   // [kEpiWG-1][2][3][128]
         int cur_p = -1;
-        uint32_t nb = 0, xi = 0, g = 0;
+        uint32_t nb = 0, g = 0;
         float maxnm = 0.f, maxsl = 0.f, maxres = 0.f;
-        for (long long u = ub; u < ue; ++u) {
+        // the unit's (problem, tile) advance incrementally; role constants change per problem
+        int p = (int)(ub / t.TT), tile = (int)(ub % t.TT);
+        int bh = 0, r = 0, ks = 1;
+        Chunks k{16, 1, 16};
+        uint16_t *assign = nullptr;
+        long long assign_bh = 0;
+        for (long long u = ub; u < ue; ++u, (++tile == t.TT ? (tile = 0, ++p) : 0)) {
             if (warp_aborted(abort_flag)) break;
-            const int p = (int)(u / t.TT), tile = (int)(u % t.TT);
-            const int bh = p / a.nroles;
-            const RoleDesc &R = a.role[a.role0 + p % a.nroles];
-            const Window w = window_of(R.ch0, R.dm);
-            const Chunks k = chunks_of(R.C);
             if (p != cur_p) {
+                bh = p / a.nroles;
+                r = p % a.nroles;
+                const RoleDesc &R = a.role[a.role0 + r];
+                ks = window_of(R.ch0, R.dm).ks;
+                k = chunks_of(R.C);
+                assign = R.assign;
+                assign_bh = R.assign_bh;
                 if (!warp_wait(&bars->b_full, nb & 1, abort_flag, a.status)) break;
                 ++nb;
                 cur_p = p;
@@ -425,30 +526,10 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
                 maxsl = n2s[k.Cr + 1];
                 maxres = n2s[k.Cr + 2];
             }
-            const int s = xi & 1;
+            const int j = tile * kTile + row;
+            // |x| of this token over the role's channels (computed once per run)
             float xn = 0.f;
-            if (e == 1) {
-                if (!warp_wait(&bars->x_full[s], (xi >> 1) & 1, abort_flag, a.status)) break;
-                // |x| over the role's channels, read from the 128-byte swizzled tile
-                const unsigned char *xt = sm + t.x_off + s * t.x_stage;
-                const int lo_c = R.ch0 - w.ws, hi_c = lo_c + R.dm;   // window-relative range
-                float ss = 0.f;
-                for (int j = lo_c >> 3; j <= (hi_c - 1) >> 3; ++j) {
-                    const uint4 v = *reinterpret_cast<const uint4 *>(
-                        xt + (j >> 3) * (kTile * 128) + row * 128 + (((j & 7) ^ (row & 7)) << 4));
-                    const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        const int c = j * 8 + q;
-                        const float x = __uint_as_float((q & 1) ? (wv[q >> 1] & 0xFFFF0000u) : (wv[q >> 1] << 16));
-                        if (c >= lo_c && c < hi_c) ss = fmaf(x, x, ss);
-                    }
-                }
-                __syncwarp();
-                if (lane == 0) bar_arrive(&bars->x_empty[s]);
-                xn = sqrtf(ss) * (1.0f + 0x1p-12f);
-            }
-            ++xi;
+            if (e == 0 && j < a.N) xn = a.xnorm[(size_t)p * a.N + j];
             // running (min, second min, winner) for the two group slots of this thread
             float a1 = INFINITY, a2 = INFINITY, b1 = INFINITY, b2 = INFINITY;
             int ai = 0, bi = 0;
@@ -462,12 +543,12 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
                     break;
                 }
                 tc_fence_after();
-                for (int gi = e; gi < ng; gi += 4) {
-                    const bool two = gi + 2 < ng;
+                for (int gi = e; gi < ng; gi += 2 * kEpiWG) {
+                    const bool two = gi + kEpiWG < ng;
                     float v[32];
                     const uint32_t ta = tmem + lane_base + buf * kChunkMax + gi * 16;
                     tmem_ld16(ta, v);
-                    if (two) tmem_ld16(ta + 32, v + 16);
+                    if (two) tmem_ld16(ta + 16 * kEpiWG, v + 16);
                     tmem_wait_ld();
                     const int c0 = n0 + gi * 16;
                     // scores two at a time: A = |mu|^2 - 2 x.mu on packed pairs, then the
@@ -481,12 +562,14 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
                         pair_update(v[4 * q + 2], v[4 * q + 3], nn.z, nn.w, c0 + 4 * q + 2, a1, a2, ai);
                     }
                     if (two) {
-                        const float4 *nb4 = reinterpret_cast<const float4 *>(n2s + c0 + 32);
+                        const float4 *nb4 = reinterpret_cast<const float4 *>(n2s + c0 + 16 * kEpiWG);
 #pragma unroll
                         for (int q = 0; q < 4; ++q) {
                             const float4 nn = nb4[q];
-                            pair_update(v[16 + 4 * q], v[16 + 4 * q + 1], nn.x, nn.y, c0 + 32 + 4 * q, b1, b2, bi);
-                            pair_update(v[16 + 4 * q + 2], v[16 + 4 * q + 3], nn.z, nn.w, c0 + 32 + 4 * q + 2, b1, b2, bi);
+                            pair_update(v[16 + 4 * q], v[16 + 4 * q + 1], nn.x, nn.y, c0 + 16 * kEpiWG + 4 * q, b1, b2,
+                                        bi);
+                            pair_update(v[16 + 4 * q + 2], v[16 + 4 * q + 3], nn.z, nn.w, c0 + 16 * kEpiWG + 4 * q + 2,
+                                        b1, b2, bi);
                         }
                     }
                 }
@@ -496,7 +579,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
                 ++g;
             }
             if (!ok) break;
-            if (u + 1 == ue || (int)((u + 1) / t.TT) != p) {
+            if (u + 1 == ue || tile + 1 == t.TT) {
                 __syncwarp();
                 if (lane == 0) bar_arrive(&bars->b_empty);
             }
@@ -506,33 +589,40 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
             int idx = b1 < a1 ? bi : ai;
             float m1 = fminf(a1, b1);
             const uint32_t mi = (uint32_t)(u - ub), slot = mi & 1;
-            if (e == 1) {
+            if (e != 0) {
                 if (!warp_wait(&bars->mg_empty[slot], ((mi >> 1) & 1) ^ 1, abort_flag, a.status)) break;
-                mg_m1[slot * kTile + row] = m1;
-                mg_m2[slot * kTile + row] = m2;
-                mg_xn[slot * kTile + row] = xn;
-                mg_ix[slot * kTile + row] = idx;
+                float *o = mg + ((size_t)((e - 1) * 2 + slot) * 3) * kTile;
+                o[row] = m1;
+                o[kTile + row] = m2;
+                reinterpret_cast<int *>(o)[2 * kTile + row] = idx;
                 __syncwarp();
                 if (lane == 0) bar_arrive(&bars->mg_full[slot]);
             } else {
                 if (!warp_wait(&bars->mg_full[slot], (mi >> 1) & 1, abort_flag, a.status)) break;
-                const float o1 = mg_m1[slot * kTile + row], o2 = mg_m2[slot * kTile + row];
-                xn = mg_xn[slot * kTile + row];
-                const int oi = mg_ix[slot * kTile + row];
+                float o1[kEpiWG - 1], o2[kEpiWG - 1];
+                int oi[kEpiWG - 1];
+#pragma unroll
+                for (int h = 0; h < kEpiWG - 1; ++h) {
+                    const float *o = mg + ((size_t)(h * 2 + slot) * 3) * kTile;
+                    o1[h] = o[row];
+                    o2[h] = o[kTile + row];
+                    oi[h] = reinterpret_cast<const int *>(o)[2 * kTile + row];
+                }
                 __syncwarp();
                 if (lane == 0) bar_arrive(&bars->mg_empty[slot]);
-                m2 = fminf(fminf(m2, o2), fmaxf(m1, o1));
-                idx = o1 < m1 ? oi : idx;
-                m1 = fminf(m1, o1);
-                const int j = tile * kTile + row;
+#pragma unroll
+                for (int h = 0; h < kEpiWG - 1; ++h) {
+                    m2 = fminf(fminf(m2, o2[h]), fmaxf(m1, o1[h]));
+                    idx = o1[h] < m1 ? oi[h] : idx;
+                    m1 = fminf(m1, o1[h]);
+                }
                 bool unsure = false;
                 if (j < a.N) {
-                    const float E = bound_E(w.ks, xn, maxnm, maxres, maxsl);
+                    const float E = bound_E(ks, xn, maxnm, maxres, maxsl);
                     const bool sure = (m2 - m1) > (E + E) * (1.0f + 0x1p-20f);
-                    R.assign[(size_t)bh * R.assign_bh + j] = sure ? (uint16_t)idx : kUnsureTc;
+                    assign[(size_t)bh * assign_bh + j] = sure ? (uint16_t)idx : kUnsureTc;
                     unsure = !sure;
                 }
-                const int r = p % a.nroles;
                 warp_append(unsure, bh * a.N + j, a.unsure_list + (size_t)r * a.BH * a.N, a.unsure_count + r);
             }
         }
@@ -549,14 +639,24 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
 
 bool km_assign_tc_supported(const KmArgs &a)
 {
-    if (!a.is_bf16 || (a.d != 64 && a.d != 128) || !a.cent_bf || !a.cn2p) return false;
+    if (!a.is_bf16 || (a.d != 64 && a.d != 128) || !a.cent_bf || !a.cn2p || !a.xnorm) return false;
     return tc_layout(a).total <= (size_t)kSmemLimit;
 }
 
 cudaError_t km_pack(const KmArgs &a, cudaStream_t s)
 {
     const TcLayout L = tc_layout(a);
-    km_pack_kernel<<<a.BH * a.nroles, 256, 0, s>>>(a, L.Cpad);
+    const int P = a.BH * a.nroles;
+    // the per-problem maxima are folded in with atomicMax: start them (and the rest) at 0
+    const cudaError_t e = cudaMemsetAsync(a.cn2p, 0, sizeof(float) * (size_t)P * (L.Cpad + 4), s);
+    if (e != cudaSuccess) return e;
+    km_pack_kernel<<<dim3(P, kPackSplit), 256, 0, s>>>(a, L.Cpad);
+    return cudaGetLastError();
+}
+
+cudaError_t km_norms(const KmArgs &a, cudaStream_t s)
+{
+    km_norms_kernel<<<dim3((a.N + 255) / 256, a.BH * a.nroles), 256, 0, s>>>(a);
     return cudaGetLastError();
 }
 

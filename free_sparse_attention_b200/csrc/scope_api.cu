@@ -96,6 +96,7 @@ KmArgs km_base(const scope_params &p, const WsLayout &L, void *ws)
     a.chunk_hist = at<int32_t>(ws, L.chunk_hist);
     a.cent_bf = at<__nv_bfloat16>(ws, L.cent_bf);
     a.cn2p = at<float>(ws, L.cn2p);
+    a.xnorm = at<float>(ws, L.xnorm);
     a.unsure_list = at<int32_t>(ws, L.unsure_list);
     a.unsure_count = at<int32_t>(ws, L.unsure_count);
     a.nchunk = (int)D.nchunk;
@@ -301,6 +302,7 @@ WsLayout ws_layout(const scope_params &p)
     const long long Cpad = (D.Cs + 15) / 16 * 16;
     L.cent_bf = take(sizeof(__nv_bfloat16) * D.P * 2 * Cpad * D.d);
     L.cn2p = take(sizeof(float) * D.P * (Cpad + 4));
+    L.xnorm = take(sizeof(float) * D.P * D.N);
     L.unsure_list = take(sizeof(int32_t) * D.P * D.N);
     L.unsure_count = take(4 * sizeof(int32_t));
     L.q_cent = take(sizeof(double) * D.BH * p.Cq * p.d);

@@ -94,7 +94,8 @@ struct Unit {
 
 // Keys are visited kBatch at a time per thread (keys j0 + k * kSelThreads + tid): the codes
 // and table entries of the batch are all loaded before any of them is used, so a thread
-// keeps 3 kBatch independent shared-memory loads in flight instead of one key's chain.
+// keeps 3 kBatch independent shared-memory loads in flight instead of one key's chain, and
+// every pass loads the next batch's codes (from L2) while it works on the current one.
 constexpr int kBatch = 2;
 
 // Codes of one batch, clamped to [0, Cm) so that a malformed caller-supplied code cannot read
@@ -271,6 +272,94 @@ struct SelectOut {
     long long rank;   // keys before it in the ranking
 };
 
+constexpr int kSampleStride = 8;     // the window sample takes one key batch in 8
+constexpr int kWindowMinN = 16384;   // below this the sample would be too small to matter
+
+// Predicts the bin of the first level's Top-p crossing from the keys of every
+// kSampleStride-th batch (their count and mass histogram over the first level's bins, and
+// the bin where their cumulative mass reaches rho times their total), then widens it to a
+// window of bins [wlo, whi] whose sampled counts, scaled up, stay within kCap / 2 keys.  The
+// window is only a guess: the caller checks it against the full histogram.  All threads call;
+// [wlo, whi] is empty (wlo > whi) when the sample finds no crossing.
+__device__ void predict_window(const SelSmem &S, const Unit &u, double rho, double hi, double scale,
+                               int &wlo, int &whi)
+{
+    const int tid = threadIdx.x;
+    for (int b = tid; b < kBins; b += kSelThreads) {
+        S.cnt[b] = 0;
+        S.mhi[b] = 0;
+        S.mlo[b] = 0;
+    }
+    __syncthreads();
+    for (int j0 = 0; j0 < u.N; j0 += kSampleStride * kBatch * kSelThreads) {
+        const KeyBatch kb = load_batch(u, j0);
+        double sc[kBatch], uw[kBatch];
+        batch_scores(S, u, kb, sc);
+        batch_weights(u, sc, uw);
+#pragma unroll
+        for (int k = 0; k < kBatch; ++k) {
+            if (!kb.v[k]) continue;
+            const int b = vbin(sc[k], hi, scale);
+            atomicAdd(&S.cnt[b], 1);
+            const unsigned long long W = weight_mass(uw[k], u);
+            atomicAdd(&S.mhi[b], W >> 32);
+            atomicAdd(&S.mlo[b], W & 0xffffffffull);
+        }
+    }
+    __syncthreads();
+    unsigned long long th = 0, tl = 0, tc = 0;
+    const int b0 = tid * kBinsPerThread;
+    for (int q = 0; q < kBinsPerThread; ++q) {
+        th += S.mhi[b0 + q];
+        tl += S.mlo[b0 + q];
+        tc += (unsigned long long)S.cnt[b0 + q];
+    }
+    unsigned long long tot[3];
+    block_excl_scan3(th, tl, tc, S.ured, tot);
+    const double target = rho * mass_to_double(tot[0], tot[1]);
+    if (tid == 0) S.misc[4] = -1;
+    __syncthreads();
+    {
+        unsigned long long eh = th, el = tl;
+        for (int q = 0; q < kBinsPerThread; ++q) {
+            const unsigned long long ih = eh + S.mhi[b0 + q], il = el + S.mlo[b0 + q];
+            if (!(mass_to_double(eh, el) >= target) && mass_to_double(ih, il) >= target) S.misc[4] = b0 + q;
+            eh = ih;
+            el = il;
+        }
+    }
+    __syncthreads();
+    if (tid == 0) {
+        const int bs = S.misc[4];
+        int lo = bs, hi2 = bs;
+        if (bs >= 0) {
+            long long est = (long long)S.cnt[bs] * kSampleStride;
+            for (bool grow = true; grow;) {
+                grow = false;
+                if (lo > 0 && est + (long long)S.cnt[lo - 1] * kSampleStride <= kCap / 2) {
+                    --lo;
+                    est += (long long)S.cnt[lo] * kSampleStride;
+                    grow = true;
+                }
+                if (hi2 < kBins - 1 && est + (long long)S.cnt[hi2 + 1] * kSampleStride <= kCap / 2) {
+                    ++hi2;
+                    est += (long long)S.cnt[hi2] * kSampleStride;
+                    grow = true;
+                }
+            }
+            S.misc[4] = lo;
+            S.misc[5] = hi2;
+        } else {
+            S.misc[4] = 1;
+            S.misc[5] = 0;
+        }
+    }
+    __syncthreads();
+    wlo = S.misc[4];
+    whi = S.misc[5];
+    __syncthreads();
+}
+
 // Finds the first key of the ranking at which the cumulative weight reaches the target.
 // mass_mode: weight = softmax mass, target = rho * (total mass); else weight = 1 and
 // target = count (1 <= count <= N).  Called by all threads of the block.
@@ -291,9 +380,18 @@ __device__ SelectOut block_select(const SelSmem &S, const Unit &u, bool mass_mod
     bool have_target = !mass_mode;
     const int tid = threadIdx.x;
     SelectOut out{smax, 0, 0};
+    // Mass mode: a histogram of every kSampleStride-th batch of keys predicts the bin where
+    // the first level's crossing lies, and a window of bins around it (about kCap / 2 keys
+    // by the sample's counts) is gathered during the first full pass, so that the separate
+    // gather pass is skipped whenever the crossing bin falls inside the window.
+    int wlo = 1, whi = 0;   // empty window
+    if (mass_mode && u.N >= kWindowMinN && hi > lo)
+        predict_window(S, u, rho, hi, (double)kBins / (hi - lo), wlo, whi);
 
     for (int iter = 0; iter < kMaxLevels + 3; ++iter) {
         const double scale = (hi > lo) ? (double)kBins / (hi - lo) : 0.0;
+        const bool gather_window = iter == 0 && wlo <= whi;
+        if (tid == 0) S.misc[3] = 0;
         for (int b = tid; b < kBins; b += kSelThreads) {
             S.cnt[b] = 0;
             S.mhi[b] = 0;
@@ -301,8 +399,10 @@ __device__ SelectOut block_select(const SelSmem &S, const Unit &u, bool mass_mod
         }
         __syncthreads();
         double cmin = DBL_MAX, cmax = -DBL_MAX, umx = 0.0;
+        KeyBatch next = load_batch(u, 0);
         for (int j0 = 0; j0 < u.N; j0 += kBatch * kSelThreads) {
-            const KeyBatch kb = load_batch(u, j0);
+            const KeyBatch kb = next;
+            if (j0 + kBatch * kSelThreads < u.N) next = load_batch(u, j0 + kBatch * kSelThreads);
             double sc[kBatch], uw[kBatch];
             batch_scores(S, u, kb, sc);
             if (mass_mode) batch_weights(u, sc, uw);
@@ -318,6 +418,14 @@ __device__ SelectOut block_select(const SelSmem &S, const Unit &u, bool mass_mod
                     const unsigned long long W = weight_mass(uw[k], u);
                     atomicAdd(&S.mhi[b], W >> 32);
                     atomicAdd(&S.mlo[b], W & 0xffffffffull);
+                    if (gather_window && b >= wlo && b <= whi) {
+                        const int slot = atomicAdd(&S.misc[3], 1);
+                        if (slot < kCap) {
+                            S.cs[slot] = s;
+                            S.cj[slot] = j;
+                            S.cw[slot] = W;
+                        }
+                    }
                 }
                 cmin = fmin(cmin, s);
                 cmax = fmax(cmax, s);
@@ -395,11 +503,47 @@ __device__ SelectOut block_select(const SelSmem &S, const Unit &u, bool mass_mod
             if (nb > kCap) {
                 if (tid == 0) set_status(status, SCOPE_DEV_SELECT_TIE);
             }
-            // gather the crossing bin's keys
+            // the crossing bin's keys: from the window gathered during this pass when the
+            // bin lies inside it (the window's keys of other bins are dropped), else by
+            // another pass over every key
+            bool have = false;
+            if (gather_window && bstar >= wlo && bstar <= whi && S.misc[3] <= kCap) {
+                const int nwin = S.misc[3];
+                double ks[kCap / kSelThreads];
+                int kj[kCap / kSelThreads];
+                unsigned long long kw[kCap / kSelThreads];
+                bool keep[kCap / kSelThreads];
+#pragma unroll
+                for (int q = 0; q < kCap / kSelThreads; ++q) {
+                    const int i = q * kSelThreads + tid;
+                    keep[q] = i < nwin && vbin(S.cs[i], hi, scale) == bstar;
+                    if (keep[q]) {
+                        ks[q] = S.cs[i];
+                        kj[q] = S.cj[i];
+                        kw[q] = S.cw[i];
+                    }
+                }
+                if (tid == 0) S.misc[1] = 0;
+                __syncthreads();
+#pragma unroll
+                for (int q = 0; q < kCap / kSelThreads; ++q)
+                    if (keep[q]) {
+                        const int slot = atomicAdd(&S.misc[1], 1);
+                        S.cs[slot] = ks[q];
+                        S.cj[slot] = kj[q];
+                        S.cw[slot] = kw[q];
+                    }
+                __syncthreads();
+                have = S.misc[1] == nb;   // every key of the bin was in the window
+                __syncthreads();
+            }
+            if (!have) {
             if (tid == 0) S.misc[1] = 0;
             __syncthreads();
+            KeyBatch next = load_batch(u, 0);
             for (int j0 = 0; j0 < u.N; j0 += kBatch * kSelThreads) {
-                const KeyBatch kb = load_batch(u, j0);
+                const KeyBatch kb = next;
+                if (j0 + kBatch * kSelThreads < u.N) next = load_batch(u, j0 + kBatch * kSelThreads);
                 double sc[kBatch];
                 batch_scores(S, u, kb, sc);
 #pragma unroll
@@ -418,6 +562,7 @@ __device__ SelectOut block_select(const SelSmem &S, const Unit &u, bool mass_mod
                 }
             }
             __syncthreads();
+            }
             const int n = min(S.misc[1], kCap);
             if (n == 0) {   // the gather pass always finds the crossing bin's keys
                 if (tid == 0) set_status(status, SCOPE_DEV_SELECT_TIE);
@@ -517,7 +662,7 @@ __global__ void sel_check_kernel(SelArgs a)
 }
 
 // Top-p count p_c and base count b_c (Eqs. 7-8).  grid (Cq, BH).
-__global__ void __launch_bounds__(kSelThreads) sel_topp_kernel(SelArgs a)
+__global__ void __launch_bounds__(kSelThreads, 2) sel_topp_kernel(SelArgs a)
 {
     extern __shared__ __align__(16) char smem_raw[];
     const SelSmem S = carve(smem_raw, a.Cm, a.d);
@@ -545,7 +690,7 @@ __global__ void __launch_bounds__(kSelThreads) sel_topp_kernel(SelArgs a)
     }
     const double smax = __dmul_rn(u.inv, __dadd_rn(__dadd_rn(tmax[0], tmax[1]), tmax[2]));
     const double smin = __dmul_rn(u.inv, __dadd_rn(__dadd_rn(tmin[0], tmin[1]), tmin[2]));
-    // Key weights u_j = E^T E^H E^W <= 1 (each exponential table peaks at 1), so masses are
+    // Key weights u_j = exp(s_j - smax) <= 1 (smax bounds every logit), so masses are
     // quantised against 1: at most N 2^-64 of absolute error in total.  That stays below
     // 1e-9 of the total mass Z >= max_j u_j unless the largest weight is tiny, in which
     // case the selection runs again normalised by the largest weight itself.
@@ -700,8 +845,10 @@ __global__ void __launch_bounds__(kSelThreads) sel_mask_kernel(SelArgs a)
     __syncthreads();
     // word w of the row holds keys 32 w .. 32 w + 31; a batch covers kBatch x 16 words, word
     // j0 / 32 + k * 16 + warp of batch j0 from warp `warp`
+    KeyBatch next = load_batch(u, 0);
     for (int j0 = 0; j0 < a.N; j0 += kBatch * kSelThreads) {
-        const KeyBatch kb = load_batch(u, j0);
+        const KeyBatch kb = next;
+        if (j0 + kBatch * kSelThreads < a.N) next = load_batch(u, j0 + kBatch * kSelThreads);
         double sc[kBatch];
         batch_scores(S, u, kb, sc);
 #pragma unroll

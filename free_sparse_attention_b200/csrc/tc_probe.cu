@@ -31,7 +31,7 @@ __global__ void __launch_bounds__(128, 1)
     unsigned char *sb = sm + (size_t)nbox * kProbeM * 128;     // [nbox][N rows][128 B]
     uint64_t *bar = reinterpret_cast<uint64_t *>(sb + (size_t)nbox * N * 128);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar + 1);
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int tid = threadIdx.x, warp = tid >> 5;
     // 16-byte chunk j (of K/8) of row r: box j/8, position r*128 + ((j%8) ^ (r%8))*16
     for (int i = tid; i < kProbeM * (K / 8); i += blockDim.x) {
         const int r = i / (K / 8), j = i % (K / 8);
