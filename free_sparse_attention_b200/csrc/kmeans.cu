@@ -438,7 +438,7 @@ __global__ void __launch_bounds__(128) sort_scatter_kernel(KmArgs a)
 // member count (one rounding).  bf16 inputs whose channel range starts and ends on an
 // even channel are read two channels (4 bytes) per load.
 constexpr int kUpdThreads = 256;
-constexpr int kUpdUnroll = 8;
+constexpr int kUpdUnroll = 16;
 
 // Value and ulp exponent of one input element (bf16: 8 significant bits, fp32: 24); a
 // subnormal gives INT_MIN (no usable bound), 0 gives INT_MAX (no ulp).

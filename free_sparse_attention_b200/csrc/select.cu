@@ -276,15 +276,40 @@ constexpr int kSampleStride = 8;     // the window sample takes one key batch in
 constexpr int kWindowMinN = 16384;   // below this the sample would be too small to matter
 
 // Predicts the bin of the first level's Top-p crossing from the keys of every
-// kSampleStride-th batch (their count and mass histogram over the first level's bins, and
-// the bin where their cumulative mass reaches rho times their total), then widens it to a
-// window of bins [wlo, whi] whose sampled counts, scaled up, stay within kCap / 2 keys.  The
-// window is only a guess: the caller checks it against the full histogram.  All threads call;
-// [wlo, whi] is empty (wlo > whi) when the sample finds no crossing.
-__device__ void predict_window(const SelSmem &S, const Unit &u, double rho, double hi, double scale,
+// kSampleStride-th batch.  The first level's value range [lo, hi] (the bounds from the
+// tables on entry) is narrowed to the sampled logits' range widened by 1/64 of it on each
+// side: keys outside it land in the end bins, which keeps the binning monotone, and the
+// bins become fine where the keys are.  The sample's count and mass histogram then gives
+// the bin where its cumulative mass reaches rho times its total, widened to a window of bins
+// [wlo, whi] whose sampled counts, scaled up, stay within kCap / 2 keys.  The window is only a
+// guess: the caller checks it against the full histogram.  All threads call; [wlo, whi] is
+// empty (wlo > whi) when the sample finds no crossing.
+__device__ void predict_window(const SelSmem &S, const Unit &u, double rho, double &hi, double &lo,
                                int &wlo, int &whi)
 {
     const int tid = threadIdx.x;
+    {
+        double cmin = DBL_MAX, cmax = -DBL_MAX;
+        for (int j0 = 0; j0 < u.N; j0 += kSampleStride * kBatch * kSelThreads) {
+            const KeyBatch kb = load_batch(u, j0);
+            double sc[kBatch];
+            batch_scores(S, u, kb, sc);
+#pragma unroll
+            for (int k = 0; k < kBatch; ++k)
+                if (kb.v[k]) {
+                    cmin = fmin(cmin, sc[k]);
+                    cmax = fmax(cmax, sc[k]);
+                }
+        }
+        cmin = block_min(cmin, S.red);
+        cmax = block_max(cmax, S.red);
+        if (cmax > cmin) {
+            const double pad = (cmax - cmin) * (1.0 / 64.0);
+            hi = fmin(hi, cmax + pad);
+            lo = fmax(lo, cmin - pad);
+        }
+    }
+    const double scale = (double)kBins / (hi - lo);
     for (int b = tid; b < kBins; b += kSelThreads) {
         S.cnt[b] = 0;
         S.mhi[b] = 0;
@@ -366,7 +391,8 @@ __device__ void predict_window(const SelSmem &S, const Unit &u, double rho, doub
 // umax_out (mass mode): the largest key weight, found in the first histogram pass.
 __device__ SelectOut block_select(const SelSmem &S, const Unit &u, bool mass_mode, double rho,
                                   long long count, double smax, double smin, int32_t *status,
-                                  double *umax_out = nullptr, int32_t *save_hist = nullptr)
+                                  double *umax_out = nullptr, int32_t *save_hist = nullptr,
+                                  double *range_out = nullptr)
 {
     Levels L;
     L.n = 0;
@@ -385,8 +411,11 @@ __device__ SelectOut block_select(const SelSmem &S, const Unit &u, bool mass_mod
     // by the sample's counts) is gathered during the first full pass, so that the separate
     // gather pass is skipped whenever the crossing bin falls inside the window.
     int wlo = 1, whi = 0;   // empty window
-    if (mass_mode && u.N >= kWindowMinN && hi > lo)
-        predict_window(S, u, rho, hi, (double)kBins / (hi - lo), wlo, whi);
+    if (mass_mode && u.N >= kWindowMinN && hi > lo) predict_window(S, u, rho, hi, lo, wlo, whi);
+    if (range_out) {
+        range_out[0] = hi;   // the first level's value range (the mask kernel bins with it)
+        range_out[1] = lo;
+    }
 
     for (int iter = 0; iter < kMaxLevels + 3; ++iter) {
         const double scale = (hi > lo) ? (double)kBins / (hi - lo) : 0.0;
@@ -700,9 +729,10 @@ __global__ void __launch_bounds__(kSelThreads, 2) sel_topp_kernel(SelArgs a)
     SelectOut so{smax, 0, 0};
     const size_t unit = (size_t)bh * a.Cq + c;
     int32_t *hist = a.hist ? a.hist + unit * kBins : nullptr;
+    double range[2] = {smax, smin};   // the first level's value range of the saved counts
     if (a.rho < 1.0) {
         double umax = 1.0;
-        so = block_select(S, u, true, a.rho, 0, smax, smin, a.status, &umax, hist);
+        so = block_select(S, u, true, a.rho, 0, smax, smin, a.status, &umax, hist, range);
         if (umax < (double)a.N * 0x1p-64 * 1e9 && umax > 0.0) {
             u.inv_umax = 1.0 / umax;
             so = block_select(S, u, true, a.rho, 0, smax, smin, a.status);
@@ -723,6 +753,8 @@ __global__ void __launch_bounds__(kSelThreads, 2) sel_topp_kernel(SelArgs a)
         st[3] = (double)so.j;
         st[4] = (double)p;
         st[5] = saved ? 1.0 : 0.0;
+        st[6] = range[0];
+        st[7] = range[1];
     }
 }
 
@@ -793,7 +825,7 @@ __global__ void __launch_bounds__(kSelThreads) sel_mask_kernel(SelArgs a)
     u.sref = a.state[unit * 8];
     u.inv_umax = 1.0;
     const double *st = a.state + unit * 8;
-    const double hi = st[0], lo = st[1];
+    const double hi = st[6], lo = st[7];   // the value range of the saved level-0 counts
     const double scale = (hi > lo) ? (double)kBins / (hi - lo) : 0.0;
     // Either the exact last selected key (s*, j*) is known -- the Top-p boundary when r_c =
     // p_c, or a count-based select -- or the level-0 counts saved by the Top-p kernel give the
