@@ -13,7 +13,10 @@
 // a target.  Keys are histogrammed into 2048 bins by value; the crossing bin is
 // resolved exactly (its keys gathered and ranked in shared memory) when it holds at
 // most 2048 keys, otherwise it is binned again over its own value range; keys with
-// identical logits are binned by index instead.
+// identical logits are binned by index instead.  For the Top-p mass, a sample of one key
+// batch in eight first narrows the first level's range to the sampled logits and predicts
+// the crossing bin; the keys of a window of bins around it are gathered during the full
+// pass, so the separate gather pass only runs when the crossing bin falls outside it.
 //
 // The softmax mass of key j is w_j = exp(s_j - s_ref), s_ref an upper bound of every
 // logit: t = (s_j - s_ref) log2 e in binary64 is split into n + f (n an integer, f in
@@ -877,10 +880,13 @@ __global__ void __launch_bounds__(kSelThreads) sel_mask_kernel(SelArgs a)
     __syncthreads();
     // word w of the row holds keys 32 w .. 32 w + 31; a batch covers kBatch x 16 words, word
     // j0 / 32 + k * 16 + warp of batch j0 from warp `warp`
-    KeyBatch next = load_batch(u, 0);
-    for (int j0 = 0; j0 < a.N; j0 += kBatch * kSelThreads) {
+    // this pass is bound by the latency of the code loads (L2): two batches are in flight
+    constexpr int kStep = kBatch * kSelThreads;
+    KeyBatch next = load_batch(u, 0), next2 = load_batch(u, kStep);
+    for (int j0 = 0; j0 < a.N; j0 += kStep) {
         const KeyBatch kb = next;
-        if (j0 + kBatch * kSelThreads < a.N) next = load_batch(u, j0 + kBatch * kSelThreads);
+        next = next2;
+        if (j0 + 2 * kStep < a.N) next2 = load_batch(u, j0 + 2 * kStep);
         double sc[kBatch];
         batch_scores(S, u, kb, sc);
 #pragma unroll
