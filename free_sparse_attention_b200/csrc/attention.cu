@@ -1,6 +1,6 @@
 // Sparse attention over each query cluster's selected original keys and values
-// (SCOPE, arXiv 2608.12780, abstract: "sparse attention is then computed over the
-// selected original keys and values"; review page, forward_implications[1]).
+// (SCOPE, arXiv 2608.12780, abstract: the attention runs over the original keys and values
+// each cluster selected, not over centroids; review page, forward_implications[1]).
 //
 //   O_i = sum_{j in S_c} softmax_j(q_i . k_j / sqrt d) v_j,   c = cluster of query i.
 //

@@ -1,5 +1,5 @@
-// Rank correlation of the Eq. 6 proxy logits with the exact logits (review page, the skeptic's
-// concrete test: "the rank correlation between Eq. (6) proxy logits and true logits").
+// Rank correlation of the Eq. 6 proxy logits with the exact logits (review page: the test the
+// skeptic asks for, how well the proxy ranking of the keys follows the true one).
 //
 // For each sampled query i of head (b, h) in cluster c: Spearman's rho over all N keys, the
 // Pearson correlation of the two vectors of average ranks (tied values share the mean of

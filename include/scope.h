@@ -69,7 +69,7 @@ typedef enum { SCOPE_F32 = 0, SCOPE_BF16 = 1 } scope_dtype;
 
 /* k_head handling (scope_params.khead_mode).  ONLINE: Eqs. 9-10, every cluster is
  * topped up to the head's k_head (the method).  OFF: the ablation the review page
- * proposes (significance; forward_implications: "disable the online k_head"): k_head is
+ * proposes (significance; forward_implications: the online k_head switched off): k_head is
  * still computed and reported, but r_c = b_c (hybrid Top-p / fixed Top-k only). */
 typedef enum { SCOPE_KHEAD_ONLINE = 0, SCOPE_KHEAD_OFF = 1 } scope_khead_mode;
 
@@ -265,8 +265,8 @@ scope_status scope_selection_recall(const scope_params *p, const void *Q, const 
                                     void *scratch, size_t scratch_bytes, void *stream);
 
 /*
- * Rank correlation of the proxy with the true logits (review page, the skeptic's concrete
- * test: "the rank correlation between Eq. (6) proxy logits and true logits").  For every
+ * Rank correlation of the proxy with the true logits (review page: the test the skeptic asks
+ * for, how well the Eq. 6 proxy ranking of the keys follows the true one).  For every
  * sampled query g = (b*H + h)*N + i: spearman[s] = Spearman's rho over the N keys of head
  * (b, h) between x_j = q_i . k_j (exact, binary64, channels in order) and y_j = s~_{c,j}, the
  * Eq. 6 proxy logits of its cluster c = q_assign[g]: the Pearson correlation of the two
@@ -283,7 +283,7 @@ scope_status scope_rank_correlation(const scope_params *p, const void *Q, const 
                                     size_t scratch_bytes, void *stream);
 
 /*
- * Channel permutation for the review page's ablation "random channel partition"
+ * Channel permutation for the review page's ablation that partitions the channels at random
  * (significance): Y[b,h,n,e] = X[b,h,n,perm[e]] for e < d.  One permutation applied to
  * both Q and K leaves every logit q.k unchanged, so the layer run on the permuted Q and K
  * (and the original V) is SCOPE with the key subspaces T, H, W made of the channel subsets
