@@ -13,14 +13,27 @@ SRC = os.path.join(HERE, "scope_oracle.c")
 LIB = os.path.join(HERE, "liboracle.so")
 
 
+FLAGS = ["-O2", "-std=c11", "-fopenmp", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared"]
+# AddressSanitizer and UndefinedBehaviorSanitizer instrumentation (any report aborts)
+SANITIZE = ["-fsanitize=address,undefined", "-fno-sanitize-recover=all", "-fno-omit-frame-pointer", "-g"]
+
+
 def build(force: bool = False) -> str:
+    # SCOPE_ORACLE_LIB: use an already-built library instead (the sanitizer test's build)
+    if os.environ.get("SCOPE_ORACLE_LIB"):
+        return os.environ["SCOPE_ORACLE_LIB"]
     if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= os.path.getmtime(SRC):
         return LIB
-    cmd = ["gcc", "-O2", "-std=c11", "-fopenmp", "-ffp-contract=off", "-fno-fast-math",
-           "-fPIC", "-shared", "-o", LIB + ".tmp", SRC, "-lm"]
-    subprocess.run(cmd, check=True)
+    subprocess.run(["gcc", *FLAGS, "-o", LIB + ".tmp", SRC, "-lm"], check=True)
     os.replace(LIB + ".tmp", LIB)
     return LIB
+
+
+def build_sanitized(out: str) -> str:
+    """The oracle with ASan + UBSan, to `out` (the process that loads it must preload the
+    sanitizer runtimes, e.g. LD_PRELOAD of gcc's libasan.so and libubsan.so)."""
+    subprocess.run(["gcc", *FLAGS, *SANITIZE, "-o", out, SRC, "-lm"], check=True)
+    return out
 
 
 if __name__ == "__main__":
