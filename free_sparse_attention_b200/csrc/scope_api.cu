@@ -2,6 +2,8 @@
 // sequences of the five entry points declared in include/scope.h.
 #include "common.cuh"
 
+#include <nvtx3/nvToolsExt.h>
+
 #include <algorithm>
 #include <cmath>
 
@@ -10,6 +12,16 @@ using namespace scope;
 namespace {
 
 constexpr size_t kAlign = 256;
+
+// An NVTX range over a scope (NVTX 3 is header-only and costs a load and a branch unless a
+// profiler has injected itself): the host side of every entry point and of the layer's three
+// stages, so that a timeline shows which launches belong to which stage.
+struct NvtxRange {
+    explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange &) = delete;
+    NvtxRange &operator=(const NvtxRange &) = delete;
+};
 
 size_t align_up(size_t x)
 {
@@ -366,6 +378,7 @@ scope_status scope_cluster_queries(const scope_params *p, const void *Q, const i
                                    uint16_t *q_assign, int32_t *q_sizes, void *ws,
                                    size_t ws_bytes, void *stream)
 {
+    NvtxRange nvtx("scope_cluster_queries");
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     WsLayout L;
     scope_status st = begin(p, ws, ws_bytes, L, s);
@@ -387,6 +400,7 @@ scope_status scope_cluster_keys(const scope_params *p, const void *K, const int3
                                 const double *init_cent, double *k_centroids, uint16_t *k_codes,
                                 void *ws, size_t ws_bytes, void *stream)
 {
+    NvtxRange nvtx("scope_cluster_keys");
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     WsLayout L;
     scope_status st = begin(p, ws, ws_bytes, L, s);
@@ -415,6 +429,7 @@ scope_status scope_build_lut_and_select(const scope_params *p, const double *q_c
                                         int32_t *final_counts, uint32_t *sel_mask, void *ws,
                                         size_t ws_bytes, void *stream)
 {
+    NvtxRange nvtx("scope_build_lut_and_select");
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     WsLayout L;
     scope_status st = begin(p, ws, ws_bytes, L, s);
@@ -518,6 +533,7 @@ scope_status scope_sparse_attention(const scope_params *p, const void *Q, const 
                                     const uint32_t *sel_mask, const int32_t *final_counts,
                                     void *O, void *ws, size_t ws_bytes, void *stream)
 {
+    NvtxRange nvtx("scope_sparse_attention");
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     WsLayout L;
     scope_status st = begin(p, ws, ws_bytes, L, s);
@@ -532,6 +548,7 @@ scope_status scope_sparse_attention(const scope_params *p, const void *Q, const 
 scope_status scope_dense_attention(const scope_params *p, const void *Q, const void *K, const void *V, void *O,
                                    void *ws, size_t ws_bytes, void *stream)
 {
+    NvtxRange nvtx("scope_dense_attention");
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     WsLayout L;
     scope_status st = begin(p, ws, ws_bytes, L, s);
@@ -543,6 +560,7 @@ scope_status scope_dense_attention(const scope_params *p, const void *Q, const v
 scope_status scope_rope3d(const scope_params *p, double base, const void *Q, const void *K, void *Qr, void *Kr,
                           void *stream)
 {
+    NvtxRange nvtx("scope_rope3d");
     scope_status st = validate(p);
     if (st != SCOPE_OK) return st;
     if ((st = validate_rope(*p, base)) != SCOPE_OK) return st;
@@ -561,6 +579,7 @@ scope_status scope_attention_layer(const scope_params *p, const scope_layer_sche
                                    const int32_t *k_init_idx, void *O, void *Qr, void *Kr, void *ws,
                                    size_t ws_bytes, void *stream)
 {
+    NvtxRange nvtx("scope_attention_layer");
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     WsLayout L;
     scope_status st = begin(p, ws, ws_bytes, L, s);
@@ -586,6 +605,7 @@ scope_status scope_selection_recall(const scope_params *p, const void *Q, const 
                                     double frac, double *recall_sel, double *recall_proxy,
                                     void *scratch, size_t scratch_bytes, void *stream)
 {
+    NvtxRange nvtx("scope_selection_recall");
     scope_status st = validate(p);
     if (st != SCOPE_OK) return st;
     if (!ok_ptr(Q) || !ok_ptr(K) || !ok_ptr(q_assign) || !ok_ptr(q_centroids) || !ok_ptr(k_centroids) ||
@@ -644,6 +664,7 @@ scope_status scope_rank_correlation(const scope_params *p, const void *Q, const 
                                     const int64_t *samples, int n_samples, double *spearman, void *scratch,
                                     size_t scratch_bytes, void *stream)
 {
+    NvtxRange nvtx("scope_rank_correlation");
     scope_status st = validate(p);
     if (st != SCOPE_OK) return st;
     if (!ok_ptr(Q) || !ok_ptr(K) || !ok_ptr(q_assign) || !ok_ptr(q_centroids) || !ok_ptr(k_centroids) ||
@@ -685,6 +706,7 @@ scope_status scope_rank_correlation(const scope_params *p, const void *Q, const 
 scope_status scope_permute_channels(const scope_params *p, const void *X, const int32_t *perm, void *Y,
                                     void *stream)
 {
+    NvtxRange nvtx("scope_permute_channels");
     scope_status st = validate(p);
     if (st != SCOPE_OK) return st;
     if (!ok_ptr(X) || !ok_ptr(perm) || !ok_ptr(Y) || X == Y) return SCOPE_ERR_INVALID_ARGUMENT;
@@ -720,6 +742,7 @@ scope_status scope_forward(const scope_params *p, const void *Q, const void *K, 
                            const scope_intermediates *inter, void *ws, size_t ws_bytes,
                            void *stream)
 {
+    NvtxRange nvtx("scope_forward");
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     WsLayout L;
     scope_status st = begin(p, ws, ws_bytes, L, s);
@@ -751,6 +774,7 @@ scope_status scope_forward(const scope_params *p, const void *Q, const void *K, 
     if (mark(0) != cudaSuccess) return SCOPE_ERR_CUDA;
 
     // stage 1: query clustering and the three key-subspace clusterings, one launch set
+    nvtxRangePushA("scope/clustering");
     KmArgs a = km_base(*p, L, ws);
     a.role0 = 0;
     a.nroles = 1 + key_roles(*p);
@@ -761,20 +785,25 @@ scope_status scope_forward(const scope_params *p, const void *Q, const void *K, 
     a.ds = p->d;
     cudaError_t e = km_run(a, p->iters, s);
     if (e == cudaSuccess) e = zero_unused_codes(*p, kk, s);
+    nvtxRangePop();
     if (e != cudaSuccess || mark(1) != cudaSuccess) return SCOPE_ERR_CUDA;
 
     // stage 2: LUT, proxy logits, Top-p, k_head, top-up, masks
     SelArgs sa = sel_args(*p, L, ws, qc, qs, kc, kk, tp, bc, kh, fc, mk);
+    nvtxRangePushA("scope/selection");
     e = select_run(sa, s);
+    nvtxRangePop();
     if (e != cudaSuccess || mark(2) != cudaSuccess) return SCOPE_ERR_CUDA;
 
     // stage 3: attention; the last clustering iteration already grouped the queries
     const Dims D = dims_of(*p);
     AttnArgs t = attn_args(*p, L, ws, Q, K, V, O, a.perm, a.nroles * D.N, a.off, a.nroles * (a.Cs + 1), mk, fc);
+    nvtxRangePushA("scope/attention");
     e = attention_items(t, s);
-    if (e != cudaSuccess || mark(3) != cudaSuccess) return SCOPE_ERR_CUDA;
-    e = attention_kernel(t, s);
-    if (e != cudaSuccess || mark(4) != cudaSuccess) return SCOPE_ERR_CUDA;
+    const bool marked = e == cudaSuccess && mark(3) == cudaSuccess;
+    if (marked) e = attention_kernel(t, s);
+    nvtxRangePop();
+    if (!marked || e != cudaSuccess || mark(4) != cudaSuccess) return SCOPE_ERR_CUDA;
     return SCOPE_OK;
 }
 
