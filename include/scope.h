@@ -75,7 +75,7 @@ typedef enum { SCOPE_KHEAD_ONLINE = 0, SCOPE_KHEAD_OFF = 1 } scope_khead_mode;
 
 /* Key clustering (scope_params.key_clustering).  SUBSPACES: the method, three k-means over
  * the temporal / height / width channel ranges.  FULL: the ablation the review page asks
- * for (significance; falsifier: "full-dimensional cluster scoring"): one k-means of the
+ * for (significance; falsifier: scoring with clusters over all channels): one k-means of the
  * keys over all d channels into Cm centroids, so that the proxy of Eq. 6 becomes the
  * cluster-level s~_cj = q_c . mu_{z_j} / sqrt d.  k_codes row 0 then holds z_j and rows 1
  * and 2 are zero; selection reads it as a one-subspace product code with split (d, 0, 0),
@@ -122,7 +122,7 @@ typedef struct {
 size_t scope_workspace_bytes(const scope_params *p);
 
 /*
- * Query clustering (abstract: "query clusters"; review page, major_comments[0]: the
+ * Query clustering (abstract: the queries are grouped into clusters; review page, major_comments[0]: the
  * cluster centroid q_c; major_comments[1]: Cq = 300).  Lloyd k-means on all d
  * channels, params->iters iterations.  One iteration assigns every token to its
  * nearest centroid in squared Euclidean distance (lowest index on a tie), then moves
