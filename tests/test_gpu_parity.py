@@ -19,6 +19,11 @@ pytestmark = pytest.mark.gpu
 RAGGED = Workload("ragged", 1, 2, 3, 9, 11, 16, 24, 24, "bf16", 13, 17, seed=5)
 MID = Workload("mid", 1, 2, 5, 16, 20, 44, 42, 42, "bf16", 50, 60, seed=6)
 COG2 = COGVIDEOX.with_(H=2)
+# channel splits whose key windows take 1, 2, 3, 5, 6 and 7 sixteen-channel MMA steps (the
+# tensor-core assignment issues a fully unrolled product sequence per step count)
+ODD = [Workload("split8_104_16", 1, 2, 4, 9, 13, 8, 104, 16, "bf16", 21, 19, seed=9),
+       Workload("split24_80_24", 1, 1, 3, 10, 11, 24, 80, 24, "bf16", 17, 23, seed=10),
+       Workload("split40_72_16", 1, 1, 5, 6, 13, 40, 72, 16, "bf16", 19, 18, seed=11)]
 CONFIGS = [TINY, RAGGED, MID]
 
 
@@ -35,7 +40,7 @@ def _run(w):
     return x, device_inputs(w, x)
 
 
-@pytest.mark.parametrize("w", CONFIGS + [COG2], ids=lambda w: w.name)
+@pytest.mark.parametrize("w", CONFIGS + [COG2] + ODD, ids=lambda w: w.name)
 def test_clustering_matches_oracle_exactly(w):
     x, t = _run(w)
     p = capi.Params.from_workload(w)
