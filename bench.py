@@ -303,6 +303,9 @@ def run_scope(args, w):
     khead_stats = {"min": int(kh.min().item()), "mean": float(kh.mean().item()), "max": int(kh.max().item()),
                    "clusters_topped_up": int((it["final_counts"] > it["base_counts"]).sum().item()),
                    "clusters": int(it["final_counts"].numel())}
+    # Top-p decisions within 1e-6 / 1e-5 of a tie (the band in which the binary64 reference
+    # logs a near tie and the selection may differ from it), counted by the selection kernel
+    near_ties = capi.get_selection_stats(p, ws)
     del it
 
     def mk_events():
@@ -462,7 +465,7 @@ def run_scope(args, w):
             "clustering_tensor": clust_flops / (stage_ms[0] * 1e-3) / 1e12 / pk["bf16_sustained"],
             "selection_hbm": sel_bytes / (stage_ms[1] * 1e-3) / 1e9 / pk["hbm_gbs"]},
         "density": density, "effective_tflop_per_layer": flops / 1e12,
-        "ms_per_step_mean": ms_mean, "k_head": khead_stats,
+        "ms_per_step_mean": ms_mean, "k_head": khead_stats, "near_ties": near_ties,
         "dense_sdpa_ms": dense_ms,
         "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),

@@ -14,7 +14,8 @@ import torch
 from .workloads import Workload
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libscope.so")
+# SCOPE_LIB_PATH selects another build of the library (the debug build's tests use it)
+LIB_PATH = os.environ.get("SCOPE_LIB_PATH") or os.path.join(HERE, "libscope.so")
 
 SCOPE_F32, SCOPE_BF16 = 0, 1
 STATUS = {0: "SCOPE_OK", 1: "SCOPE_ERR_INVALID_ARGUMENT", 2: "SCOPE_ERR_UNSUPPORTED",
@@ -24,7 +25,8 @@ DEV_BAD_INIT_INDEX, DEV_SELECT_TIE, DEV_BAD_ASSIGN = 0x1, 0x2, 0x4
 
 EXPORTS = ("scope_workspace_bytes", "scope_cluster_queries", "scope_cluster_keys",
            "scope_build_lut_and_select", "scope_sparse_attention", "scope_forward",
-           "scope_status_string", "scope_get_device_status", "scope_build_lut_and_select_noalloc",
+           "scope_status_string", "scope_get_device_status", "scope_get_selection_stats",
+           "scope_build_lut_and_select_noalloc",
            "scope_selection_recall", "scope_permute_channels", "scope_dense_attention",
            "scope_rope3d", "scope_layer_is_dense", "scope_attention_layer",
            "scope_rank_correlation_scratch_bytes", "scope_rank_correlation", "scope_check_wait_timeout",
@@ -130,6 +132,8 @@ def lib() -> ctypes.CDLL:
         L.scope_status_string.argtypes = [i]
         L.scope_get_device_status.restype = i
         L.scope_get_device_status.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_int32)]
+        L.scope_get_selection_stats.restype = i
+        L.scope_get_selection_stats.argtypes = [ctypes.POINTER(Params), vp, vp, ctypes.POINTER(ctypes.c_int32)]
         L.scope_check_wait_timeout.restype = i
         L.scope_check_wait_timeout.argtypes = [P, ctypes.c_uint64, vp, sz, vp]
         L.scope_tc_accumulation_probe.restype = i
@@ -383,6 +387,14 @@ def device_status_code(ws, stream=None):
     out = ctypes.c_int32(0)
     code = lib().scope_get_device_status(_ptr(ws), _stream(stream), ctypes.byref(out))
     return int(code), int(out.value)
+
+
+def get_selection_stats(p, ws, stream=None) -> dict:
+    """Top-p decisions of the last selection on `ws` and how many lay within 1e-6 / 1e-5 of a
+    tie (the margin the binary64 reference logs; scope_get_selection_stats)."""
+    out = (ctypes.c_int32 * 4)()
+    _check("scope_get_selection_stats", lib().scope_get_selection_stats(ctypes.byref(p), _ptr(ws), _stream(stream), out))
+    return {"decisions": int(out[0]), "margin_below_1e-6": int(out[1]), "margin_below_1e-5": int(out[2])}
 
 
 def get_device_status(ws, stream=None) -> int:

@@ -260,7 +260,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int g = gw * 16 + lane, q = g >> 5, r0 = (g & 31) * 4;
                     int rr[4];
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) rr[k] = rowbase + perm[min(q * kBM + r0 + k, nq - 1)];
+                    for (int k = 0; k < 4; ++k)
+                        rr[k] = rowbase + SCOPE_DCHECK(perm[min(q * kBM + r0 + k, nq - 1)], a.N, a.status);
 #pragma unroll
                     for (int b = 0; b < NB; ++b)
                         tma_gather4(sbase + L::kQ + q * L::kQTile + b * (kBM * 128) + r0 * 128, &tmQ, b * 64,
@@ -294,8 +295,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __syncwarp();
                 if (active)
                     tma_gather4(sbase + (is_k ? L::kK : L::kV) + s * L::kKVTile + blk * (kBN * 128) + grp * 512,
-                                tm, blk * 64, rowbase + g0.x, rowbase + g0.y, rowbase + g0.z,
-                                rowbase + g0.w, full);
+                                tm, blk * 64, rowbase + SCOPE_DCHECK(g0.x, a.N, a.status),
+                                rowbase + SCOPE_DCHECK(g0.y, a.N, a.status), rowbase + SCOPE_DCHECK(g0.z, a.N, a.status),
+                                rowbase + SCOPE_DCHECK(g0.w, a.N, a.status), full);
                 g0 = g1;
                 if (t + 2 < T) g1 = keys_of(t + 2);
                 ++stage_it;
@@ -501,7 +503,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool valid = q * kBM + row < nq;
             __nv_bfloat16 *dst = nullptr;
             if (valid) {
-                const int tok = a.perm[(size_t)bh * a.perm_bh + q0 + q * kBM + row];
+                const int tok = SCOPE_DCHECK(a.perm[(size_t)bh * a.perm_bh + q0 + q * kBM + row], a.N, a.status);
                 dst = reinterpret_cast<__nv_bfloat16 *>(a.O) + ((size_t)bh * a.N + tok) * D;
             }
 #pragma unroll 1

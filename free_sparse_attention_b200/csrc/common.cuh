@@ -64,7 +64,7 @@ struct WsLayout {
     size_t cent32, cent64T, cnorm, cnrm2, cslack, perm, off, chunk_hist, cent_bf, cn2p, xnorm, unsure_list,
         unsure_count;
     size_t q_cent, q_assign, q_sizes, k_cent, k_codes, k_sizes;
-    size_t topp, base, khead, final_cnt, mask, sel_state, sel_hist;
+    size_t topp, base, khead, final_cnt, mask, sel_state, sel_hist, sel_stats;
     size_t q_perm, q_off, q_hist, work_items, attn_counter, key_lists;
     size_t total;
 };
@@ -88,6 +88,7 @@ struct SelArgs {
     uint32_t *mask;           // [BH, Cq, nw]
     double *state;            // [BH*Cq, 8] per-unit selection state
     int32_t *hist;            // [BH*Cq, 2048] level-0 key counts of the Top-p pass (or NULL)
+    int32_t *stats;           // [4] Top-p decisions: made, with margin < 1e-6, < 1e-5 (or NULL)
     int BH, N, d, dt, dh, dw, Cq, Cm, nw;
     double rho, inv_sqrt_d;
     int kfix;
@@ -183,6 +184,24 @@ __device__ __forceinline__ void set_status(int32_t *status, int bits)
 {
     if (status) atomicOr(status, bits);
 }
+
+// Debug builds (-DSCOPE_DEBUG): the internal indices the kernels derive (token rows taken from
+// permutations and key lists, cluster indices about to be stored) are checked before use; an
+// index outside [0, n) sets SCOPE_DEV_DEBUG_CHECK and is replaced by 0, so the access stays in
+// bounds and the kernel carries on.  Release builds compile the check away.
+#ifdef SCOPE_DEBUG
+__device__ __forceinline__ long long debug_index(long long i, long long n, int32_t *status)
+{
+    if (i < 0 || i >= n) {
+        set_status(status, SCOPE_DEV_DEBUG_CHECK);
+        return 0;
+    }
+    return i;
+}
+#define SCOPE_DCHECK(i, n, status) ((int)::scope::debug_index((i), (n), (status)))
+#else
+#define SCOPE_DCHECK(i, n, status) (i)
+#endif
 
 // Appends `value` for every lane with `take` to list[*count ...] with one atomic per
 // warp.  All 32 lanes of the warp must call it.

@@ -224,7 +224,7 @@ __global__ void __launch_bounds__(kAssignThreads) km_assign_fast_kernel(KmArgs a
             int j = j0 + ty * 8 + t;
             if (j < a.N) {
                 bool sure = min2L[t] > minU[t];
-                R.assign[(size_t)bh * R.assign_bh + j] = sure ? (uint16_t)idxL[t] : kUnsure;
+                R.assign[(size_t)bh * R.assign_bh + j] = sure ? (uint16_t)SCOPE_DCHECK(idxL[t], R.C, a.status) : kUnsure;
                 unsure = !sure;
                 entry = bh * a.N + j;
             }
@@ -418,7 +418,7 @@ __global__ void __launch_bounds__(128) sort_scatter_kernel(KmArgs a)
         const int rank = __popc(peers & ((1u << lane) - 1u));
         int base = (lane == leader && z >= 0) ? cnt[z] : 0;
         base = __shfl_sync(0xffffffffu, base, leader);
-        if (z >= 0) perm[base + rank] = j;
+        if (z >= 0) perm[SCOPE_DCHECK(base + rank, a.N, a.status)] = j;
         __syncwarp();
         if (lane == leader && z >= 0) cnt[z] = base + __popc(peers);
         __syncwarp();
@@ -508,14 +508,14 @@ __global__ void __launch_bounds__(kUpdThreads) km_update_kernel(KmArgs a)
         for (; m + kUpdUnroll <= m1; m += kUpdUnroll) {
             int tok[kUpdUnroll];
 #pragma unroll
-            for (int q = 0; q < kUpdUnroll; ++q) tok[q] = perm[m + q];
+            for (int q = 0; q < kUpdUnroll; ++q) tok[q] = SCOPE_DCHECK(perm[m + q], a.N, a.status);
             uint32_t bits[kUpdUnroll];
 #pragma unroll
             for (int q = 0; q < kUpdUnroll; ++q) bits[q] = load(tok[q]);
 #pragma unroll
             for (int q = 0; q < kUpdUnroll; ++q) take(bits[q]);
         }
-        for (; m < m1; ++m) take(load(perm[m]));
+        for (; m < m1; ++m) take(load(SCOPE_DCHECK(perm[m], a.N, a.status)));
 #pragma unroll
         for (int h = 0; h < CH; ++h) {
             psum[threadIdx.x * CH + h] = acc[h];

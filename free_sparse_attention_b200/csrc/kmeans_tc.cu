@@ -505,7 +505,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
         float maxnm = 0.f, maxsl = 0.f, maxres = 0.f;
         // the unit's (problem, tile) advance incrementally; role constants change per problem
         int p = (int)(ub / t.TT), tile = (int)(ub % t.TT);
-        int bh = 0, r = 0, ks = 1;
+        int bh = 0, r = 0, ks = 1, Cn = 1;
         Chunks k{16, 1, 16};
         uint16_t *assign = nullptr;
         long long assign_bh = 0;
@@ -517,6 +517,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
                 const RoleDesc &R = a.role[a.role0 + r];
                 ks = window_of(R.ch0, R.dm).ks;
                 k = chunks_of(R.C);
+                Cn = R.C;
                 assign = R.assign;
                 assign_bh = R.assign_bh;
                 if (!warp_wait(&bars->b_full, nb & 1, abort_flag, a.status)) break;
@@ -620,7 +621,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
                 if (j < a.N) {
                     const float E = bound_E(ks, xn, maxnm, maxres, maxsl);
                     const bool sure = (m2 - m1) > (E + E) * (1.0f + 0x1p-20f);
-                    assign[(size_t)bh * assign_bh + j] = sure ? (uint16_t)idx : kUnsureTc;
+                    assign[(size_t)bh * assign_bh + j] = sure ? (uint16_t)SCOPE_DCHECK(idx, Cn, a.status) : kUnsureTc;
                     unsure = !sure;
                 }
                 warp_append(unsure, bh * a.N + j, a.unsure_list + (size_t)r * a.BH * a.N, a.unsure_count + r);

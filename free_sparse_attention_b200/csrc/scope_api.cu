@@ -232,6 +232,7 @@ SelArgs sel_args(const scope_params &p, const WsLayout &L, void *ws, const doubl
     a.mask = mask;
     a.state = at<double>(ws, L.sel_state);
     a.hist = at<int32_t>(ws, L.sel_hist);
+    a.stats = at<int32_t>(ws, L.sel_stats);
     a.BH = (int)D.BH;
     a.N = (int)D.N;
     a.d = p.d;
@@ -330,6 +331,7 @@ WsLayout ws_layout(const scope_params &p)
     L.mask = take(sizeof(uint32_t) * D.BH * p.Cq * D.nw);
     L.sel_state = take(sizeof(double) * 8 * D.BH * p.Cq);
     L.sel_hist = take(sizeof(int32_t) * kSelBins * D.BH * p.Cq);
+    L.sel_stats = take(4 * sizeof(int32_t));
     L.work_items = take(sizeof(int4) * D.BH * ((D.N + kAttnTile - 1) / kAttnTile + p.Cq));
     L.key_lists = take(sizeof(int32_t) * D.BH * p.Cq * ((D.N + 3) / 4 * 4));
     L.total = o;
@@ -371,6 +373,20 @@ scope_status scope_get_device_status(const void *ws, void *stream, int32_t *out)
     *out = v;
     if (v & SCOPE_DEV_TIMEOUT) return SCOPE_ERR_TIMEOUT;
     return v ? SCOPE_ERR_DEVICE_CHECK : SCOPE_OK;
+}
+
+scope_status scope_get_selection_stats(const scope_params *p, const void *ws, void *stream, int32_t *out)
+{
+    if (!ws || !out || validate(p) != SCOPE_OK) return SCOPE_ERR_INVALID_ARGUMENT;
+    const WsLayout L = ws_layout(*p);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int32_t v[4] = {0, 0, 0, 0};
+    cudaError_t e = cudaMemcpyAsync(v, static_cast<const char *>(ws) + L.sel_stats, sizeof(v),
+                                    cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return SCOPE_ERR_CUDA;
+    for (int k = 0; k < 4; ++k) out[k] = v[k];
+    return SCOPE_OK;
 }
 
 scope_status scope_cluster_queries(const scope_params *p, const void *Q, const int32_t *init_idx,

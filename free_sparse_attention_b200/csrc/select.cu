@@ -273,6 +273,7 @@ struct SelectOut {
     double s;
     int j;
     long long rank;   // keys before it in the ranking
+    double margin;    // mass mode: min(|mass before - target|, |mass through it - target|) / Z
 };
 
 constexpr int kSampleStride = 8;     // the window sample takes one key batch in 8
@@ -408,7 +409,7 @@ __device__ SelectOut block_select(const SelSmem &S, const Unit &u, bool mass_mod
     double target = 0.0;
     bool have_target = !mass_mode;
     const int tid = threadIdx.x;
-    SelectOut out{smax, 0, 0};
+    SelectOut out{smax, 0, 0, INFINITY};
     // Mass mode: a histogram of every kSampleStride-th batch of keys predicts the bin where
     // the first level's crossing lies, and a window of bins around it (about kCap / 2 keys
     // by the sample's counts) is gathered during the first full pass, so that the separate
@@ -614,6 +615,8 @@ __device__ SelectOut block_select(const SelSmem &S, const Unit &u, bool mass_mod
             }
             __syncthreads();
             int pos = -1;
+            if (tid == 0) S.red[31] = INFINITY;
+            __syncthreads();
             if (mass_mode) {
                 if (tid < 32) {
                     unsigned long long rh = bhi, rl = blo;
@@ -624,7 +627,17 @@ __device__ SelectOut block_select(const SelSmem &S, const Unit &u, bool mass_mod
                         warp_scan3(h, l, z);
                         const bool ok = idx < n && mass_to_double(rh + h, rl + l) >= target;
                         const unsigned bal = __ballot_sync(0xffffffffu, ok);
-                        if (bal) pos = base + __ffs(bal) - 1;
+                        if (bal) {
+                            pos = base + __ffs(bal) - 1;
+                            // the decision's closeness to a tie, as the oracle measures it:
+                            // the masses before and through the crossing key against rho Z
+                            if (tid == pos - base) {
+                                const double incl = mass_to_double(rh + h, rl + l);
+                                const double excl = mass_to_double(rh + h - (W >> 32), rl + l - (W & 0xffffffffull));
+                                const double Z = target / rho;
+                                S.red[31] = fmin(fabs(incl - target), fabs(excl - target)) / Z;
+                            }
+                        }
                         rh += __shfl_sync(0xffffffffu, h, 31);
                         rl += __shfl_sync(0xffffffffu, l, 31);
                     }
@@ -640,6 +653,7 @@ __device__ SelectOut block_select(const SelSmem &S, const Unit &u, bool mass_mod
             out.s = S.cs[i];
             out.j = S.cj[i];
             out.rank = bcnt + pos;
+            if (mass_mode) out.margin = S.red[31];
             __syncthreads();
             return out;
         }
@@ -741,6 +755,11 @@ __global__ void __launch_bounds__(kSelThreads, 2) sel_topp_kernel(SelArgs a)
             so = block_select(S, u, true, a.rho, 0, smax, smin, a.status);
         }
         p = so.rank + 1;
+        if (tid == 0 && a.stats) {
+            atomicAdd(&a.stats[0], 1);
+            if (so.margin < 1e-6) atomicAdd(&a.stats[1], 1);
+            if (so.margin < 1e-5) atomicAdd(&a.stats[2], 1);
+        }
     }
     // rho = 1 selects every key: no pass ran, so the level-0 counts are only saved when a
     // count-based selection will need them (never: r = N then)
@@ -948,6 +967,10 @@ cudaError_t select_run(const SelArgs &a, cudaStream_t s)
     cudaFuncSetAttribute(sel_topp_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     cudaFuncSetAttribute(sel_mask_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     dim3 grid(a.Cq, a.BH);
+    if (a.stats) {
+        const cudaError_t e = cudaMemsetAsync(a.stats, 0, 4 * sizeof(int32_t), s);
+        if (e != cudaSuccess) return e;
+    }
     sel_check_kernel<<<256, 256, 0, s>>>(a);
     sel_topp_kernel<<<grid, kSelThreads, smem, s>>>(a);
     sel_khead_kernel<<<a.BH, 256, 0, s>>>(a);

@@ -66,6 +66,8 @@ typedef enum { SCOPE_F32 = 0, SCOPE_BF16 = 1 } scope_dtype;
 #define SCOPE_DEV_TIMEOUT        0x8   /* an on-chip pipeline wait gave up (~4 s); outputs invalid */
 #define SCOPE_DEV_BAD_COUNTS     0x10  /* a selection mask row holds fewer keys than its r_c; the
                                           missing keys were taken as key 0 */
+#define SCOPE_DEV_DEBUG_CHECK    0x20  /* debug builds (-DSCOPE_DEBUG) only: an internal index was
+                                          out of range; the access used element 0 instead */
 
 /* k_head handling (scope_params.khead_mode).  ONLINE: Eqs. 9-10, every cluster is
  * topped up to the head's k_head (the method).  OFF: the ablation the review page
@@ -406,6 +408,17 @@ const char *scope_status_string(scope_status s);
  * that call are invalid, the context stays usable), SCOPE_ERR_DEVICE_CHECK for any other
  * bit, SCOPE_ERR_CUDA if the copy or the synchronisation failed. */
 scope_status scope_get_device_status(const void *ws, void *stream, int32_t *out);
+
+/* Top-p decision statistics of the last selection that used `ws` (scope_forward or
+ * scope_build_lut_and_select with parameters `p`): synchronises `stream` and writes
+ * out[0] = Top-p decisions made (one per unit (b, h, c) when rho < 1), out[1] = those whose
+ * margin is below 1e-6, out[2] = below 1e-5, out[3] = 0.  The margin of a decision is
+ * min(|M_{p-1} - rho Z|, |M_p - rho Z|) / Z, with M_r the softmax mass of the first r keys of
+ * the ranking and Z the total (Eq. 7; the same quantity the binary64 reference logs as a near
+ * tie below 1e-6), computed from the fixed-point masses of the selection (relative error below
+ * 3e-7).  SCOPE_ERR_INVALID_ARGUMENT for a NULL pointer or invalid `p`, SCOPE_ERR_CUDA if the
+ * copy or the synchronisation failed. */
+scope_status scope_get_selection_stats(const scope_params *p, const void *ws, void *stream, int32_t *out);
 
 #ifdef __cplusplus
 }

@@ -236,6 +236,18 @@ def test_device_status_rejections(L):
     assert L.scope_get_device_status(ctypes.c_void_p(1 << 20), None, None) == 1
 
 
+def test_selection_stats_rejections(L):
+    """scope_get_selection_stats validates before touching the device."""
+    from free_sparse_attention_b200.workloads import COGVIDEOX
+    p = capi.Params.from_workload(COGVIDEOX)
+    out = (ctypes.c_int32 * 4)()
+    f = L.scope_get_selection_stats
+    assert f(ctypes.byref(p), None, None, out) == 1
+    assert f(ctypes.byref(p), ctypes.c_void_p(1 << 20), None, None) == 1
+    bad = capi.Params.from_workload(COGVIDEOX, rho=0.0)
+    assert f(ctypes.byref(bad), ctypes.c_void_p(1 << 20), None, out) == 1
+
+
 def test_wait_timeout_check_rejections(L):
     """scope_check_wait_timeout validates on the host before launching anything."""
     from free_sparse_attention_b200.workloads import COGVIDEOX

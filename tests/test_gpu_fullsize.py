@@ -69,6 +69,11 @@ def _run(w, heads_to_check, rhos=None):
         O, it = capi.forward(p, t["q"], t["k"], t["v"], t["qi"], t["ki"], ws=ws, intermediates=True)
         torch.cuda.synchronize()
         assert capi.get_device_status(ws) == 0
+        # the selection's own count of Top-p decisions near a tie (every unit decides once)
+        st = capi.get_selection_stats(p, ws)
+        assert st["decisions"] == (w.B * w.H * w.Cq if rho < 1.0 else 0), st
+        assert 0 <= st["margin_below_1e-6"] <= st["margin_below_1e-5"] <= st["decisions"], st
+        print(f"rho={rho}: Top-p decisions {st}")
         n = it["q_sizes"].double()
         r = it["final_counts"].double()
         densities[rho] = float((n * r).sum() / (w.B * w.H * w.N * w.N))
