@@ -390,11 +390,11 @@ def device_status_code(ws, stream=None):
 
 
 def get_selection_stats(p, ws, stream=None) -> dict:
-    """Top-p decisions of the last selection on `ws` and how many lay within 1e-6 / 1e-5 of a
+    """Top-p decisions of the last selection on `ws` and how many lay within 1e-6 / 3e-7 of a
     tie (the margin the binary64 reference logs; scope_get_selection_stats)."""
     out = (ctypes.c_int32 * 4)()
     _check("scope_get_selection_stats", lib().scope_get_selection_stats(ctypes.byref(p), _ptr(ws), _stream(stream), out))
-    return {"decisions": int(out[0]), "margin_below_1e-6": int(out[1]), "margin_below_1e-5": int(out[2])}
+    return {"decisions": int(out[0]), "margin_below_1e-6": int(out[1]), "margin_below_3e-7": int(out[2])}
 
 
 def get_device_status(ws, stream=None) -> int:

@@ -88,7 +88,7 @@ struct SelArgs {
     uint32_t *mask;           // [BH, Cq, nw]
     double *state;            // [BH*Cq, 8] per-unit selection state
     int32_t *hist;            // [BH*Cq, 2048] level-0 key counts of the Top-p pass (or NULL)
-    int32_t *stats;           // [4] Top-p decisions: made, with margin < 1e-6, < 1e-5 (or NULL)
+    int32_t *stats;           // [4] Top-p decisions: made, with margin < 1e-6, < 3e-7 (or NULL)
     int BH, N, d, dt, dh, dw, Cq, Cm, nw;
     double rho, inv_sqrt_d;
     int kfix;

@@ -758,7 +758,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) sel_topp_kernel(SelArgs a)
         if (tid == 0 && a.stats) {
             atomicAdd(&a.stats[0], 1);
             if (so.margin < 1e-6) atomicAdd(&a.stats[1], 1);
-            if (so.margin < 1e-5) atomicAdd(&a.stats[2], 1);
+            if (so.margin < 3e-7) atomicAdd(&a.stats[2], 1);
         }
     }
     // rho = 1 selects every key: no pass ran, so the level-0 counts are only saved when a

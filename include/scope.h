@@ -412,11 +412,13 @@ scope_status scope_get_device_status(const void *ws, void *stream, int32_t *out)
 /* Top-p decision statistics of the last selection that used `ws` (scope_forward or
  * scope_build_lut_and_select with parameters `p`): synchronises `stream` and writes
  * out[0] = Top-p decisions made (one per unit (b, h, c) when rho < 1), out[1] = those whose
- * margin is below 1e-6, out[2] = below 1e-5, out[3] = 0.  The margin of a decision is
+ * margin is below 1e-6, out[2] = below 3e-7, out[3] = 0.  The margin of a decision is
  * min(|M_{p-1} - rho Z|, |M_p - rho Z|) / Z, with M_r the softmax mass of the first r keys of
  * the ranking and Z the total (Eq. 7; the same quantity the binary64 reference logs as a near
  * tie below 1e-6), computed from the fixed-point masses of the selection (relative error below
- * 3e-7).  SCOPE_ERR_INVALID_ARGUMENT for a NULL pointer or invalid `p`, SCOPE_ERR_CUDA if the
+ * 3e-7, so only a decision with a margin below 3e-7 can differ from the binary64 one).  The
+ * margin is at most half the mass of the crossing key, so at large N a sizeable share of the
+ * decisions falls below 1e-6.  SCOPE_ERR_INVALID_ARGUMENT for a NULL pointer or invalid `p`, SCOPE_ERR_CUDA if the
  * copy or the synchronisation failed. */
 scope_status scope_get_selection_stats(const scope_params *p, const void *ws, void *stream, int32_t *out);
 

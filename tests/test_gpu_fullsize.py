@@ -72,7 +72,7 @@ def _run(w, heads_to_check, rhos=None):
         # the selection's own count of Top-p decisions near a tie (every unit decides once)
         st = capi.get_selection_stats(p, ws)
         assert st["decisions"] == (w.B * w.H * w.Cq if rho < 1.0 else 0), st
-        assert 0 <= st["margin_below_1e-6"] <= st["margin_below_1e-5"] <= st["decisions"], st
+        assert 0 <= st["margin_below_3e-7"] <= st["margin_below_1e-6"] <= st["decisions"], st
         print(f"rho={rho}: Top-p decisions {st}")
         n = it["q_sizes"].double()
         r = it["final_counts"].double()
