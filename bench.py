@@ -416,7 +416,31 @@ def run_scope(args, w):
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, device="cuda")
     # every step computes the same layer: its read-back output equals the device-resident run
     e2e_match = bool(torch.equal(Oh[0], Oh[1]) and torch.equal(Oh[0].cuda(), O_dev))
-    del dev2, O2, O_dev
+    del dev2, O2
+
+    # the same layer captured once into a CUDA graph and replayed (device-resident inputs):
+    # what the per-launch host overhead of the ~60 launches and memsets of a layer costs
+    graph = None
+    if world == 1:
+        try:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                capi.forward(p, dev["q"], dev["k"], dev["v"], dev["qi"], dev["ki"], ws=ws, out=O)
+            for _ in range(args.warmup):
+                g.replay()
+            torch.cuda.synchronize()
+            e0.record()
+            for _ in range(args.steps):
+                g.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            graph = {"ms_per_step": e0.elapsed_time(e1) / args.steps,
+                     "output_matches_device_run": bool(torch.equal(O, O_dev)),
+                     "device_status": capi.get_device_status(ws)}
+            del g
+        except Exception as ex:   # report, do not fail the bench line
+            graph = {"error": f"{type(ex).__name__}: {ex}"[:300]}
+    del O_dev
 
     # dense attention on the same shape (library comparator, not part of the path)
     dense_ms = None
@@ -474,6 +498,7 @@ def run_scope(args, w):
                               "copy streams under step i's layer",
                 "output_matches_device_run": e2e_match,
                 "serial": {"value": world * flops / (e2e_serial_ms * 1e-3) / 1e12, "ms_per_step": e2e_serial_ms}},
+        "graph": graph,
         "gpu_launches": kernels_per_forward(w.iters) * args.steps,
         "device_status": status,
         "clocks": clk,
