@@ -58,13 +58,15 @@ struct KmArgs {
     int32_t *unsure_count;    // [4], cleared before every assignment launch
 };
 
-// Workspace layout (byte offsets); computed identically by every entry point.
+// Workspace layout (byte offsets); computed identically by every entry point.  The selection
+// stage keeps its per-key bins in the key-list region, which only the attention stage
+// writes afterwards (2 bytes per key and unit fit in the 4 of a list entry).
 struct WsLayout {
     size_t status, counters;
     size_t cent32, cent64T, cnorm, cnrm2, cslack, perm, off, chunk_hist, cent_bf, cn2p, xnorm, unsure_list,
         unsure_count;
     size_t q_cent, q_assign, q_sizes, k_cent, k_codes, k_sizes;
-    size_t topp, base, khead, final_cnt, mask, sel_state, sel_hist, sel_stats;
+    size_t topp, base, khead, final_cnt, mask, sel_state, sel_hist, sel_stats, sel_lut;
     size_t q_perm, q_off, q_hist, work_items, attn_counter, key_lists;
     size_t total;
 };
@@ -88,6 +90,9 @@ struct SelArgs {
     uint32_t *mask;           // [BH, Cq, nw]
     double *state;            // [BH*Cq, 8] per-unit selection state
     int32_t *hist;            // [BH*Cq, 2048] level-0 key counts of the Top-p pass (or NULL)
+    uint16_t *bins;           // [BH*Cq, bins_stride] each key's level-0 bin (or NULL)
+    long long bins_stride;    // N rounded up to a multiple of 8
+    double *lut;              // [BH*Cq, 3*Cm] the Top-p kernel's tables (or NULL)
     int32_t *stats;           // [4] Top-p decisions: made, with margin < 1e-6, < 3e-7 (or NULL)
     int BH, N, d, dt, dh, dw, Cq, Cm, nw;
     double rho, inv_sqrt_d;

@@ -232,6 +232,9 @@ SelArgs sel_args(const scope_params &p, const WsLayout &L, void *ws, const doubl
     a.mask = mask;
     a.state = at<double>(ws, L.sel_state);
     a.hist = at<int32_t>(ws, L.sel_hist);
+    a.bins = at<uint16_t>(ws, L.key_lists);
+    a.bins_stride = (D.N + 7) / 8 * 8;
+    a.lut = at<double>(ws, L.sel_lut);
     a.stats = at<int32_t>(ws, L.sel_stats);
     a.BH = (int)D.BH;
     a.N = (int)D.N;
@@ -332,6 +335,7 @@ WsLayout ws_layout(const scope_params &p)
     L.sel_state = take(sizeof(double) * 8 * D.BH * p.Cq);
     L.sel_hist = take(sizeof(int32_t) * kSelBins * D.BH * p.Cq);
     L.sel_stats = take(4 * sizeof(int32_t));
+    L.sel_lut = take(sizeof(double) * 3 * p.Cm * D.BH * p.Cq);
     L.work_items = take(sizeof(int4) * D.BH * ((D.N + kAttnTile - 1) / kAttnTile + p.Cq));
     L.key_lists = take(sizeof(int32_t) * D.BH * p.Cq * ((D.N + 3) / 4 * 4));
     L.total = o;

@@ -27,10 +27,12 @@
 // where the mass of a prefix is within ~3e-7 (relative) of rho times the total, inside the
 // 1e-6 band in which the oracle logs a near tie.
 //
-// The Top-p kernel saves the count histogram of its first (full-range) pass; the mask
-// kernel uses it to find the bin where the r_c-th key of the ranking lies, so that one
-// pass over the keys writes the selected set (keys of higher bins set directly, the keys
-// of that bin ranked exactly in shared memory).
+// The Top-p kernel saves the count histogram of its first pass, every key's bin in that
+// pass (2 bytes per key) and its tables.  The mask kernel finds from the counts the bin
+// where the r_c-th key of the ranking lies (or takes the bin of the Top-p boundary key when
+// r_c = p_c), and one pass over the saved bins writes the selected set: keys of lower bins
+// (higher logits) are set directly, and only the keys of the boundary bin get their logit
+// computed again, to be compared with the boundary key or ranked exactly in shared memory.
 #include "common.cuh"
 
 #include <cfloat>
@@ -135,6 +137,14 @@ __device__ __forceinline__ void batch_scores(const SelSmem &S, const Unit &u, co
     }
 #pragma unroll
     for (int k = 0; k < kBatch; ++k) s[k] = __dmul_rn(u.inv, __dadd_rn(__dadd_rn(a[k], b[k]), c[k]));
+}
+
+// s_j of Eq. 6 for one key (the same operations as batch_scores)
+__device__ __forceinline__ double key_score(const SelSmem &S, const Unit &u, int j)
+{
+    const int zt = min((int)u.zt[j], u.Cm - 1), zh = min((int)u.zh[j], u.Cm - 1),
+              zw = min((int)u.zw[j], u.Cm - 1);
+    return __dmul_rn(u.inv, __dadd_rn(__dadd_rn(S.lut[zt], S.lut[u.Cm + zh]), S.lut[2 * u.Cm + zw]));
 }
 
 // Softmax weight of a key of logit s: exp(s - sref) = 2^n 2^f with t = (s - sref) log2 e
@@ -396,7 +406,7 @@ __device__ void predict_window(const SelSmem &S, const Unit &u, double rho, doub
 __device__ SelectOut block_select(const SelSmem &S, const Unit &u, bool mass_mode, double rho,
                                   long long count, double smax, double smin, int32_t *status,
                                   double *umax_out = nullptr, int32_t *save_hist = nullptr,
-                                  double *range_out = nullptr)
+                                  double *range_out = nullptr, uint16_t *save_bins = nullptr)
 {
     Levels L;
     L.n = 0;
@@ -419,6 +429,7 @@ __device__ SelectOut block_select(const SelSmem &S, const Unit &u, bool mass_mod
     if (range_out) {
         range_out[0] = hi;   // the first level's value range (the mask kernel bins with it)
         range_out[1] = lo;
+        range_out[2] = 0.0;  // set to 1 once the first level's counts (and bins) are saved
     }
 
     for (int iter = 0; iter < kMaxLevels + 3; ++iter) {
@@ -445,6 +456,7 @@ __device__ SelectOut block_select(const SelSmem &S, const Unit &u, bool mass_mod
                 if (!kb.v[k] || !in_candidates(L, s)) continue;
                 const int j = j0 + k * kSelThreads + tid;
                 const int b = L.jmode ? jbin(j, u.N) : vbin(s, hi, scale);
+                if (iter == 0 && save_bins) save_bins[j] = (uint16_t)b;
                 atomicAdd(&S.cnt[b], 1);
                 if (mass_mode) {
                     umx = fmax(umx, uw[k]);
@@ -467,8 +479,10 @@ __device__ SelectOut block_select(const SelSmem &S, const Unit &u, bool mass_mod
         cmin = block_min(cmin, S.red);
         cmax = block_max(cmax, S.red);
         if (mass_mode && iter == 0 && umax_out) *umax_out = block_max(umx, S.red);
-        if (iter == 0 && save_hist && !(cmin == cmax))   // the full-range counts, for the mask kernel
+        if (iter == 0 && save_hist && !(cmin == cmax)) {   // the first level's counts, for the mask kernel
             for (int b = tid; b < kBins; b += kSelThreads) save_hist[b] = S.cnt[b];
+            if (range_out) range_out[2] = 1.0;
+        }
         if (!L.jmode && cmin == cmax) {
             // every candidate has the same logit: the ranking among them is by index
             L.jmode = true;
@@ -746,10 +760,15 @@ __global__ void __launch_bounds__(kSelThreads, 2) sel_topp_kernel(SelArgs a)
     SelectOut so{smax, 0, 0};
     const size_t unit = (size_t)bh * a.Cq + c;
     int32_t *hist = a.hist ? a.hist + unit * kBins : nullptr;
-    double range[2] = {smax, smin};   // the first level's value range of the saved counts
+    // every key's first-level bin, kept beside the counts when the mask kernel can use them
+    uint16_t *bins = hist && a.bins && a.lut ? a.bins + unit * a.bins_stride : nullptr;
+    if (bins)   // the unit's tables, so that the mask kernel need not build them again
+        for (int i = tid; i < 3 * a.Cm; i += kSelThreads) a.lut[unit * 3 * a.Cm + i] = S.lut[i];
+    // the first level's value range of the saved counts, and whether they were saved
+    double range[3] = {smax, smin, 0.0};
     if (a.rho < 1.0) {
         double umax = 1.0;
-        so = block_select(S, u, true, a.rho, 0, smax, smin, a.status, &umax, hist, range);
+        so = block_select(S, u, true, a.rho, 0, smax, smin, a.status, &umax, hist, range, bins);
         if (umax < (double)a.N * 0x1p-64 * 1e9 && umax > 0.0) {
             u.inv_umax = 1.0 / umax;
             so = block_select(S, u, true, a.rho, 0, smax, smin, a.status);
@@ -761,9 +780,9 @@ __global__ void __launch_bounds__(kSelThreads, 2) sel_topp_kernel(SelArgs a)
             if (so.margin < 3e-7) atomicAdd(&a.stats[2], 1);
         }
     }
-    // rho = 1 selects every key: no pass ran, so the level-0 counts are only saved when a
-    // count-based selection will need them (never: r = N then)
-    const bool saved = hist && a.rho < 1.0 && smax > smin;
+    // The counts are saved only by a first level that binned by value (not when every logit
+    // is the same, and not at rho = 1, where no pass runs and r = N selects every key).
+    const bool saved = hist && range[2] != 0.0;
     if (tid == 0) {
         const long long b = p > a.kfix ? p : a.kfix;
         if (a.topp) a.topp[unit] = (int32_t)p;
@@ -836,7 +855,17 @@ __global__ void __launch_bounds__(kSelThreads) sel_mask_kernel(SelArgs a)
         }
         return;
     }
-    build_tables(a, S, bh, c);
+    const double *st = a.state + unit * 8;
+    // With the Top-p kernel's saved bins (and its copy of the tables), the pass below reads
+    // each key's first-level bin and computes a logit only for the keys of the boundary bin.
+    const bool use_bins = a.bins && a.lut && a.hist && st[5] != 0.0;
+    if (use_bins) {
+        const double *lut = a.lut + unit * 3 * a.Cm;
+        for (int i = tid; i < 3 * a.Cm; i += kSelThreads) S.lut[i] = lut[i];
+        __syncthreads();
+    } else {
+        build_tables(a, S, bh, c);
+    }
     Unit u;
     u.zt = a.codes + (size_t)bh * 3 * a.N;
     u.zh = u.zt + a.N;
@@ -846,7 +875,6 @@ __global__ void __launch_bounds__(kSelThreads) sel_mask_kernel(SelArgs a)
     u.inv = a.inv_sqrt_d;
     u.sref = a.state[unit * 8];
     u.inv_umax = 1.0;
-    const double *st = a.state + unit * 8;
     const double hi = st[6], lo = st[7];   // the value range of the saved level-0 counts
     const double scale = (hi > lo) ? (double)kBins / (hi - lo) : 0.0;
     // Either the exact last selected key (s*, j*) is known -- the Top-p boundary when r_c =
@@ -897,6 +925,56 @@ __global__ void __launch_bounds__(kSelThreads) sel_mask_kernel(SelArgs a)
     }
     if (tid == 0) S.misc[2] = 0;
     __syncthreads();
+    if (use_bins) {
+        // Bins are monotone in the logit (a lower bin holds strictly higher logits), so a key
+        // of a bin below the boundary bin is selected, one above it is not, and only the keys
+        // of the boundary bin need their logit: compared with (s*, j*), or gathered for ranking.
+        const bool gather = bstar >= 0;
+        const int bsel = gather ? bstar : vbin(s_star, hi, scale);
+        const uint16_t *bn = a.bins + unit * a.bins_stride;
+        // thread t takes keys 8 t .. 8 t + 7 of each step (one 16-byte load; rows are padded
+        // to a multiple of 8 keys); lanes 4 q .. 4 q + 3 fill word q of the warp's 8 words
+        constexpr int kPer = 8, kStep = kPer * kSelThreads;
+        auto load8 = [&](int j0) -> uint4 {
+            const int j = j0 + kPer * tid;
+            return j < a.N ? *reinterpret_cast<const uint4 *>(bn + j) : make_uint4(0u, 0u, 0u, 0u);
+        };
+        uint4 next = load8(0), next2 = load8(kStep);
+        for (int j0 = 0; j0 < a.N; j0 += kStep) {
+            const uint4 cur = next;
+            next = next2;
+            if (j0 + 2 * kStep < a.N) next2 = load8(j0 + 2 * kStep);
+            const uint32_t pair[4] = {cur.x, cur.y, cur.z, cur.w};
+            const int jb = j0 + kPer * tid;
+            uint32_t m8 = 0;
+#pragma unroll
+            for (int i = 0; i < kPer; ++i) {
+                const int j = jb + i;
+                const int b = (int)((pair[i >> 1] >> (16 * (i & 1))) & 0xffffu);
+                if (j >= a.N || b > bsel) continue;
+                bool sel = b < bsel;
+                if (b == bsel) {
+                    const double sj = key_score(S, u, j);
+                    if (gather) {
+                        const int slot = atomicAdd(&S.misc[2], 1);
+                        if (slot < kCap) {
+                            S.cs[slot] = sj;
+                            S.cj[slot] = j;
+                        }
+                    } else {
+                        sel = (sj > s_star) || (sj == s_star && j <= j_star);
+                    }
+                }
+                m8 |= (uint32_t)sel << i;
+            }
+            uint32_t bits = m8 << (8 * (lane & 3));
+            bits |= __shfl_xor_sync(0xffffffffu, bits, 1);
+            bits |= __shfl_xor_sync(0xffffffffu, bits, 2);
+            const int w = jb >> 5;
+            if ((lane & 3) == 0 && w < a.nw) row[w] = bits;
+        }
+        if (!gather) return;
+    } else {
     // word w of the row holds keys 32 w .. 32 w + 31; a batch covers kBatch x 16 words, word
     // j0 / 32 + k * 16 + warp of batch j0 from warp `warp`
     // this pass is bound by the latency of the code loads (L2): two batches are in flight
@@ -929,6 +1007,7 @@ __global__ void __launch_bounds__(kSelThreads) sel_mask_kernel(SelArgs a)
             const int w = (j0 + k * kSelThreads) / 32 + warp;
             if (lane == 0 && w < a.nw) row[w] = bits;
         }
+    }
     }
     if (bstar < 0) return;
     // rank the keys of b* (logit descending, index ascending) and add the first r - before

@@ -122,6 +122,43 @@ def test_explicit_initial_centroids_warm_start():
         np.testing.assert_array_equal(to_np(kc)[0, h], rk["centroids"])
 
 
+def test_equal_logits_with_spread_tables_and_a_topup():
+    """Every key carries the same three codes, so inside a cluster all logits are equal,
+    while the memberless centroids keep each table spread (its bounds differ).  The Top-p
+    pass then sees one logit value and bins nothing by value; with rho below alpha every
+    cluster is topped up to k_fix keys (Eq. 10), which the ranking by index makes the first
+    k_fix keys.  An earlier call on the same workspace leaves real first-level counts
+    behind, which the mask kernel must not take for this call's."""
+    w = W
+    rho = 0.0513   # rho N = 18.47: the Top-p count is 19 keys, far from a mass tie
+    p = capi.Params.from_workload(w, rho=rho)
+    ws = capi.alloc_workspace(p)
+    rng = np.random.default_rng(8)
+    BH = w.B * w.H
+    qc = rng.standard_normal((BH, w.Cq, w.d))
+    qs = (1 + rng.multinomial(w.N - w.Cq, np.full(w.Cq, 1.0 / w.Cq), size=BH)).astype(np.int32)
+    kc = rng.standard_normal((BH, w.Cm, w.d))
+    spread = rng.integers(0, w.Cm, (BH, 3, w.N)).astype(np.uint16)
+    equal = np.zeros((BH, 3, w.N), np.uint16)
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).reshape((w.B, w.H) + a.shape[1:]).cuda()
+    capi.build_lut_and_select(p, dev(qc), dev(qs), dev(kc), dev(spread), ws=ws)
+    out = capi.build_lut_and_select(p, dev(qc), dev(qs), dev(kc), dev(equal), ws=ws)
+    torch.cuda.synchronize()
+    assert capi.get_device_status(ws) == 0
+    g = {k: to_np(v).reshape((BH,) + tuple(v.shape[2:])) for k, v in out.items()}
+    for i in range(BH):
+        ref = oracle.select(qc[i], qs[i], kc[i], equal[i], (w.d_t, w.d_h, w.d_w), rho, w.alpha)
+        assert np.all(g["topp_counts"][i] == 19)
+        kfix = int(ref["r"][0])
+        assert kfix > 19 and np.all(ref["r"] == kfix)
+        first = np.zeros(p.nw, np.uint32)
+        for j in range(kfix):
+            first[j >> 5] |= np.uint32(1 << (j & 31))
+        assert np.all(ref["mask"] == first)
+        np.testing.assert_array_equal(g["final_counts"][i], ref["r"])
+        np.testing.assert_array_equal(g["sel_mask"][i].view(np.uint32), ref["mask"])
+
+
 def test_bad_init_index_sets_status():
     x = synth.layer_inputs(W)
     qi = x["q_init"].copy()
