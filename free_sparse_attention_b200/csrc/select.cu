@@ -946,26 +946,32 @@ __global__ void __launch_bounds__(kSelThreads) sel_mask_kernel(SelArgs a)
             if (j0 + 2 * kStep < a.N) next2 = load8(j0 + 2 * kStep);
             const uint32_t pair[4] = {cur.x, cur.y, cur.z, cur.w};
             const int jb = j0 + kPer * tid;
-            uint32_t m8 = 0;
+            const int nv = min(max(a.N - jb, 0), kPer);   // keys of this thread below N
+            // bit i: key jb + i lies below (lt) or in (eq) the boundary bin
+            uint32_t lt = 0, eq = 0;
 #pragma unroll
             for (int i = 0; i < kPer; ++i) {
+                const uint32_t b = (pair[i >> 1] >> (16 * (i & 1))) & 0xffffu;
+                lt |= (uint32_t)(b < (uint32_t)bsel) << i;
+                eq |= (uint32_t)(b == (uint32_t)bsel) << i;
+            }
+            const uint32_t valid = (1u << nv) - 1u;
+            uint32_t m8 = lt & valid;
+            eq &= valid;
+            while (eq) {   // the boundary bin's keys (a few per unit)
+                const int i = __ffs(eq) - 1;
+                eq &= eq - 1u;
                 const int j = jb + i;
-                const int b = (int)((pair[i >> 1] >> (16 * (i & 1))) & 0xffffu);
-                if (j >= a.N || b > bsel) continue;
-                bool sel = b < bsel;
-                if (b == bsel) {
-                    const double sj = key_score(S, u, j);
-                    if (gather) {
-                        const int slot = atomicAdd(&S.misc[2], 1);
-                        if (slot < kCap) {
-                            S.cs[slot] = sj;
-                            S.cj[slot] = j;
-                        }
-                    } else {
-                        sel = (sj > s_star) || (sj == s_star && j <= j_star);
+                const double sj = key_score(S, u, j);
+                if (gather) {
+                    const int slot = atomicAdd(&S.misc[2], 1);
+                    if (slot < kCap) {
+                        S.cs[slot] = sj;
+                        S.cj[slot] = j;
                     }
+                } else if ((sj > s_star) || (sj == s_star && j <= j_star)) {
+                    m8 |= 1u << i;
                 }
-                m8 |= (uint32_t)sel << i;
             }
             uint32_t bits = m8 << (8 * (lane & 3));
             bits |= __shfl_xor_sync(0xffffffffu, bits, 1);
