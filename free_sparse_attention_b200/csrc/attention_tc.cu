@@ -24,10 +24,11 @@
 //   S_q  = Q_q K^T     tcgen05.mma kind::f16, M=128, N=64 keys, K=d, fp32 in TMEM
 //   O_q += P_q V       M=128, N=d, K=64, P_q bf16 written by the softmax over the first
 //                      columns of its own S buffer (A operand from TMEM), V from smem
-// Both Q tiles reuse every gathered K/V tile.  S is double-buffered per Q tile (two
-// 64-column buffers; 2 x (2 x 64 + 128) = 512 TMEM columns at d = 128): the MMA thread
-// of tile q issues S(0), S(1), then P(t) V(t) followed by S(t+2) into the buffer P(t)
-// occupied, so the softmax of step t+1 runs while the tensor core works on step t.  A
+// Both Q tiles reuse every gathered K/V tile.  S has NSB 64-column buffers per Q tile,
+// as many as TMEM holds beside O (2 at d = 128: 2 x (2 x 64 + 128) = 512 columns; 3 at
+// d = 64): the MMA thread of tile q issues S(0) .. S(NSB-1), then P(t) V(t) followed by
+// S(t+NSB) into the buffer P(t) occupied, so the softmax of the next steps runs while the
+// tensor core works on step t.  A
 // thread's tcgen05.commit costs it roughly one pipe latency before its next MMA starts,
 // which is why each Q tile has its own issuing thread.  The softmax keeps a running row
 // maximum and rescales O (TMEM load/store) only when the maximum grows by more than
@@ -54,6 +55,13 @@ constexpr int kOtherRegs = 64;     //  + 2 warpgroups x 128 threads x 64 = 65536
 constexpr int kMaxStages = 8;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kRing = 4;           // work items fetched ahead by the scheduler thread
+constexpr int kMaxSB = 3;          // S buffers per Q tile, at most
+// S buffers per Q tile: as many 64-column buffers as TMEM holds beside the two O tiles
+// (d = 128: 2 x (2 x 64 + 128) = 512 columns; d = 64: 2 x (3 x 64 + 64) = 512)
+template <int D>
+struct SBuf {
+    static constexpr int n = D == 128 ? 2 : 3;
+};
 constexpr int kWarps = kThreads / 32;
 
 // max(a, b, c) in one instruction (the three-input form of max.f32 on sm_100)
@@ -69,7 +77,7 @@ struct __align__(8) Bars {
     uint64_t k_full[kMaxStages], k_empty[kMaxStages];
     uint64_t v_full[kMaxStages], v_empty[kMaxStages];
     // per Q tile and S buffer: S ready (MMA commit), P written (softmax), P V done (commit)
-    uint64_t s_full[kQT][2], p_full[kQT][2], o_done[kQT][2];
+    uint64_t s_full[kQT][kMaxSB], p_full[kQT][kMaxSB], o_done[kQT][kMaxSB];
     uint64_t o_free[kQT];  // epilogue has read O_q
     uint64_t item_full[kRing], item_empty[kRing];   // work-item ring (dynamic scheduler)
     uint64_t drain[kQT];                            // the issuing threads' last products
@@ -118,8 +126,8 @@ __device__ __forceinline__ void drain_wait(uint64_t *b, uint32_t parity, unsigne
 }
 
 // Shared memory: two Q tiles, a K ring and a V ring (bf16, 128-byte swizzled, K-major).
-// TMEM: two S buffers per Q tile (fp32, 64 columns each; P bf16 pairs over the first 32
-// columns of its own buffer) at q*128 + b*64, O_q (fp32, D columns) at 256 + q*D.
+// TMEM: NSB S buffers per Q tile (fp32, 64 columns each; P bf16 pairs over the first 32
+// columns of its own buffer) at (q NSB + b) 64, O_q (fp32, D columns) at 2 NSB 64 + q D.
 template <int D>
 struct Smem {
     static constexpr int kKS = D == 128 ? 5 : 8;       // K ring depth
@@ -167,7 +175,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             bar_init(&bars->v_empty[s], kMmaWarps);
         }
         for (int q = 0; q < kQT; ++q) {
-            for (int b = 0; b < 2; ++b) {
+            for (int b = 0; b < kMaxSB; ++b) {
                 bar_init(&bars->s_full[q][b], 1);
                 bar_init(&bars->p_full[q][b], 4);
                 bar_init(&bars->o_done[q][b], 1);
@@ -315,9 +323,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
         // ------------------------------------------------------------ MMA issuers (warps 14, 15)
         // Lane 0 of warp 14 + q issues Q tile q's products alone (lanes 1-31 wait at the end):
-        // S(0), S(1), then for every t: O += P(t) V(t), S(t+2).  S(t+2) reuses the buffer
-        // whose first columns hold P(t); issuing it after P(t) V(t) from the same thread keeps
-        // the in-order tensor pipe from overwriting P(t) early.  Both issuers consume every K
+        // S(0) .. S(NSB-1), then for every t: O += P(t) V(t), S(t+NSB).  S(t+NSB) reuses the
+        // buffer whose first columns hold P(t); issuing it after P(t) V(t) from the same thread
+        // keeps the in-order tensor pipe from overwriting P(t) early.  Both issuers consume every K
         // and V stage in the same order (an idle Q tile only waits for the data and releases
         // the stage), so the ring phases advance in step.
         if (lane == 0) {
@@ -325,6 +333,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             constexpr uint32_t idesc_qk = f16_idesc(kBM, kBN, false);
             constexpr uint32_t idesc_pv = f16_idesc(kBM, D, true);
             uint32_t k_it = 0, v_it = 0, q_it = 0, o_items = 0;
+            constexpr int NSB = SBuf<D>::n;
+            const uint32_t s_base = tmem + q * NSB * kBN, o_tm = tmem + kQT * NSB * kBN + q * D;
             uint32_t p_par = 0;   // bit b: parity of the next p_full[q][b] phase
             bool issued = false;
             const uint64_t qd = sw128_desc(sbase + L::kQ + q * L::kQTile, 16, 1024);
@@ -340,21 +350,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const bool active = q == 0 || item.w > kBM;   // Q tile 1 idles on items of <= 128 queries
                 if (!wait1(&bars->q_full, q_it & 1, W)) break;
                 ++q_it;
-                // S_q(j) = Q_q K(j)^T into buffer j & 1
+                // S_q(j) = Q_q K(j)^T into buffer j % NSB
                 auto qk_step = [&](int j) -> bool {
                     const int ks = k_it % L::kKS;
                     if (!wait1(&bars->k_full[ks], (k_it / L::kKS) & 1, W)) return false;
                     tc_fence_after();
                     if (active) {
                         const uint64_t kd = sw128_desc(sbase + L::kK + ks * L::kKVTile, 16, 1024);
-                        const uint32_t dst = tmem + q * 128 + (j & 1) * kBN;
+                        const uint32_t dst = s_base + (j % NSB) * kBN;
 #pragma unroll
                         for (int kk = 0; kk < D / 16; ++kk) {
                             const uint64_t offa = (uint64_t)(((kk >> 2) * (kBM * 128) + (kk & 3) * 32) >> 4);
                             const uint64_t offb = (uint64_t)(((kk >> 2) * (kBN * 128) + (kk & 3) * 32) >> 4);
                             mma_bf16(dst, qd + offa, kd + offb, idesc_qk, kk > 0);
                         }
-                        mma_commit(&bars->s_full[q][j & 1]);
+                        mma_commit(&bars->s_full[q][j % NSB]);
                     }
                     mma_commit(&bars->k_empty[ks]);
                     if (j == T - 1) mma_commit(&bars->q_empty);
@@ -362,11 +372,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     return true;
                 };
                 issued = true;
-                bool ok = qk_step(0);
-                if (ok && T > 1) ok = qk_step(1);
+                bool ok = true;
+#pragma unroll
+                for (int j = 0; j < NSB; ++j)
+                    if (ok && j < T) ok = qk_step(j);
                 for (int t = 0; t < T && ok; ++t) {
                     const int vs = v_it % L::kVS;
-                    const int b = t & 1;
+                    const int b = t % NSB;
                     ok = wait1(&bars->v_full[vs], (v_it / L::kVS) & 1, W);
                     if (ok && active) {
                         ok = wait1(&bars->p_full[q][b], (p_par >> b) & 1u, W);
@@ -374,11 +386,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (ok) {
                             p_par ^= 1u << b;
                             tc_fence_after();
-                            // O_q += P_q(t) V(t), P_q(t) from TMEM (columns q*128 + b*64 + [0, 32))
+                            // O_q += P_q(t) V(t), P_q(t) from TMEM (the first 32 columns of buffer b)
                             const uint64_t vd = sw128_desc(sbase + L::kV + vs * L::kKVTile, kBN * 128, 1024);
 #pragma unroll
                             for (int kk = 0; kk < kBN / 16; ++kk)
-                                mma_bf16_ts(tmem + 256 + q * D, tmem + q * 128 + b * kBN + kk * 8,
+                                mma_bf16_ts(o_tm, s_base + b * kBN + kk * 8,
                                             vd + (uint64_t)(kk * 2048 >> 4), idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
                             mma_commit(&bars->o_done[q][b]);
                         }
@@ -386,7 +398,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (!ok) break;
                     mma_commit(&bars->v_empty[vs]);
                     ++v_it;
-                    if (t + 2 < T) ok = qk_step(t + 2);
+                    if (t + NSB < T) ok = qk_step(t + NSB);
                 }
                 if (!ok) break;
                 if (active) ++o_items;
@@ -405,14 +417,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int q = warp >> 2;                       // Q tile of this warpgroup
         const int row = threadIdx.x - q * kBM;         // 0..127 = TMEM lane
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-        const uint32_t s_col = q * 128, o_col = 256 + q * D;
+        constexpr int NSB = SBuf<D>::n;
+        const uint32_t s_col = q * NSB * kBN, o_col = kQT * NSB * kBN + q * D;
         // bit b of s_par: parity of the next s_full[q][b] phase; bit b of o_par: parity of
         // the P V commits on o_done[q][b] before the current item (the softmax waits on
         // o_done only when it must, so it counts the phases per item instead)
         uint32_t s_par = 0, o_par = 0;
         const float c = a.scale_log2;
-        // parity of the o_done[q][j & 1] phase that completes when P(j) V(j) is done
-        auto pv_parity = [&](int j) -> uint32_t { return ((o_par >> (j & 1)) + (uint32_t)(j >> 1)) & 1u; };
+        // parity of the o_done[q][j % NSB] phase that completes when P(j) V(j) is done
+        auto pv_parity = [&](int j) -> uint32_t { return ((o_par >> (j % NSB)) + (uint32_t)(j / NSB)) & 1u; };
         for (uint32_t item_k = 0; !warp_aborted(abort_flag); ++item_k) {
             const int it = next_item(item_k);
             if (it < 0) break;
@@ -424,7 +437,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             float m_run = -INFINITY, l = 0.f;
             bool ok = true;
             for (int t = 0; t < T; ++t) {
-                const int b = t & 1;
+                const int b = t % NSB;
                 ok = waitw(&bars->s_full[q][b], (s_par >> b) & 1u, W);
                 if (!ok) break;
                 s_par ^= 1u << b;
@@ -453,7 +466,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const bool need = mt > m_run + 8.f;
                 if (t > 0 && __any_sync(0xffffffffu, need)) {
                     // rescaling O needs every earlier P V done; the last one is P(t-1) V(t-1)
-                    ok = waitw(&bars->o_done[q][(t - 1) & 1], pv_parity(t - 1), W);
+                    ok = waitw(&bars->o_done[q][(t - 1) % NSB], pv_parity(t - 1), W);
                     if (!ok) break;
                     tc_fence_after();
                     const float alpha = need ? fast_exp2(m_run - mt) : 1.f;
@@ -496,8 +509,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (!ok) break;
             // epilogue: O / l for the valid rows of this Q tile, once P(T-1) V(T-1) is done
-            if (!waitw(&bars->o_done[q][(T - 1) & 1], pv_parity(T - 1), W)) break;
-            o_par ^= (uint32_t)(((T + 1) >> 1) & 1) | ((uint32_t)((T >> 1) & 1) << 1);
+            if (!waitw(&bars->o_done[q][(T - 1) % NSB], pv_parity(T - 1), W)) break;
+            // buffer b took the P V commits of steps b, b + NSB, ... of this item
+#pragma unroll
+            for (int b = 0; b < NSB; ++b) o_par ^= (uint32_t)(((T + NSB - 1 - b) / NSB) & 1) << b;
             tc_fence_after();
             const float inv = l > 0.f ? 1.f / l : 0.f;
             const bool valid = q * kBM + row < nq;
