@@ -260,26 +260,34 @@ __global__ void __launch_bounds__(kExactWarps * 32) km_assign_exact_kernel(KmArg
         __syncwarp();
         for (int i = lane; i < R.dm; i += 32) xs[wib][i] = (double)load_x(R.X, xrow + i, a.is_bf16);
         __syncwarp();
+        // lane takes centroids lane, lane + 32, ... in ascending order, four at a time (four
+        // independent binary64 sums, each over the channels in order)
         double best = INFINITY;
         int bi = 0x7fffffff;
-        for (int c = lane; c < R.C; c += 64) {
-            const bool two = c + 32 < R.C;
-            const int c2 = two ? c + 32 : c;
-            double d0 = 0.0, d1 = 0.0;
+        constexpr int kChains = 4;
+        for (int c = lane; c < R.C; c += 32 * kChains) {
+            int cc[kChains];
+            double dd[kChains];
+#pragma unroll
+            for (int k = 0; k < kChains; ++k) {
+                cc[k] = min(c + 32 * k, R.C - 1);
+                dd[k] = 0.0;
+            }
             for (int i = 0; i < R.dm; ++i) {
                 const double x = xs[wib][i];
-                const double e0 = __dsub_rn(x, muT[(size_t)i * a.Cs + c]);
-                const double e1 = __dsub_rn(x, muT[(size_t)i * a.Cs + c2]);
-                d0 = __dadd_rn(d0, __dmul_rn(e0, e0));
-                d1 = __dadd_rn(d1, __dmul_rn(e1, e1));
+                const double *mrow = muT + (size_t)i * a.Cs;
+#pragma unroll
+                for (int k = 0; k < kChains; ++k) {
+                    const double e = __dsub_rn(x, mrow[cc[k]]);
+                    dd[k] = __dadd_rn(dd[k], __dmul_rn(e, e));
+                }
             }
-            if (d0 < best) {
-                best = d0;
-                bi = c;
-            }
-            if (two && d1 < best) {
-                best = d1;
-                bi = c2;
+#pragma unroll
+            for (int k = 0; k < kChains; ++k) {
+                if (c + 32 * k < R.C && dd[k] < best) {
+                    best = dd[k];
+                    bi = c + 32 * k;
+                }
             }
         }
         for (int off = 16; off; off >>= 1) {
