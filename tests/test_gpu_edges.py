@@ -9,7 +9,7 @@ import oracle
 from free_sparse_attention_b200 import capi, synth
 from free_sparse_attention_b200.workloads import Workload
 
-from gpu_common import compare_attention, to_np
+from gpu_common import check_selection, compare_attention, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -78,6 +78,19 @@ def test_duplicate_init_rows_give_empty_clusters():
     assert np.all(to_np(qs)[0, :, 5] == 0)
     first = np.stack([x["q"][h][qi[h, 2]] for h in range(W.H)]).astype(np.float64)
     np.testing.assert_array_equal(to_np(qc)[0, :, 5], first)
+
+
+@pytest.mark.parametrize("grid,Cq,Cm", [((1, 1, 1), 1, 1), ((1, 2, 3), 2, 3), ((1, 3, 11), 5, 4)],
+                         ids=["N1", "N6", "N33"])
+def test_tiny_token_counts(grid, Cq, Cm):
+    """Layers of 1, 6 and 33 tokens: fewer keys than one 64-key attention tile, than one
+    32-bit mask word or one 8-key row of saved bins (33: one word and one key more).  The
+    whole layer must equal the oracle's."""
+    w = Workload("tiny_n", 1, 2, *grid, 44, 42, 42, "bf16", Cq, Cm, seed=27)
+    x = synth.layer_inputs(w)
+    t = _dev(w, x)
+    _forward_and_compare(w, x, t, x["q_init"], x["k_init"])
+    _forward_and_compare(w, x, t, x["q_init"], x["k_init"], rho=0.5)
 
 
 def test_single_centroid_everywhere():
@@ -157,6 +170,39 @@ def test_equal_logits_with_spread_tables_and_a_topup():
         assert np.all(ref["mask"] == first)
         np.testing.assert_array_equal(g["final_counts"][i], ref["r"])
         np.testing.assert_array_equal(g["sel_mask"][i].view(np.uint32), ref["mask"])
+
+
+@pytest.mark.parametrize("rho", [0.3, 0.75])
+def test_two_logit_values_in_bins_larger_than_the_gather_capacity(rho):
+    """The keys take only two codes in the temporal subspace and one in the others, so every
+    cluster sees two logit values, each shared by ~3456 keys: the Top-p crossing and the
+    top-up boundary both fall inside a bin of more keys than one gather holds (2048), where
+    the ranking among equal logits is by key index.  Selection must equal the oracle's (a
+    logged near tie excepted, as everywhere)."""
+    w = Workload("twovalues", 1, 1, 3, 48, 48, 44, 42, 42, "bf16", 16, 4, seed=23)
+    p = capi.Params.from_workload(w, rho=rho)
+    rng = np.random.default_rng(12)
+    BH = w.B * w.H
+    qc = rng.standard_normal((BH, w.Cq, w.d))
+    qs = (1 + rng.multinomial(w.N - w.Cq, np.full(w.Cq, 1.0 / w.Cq), size=BH)).astype(np.int32)
+    kc = rng.standard_normal((BH, w.Cm, w.d))
+    codes = np.zeros((BH, 3, w.N), np.uint16)
+    codes[:, 0] = rng.integers(0, 2, (BH, w.N))
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).reshape((w.B, w.H) + a.shape[1:]).cuda()
+    ws = capi.alloc_workspace(p)
+    out = capi.build_lut_and_select(p, dev(qc), dev(qs), dev(kc), dev(codes), ws=ws)
+    torch.cuda.synchronize()
+    assert capi.get_device_status(ws) == 0
+    g = {k: to_np(v).reshape((BH,) + tuple(v.shape[2:])) for k, v in out.items()}
+    split = (w.d_t, w.d_h, w.d_w)
+    for i in range(BH):
+        args = (qc[i], qs[i], kc[i], codes[i], split, rho, w.alpha)
+        sel = oracle.select(*args)
+        gi = {k: g[k][i] for k in g}
+        check_selection(w, gi, sel, qs[i], lambda: oracle.select(*args, want_scores=True))
+        # each logit value is shared by more than 2048 keys, and some clusters are topped up
+        assert min((codes[i, 0] == 0).sum(), (codes[i, 0] == 1).sum()) > 2048
+        assert np.any(sel["r"] != sel["p"]) and np.all(sel["r"] < w.N)
 
 
 def test_bad_init_index_sets_status():
