@@ -505,7 +505,10 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
         float maxnm = 0.f, maxsl = 0.f, maxres = 0.f;
         // the unit's (problem, tile) advance incrementally; role constants change per problem
         int p = (int)(ub / t.TT), tile = (int)(ub % t.TT);
-        int bh = 0, r = 0, ks = 1, Cn = 1;
+        int bh = 0, r = 0, ks = 1;
+#ifdef SCOPE_DEBUG
+        int Cn = 1;   // the centroid count, the bound of the debug build's index check
+#endif
         Chunks k{16, 1, 16};
         uint16_t *assign = nullptr;
         long long assign_bh = 0;
@@ -517,7 +520,9 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
                 const RoleDesc &R = a.role[a.role0 + r];
                 ks = window_of(R.ch0, R.dm).ks;
                 k = chunks_of(R.C);
+#ifdef SCOPE_DEBUG
                 Cn = R.C;
+#endif
                 assign = R.assign;
                 assign_bh = R.assign_bh;
                 if (!warp_wait(&bars->b_full, nb & 1, abort_flag, a.status)) break;
